@@ -1,0 +1,461 @@
+"""Decode attention-stage benchmark of the JSSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jssa|reference] [--workload NAME]
+
+A step is one decode step of one attention layer at the workload's shape:
+append the new token's low-rank key row, score the low-rank cache, select a
+top-k token set per (batch, KV head), and run gather-free indexed attention
+(jssa_decode_step: three kernels).  The default workload is the 128K-context,
+batch-16 GQA layer (B=16, Hq=32, Hkv=8, d=128, T=131072, r=32, k=256).
+
+value  = steps/s of the whole job (N replicas, one per GPU, each running the
+         full workload: weak scaling, no collective on the data path), timed
+         on the device with CUDA events over exactly K steps, max over ranks.
+e2e    = the same metric through the public session API with host buffers:
+         every step copies q and the new K/V rows from pinned host memory and
+         reads the output back (synchronising per step).
+roofline = the dominant kernel (the fused score + top-k pass, jssa_select)
+         timed alone, algorithmic bytes / duration against the measured HBM copy
+         bandwidth.
+cpu_baseline / --impl reference = the fp64 C oracle on the host cores over a
+         bounded sample of (batch, KV head) pairs, scaled to a whole step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode attn-stage steps/s at 128K ctx, batch 16; achieved HBM GB/s vs peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w):
+    """Bytes the method must move per step: the low-rank key cache, the k
+    selected K and V rows per (b, h), the queries and the outputs."""
+    es = 2
+    kt = w.B * w.Hkv * w.T * w.r * es
+    sel = w.B * w.Hkv * min(w.k, w.T) * (w.d + w.Dv) * es
+    qo = w.B * w.Hq * (w.d + w.Dv) * es
+    return kt + sel + qo, kt
+
+
+def select_bytes(w):
+    """Algorithmic bytes of the fused score + top-k pass: the low-rank cache,
+    the queries and the index lists it writes."""
+    return w.B * w.Hkv * w.T * w.r * 2 + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * (w.k + 1) * 4
+
+
+def profile_traffic(kernel_file, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the summary's
+    source hash matches the kernel source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", "scan_select_%s.txt" % workload)
+    src = os.path.join(ROOT, "token_level_sparse_kv_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != h:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup_dist(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# --------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """The fp64 C oracle on a bounded sample of one workload: n_rows batch rows
+    drawn on the host (all KV heads), the prefix low-rank cache built by the
+    oracle itself; a timed unit is one decode step (append one row, score,
+    select, attend) over a chosen number of (batch, KV head) pairs."""
+
+    def __init__(self, w, n_rows, threads):
+        import oracle
+        from token_level_sparse_kv_b200.inputs import Workload, make_inputs
+
+        self.w = w
+        self.threads = threads
+        oracle.set_threads(threads)
+        ws = Workload(**{**w.__dict__, "B": n_rows, "name": w.name + "_sample"})
+        self.q, self.K, self.V, self.P, self.sl = make_inputs(ws, device="cpu")
+        self.Kt = oracle.append_lowrank(self.K, self.P, [0] * n_rows, ws.T)
+        self.pos = (self.sl - 1).clamp_min(0).tolist()
+        self.n_pairs_avail = n_rows * w.Hkv
+        self.cursor = 0
+
+    def run(self, n_pairs):
+        """One timed oracle step over n_pairs (b, h) pairs; returns seconds."""
+        import oracle
+
+        w = self.w
+        bh = [(self.cursor + i) % self.n_pairs_avail for i in range(n_pairs)]
+        self.cursor = (self.cursor + n_pairs) % self.n_pairs_avail
+        rows = sorted(set(x // w.Hkv for x in bh))
+        t0 = time.perf_counter()
+        Kt = self.Kt  # the append touches only the sampled rows' newest position
+        oracle.append_lowrank(self.K[rows[0]:rows[-1] + 1], self.P, [self.pos[r] for r in range(rows[0], rows[-1] + 1)],
+                              1, Kt=Kt[rows[0]:rows[-1] + 1])
+        s = oracle.score(self.q, self.P, Kt, self.sl, bh_list=bh)
+        idx, cnt = oracle.topk(s, self.sl, w.k, bh_list=bh)
+        oracle.attend(self.q, self.K, self.V, idx, cnt, self.sl, w.scale, dv=w.Dv, bh_list=bh,
+                      v_aliases_k=self.V is None)
+        return time.perf_counter() - t0
+
+    def describe(self, n_pairs, repeats):
+        w = self.w
+        return ("%d of %d (batch, KV head) pairs per timed step (T=%d, r=%d, k=%d): append 1 row, score, select, "
+                "attend; mean of %d, scaled x%g to a full step" % (n_pairs, w.B * w.Hkv, w.T, w.r, w.k, repeats,
+                                                                  w.B * w.Hkv / n_pairs))
+
+
+def oracle_baseline(w, budget_s, n_rows, threads):
+    """Oracle steps/s over about budget_s seconds of host work."""
+    smp = OracleSample(w, n_rows, threads)
+    n_pairs = smp.n_pairs_avail
+    smp.run(n_pairs)  # warm
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 3:
+        times.append(smp.run(n_pairs))
+    per_step = statistics.mean(times) * (w.B * w.Hkv / n_pairs)
+    return 1.0 / per_step, smp.describe(n_pairs, len(times)), threads
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from token_level_sparse_kv_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    threads = os.cpu_count() or 1
+    smp = OracleSample(w, max(1, min(w.B, args.cpu_rows)), threads)
+    # size the per-step sample so that warm-up + timed steps take about 2 minutes
+    t1 = smp.run(1)
+    t1 = min(t1, smp.run(1))
+    n_pairs = int(max(1, min(smp.n_pairs_avail, 120.0 / (args.steps + args.warmup) / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        smp.run(n_pairs)
+    times = [smp.run(n_pairs) for _ in range(args.steps)]
+    sec = statistics.mean(times) * (w.B * w.Hkv / n_pairs)
+    v = 1.0 / sec
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, world),
+            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                             "sample": smp.describe(n_pairs, args.steps)},
+            "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "dv": w.Dv, "T": w.T, "r": w.r,
+            "k": w.k, "inputs": ("N(0,1) Gaussian" if w.kind == "plain" else
+                                 "spiked Gaussian (q spike 2, key spike 3 along one direction on 1% of tokens)"),
+            "l2": ("inputs larger than L2 (%.0f MiB low-rank cache streamed per step; 4 rotating queries)"
+                   % (w.B * w.Hkv * w.T * w.r * 2 / 2**20)),
+            "parallelism": "replicas x%d (one full workload per GPU)" % world}
+
+
+# --------------------------------------------------------------- GPU timing
+def time_loop(fn, steps, stream, events_inside=None):
+    import torch
+
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        fn(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def run_jssa(args, world, rank, local):
+    import torch
+
+    from token_level_sparse_kv_b200 import ops
+    from token_level_sparse_kv_b200.inputs import WORKLOADS, Workload, make_inputs, make_queries
+
+    w0 = WORKLOADS[args.workload]
+    w = Workload(**{**w0.__dict__, "seed": w0.seed + 1000 * rank})
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    t_setup = time.perf_counter()
+    q, K, V, P, sl = make_inputs(w, device=dev)
+    qs = [q] + make_queries(w, 3, device=dev)
+    Kt = ops.build_lowrank_cache(K, P)
+    pos = (sl - 1).clamp_min(0).contiguous()
+    dims = ops.make_dims(q, K, V, P=P, Kt=Kt)
+    ws = ops.new_workspace(dims, w.k, ops.OP_DECODE_STEP, dev)
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
+    out = torch.empty((w.B, w.Hq, w.Dv), dtype=q.dtype, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    Vv = V
+    torch.cuda.synchronize()
+    log("rank %d: setup %.1f s" % (rank, time.perf_counter() - t_setup))
+
+    def step(i):
+        ops.decode_step(qs[i & 3], K, Vv, P, Kt, sl, pos, w.k, w.scale, ws=ws, idx=idx, count=cnt, out=out, lse=lse)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    status = ops.device_status(ws)
+    if status:
+        raise RuntimeError("device status 0x%x after warm-up" % status)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier(world)
+        secs = time_loop(step, args.steps, stream)
+        barrier(world)
+        # dominant kernel alone: the fused score + top-k pass (jssa_select)
+        ws_sel = ops.new_workspace(dims, w.k, ops.OP_SELECT, dev)
+        sel_steps = max(args.steps, 20)
+
+        def sel(i):
+            ops.select(qs[i & 3], P, Kt, sl, w.k, ws=ws_sel, idx=idx, count=cnt)
+
+        for i in range(3):
+            sel(i)
+        sel_secs = time_loop(sel, sel_steps, stream)
+    clocks = sampler.summary()
+    secs_max = max_over_ranks(secs, world)
+    ms = secs_max / args.steps * 1e3
+    value = world * args.steps / secs_max
+
+    peak, peak_kind = measured_peaks()
+    step_bytes, kt_bytes = algorithmic_bytes(w)
+    sbytes = select_bytes(w)
+    sel_s = sel_secs / sel_steps
+    achieved = sbytes / sel_s / 1e9
+    traffic = profile_traffic("jssa_scan.cu", w.name)
+
+    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
+            "roofline": {"bound": "hbm", "kernel": "scan_kernel (jssa_select: fused score + top-k)",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind + " (burst copy)", "traffic": traffic,
+                         "algorithmic_bytes_per_launch": sbytes, "us_per_launch": sel_s * 1e6},
+            "step_hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms / 1e3) / 1e9,
+                         "frac_of_peak": step_bytes / (ms / 1e3) / 1e9 / peak, "peak_gbs": peak},
+            "gpu_launches": 3 * args.steps}
+    if clocks:
+        line["clocks"] = clocks
+
+    if not args.quick:
+        # comparison paths from the same build, same inputs
+        ws_d = ops.new_workspace(dims, 1, ops.OP_DENSE_DECODE, dev)
+        ws_a = ops.new_workspace(dims, 1, ops.OP_APPEND, dev)
+        ws_g = ops.new_workspace(dims, w.k, ops.OP_GATHER_THEN_DENSE, dev)
+        gbuf = torch.empty(ops.gather_buffer_bytes(dims, w.k), dtype=torch.uint8, device=dev)
+        cmp_steps = max(5, min(args.steps, args.cmp_steps))
+
+        def dense(i):
+            ops.dense_decode(qs[i & 3], K, Vv, sl, w.scale, window=w.window, ws=ws_d, out=out, lse=lse)
+
+        def gather(i):
+            ops.append_lowrank(K, P, Kt, pos, 1, ws=ws_a)
+            ops.select(qs[i & 3], P, Kt, sl, w.k, ws=ws_sel, idx=idx, count=cnt)
+            ops.gather_then_dense(qs[i & 3], K, Vv, idx, cnt, sl, w.scale, gather_buf=gbuf, ws=ws_g, out=out,
+                                  lse=lse)
+
+        def split(i):
+            ops.append_lowrank(K, P, Kt, pos, 1, ws=ws_a)
+            ops.select(qs[i & 3], P, Kt, sl, w.k, ws=ws_sel, idx=idx, count=cnt)
+            ops.indexed_decode(qs[i & 3], K, Vv, idx, cnt, sl, w.scale, ws=ws_g, out=out, lse=lse)
+
+        res = {}
+        for name, fn in (("dense_full_kv", dense), ("gather_then_dense", gather), ("split_calls_gather_free", split)):
+            for i in range(3):
+                fn(i)
+            t = max_over_ranks(time_loop(fn, cmp_steps, stream), world)
+            res[name] = {"steps_per_s": world * cmp_steps / t, "ms_per_step": t / cmp_steps * 1e3}
+        res["speedup_vs_dense"] = value / res["dense_full_kv"]["steps_per_s"]
+        res["speedup_vs_gather_then_dense"] = value / res["gather_then_dense"]["steps_per_s"]
+        if w.window:
+            res["dense_full_kv"]["note"] = "sliding window %d (the local layer of the hybrid pair)" % w.window
+        line["comparison"] = res
+
+        # end to end through the session API with host buffers
+        sess = ops.DecodeSession(K, Vv, P, sl, w.k, w.scale, Kt=Kt)
+        qh = [x.cpu().pin_memory() for x in qs]
+        kh = torch.randn((w.B, w.Hkv, w.d), dtype=torch.float32).to(q.dtype).pin_memory()
+        vh = torch.randn((w.B, w.Hkv, w.Dv), dtype=torch.float32).to(q.dtype).pin_memory()
+        e2e_steps = max(5, min(args.steps, args.e2e_steps))
+        for i in range(3):
+            sess.step_from_host(qh[i & 3], kh, vh)
+            stream.synchronize()
+        barrier(world)
+        t0 = time.perf_counter()
+        for i in range(e2e_steps):
+            o = sess.step_from_host(qh[i & 3], kh, vh)
+            stream.synchronize()  # the host reads the output every step
+        te = max_over_ranks(time.perf_counter() - t0, world)
+        h2d = qh[0].numel() * qh[0].element_size() + kh.numel() * kh.element_size() + vh.numel() * vh.element_size()
+        d2h = o.numel() * o.element_size()
+        line["e2e"] = {"value": world * e2e_steps / te, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "api": "DecodeSession.step_from_host (pinned host in/out)"}
+
+    if rank == 0 and not args.no_cpu:
+        v, desc, thr = oracle_baseline(w0, args.cpu_seconds, max(1, min(w0.B, args.cpu_rows)), os.cpu_count() or 1)
+        line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": thr, "kind": "oracle", "sample": desc}
+    if status := ops.device_status(ws):
+        raise RuntimeError("device status 0x%x after the timed region" % status)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="jssa", choices=["jssa", "reference"])
+    ap.add_argument("--workload", default="gqa_128k_b16")
+    ap.add_argument("--cmp-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--cpu-rows", type=int, default=2, help="batch rows in the oracle's timed sample")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host seconds of oracle work to time")
+    ap.add_argument("--quick", action="store_true", help="skip the comparison and end-to-end passes")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = setup_dist(args)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_jssa(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

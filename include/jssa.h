@@ -1,0 +1,219 @@
+/*
+ * jssa.h -- C ABI of libjssa.so, the B200 (sm_100a) decode hot path of
+ * Joint Subspace Sparse Attention (JSSA).
+ *
+ * Method pages, cited by title and section:
+ *   [ABS]  "Joint Subspace Sparse Attention for Efficient Long-Context
+ *          Decoding" (arXiv 2610.19026), Abstract.
+ *   [NEWS] "JSSA makes token-level sparse decoding gather-free, reaching up
+ *          to full-KV throughput at 128K context" (news item), Synopsis,
+ *          Interpretation, Perspective.
+ *
+ * One decode step of one attention layer is
+ *   jssa_append_lowrank (n_new = 1)  ->  jssa_select (= jssa_score + jssa_topk)
+ *   ->  jssa_indexed_decode,
+ * or all three at once with jssa_decode_step.  jssa_dense_decode and
+ * jssa_gather_then_dense are the comparison paths the pages measure against
+ * (full-KV attention [ABS]; gather into a contiguous buffer, then a dense
+ * kernel [NEWS Interpretation para 3]).
+ *
+ * ------------------------------------------------------------ conventions --
+ * Notation: G = Hq / Hkv query heads share KV head h; query head g belongs to
+ * KV head g / G (heads h*G .. h*G+G-1).  T_b = seq_lens[b] <= T_cap.
+ * k_b = min(k, T_b).
+ *
+ * Layouts (row-major, contiguous, all device memory, all caller-owned):
+ *   q      [B, Hq, d]            dtype kv_dtype
+ *   K      [B, T_cap, Hkv, d]    dtype kv_dtype (standard GQA cache layout)
+ *   V      [B, T_cap, Hkv, dv]   dtype kv_dtype; for a latent (MLA) cache pass
+ *                                V == K, Hkv = 1, dv < d: the value of a token
+ *                                is the first dv entries of its key row
+ *   P      [Hkv, d, r]           fp32, the per-KV-head shared basis
+ *   Kt     [B, Hkv, T_cap, r]    dtype kt_dtype, the low-rank key cache
+ *   scores [B, Hkv, T_cap]       fp32
+ *   idx    [B, Hkv, k]           int32, selected token indices, ascending,
+ *                                slots >= count hold -1
+ *   count  [B, Hkv]              int32, k_b
+ *   out    [B, Hq, dv]           dtype kv_dtype
+ *   lse    [B, Hq]               fp32, natural-log log-sum-exp of the scaled
+ *                                logits (-inf for an empty token set); optional
+ * Every pointer must be 16-byte aligned.  Supported shapes: d in {64, 128,
+ * 256} with dv == d, or the latent form d = 576, dv = 512, Hkv = 1; r a
+ * power of two in [8, 128] with r <= d; G <= 16 (any G for the latent form);
+ * 1 <= k <= 2048.
+ *
+ * Status: every entry point returns JSSA_OK or a negative JSSA_ERR_* code.
+ * Arguments are checked on the host, synchronously, before anything is
+ * enqueued; on an error nothing is enqueued and jssa_last_error() returns a
+ * thread-local message.  Work is enqueued asynchronously on `stream` (a
+ * cudaStream_t; NULL = the legacy default stream).  The library never
+ * synchronises, allocates device memory or traps.
+ *
+ * Workspace: each call takes caller-owned device scratch `ws` of at least
+ * jssa_workspace_size(...) bytes.  Zero it once with jssa_workspace_init()
+ * before first use; afterwards the library keeps it valid (its arrival
+ * counters reset themselves).  Calls that share one workspace must be
+ * ordered (same stream, or events); concurrent calls need separate ones.
+ * Word 0 of the workspace is a sticky status word: kernels OR in
+ * JSSA_DEV_* bits for bad data they meet (and skip that item); read it back
+ * with a device-to-host copy of 4 bytes; jssa_workspace_init() clears it.
+ */
+#ifndef JSSA_H
+#define JSSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define JSSA_VERSION 1
+
+#if defined(__GNUC__)
+#define JSSA_API __attribute__((visibility("default")))
+#else
+#define JSSA_API
+#endif
+
+typedef void *jssa_stream_t; /* a cudaStream_t */
+
+enum {
+    JSSA_OK = 0,
+    JSSA_ERR_INVALID_ARG = -1, /* null pointer, bad dimension, k < 1, r > d, misaligned pointer */
+    JSSA_ERR_UNSUPPORTED = -2, /* a shape / dtype combination without a kernel */
+    JSSA_ERR_WORKSPACE = -3,   /* ws_bytes below jssa_workspace_size() */
+    JSSA_ERR_CUDA = -4         /* a CUDA runtime call or launch failed */
+};
+
+/* Device status bits (workspace word 0). */
+enum {
+    JSSA_DEV_SEQLEN = 1u,  /* a seq_lens entry outside [0, T_cap] (clamped) */
+    JSSA_DEV_INDEX = 2u,   /* an index outside [0, T_b) or a count outside [0, k] (skipped) */
+    JSSA_DEV_POS = 4u,     /* an append position outside [0, T_cap - n_new] (row skipped) */
+    JSSA_DEV_TIMEOUT = 8u  /* a bounded on-chip wait gave up (the kernel returned early) */
+};
+
+typedef enum { JSSA_BF16 = 0, JSSA_FP32 = 1 } jssa_dtype;
+
+/* How the G query heads of one KV head combine into one token score.  The
+ * pages do not say; SUM (the default, the timed path) adds the subspace
+ * logits of the group, MAX takes their maximum. */
+typedef enum { JSSA_AGG_SUM = 0, JSSA_AGG_MAX = 1 } jssa_agg;
+
+typedef enum {
+    JSSA_OP_APPEND = 0,
+    JSSA_OP_SCORE = 1,
+    JSSA_OP_TOPK = 2,
+    JSSA_OP_SELECT = 3,
+    JSSA_OP_INDEXED_DECODE = 4,
+    JSSA_OP_DENSE_DECODE = 5,
+    JSSA_OP_GATHER_THEN_DENSE = 6,
+    JSSA_OP_DECODE_STEP = 7
+} jssa_op;
+
+typedef struct {
+    int32_t B, Hq, Hkv, d, dv, r, T_cap;
+    int32_t kv_dtype; /* jssa_dtype of q, K, V, out */
+    int32_t kt_dtype; /* jssa_dtype of Kt */
+} jssa_dims;
+
+/* Library version (JSSA_VERSION). */
+JSSA_API int jssa_version(void);
+
+/* Text for a JSSA_OK / JSSA_ERR_* code (static storage). */
+JSSA_API const char *jssa_status_string(int status);
+
+/* Message of the last failing call on this host thread (static per thread). */
+JSSA_API const char *jssa_last_error(void);
+
+/* Bytes of workspace `op` needs for these dims and k (k is ignored by ops
+ * without a selection).  The size covers either aggregation and any sliding
+ * window, and depends on the current device's SM count.  Writes *bytes;
+ * returns a status. */
+JSSA_API int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes);
+
+/* Zero `ws_bytes` bytes of workspace on `stream` (clears the status word and
+ * the arrival counters).  Needed once per workspace before first use. */
+JSSA_API int jssa_workspace_init(void *ws, size_t ws_bytes, jssa_stream_t stream);
+
+/* Low-rank key append [ABS: shared low-dimensional query-key subspace; NEWS
+ * Synopsis: candidate tokens are scored in that subspace].
+ *   Kt[b,h,t,:] = round(sum_i K[b,t,h,i] * P[h,i,:])   (fp32 accumulation,
+ *   one round-to-nearest-even into kt_dtype)
+ * for t in [pos_begin[b], pos_begin[b] + n_new), every b and h.  pos_begin is
+ * device int32 [B].  A row whose range leaves [0, T_cap) is skipped and sets
+ * JSSA_DEV_POS.  n_new = 1 is the per-step append; n_new = T builds a prefix. */
+JSSA_API int jssa_append_lowrank(const jssa_dims *dims, const void *K, const float *P, void *Kt,
+                        const int32_t *pos_begin, int n_new, void *ws, size_t ws_bytes,
+                        jssa_stream_t stream);
+
+/* Subspace scores [NEWS Synopsis and Interpretation para 2: queries and keys
+ * share one scoring space].  With qt_g = P_h^T q_g (fp32):
+ *   SUM: scores[b,h,t] = (sum_g qt_g) . Kt[b,h,t,:]
+ *   MAX: scores[b,h,t] = max_g qt_g . Kt[b,h,t,:]
+ * for t < T_b (entries t >= T_b are not written).  fp32 arithmetic. */
+JSSA_API int jssa_score(const jssa_dims *dims, const void *q, const float *P, const void *Kt,
+               const int32_t *seq_lens, int agg, float *scores, void *ws, size_t ws_bytes,
+               jssa_stream_t stream);
+
+/* Per-(b, h) top-k [ABS: distinct per-KV-head selections; NEWS Synopsis]:
+ * the k_b tokens t < T_b that come first under (scores desc, t asc); -0.0 and
+ * +0.0 are one value; written in ascending t, -1 padded.  count may be NULL. */
+JSSA_API int jssa_topk(const jssa_dims *dims, const float *scores, const int32_t *seq_lens, int k,
+              int32_t *idx, int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream);
+
+/* jssa_score followed by jssa_topk in one pass over Kt, without writing the
+ * score array.  Results are bit-identical to the two-call path (same fp32
+ * scores, same order): the global top-k of a strict total order is the top-k
+ * of the union of the per-chunk top-k sets. */
+JSSA_API int jssa_select(const jssa_dims *dims, const void *q, const float *P, const void *Kt,
+                const int32_t *seq_lens, int agg, int k, int32_t *idx, int32_t *count,
+                void *ws, size_t ws_bytes, jssa_stream_t stream);
+
+/* Gather-free indexed attention [ABS: token-level indexed-attention kernel
+ * with distinct per-KV-head selections under the standard GQA cache layout;
+ * NEWS Interpretation para 3: selected tokens are read in place through their
+ * indices].  For every query head g of KV head h, over t in
+ * idx[b,h,0:count[b,h]]:
+ *   l_t = softmax_scale * q[b,g,:] . K[b,t,h,:]
+ *   out[b,g,:] = sum_t softmax(l)_t * V[b,t,h,:],  lse[b,g] = ln sum_t e^{l_t}
+ * fp32 accumulation, split over the index list, log-sum-exp combine.
+ * count may be NULL (then the count is the number of leading non-negative
+ * slots).  An empty set gives out = 0, lse = -inf.  An index outside [0, T_b)
+ * is skipped and sets JSSA_DEV_INDEX.  lse may be NULL. */
+JSSA_API int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                        const int32_t *idx, const int32_t *count, int k,
+                        const int32_t *seq_lens, float softmax_scale, void *out, float *lse,
+                        void *ws, size_t ws_bytes, jssa_stream_t stream);
+
+/* Full-KV decode attention (window = 0: t < T_b) or sliding-window decode
+ * (window = W > 0: t in [max(0, T_b - W), T_b)), same arithmetic as above. */
+JSSA_API int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                      const int32_t *seq_lens, int window, float softmax_scale, void *out,
+                      float *lse, void *ws, size_t ws_bytes, jssa_stream_t stream);
+
+/* The gather-then-dense comparison path [NEWS Interpretation para 3]: copy the
+ * selected K and V rows into gather_buf (laid out [2][B, Hkv, k, d]; needs
+ * 2*B*Hkv*k*d*sizeof(kv_dtype) bytes, 16-byte aligned), then run dense decode
+ * over the contiguous rows.  Same results as jssa_indexed_decode. */
+JSSA_API int jssa_gather_then_dense(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                           const int32_t *idx, const int32_t *count, int k,
+                           const int32_t *seq_lens, float softmax_scale, void *gather_buf,
+                           size_t gather_bytes, void *out, float *lse, void *ws,
+                           size_t ws_bytes, jssa_stream_t stream);
+
+/* One whole decode step: append the row at pos_begin[b] (n_new = 1), select
+ * (score + top-k, fused), then indexed decode.  Equal to the three calls in a
+ * row; idx and count receive the selection. */
+JSSA_API int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                     const float *P, void *Kt, const int32_t *seq_lens,
+                     const int32_t *pos_begin, int k, int agg, float softmax_scale,
+                     int32_t *idx, int32_t *count, void *out, float *lse, void *ws,
+                     size_t ws_bytes, jssa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JSSA_H */

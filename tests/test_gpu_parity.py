@@ -1,0 +1,412 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Every case draws seeded inputs (token_level_sparse_kv_b200.inputs), runs the
+kernels through ops.* (ctypes -> libjssa.so) and compares with oracle.*
+under the rules in tests/parity.py.  Stage-isolated checks feed the oracle the
+GPU's own upstream result (its low-rank cache, its scores, its indices), so a
+near-tie resolved differently upstream cannot leak downstream.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import check_append, check_attention, check_scores, check_selection, host
+from token_level_sparse_kv_b200 import ops
+from token_level_sparse_kv_b200.inputs import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests selected but no CUDA device is visible")
+    ops.lib()
+
+
+def W(**kw):
+    base = dict(name="t", B=2, Hq=8, Hkv=2, d=128, T=1500, r=32, k=64, kind="spiked", seed=11)
+    base.update(kw)
+    return Workload(**base)
+
+
+def draw(w, dtype=torch.bfloat16, seq_lens=None):
+    q, K, V, P, sl = make_inputs(w, device="cpu", dtype=dtype, seq_lens=seq_lens)
+    dev = lambda t: None if t is None else t.to(DEV).contiguous()
+    return (q, K, V, P, sl), (dev(q), dev(K), dev(V), dev(P), dev(sl))
+
+
+def score_scale(q, P, Kt_host, G, agg):
+    """sum_j (sum_i |q_i| |P_ij|) |Kt_j| per (b,h,t): the size of the terms of a score."""
+    qa = np.abs(oracle.to_f64(q))
+    B, Hq, d = qa.shape
+    Hkv = Hq // G
+    qa = qa.reshape(B, Hkv, G, d).sum(2)
+    pa = np.abs(P.to(torch.float64).numpy())
+    qp = np.einsum("bhi,hij->bhj", qa, pa)
+    return np.einsum("bhj,bhtj->bht", qp, np.abs(oracle.to_f64(Kt_host)))
+
+
+# ------------------------------------------------------------------ append
+@pytest.mark.parametrize("d,r,Hkv,kt", [(128, 32, 2, torch.bfloat16), (128, 32, 2, torch.float32),
+                                        (256, 64, 2, torch.bfloat16), (64, 8, 3, torch.bfloat16),
+                                        (576, 64, 1, torch.bfloat16)])
+def test_append_prefix_and_step(d, r, Hkv, kt):
+    w = W(d=d, r=r, Hkv=Hkv, Hq=Hkv * 2, T=333, dv=512 if d == 576 else None, latent=d == 576)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    Kt = ops.build_lowrank_cache(Kd, Pd, kt_dtype=kt)
+    torch.cuda.synchronize()
+    check_append(Kt, K, P, [0] * w.B, w.T)
+    # per-step append at a different position per batch row; rows elsewhere untouched
+    before = Kt.clone()
+    K2 = K.clone()
+    pos = [5, 300][: w.B]
+    for b, p in enumerate(pos):
+        K2[b, p] = torch.randn(K2[b, p].shape, generator=torch.Generator().manual_seed(b)).to(K2.dtype)
+    Kd.copy_(K2.to(DEV))
+    ops.append_lowrank(Kd, Pd, Kt, torch.tensor(pos, dtype=torch.int32, device=DEV), 1)
+    torch.cuda.synchronize()
+    check_append(Kt, K2, P, pos, 1)
+    changed = (Kt != before).reshape(w.B, Hkv, w.T, -1).any(-1).cpu()
+    for b in range(w.B):
+        rows = torch.nonzero(changed[b].any(0)).flatten().tolist()
+        assert set(rows) <= {pos[b]}
+
+
+# ------------------------------------------------------------------- score
+@pytest.mark.parametrize("agg", [ops.AGG_SUM, ops.AGG_MAX])
+@pytest.mark.parametrize("kt", [torch.bfloat16, torch.float32])
+def test_score_parity(agg, kt):
+    w = W(T=2049, Hq=8, Hkv=2)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[2049, 700])
+    Kt = ops.build_lowrank_cache(Kd, Pd, kt_dtype=kt)
+    s = ops.score(qd, Pd, Kt, sld, agg=agg)
+    torch.cuda.synchronize()
+    Kt_h = host(Kt)
+    ref = oracle.score(q, P, Kt_h, sl, agg=agg)
+    sg = host(s).numpy()
+    check_scores(sg, ref, score_scale(q, P, Kt_h, w.G, agg))
+    assert np.all(np.isnan(sg[1, :, 700:])), "entries past T_b were written"
+
+
+# -------------------------------------------------------------------- topk
+def test_topk_is_exact_on_the_same_scores():
+    w = W(B=3, Hkv=2, Hq=4, T=9000)
+    g = torch.Generator().manual_seed(3)
+    s = torch.randn(w.B, w.Hkv, w.T, generator=g)
+    s[0, 0, 100:4000] = torch.round(s[0, 0, 100:4000] * 4) / 4  # heavy exact ties
+    s[1, 1, :] = 0.0
+    s[1, 1, ::3] = -0.0  # -0.0 and +0.0 are one value
+    s[2, 0, 10:20] = 1e30
+    sl = torch.tensor([9000, 8999, 300], dtype=torch.int32)
+    for k in (1, 64, 300, 2048):
+        idx, cnt = ops.topk(s.to(DEV), sl.to(DEV), k)
+        torch.cuda.synchronize()
+        ref_idx, ref_cnt = oracle.topk(s.double().numpy(), sl, k)
+        np.testing.assert_array_equal(host(idx).numpy(), ref_idx)
+        np.testing.assert_array_equal(host(cnt).numpy(), ref_cnt)
+
+
+def test_topk_ragged_and_empty():
+    g = torch.Generator().manual_seed(4)
+    s = torch.randn(4, 1, 5000, generator=g)
+    sl = torch.tensor([0, 1, 255, 5000], dtype=torch.int32)
+    idx, cnt = ops.topk(s.to(DEV), sl.to(DEV), 256)
+    torch.cuda.synchronize()
+    ref_idx, ref_cnt = oracle.topk(s.double().numpy(), sl, 256)
+    np.testing.assert_array_equal(host(idx).numpy(), ref_idx)
+    np.testing.assert_array_equal(host(cnt).numpy(), ref_cnt)
+
+
+# ------------------------------------------------------------------ select
+@pytest.mark.parametrize("case", ["small", "multi_segment", "r64", "fp32", "max"])
+def test_select_equals_score_then_topk_and_matches_oracle(case):
+    kt = torch.bfloat16
+    agg = ops.AGG_SUM
+    if case == "small":
+        w, sl = W(T=1500, k=64), [1500, 1111]
+    elif case == "multi_segment":
+        w, sl = W(B=4, Hkv=8, Hq=32, T=40000, k=256, seed=12), [40000, 39999, 12345, 257]
+    elif case == "r64":
+        w, sl = W(d=256, r=64, Hq=16, Hkv=2, T=5000, k=256, seed=13), [5000, 4097]
+    elif case == "fp32":
+        w, sl, kt = W(T=3000, k=100, seed=14), [3000, 2999], torch.float32
+    else:
+        w, sl, agg = W(T=3000, k=128, seed=15), [3000, 1500], ops.AGG_MAX
+    dtype = torch.float32 if kt == torch.float32 else torch.bfloat16
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, dtype=dtype, seq_lens=sl)
+    Kt = ops.build_lowrank_cache(Kd, Pd, kt_dtype=kt)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k, agg=agg)
+    s = ops.score(qd, Pd, Kt, sld, agg=agg)
+    idx2, cnt2 = ops.topk(s, sld, w.k)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(idx).numpy(), host(idx2).numpy())
+    np.testing.assert_array_equal(host(cnt).numpy(), host(cnt2).numpy())
+    ref = oracle.score(q, P, host(Kt), slh, agg=agg)
+    check_selection(host(idx).numpy(), host(cnt).numpy(), ref, slh.numpy(), w.k)
+
+
+def test_select_exact_ties_take_lowest_index():
+    w = W(B=1, Hkv=2, Hq=4, T=3000, k=50, kind="plain", seed=16)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    # head 0: every row equal -> every score equal -> the first k tokens
+    Kd[0, :, 0, :] = Kd[0, 7, 0, :]
+    # head 1: a block of 100 identical rows at 1000..1099 along P P^T (sum of the
+    # group's queries), far above every other token -> the first 50 of the block
+    x = q[0, 2:4, :].float().sum(0)
+    y = P[1] @ (P[1].T @ x)
+    Kd[0, 1000:1100, 1, :] = (50.0 * y / y.norm()).to(Kd.dtype).to(DEV)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    torch.cuda.synchronize()
+    assert host(idx)[0, 0].tolist() == list(range(50))
+    assert host(idx)[0, 1].tolist() == list(range(1000, 1050))
+    # permuting the tokens permutes the selection (distinct scores)
+    perm = torch.randperm(w.T, generator=torch.Generator().manual_seed(1))
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(W(B=1, Hkv=2, Hq=4, T=3000, k=50, seed=17))
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    i1, _ = ops.select(qd, Pd, Kt, sld, w.k)
+    Kp = Kd[:, perm.to(DEV)].contiguous()
+    Ktp = ops.build_lowrank_cache(Kp, Pd)
+    i2, _ = ops.select(qd, Pd, Ktp, sld, w.k)
+    torch.cuda.synchronize()
+    for h in range(2):
+        assert sorted(perm[host(i2)[0, h].long()].tolist()) == host(i1)[0, h].tolist()
+
+
+# ------------------------------------------------------------------ attend
+@pytest.mark.parametrize("d,G,dtype", [(128, 4, torch.bfloat16), (128, 4, torch.float32), (256, 8, torch.bfloat16),
+                                       (64, 1, torch.bfloat16), (128, 16, torch.bfloat16), (256, 2, torch.float32)])
+def test_indexed_decode_parity(d, G, dtype):
+    w = W(d=d, Hq=2 * G, Hkv=2, T=1000, k=200, r=8, seed=20 + d + G)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, dtype=dtype, seq_lens=[1000, 450])
+    g = torch.Generator().manual_seed(5)
+    idx = torch.full((w.B, w.Hkv, w.k), -1, dtype=torch.int32)
+    cnt = torch.tensor([[200, 131], [1, 0]], dtype=torch.int32)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            c = int(cnt[b, h])
+            idx[b, h, :c] = torch.sort(torch.randperm(int(sl[b]), generator=g)[:c])[0].to(torch.int32)
+    out, lse = ops.indexed_decode(qd, Kd, Vd, idx.to(DEV), cnt.to(DEV), sld, w.scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attend(q, K, V, idx, cnt, sl, w.scale)
+    check_attention(out, lse, ref_o, ref_l, dtype)
+    # count = NULL: the count is the number of leading non-negative slots
+    out2, lse2 = ops.indexed_decode(qd, Kd, Vd, idx.to(DEV), None, sld, w.scale)
+    torch.cuda.synchronize()
+    check_attention(out2, lse2, ref_o, ref_l, dtype)
+
+
+@pytest.mark.parametrize("window", [0, 100, 5000])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_dense_decode_parity(window, dtype):
+    w = W(T=3000, Hq=8, Hkv=2, seed=30)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, dtype=dtype, seq_lens=[3000, 77])
+    out, lse = ops.dense_decode(qd, Kd, Vd, sld, w.scale, window=window)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.dense(q, K, V, sl, w.scale, window=window)
+    check_attention(out, lse, ref_o, ref_l, dtype)
+
+
+def test_dense_decode_long_many_splits():
+    w = W(B=1, T=70000, Hq=16, Hkv=2, d=256, r=8, seed=31)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    out, lse = ops.dense_decode(qd, Kd, Vd, sld, w.scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.dense(q, K, V, sl, w.scale)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
+def test_sparse_with_k_equal_T_equals_dense():
+    w = W(T=640, k=640, seed=32)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    o1, l1 = ops.indexed_decode(qd, Kd, Vd, idx, cnt, sld, w.scale)
+    o2, l2 = ops.dense_decode(qd, Kd, Vd, sld, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(idx[:, :, :640].cpu(), torch.arange(640, dtype=torch.int32).expand(2, 2, 640))
+    torch.testing.assert_close(o1.float(), o2.float(), rtol=0, atol=2e-2)
+    torch.testing.assert_close(l1, l2, rtol=0, atol=1e-3)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gather_then_dense_matches_indexed_and_oracle(dtype):
+    w = W(T=4000, k=256, seed=33)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, dtype=dtype, seq_lens=[4000, 100])
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    o1, l1 = ops.indexed_decode(qd, Kd, Vd, idx, cnt, sld, w.scale)
+    o2, l2 = ops.gather_then_dense(qd, Kd, Vd, idx, cnt, sld, w.scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attend(q, K, V, host(idx), host(cnt), sl, w.scale)
+    check_attention(o1, l1, ref_o, ref_l, dtype)
+    check_attention(o2, l2, ref_o, ref_l, dtype)
+
+
+# ------------------------------------------------------------- whole step
+@pytest.mark.parametrize("agg", [ops.AGG_SUM, ops.AGG_MAX])
+def test_decode_step_end_to_end(agg):
+    w = W(B=3, T=6000, k=256, seed=40)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[6000, 5999, 1])
+    pos = (sl - 1).clamp_min(0)
+    # prefix cache built without the newest row, which the step appends
+    Kt0 = ops.build_lowrank_cache(Kd, Pd)
+    for b in range(w.B):
+        Kt0[b, :, int(pos[b])] = 0
+    out, lse, idx, cnt = ops.decode_step(qd, Kd, Vd, Pd, Kt0, sld, pos.to(DEV), w.k, w.scale, agg=agg)
+    torch.cuda.synchronize()
+    # stage-isolated: oracle scores on the GPU's low-rank cache (after the append)
+    check_append(Kt0, K, P, pos.tolist(), 1)
+    ref_s = oracle.score(q, P, host(Kt0), sl, agg=agg)
+    check_selection(host(idx).numpy(), host(cnt).numpy(), ref_s, sl.numpy(), w.k)
+    ref_o, ref_l = oracle.attend(q, K, V, host(idx), host(cnt), sl, w.scale)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+    # end to end: the oracle's own step from its own low-rank cache
+    Kt_or = oracle.append_lowrank(K, P, [0] * w.B, w.T)
+    _, s_or, idx_or, cnt_or, out_or, lse_or = oracle.step(q, K, V, P, Kt_or, sl, w.k, w.scale, agg=agg)
+    same = np.all(host(idx).numpy() == idx_or, axis=2)
+    assert same.mean() >= 0.5, "selections differ from the oracle's own in most heads"
+    o = host(out).double().numpy()
+    G = w.G
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            if same[b, h]:
+                assert np.abs(o[b, h * G:(h + 1) * G] - out_or[b, h * G:(h + 1) * G]).max() <= 2e-2
+
+
+# -------------------------------------------------------------- edge cases
+def test_empty_and_short_sequences():
+    w = W(B=3, T=300, k=64, seed=50)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[0, 5, 300])
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    out, lse = ops.indexed_decode(qd, Kd, Vd, idx, cnt, sld, w.scale)
+    do, dl = ops.dense_decode(qd, Kd, Vd, sld, w.scale)
+    torch.cuda.synchronize()
+    c = host(cnt)
+    assert c[0].tolist() == [0, 0] and c[1].tolist() == [5, 5] and c[2].tolist() == [64, 64]
+    assert torch.all(host(idx)[0] == -1)
+    assert host(idx)[1, 0, :5].tolist() == [0, 1, 2, 3, 4]
+    assert torch.all(host(out)[0] == 0) and torch.all(torch.isneginf(host(lse)[0]))
+    assert torch.all(host(do)[0] == 0) and torch.all(torch.isneginf(host(dl)[0]))
+    ref_o, ref_l = oracle.attend(q, K, V, host(idx), c, sl, w.scale)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
+def test_device_status_flags_bad_data_without_fault():
+    w = W(B=2, T=500, k=16, seed=51)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    idx = torch.arange(16, dtype=torch.int32).expand(2, 2, 16).contiguous()
+    bad = idx.clone()
+    bad[1, 1, 3] = 100000  # outside [0, T_b): skipped and flagged
+    cnt = torch.full((2, 2), 16, dtype=torch.int32)
+    dims = ops.make_dims(qd, Kd, Vd, r=8)
+    ws = ops.new_workspace(dims, 16, ops.OP_INDEXED_DECODE, qd.device)
+    out, lse = ops.indexed_decode(qd, Kd, Vd, bad.to(DEV), cnt.to(DEV), sld, w.scale, ws=ws)
+    assert ops.device_status(ws) & ops.DEV_INDEX
+    keep = bad.clone()
+    keep[1, 1, 3:15] = keep[1, 1, 4:16].clone()
+    kc = cnt.clone()
+    kc[1, 1] = 15
+    ref_o, ref_l = oracle.attend(q, K, V, keep, kc, sl, w.scale)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+    # seq_lens above T_cap: clamped and flagged
+    ops.workspace_init(ws)
+    big = torch.tensor([10**6, 500], dtype=torch.int32, device=DEV)
+    ops.indexed_decode(qd, Kd, Vd, idx.to(DEV), cnt.to(DEV), big, w.scale, ws=ws)
+    assert ops.device_status(ws) & ops.DEV_SEQLEN
+    # append position out of range: row skipped and flagged
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    before = Kt.clone()
+    wsa = ops.new_workspace(dims, 1, ops.OP_APPEND, qd.device)
+    ops.append_lowrank(Kd, Pd, Kt, torch.tensor([499, 500], dtype=torch.int32, device=DEV), 1, ws=wsa)
+    assert ops.device_status(wsa) & ops.DEV_POS
+    assert torch.equal(Kt[1], before[1])
+
+
+def test_invalid_arguments_raise():
+    w = W(B=1, Hq=64, Hkv=2, T=100, k=8, seed=52)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    idx = torch.zeros((1, 2, 8), dtype=torch.int32, device=DEV)
+    with pytest.raises(ops.JssaError) as e:
+        ops.indexed_decode(qd, Kd, Vd, idx, None, sld, 1.0)  # G = 32 > 16
+    assert e.value.code == -2
+    w = W(B=1, T=100, k=8, seed=53)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    dims = ops.make_dims(qd, Kd, Vd, r=8)
+    small = torch.zeros(64, dtype=torch.uint8, device=DEV)
+    with pytest.raises(ops.JssaError) as e:
+        ops.indexed_decode(qd, Kd, Vd, idx, None, sld, 1.0, ws=small)
+    assert e.value.code == -3
+    with pytest.raises(ops.JssaError) as e:
+        ops.select(qd, Pd, ops.build_lowrank_cache(Kd, Pd), sld, 4096)
+    assert e.value.code == -1
+    assert dims.B == 1
+
+
+# ------------------------------------------------------- full-size samples
+def _full_size_sampled(wname, pairs, dense_check=True):
+    from token_level_sparse_kv_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[wname]
+    q, K, V, P, sl = make_inputs(w, device=DEV)
+    Kt = ops.build_lowrank_cache(K, P)
+    pos = (sl - 1).clamp_min(0)
+    out, lse, idx, cnt = ops.decode_step(q, K, V, P, Kt, sl, pos, w.k, w.scale)
+    s = ops.score(q, P, Kt, sl)
+    idx2, cnt2 = ops.topk(s, sl, w.k)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(cnt, cnt2)
+    G = w.G
+    for b, h in pairs:
+        qs = q[b:b + 1, h * G:(h + 1) * G].contiguous()
+        Ks = K[b:b + 1, :, h:h + 1].contiguous()
+        Vs = V[b:b + 1, :, h:h + 1].contiguous()
+        Ps = P[h:h + 1].contiguous()
+        Kts = Kt[b:b + 1, h:h + 1].contiguous()
+        slh = sl[b:b + 1].cpu()
+        # the newest row was appended by the step: check it, then score the GPU cache
+        check_append(Kt[b:b + 1, h:h + 1], host(Ks), host(Ps), [int(pos[b])], 1)
+        ref_s = oracle.score(host(qs), host(Ps), host(Kts), slh)
+        sg = host(s[b:b + 1, h:h + 1]).numpy()
+        check_scores(sg, ref_s, score_scale(host(qs), host(Ps), host(Kts), G, 0))
+        check_selection(host(idx[b:b + 1, h:h + 1]).numpy(), host(cnt[b:b + 1, h:h + 1]).numpy(), ref_s,
+                        slh.numpy(), w.k)
+        ref_o, ref_l = oracle.attend(host(qs), host(Ks), host(Vs), host(idx[b:b + 1, h:h + 1]),
+                                     host(cnt[b:b + 1, h:h + 1]), slh, w.scale)
+        check_attention(out[b:b + 1, h * G:(h + 1) * G], lse[b:b + 1, h * G:(h + 1) * G], ref_o, ref_l,
+                        torch.bfloat16)
+    if dense_check:
+        do, dl = ops.dense_decode(q, K, V, sl, w.scale, window=w.window)
+        torch.cuda.synchronize()
+        for b, h in pairs[:2]:
+            ref_o, ref_l = oracle.dense(host(q[b:b + 1, h * G:(h + 1) * G].contiguous()),
+                                        host(K[b:b + 1, :, h:h + 1].contiguous()),
+                                        host(V[b:b + 1, :, h:h + 1].contiguous()), sl[b:b + 1].cpu(), w.scale,
+                                        window=w.window)
+            check_attention(do[b:b + 1, h * G:(h + 1) * G], dl[b:b + 1, h * G:(h + 1) * G], ref_o, ref_l,
+                            torch.bfloat16)
+    del q, K, V, Kt, s
+    torch.cuda.empty_cache()
+
+
+def test_full_size_gqa_128k_b16_sampled():
+    _full_size_sampled("gqa_128k_b16", [(0, 0), (7, 3), (15, 7), (9, 5)])
+
+
+def test_full_size_gqa_32k_b4_sampled():
+    _full_size_sampled("gqa_32k_b4", [(0, 0), (3, 7), (2, 4)])
+
+
+def test_full_size_hybrid_global_sampled():
+    _full_size_sampled("hybrid_global_128k_b8", [(0, 0), (7, 1), (4, 0)])
+
+
+def test_full_size_gqa_4k_b1_all_heads():
+    _full_size_sampled("gqa_4k_b1", [(0, h) for h in range(8)])

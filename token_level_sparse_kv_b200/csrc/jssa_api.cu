@@ -1,0 +1,537 @@
+// C ABI of libjssa (declared in include/jssa.h): host-side argument checks,
+// workspace layout and kernel launches.  No allocation, no synchronisation.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "jssa_internal.h"
+
+namespace jssa {
+
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        dev = 0;
+    }
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+}  // namespace jssa
+
+using namespace jssa;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    cudaGetLastError();  // clear this runtime's last-error slot
+    return fail(JSSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Shape {
+    bool latent;
+    int G, es_kv, es_kt;
+    int BH;
+};
+
+int check_dims(const jssa_dims *d, Shape *sh) {
+    if (!d) return fail(JSSA_ERR_INVALID_ARG, "dims is NULL");
+    if (d->B < 0 || d->Hq < 1 || d->Hkv < 1 || d->T_cap < 1 || d->d < 1 || d->dv < 1 || d->r < 1)
+        return fail(JSSA_ERR_INVALID_ARG, "bad dimension (B=%d Hq=%d Hkv=%d d=%d dv=%d r=%d T_cap=%d)", d->B, d->Hq,
+                    d->Hkv, d->d, d->dv, d->r, d->T_cap);
+    if (d->Hq % d->Hkv != 0) return fail(JSSA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", d->Hq, d->Hkv);
+    if ((long long)d->B * d->Hkv > 65535) return fail(JSSA_ERR_UNSUPPORTED, "B*Hkv above 65535");
+    if ((d->kv_dtype != JSSA_BF16 && d->kv_dtype != JSSA_FP32) || (d->kt_dtype != JSSA_BF16 && d->kt_dtype != JSSA_FP32))
+        return fail(JSSA_ERR_INVALID_ARG, "bad dtype code (kv=%d kt=%d)", d->kv_dtype, d->kt_dtype);
+    if (d->r > d->d) return fail(JSSA_ERR_INVALID_ARG, "r=%d exceeds d=%d", d->r, d->d);
+    if (d->r < 8 || d->r > 128 || (d->r & (d->r - 1)) != 0)
+        return fail(JSSA_ERR_UNSUPPORTED, "r=%d: supported ranks are powers of two in [8, 128]", d->r);
+    const bool latent = d->d == 576 && d->dv == 512 && d->Hkv == 1;
+    const bool gqa = (d->d == 64 || d->d == 128 || d->d == 256) && d->dv == d->d;
+    if (!latent && !gqa)
+        return fail(JSSA_ERR_UNSUPPORTED, "d=%d dv=%d: supported are d in {64,128,256} with dv=d, or d=576 dv=512 Hkv=1",
+                    d->d, d->dv);
+    sh->latent = latent;
+    sh->G = d->Hq / d->Hkv;
+    sh->es_kv = d->kv_dtype == JSSA_BF16 ? 2 : 4;
+    sh->es_kt = d->kt_dtype == JSSA_BF16 ? 2 : 4;
+    sh->BH = d->B * d->Hkv;
+    return JSSA_OK;
+}
+
+int check_k(int k) {
+    if (k < 1 || k > kMaxK) return fail(JSSA_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, kMaxK);
+    return JSSA_OK;
+}
+
+int check_attn_shape(const jssa_dims *d, const Shape &sh) {
+    if (sh.latent) return fail(JSSA_ERR_UNSUPPORTED, "latent-cache attention (d=576) has no kernel in this build");
+    if (sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "G=%d query heads per KV head above %d", sh.G, kMaxG);
+    (void)d;
+    return JSSA_OK;
+}
+
+#define REQUIRE_PTR(p)                                                                          \
+    do {                                                                                        \
+        if (!(p)) return fail(JSSA_ERR_INVALID_ARG, "%s is NULL", #p);                          \
+        if (!aligned16(p)) return fail(JSSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+#define OPTIONAL_PTR(p)                                                                         \
+    do {                                                                                        \
+        if ((p) && !aligned16(p)) return fail(JSSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+// ----------------------------------------------------------- workspace ---
+struct Layout {
+    size_t qproj = 0, cand_key = 0, cand_idx = 0, cand_cnt = 0, sel_ctr = 0;
+    size_t part_o = 0, part_ml = 0, att_ctr = 0, gcount = 0;
+    size_t total = 256;  // [0, 256): status word
+    ScanPlan sp{};
+    AttnPlan ap{};
+};
+
+size_t take(size_t &off, size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return o;
+}
+
+int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, Layout &L) {
+    const int nq = (src != SRC_SCORES && agg == JSSA_AGG_MAX) ? sh.G : 1;
+    cudaError_t e = plan_scan(src, MODE_SELECT, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.sp);
+    if (e != cudaSuccess) return cuda_fail(e, "planning the selection pass");
+    const size_t nc = (size_t)sh.BH * L.sp.max_seg * k;
+    L.cand_key = take(L.total, nc * 4);
+    L.cand_idx = take(L.total, nc * 4);
+    L.cand_cnt = take(L.total, (size_t)sh.BH * L.sp.max_seg * 4);
+    L.sel_ctr = take(L.total, (size_t)sh.BH * 4);
+    return JSSA_OK;
+}
+
+int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout &L) {
+    cudaError_t e = plan_attend(src, d->kv_dtype, d->d, sh.G, d->B, d->Hkv, npos, &L.ap);
+    if (e != cudaSuccess) return cuda_fail(e, "planning the attention pass");
+    L.part_o = take(L.total, (size_t)sh.BH * L.ap.splits * sh.G * d->dv * 4);
+    L.part_ml = take(L.total, (size_t)sh.BH * L.ap.splits * sh.G * 2 * 4);
+    L.att_ctr = take(L.total, (size_t)sh.BH * 4);
+    return JSSA_OK;
+}
+
+int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L) {
+    L = Layout();
+    int st = JSSA_OK;
+    const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
+    switch (op) {
+        case JSSA_OP_APPEND: break;
+        case JSSA_OP_SCORE: {
+            L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
+            cudaError_t e = plan_scan(d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, MODE_WRITE, agg, d->B,
+                                      d->Hkv, d->T_cap, d->r, nq, 0, &L.sp);
+            if (e != cudaSuccess) return cuda_fail(e, "planning the score pass");
+            break;
+        }
+        case JSSA_OP_TOPK: st = layout_select(d, sh, SRC_SCORES, k, agg, L); break;
+        case JSSA_OP_SELECT:
+            L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
+            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L);
+            break;
+        case JSSA_OP_INDEXED_DECODE: st = layout_attend(d, sh, ATT_INDEXED, k, L); break;
+        case JSSA_OP_DENSE_DECODE:
+            st = layout_attend(d, sh, ATT_RANGE, window > 0 && window < d->T_cap ? window : d->T_cap, L);
+            break;
+        case JSSA_OP_GATHER_THEN_DENSE:
+            st = layout_attend(d, sh, ATT_RANGE_BH, k, L);
+            if (st == JSSA_OK) L.gcount = take(L.total, (size_t)sh.BH * 4);
+            break;
+        case JSSA_OP_DECODE_STEP:
+            L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
+            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L);
+            if (st == JSSA_OK) st = layout_attend(d, sh, ATT_INDEXED, k, L);
+            break;
+        default: return fail(JSSA_ERR_INVALID_ARG, "unknown op %d", op);
+    }
+    return st;
+}
+
+int check_ws(void *ws, size_t ws_bytes, const Layout &L) {
+    if (!ws) return fail(JSSA_ERR_INVALID_ARG, "ws is NULL");
+    if (!aligned16(ws)) return fail(JSSA_ERR_INVALID_ARG, "ws is not 16-byte aligned");
+    if (ws_bytes < L.total)
+        return fail(JSSA_ERR_WORKSPACE, "workspace of %zu bytes is below the %zu bytes needed", ws_bytes, L.total);
+    return JSSA_OK;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<char *>(ws) + off);
+}
+
+cudaStream_t S(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+void fill_attn(AttnArgs &a, const jssa_dims *d, const Shape &sh, const void *q, const void *K, const void *V,
+               const int32_t *seq_lens, float scale, void *out, float *lse, void *ws, const Layout &L) {
+    memset(&a, 0, sizeof a);
+    a.q = q;
+    a.K = K;
+    a.V = V;
+    a.k_sb = (long long)d->T_cap * d->Hkv * d->d;
+    a.k_st = (long long)d->Hkv * d->d;
+    a.k_sh = d->d;
+    a.v_sb = (long long)d->T_cap * d->Hkv * d->dv;
+    a.v_st = (long long)d->Hkv * d->dv;
+    a.v_sh = d->dv;
+    a.seq_lens = seq_lens;
+    a.B = d->B;
+    a.Hq = d->Hq;
+    a.Hkv = d->Hkv;
+    a.G = sh.G;
+    a.T_cap = d->T_cap;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.part_o = at<float>(ws, L.part_o);
+    a.part_ml = at<float>(ws, L.part_ml);
+    a.counters = at<uint32_t>(ws, L.att_ctr);
+    a.out = out;
+    a.lse = lse;
+    a.status = at<uint32_t>(ws, 0);
+}
+
+int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *P, const void *Kt,
+               const int32_t *seq_lens, int agg, int k, int32_t *idx, int32_t *count, void *ws, const Layout &L,
+               cudaStream_t s, bool with_project) {
+    const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
+    if (with_project) {
+        ProjArgs pj{q, P, at<float>(ws, L.qproj), d->B, d->Hq, d->Hkv, d->d, d->r, agg};
+        cudaError_t e = launch_project(pj, s, true, d->kv_dtype);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the query projection");
+    }
+    ScanArgs sa;
+    memset(&sa, 0, sizeof sa);
+    sa.src = Kt;
+    sa.qproj = at<float>(ws, L.qproj);
+    sa.seq_lens = seq_lens;
+    sa.cand_key = at<uint32_t>(ws, L.cand_key);
+    sa.cand_idx = at<int32_t>(ws, L.cand_idx);
+    sa.cand_cnt = at<int32_t>(ws, L.cand_cnt);
+    sa.counters = at<uint32_t>(ws, L.sel_ctr);
+    sa.idx_out = idx;
+    sa.count_out = count;
+    sa.status = at<uint32_t>(ws, 0);
+    sa.B = d->B;
+    sa.Hkv = d->Hkv;
+    sa.T_cap = d->T_cap;
+    sa.r = d->r;
+    sa.nq = nq;
+    sa.k = k;
+    cudaError_t e = launch_scan(L.sp, sa, agg, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the selection pass");
+    return JSSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int jssa_version(void) { return JSSA_VERSION; }
+
+const char *jssa_status_string(int status) {
+    switch (status) {
+        case JSSA_OK: return "JSSA_OK";
+        case JSSA_ERR_INVALID_ARG: return "JSSA_ERR_INVALID_ARG: invalid argument";
+        case JSSA_ERR_UNSUPPORTED: return "JSSA_ERR_UNSUPPORTED: shape or dtype without a kernel";
+        case JSSA_ERR_WORKSPACE: return "JSSA_ERR_WORKSPACE: workspace too small";
+        case JSSA_ERR_CUDA: return "JSSA_ERR_CUDA: CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+const char *jssa_last_error(void) { return g_err; }
+
+int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if (!bytes) return fail(JSSA_ERR_INVALID_ARG, "bytes is NULL");
+    const bool needs_k = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_INDEXED_DECODE ||
+                         op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP;
+    if (needs_k && (st = check_k(k))) return st;
+    if ((op == JSSA_OP_INDEXED_DECODE || op == JSSA_OP_DENSE_DECODE || op == JSSA_OP_GATHER_THEN_DENSE ||
+         op == JSSA_OP_DECODE_STEP) &&
+        (st = check_attn_shape(dims, sh)))
+        return st;
+    size_t best = 0;
+    for (int agg = 0; agg < 2; ++agg) {
+        if (agg == JSSA_AGG_MAX && sh.G > kMaxG) continue;
+        Layout L;
+        st = build_layout(dims, sh, k, op, agg, 0, L);
+        if (st) return st;
+        if (L.total > best) best = L.total;
+    }
+    *bytes = best;
+    return JSSA_OK;
+}
+
+int jssa_workspace_init(void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    if (!ws) return fail(JSSA_ERR_INVALID_ARG, "ws is NULL");
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace");
+    return JSSA_OK;
+}
+
+int jssa_append_lowrank(const jssa_dims *dims, const void *K, const float *P, void *Kt, const int32_t *pos_begin,
+                        int n_new, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(P);
+    REQUIRE_PTR(Kt);
+    REQUIRE_PTR(pos_begin);
+    if (n_new < 0 || n_new > dims->T_cap) return fail(JSSA_ERR_INVALID_ARG, "n_new=%d outside [0, T_cap]", n_new);
+    Layout L;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_APPEND, 0, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (n_new == 0 || dims->B == 0) return JSSA_OK;
+    AppendArgs a{K, P, Kt, pos_begin, at<uint32_t>(ws, 0), dims->B, dims->T_cap, dims->Hkv, dims->d, dims->r, n_new, 0};
+    cudaError_t e = launch_append(a, S(stream), true, dims->kv_dtype, dims->kt_dtype);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the low-rank append");
+    return JSSA_OK;
+}
+
+int jssa_score(const jssa_dims *dims, const void *q, const float *P, const void *Kt, const int32_t *seq_lens,
+               int agg, float *scores, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(P);
+    REQUIRE_PTR(Kt);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(scores);
+    if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
+    if (agg == JSSA_AGG_MAX && sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "MAX aggregation needs G <= %d", kMaxG);
+    Layout L;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_SCORE, agg, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
+    ProjArgs pj{q, P, at<float>(ws, L.qproj), dims->B, dims->Hq, dims->Hkv, dims->d, dims->r, agg};
+    cudaError_t e = launch_project(pj, S(stream), true, dims->kv_dtype);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the query projection");
+    ScanArgs sa;
+    memset(&sa, 0, sizeof sa);
+    sa.src = Kt;
+    sa.qproj = at<float>(ws, L.qproj);
+    sa.seq_lens = seq_lens;
+    sa.scores_out = scores;
+    sa.status = at<uint32_t>(ws, 0);
+    sa.B = dims->B;
+    sa.Hkv = dims->Hkv;
+    sa.T_cap = dims->T_cap;
+    sa.r = dims->r;
+    sa.nq = nq;
+    e = launch_scan(L.sp, sa, agg, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the score pass");
+    return JSSA_OK;
+}
+
+int jssa_topk(const jssa_dims *dims, const float *scores, const int32_t *seq_lens, int k, int32_t *idx,
+              int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    REQUIRE_PTR(scores);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(idx);
+    OPTIONAL_PTR(count);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_TOPK, 0, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    return run_select(dims, sh, nullptr, nullptr, scores, seq_lens, JSSA_AGG_SUM, k, idx, count, ws, L, S(stream),
+                      false);
+}
+
+int jssa_select(const jssa_dims *dims, const void *q, const float *P, const void *Kt, const int32_t *seq_lens,
+                int agg, int k, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(P);
+    REQUIRE_PTR(Kt);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(idx);
+    OPTIONAL_PTR(count);
+    if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
+    if (agg == JSSA_AGG_MAX && sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "MAX aggregation needs G <= %d", kMaxG);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_SELECT, agg, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    return run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), true);
+}
+
+int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, const void *V, const int32_t *idx,
+                        const int32_t *count, int k, const int32_t *seq_lens, float softmax_scale, void *out,
+                        float *lse, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    if ((st = check_attn_shape(dims, sh))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(out);
+    OPTIONAL_PTR(count);
+    OPTIONAL_PTR(lse);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    AttnArgs a;
+    fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
+    a.idx = idx;
+    a.count = count;
+    a.k = k;
+    cudaError_t e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the indexed decode");
+    return JSSA_OK;
+}
+
+int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const void *V, const int32_t *seq_lens,
+                      int window, float softmax_scale, void *out, float *lse, void *ws, size_t ws_bytes,
+                      jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_attn_shape(dims, sh))) return st;
+    if (window < 0) return fail(JSSA_ERR_INVALID_ARG, "window=%d is negative", window);
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(out);
+    OPTIONAL_PTR(lse);
+    Layout L;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_DENSE_DECODE, 0, window, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    AttnArgs a;
+    fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
+    a.window = window;
+    cudaError_t e = launch_attend(L.ap, ATT_RANGE, a, dims->kv_dtype, dims->d, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the dense decode");
+    return JSSA_OK;
+}
+
+int jssa_gather_then_dense(const jssa_dims *dims, const void *q, const void *K, const void *V, const int32_t *idx,
+                           const int32_t *count, int k, const int32_t *seq_lens, float softmax_scale,
+                           void *gather_buf, size_t gather_bytes, void *out, float *lse, void *ws, size_t ws_bytes,
+                           jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    if ((st = check_attn_shape(dims, sh))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(out);
+    REQUIRE_PTR(gather_buf);
+    OPTIONAL_PTR(count);
+    OPTIONAL_PTR(lse);
+    const size_t half = (size_t)sh.BH * k * dims->d * sh.es_kv;
+    if (gather_bytes < 2 * half)
+        return fail(JSSA_ERR_INVALID_ARG, "gather_buf of %zu bytes is below the %zu bytes needed", gather_bytes,
+                    2 * half);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_GATHER_THEN_DENSE, 0, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    void *gK = gather_buf;
+    void *gV = static_cast<char *>(gather_buf) + half;
+    GatherArgs g{K, V, idx, count, seq_lens, gK, gV, at<int32_t>(ws, L.gcount), at<uint32_t>(ws, 0),
+                 dims->B, dims->Hkv, dims->T_cap, dims->d, k};
+    cudaError_t e = launch_gather(g, dims->kv_dtype, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the gather");
+    AttnArgs a;
+    fill_attn(a, dims, sh, q, gK, gV, seq_lens, softmax_scale, out, lse, ws, L);
+    a.k_sb = a.v_sb = (long long)dims->Hkv * k * dims->d;
+    a.k_st = a.v_st = dims->d;
+    a.k_sh = a.v_sh = (long long)k * dims->d;
+    a.count = at<int32_t>(ws, L.gcount);
+    a.k = k;
+    e = launch_attend(L.ap, ATT_RANGE_BH, a, dims->kv_dtype, dims->d, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the dense decode over gathered rows");
+    return JSSA_OK;
+}
+
+int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const void *V, const float *P, void *Kt,
+                     const int32_t *seq_lens, const int32_t *pos_begin, int k, int agg, float softmax_scale,
+                     int32_t *idx, int32_t *count, void *out, float *lse, void *ws, size_t ws_bytes,
+                     jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    if ((st = check_attn_shape(dims, sh))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    REQUIRE_PTR(P);
+    REQUIRE_PTR(Kt);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(pos_begin);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(count);
+    REQUIRE_PTR(out);
+    OPTIONAL_PTR(lse);
+    if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_DECODE_STEP, agg, 0, L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    AppendArgs ap{K, P, Kt, pos_begin, at<uint32_t>(ws, 0), dims->B, dims->T_cap, dims->Hkv, dims->d, dims->r, 1, 1};
+    ProjArgs pj{q, P, at<float>(ws, L.qproj), dims->B, dims->Hq, dims->Hkv, dims->d, dims->r, agg};
+    cudaError_t e = launch_prep(ap, pj, S(stream), true, dims->kv_dtype, dims->kt_dtype);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the append + projection prologue");
+    if ((st = run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), false))) return st;
+    AttnArgs a;
+    fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
+    a.idx = idx;
+    a.count = count;
+    a.k = k;
+    e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the indexed decode");
+    return JSSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+// Host-side plans, kernel argument blocks and launcher declarations shared
+// by the translation units of libjssa.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <utility>
+
+#include "../../include/jssa.h"
+
+namespace jssa {
+
+constexpr int kMaxK = 2048;
+constexpr int kMaxG = 16;
+constexpr int kScanThreads = 256;
+constexpr int kScanStageBytes = 16384;
+constexpr int kScoreTileTokens = 4096;  // tokens per tile when the source is a score array
+constexpr int kAttnThreads = 128;
+
+// ------------------------------------------------------------------ scan ---
+// One persistent pass over per-(b,h) token streams.  Source: the low-rank key
+// cache (scores computed on the fly) or a score array.  Mode: write the scores,
+// or keep a per-segment top-k and merge segments into the final selection.
+enum ScanSrc { SRC_KT_BF16 = 0, SRC_KT_FP32 = 1, SRC_SCORES = 2 };
+enum ScanMode { MODE_WRITE = 0, MODE_SELECT = 1 };
+
+struct ScanArgs {
+    const void *src;          // Kt [B,Hkv,T_cap,r] or scores [B,Hkv,T_cap]
+    const float *qproj;       // [B*Hkv, nq, r] projected (folded) queries
+    const int32_t *seq_lens;  // [B]
+    float *scores_out;        // MODE_WRITE
+    uint32_t *cand_key;       // [BH, max_seg, k]
+    int32_t *cand_idx;        // [BH, max_seg, k]
+    int32_t *cand_cnt;        // [BH, max_seg]
+    uint32_t *counters;       // [BH] arrival tickets (self-resetting)
+    int32_t *idx_out;         // [BH, k]
+    int32_t *count_out;       // [BH] or null
+    uint32_t *status;
+    int B, Hkv, T_cap, r, nq, k;
+    int tile_tokens, tiles_per_bh;
+    long long total_tiles;
+    int grid, max_seg, cap, nstages;
+};
+
+struct ScanPlan {
+    int src, mode, tile_tokens, tiles_per_bh, grid, max_seg, cap, nstages;
+    long long total_tiles;
+    size_t smem;
+};
+
+struct ProjArgs {
+    const void *q;   // [B, Hq, d] kv dtype
+    const float *P;  // [Hkv, d, r]
+    float *qproj;    // [B*Hkv, nq, r]
+    int B, Hq, Hkv, d, r, agg;
+};
+
+struct AppendArgs {
+    const void *K;  // [B, T_cap, Hkv, d]
+    const float *P;
+    void *Kt;       // [B, Hkv, T_cap, r]
+    const int32_t *pos_begin;
+    uint32_t *status;
+    int B, T_cap, Hkv, d, r, n_new, rows_per_cta;
+};
+
+// ---------------------------------------------------------------- attend ---
+enum AttnSrc { ATT_INDEXED = 0, ATT_RANGE = 1, ATT_RANGE_BH = 2 };
+
+struct AttnArgs {
+    const void *q;  // [B, Hq, d]
+    const void *K;
+    const void *V;
+    long long k_sb, k_st, k_sh;  // element strides of K: batch, token, head
+    long long v_sb, v_st, v_sh;
+    const int32_t *idx;      // ATT_INDEXED: [BH, k]
+    const int32_t *count;    // ATT_INDEXED / ATT_RANGE_BH: [BH] (indexed: may be null)
+    const int32_t *seq_lens; // [B]
+    int k, window;
+    int B, Hq, Hkv, G, T_cap;
+    float scale_log2;        // softmax_scale * log2(e)
+    int splits, pos_per_split;
+    float *part_o;           // [BH, splits, G, D]
+    float *part_ml;          // [BH, splits, G, 2]
+    uint32_t *counters;      // [BH]
+    void *out;               // [B, Hq, D]
+    float *lse;              // [B, Hq] or null
+    uint32_t *status;
+};
+
+struct AttnPlan {
+    int nt, splits, pos_per_split, stages;
+    size_t smem;
+};
+
+struct GatherArgs {
+    const void *K;
+    const void *V;
+    const int32_t *idx;
+    const int32_t *count;
+    const int32_t *seq_lens;
+    void *gK;  // [B, Hkv, k, d]
+    void *gV;
+    int32_t *gcount;  // [BH] rows actually gathered
+    uint32_t *status;
+    int B, Hkv, T_cap, d, k;
+};
+
+// --------------------------------------------------------------- helpers ---
+int device_sm_count();
+cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype);
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t s, bool pdl, int kv_dtype, int kt_dtype);
+cudaError_t launch_prep(const AppendArgs &ap, const ProjArgs &pj, cudaStream_t s, bool pdl, int kv_dtype,
+                        int kt_dtype);
+cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, ScanPlan *p);
+cudaError_t launch_scan(const ScanPlan &p, const ScanArgs &a, int agg, cudaStream_t s, bool pdl);
+cudaError_t plan_attend(int src, int kv_dtype, int d, int G, int B, int Hkv, int npos, AttnPlan *p);
+cudaError_t launch_attend(const AttnPlan &p, int src, const AttnArgs &a, int kv_dtype, int d, cudaStream_t s,
+                          bool pdl);
+cudaError_t launch_gather(const GatherArgs &a, int kv_dtype, cudaStream_t s, bool pdl);
+
+// Launch with the programmatic-stream-serialisation attribute (PDL) if asked.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                          Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+}  // namespace jssa

@@ -1,0 +1,203 @@
+// Low-rank key append and query projection.
+//
+// Append ("Joint Subspace Sparse Attention for Efficient Long-Context
+// Decoding", Abstract: a shared low-dimensional query-key subspace; news item
+// "JSSA makes token-level sparse decoding gather-free", Synopsis: candidate
+// tokens are scored in that subspace):
+//   Kt[b,h,t,:] = round(K[b,t,h,:] . P[h])   for t in [pos_b, pos_b + n_new).
+// Projection (same pages, Interpretation para 2: queries and keys share the
+// scoring space): qt_g = P_h^T q_g; the SUM score folds the group first,
+// qbar_h = P_h^T (sum_g q_g), which is the same linear map applied once.
+//
+// Every dot product over d is evaluated in one fixed order, independent of
+// the launch shape: partial sums over consecutive chunks of kChunk inputs
+// (fma chains from 0), then the chunk partials added left to right.  So the
+// per-step append, the prefix append and the fused decode-step prologue give
+// bit-identical rows, and the score and select paths see the same qbar.
+#include "jssa_common.cuh"
+#include "jssa_internal.h"
+
+namespace jssa {
+
+namespace {
+
+constexpr int kPrepThreads = 256;
+constexpr int kChunk = 16;  // d is a multiple of 16 for every supported shape
+
+// out[o] for o < n_out, with out[o] = sum_i x[row(o)][i] * P[i][col(o)], x in
+// shared memory (fp32, rows of d), P global [d][r].  `part` is shared scratch
+// of n_out * (d / kChunk) floats.
+__device__ __forceinline__ void chunked_dots(const float *x, const float *__restrict__ P, int d, int r, int n_out,
+                                             float *part) {
+    const int nch = d / kChunk;
+    for (int p = threadIdx.x; p < n_out * nch; p += blockDim.x) {
+        const int o = p / nch, c = p - o * nch;
+        const int row = o / r, j = o - row * r;
+        const float *xr = x + (size_t)row * d + c * kChunk;
+        const float *pc = P + (size_t)(c * kChunk) * r + j;
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kChunk; ++i) acc = fmaf(xr[i], __ldg(pc + (size_t)i * r), acc);
+        part[p] = acc;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ float sum_chunks(const float *part, int o, int nch) {
+    float s = part[(size_t)o * nch];
+    for (int c = 1; c < nch; ++c) s += part[(size_t)o * nch + c];
+    return s;
+}
+
+// Append rows [row0, row0 + nrows) of KV head bh's new range.
+template <typename KV, typename KT>
+__device__ void append_rows(const AppendArgs &a, int bh, int row0, int nrows, float *xs, float *part) {
+    const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+    const int pos = a.pos_begin[b];
+    if (pos < 0 || pos > a.T_cap - a.n_new) {
+        if (threadIdx.x == 0 && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_POS);
+        return;
+    }
+    const int d = a.d, r = a.r;
+    const KV *K = static_cast<const KV *>(a.K);
+    for (int p = threadIdx.x; p < nrows * d; p += blockDim.x) {
+        const int rr = p / d, i = p - rr * d;
+        const size_t t = (size_t)pos + row0 + rr;
+        xs[p] = to_f32(K[(((size_t)b * a.T_cap + t) * a.Hkv + h) * d + i]);
+    }
+    __syncthreads();
+    const float *P = a.P + (size_t)h * d * r;
+    chunked_dots(xs, P, d, r, nrows * r, part);
+    KT *Kt = static_cast<KT *>(a.Kt);
+    const int nch = d / kChunk;
+    for (int o = threadIdx.x; o < nrows * r; o += blockDim.x) {
+        const int rr = o / r, j = o - rr * r;
+        const size_t t = (size_t)pos + row0 + rr;
+        store_elem(Kt + (((size_t)b * a.Hkv + h) * a.T_cap + t) * r + j, sum_chunks(part, o, nch));
+    }
+}
+
+// Projected queries of KV head bh: SUM -> qproj[bh][0][:] = P_h^T sum_g q_g;
+// MAX -> qproj[bh][g][:] = P_h^T q_g.
+template <typename KV>
+__device__ void project_bh(const ProjArgs &a, int bh, float *xs, float *part) {
+    const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+    const int G = a.Hq / a.Hkv, d = a.d, r = a.r;
+    const KV *q = static_cast<const KV *>(a.q) + ((size_t)b * a.Hq + (size_t)h * G) * d;
+    const int nrow = a.agg == JSSA_AGG_SUM ? 1 : G;
+    if (a.agg == JSSA_AGG_SUM) {
+        for (int i = threadIdx.x; i < d; i += blockDim.x) {
+            float s = 0.f;
+            for (int g = 0; g < G; ++g) s += to_f32(q[(size_t)g * d + i]);
+            xs[i] = s;
+        }
+    } else {
+        for (int p = threadIdx.x; p < G * d; p += blockDim.x) xs[p] = to_f32(q[p]);
+    }
+    __syncthreads();
+    chunked_dots(xs, a.P + (size_t)h * d * r, d, r, nrow * r, part);
+    const int nch = d / kChunk;
+    for (int o = threadIdx.x; o < nrow * r; o += blockDim.x)
+        a.qproj[(size_t)bh * nrow * r + o] = sum_chunks(part, o, nch);
+}
+
+template <typename KV, typename KT>
+__global__ void __launch_bounds__(kPrepThreads) append_kernel(AppendArgs a) {
+    extern __shared__ __align__(16) float sm_prep[];
+    pdl_trigger();
+    pdl_wait();
+    const int bh = blockIdx.y;
+    const int row0 = blockIdx.x * a.rows_per_cta;
+    const int nrows = min(a.rows_per_cta, a.n_new - row0);
+    if (nrows <= 0) return;
+    append_rows<KV, KT>(a, bh, row0, nrows, sm_prep, sm_prep + (size_t)a.rows_per_cta * a.d);
+}
+
+template <typename KV>
+__global__ void __launch_bounds__(kPrepThreads) project_kernel(ProjArgs a) {
+    extern __shared__ __align__(16) float sm_prep[];
+    pdl_trigger();
+    pdl_wait();
+    const int G = a.Hq / a.Hkv;
+    const int xrows = a.agg == JSSA_AGG_SUM ? 1 : G;
+    project_bh<KV>(a, blockIdx.x, sm_prep, sm_prep + (size_t)xrows * a.d);
+}
+
+// Decode-step prologue: one CTA per (b, h) appends the new row and projects
+// the queries; equal to append_kernel (n_new = 1) followed by project_kernel.
+template <typename KV, typename KT>
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(AppendArgs ap, ProjArgs pj) {
+    extern __shared__ __align__(16) float sm_prep[];
+    pdl_trigger();
+    pdl_wait();
+    const int G = pj.Hq / pj.Hkv;
+    const int xrows = pj.agg == JSSA_AGG_SUM ? 1 : G;
+    float *xs = sm_prep;
+    float *part = sm_prep + (size_t)xrows * pj.d;
+    append_rows<KV, KT>(ap, blockIdx.x, 0, 1, xs, part);
+    __syncthreads();
+    project_bh<KV>(pj, blockIdx.x, xs, part);
+}
+
+size_t prep_smem(int rows, int d, int r) {
+    return ((size_t)rows * d + (size_t)rows * r * (d / kChunk)) * sizeof(float);
+}
+
+template <typename Kern>
+cudaError_t allow_smem(Kern k, size_t smem) {
+    if (smem <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendArgs &a0, cudaStream_t s, bool pdl, int kv_dtype, int kt_dtype) {
+    AppendArgs a = a0;
+    // rows per CTA: as many as keep the staging under ~96 KiB
+    int rows = 32;
+    while (rows > 1 && prep_smem(rows, a.d, a.r) > 96 * 1024) rows >>= 1;
+    if (rows > a.n_new) rows = a.n_new;
+    a.rows_per_cta = rows;
+    const size_t smem = prep_smem(rows, a.d, a.r);
+    dim3 grid((a.n_new + rows - 1) / rows, a.B * a.Hkv);
+    void (*k)(AppendArgs);
+    if (kv_dtype == JSSA_BF16)
+        k = kt_dtype == JSSA_BF16 ? append_kernel<__nv_bfloat16, __nv_bfloat16> : append_kernel<__nv_bfloat16, float>;
+    else
+        k = kt_dtype == JSSA_BF16 ? append_kernel<float, __nv_bfloat16> : append_kernel<float, float>;
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(k, grid, dim3(kPrepThreads), smem, s, pdl, a);
+}
+
+cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype) {
+    const int G = a.Hq / a.Hkv;
+    const int nrow = a.agg == JSSA_AGG_SUM ? 1 : G;
+    const size_t smem = ((size_t)nrow * a.d + (size_t)nrow * a.r * (a.d / kChunk)) * sizeof(float);
+    void (*k)(ProjArgs) = kv_dtype == JSSA_BF16 ? project_kernel<__nv_bfloat16> : project_kernel<float>;
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(k, dim3(a.B * a.Hkv), dim3(kPrepThreads), smem, s, pdl, a);
+}
+
+cudaError_t launch_prep(const AppendArgs &ap0, const ProjArgs &pj, cudaStream_t s, bool pdl, int kv_dtype,
+                        int kt_dtype) {
+    AppendArgs ap = ap0;
+    ap.n_new = 1;
+    ap.rows_per_cta = 1;
+    const int G = pj.Hq / pj.Hkv;
+    const int nrow = pj.agg == JSSA_AGG_SUM ? 1 : G;
+    size_t xs = (size_t)nrow * pj.d;
+    size_t part = (size_t)(nrow > 1 ? nrow : 1) * pj.r * (pj.d / kChunk);
+    const size_t smem = (xs + part) * sizeof(float);
+    void (*k)(AppendArgs, ProjArgs);
+    if (kv_dtype == JSSA_BF16)
+        k = kt_dtype == JSSA_BF16 ? prep_kernel<__nv_bfloat16, __nv_bfloat16> : prep_kernel<__nv_bfloat16, float>;
+    else
+        k = kt_dtype == JSSA_BF16 ? prep_kernel<float, __nv_bfloat16> : prep_kernel<float, float>;
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(k, dim3(pj.B * pj.Hkv), dim3(kPrepThreads), smem, s, pdl, ap, pj);
+}
+
+}  // namespace jssa

@@ -1,0 +1,360 @@
+"""Python binding of libjssa.so: torch CUDA tensors in, C-ABI calls out.
+
+Argument marshalling only.  Every step of the decode path runs in the CUDA
+kernels behind ``include/jssa.h``; there is no Python or CPU fallback, and a
+missing library or a call on tensors that are not on a CUDA device raises.
+
+Layouts (see the header for the full contract):
+  q [B, Hq, d]   K [B, T_cap, Hkv, d]   V [B, T_cap, Hkv, dv] (None = latent cache, V is K)
+  P [Hkv, d, r] fp32   Kt [B, Hkv, T_cap, r]   seq_lens int32 [B]
+  idx int32 [B, Hkv, k] (ascending, -1 padded)   count int32 [B, Hkv]
+  out [B, Hq, dv]   lse fp32 [B, Hq]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libjssa.so")
+
+BF16, FP32 = 0, 1
+AGG_SUM, AGG_MAX = 0, 1
+OP_APPEND, OP_SCORE, OP_TOPK, OP_SELECT, OP_INDEXED_DECODE, OP_DENSE_DECODE, OP_GATHER_THEN_DENSE, OP_DECODE_STEP = \
+    range(8)
+DEV_SEQLEN, DEV_INDEX, DEV_POS, DEV_TIMEOUT = 1, 2, 4, 8
+
+
+class JssaError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("libjssa status %d: %s" % (code, msg))
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "d", "dv", "r", "T_cap", "kv_dtype", "kt_dtype")]
+
+    def key(self):
+        return tuple(getattr(self, n) for n, _ in self._fields_)
+
+
+_lib = None
+
+EXPORTS = ("jssa_version", "jssa_status_string", "jssa_last_error", "jssa_workspace_size", "jssa_workspace_init",
+           "jssa_append_lowrank", "jssa_score", "jssa_topk", "jssa_select", "jssa_indexed_decode",
+           "jssa_dense_decode", "jssa_gather_then_dense", "jssa_decode_step")
+
+
+def lib():
+    """Load libjssa.so (raises if it is missing; there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libjssa.so not found at %s: build it with `python -m token_level_sparse_kv_b200.build`"
+                           % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    D = ctypes.POINTER(Dims)
+    L.jssa_version.restype = i32
+    L.jssa_status_string.restype = ctypes.c_char_p
+    L.jssa_status_string.argtypes = [i32]
+    L.jssa_last_error.restype = ctypes.c_char_p
+    L.jssa_workspace_size.restype = i32
+    L.jssa_workspace_size.argtypes = [D, i32, i32, ctypes.POINTER(sz)]
+    L.jssa_workspace_init.restype = i32
+    L.jssa_workspace_init.argtypes = [vp, sz, vp]
+    L.jssa_append_lowrank.restype = i32
+    L.jssa_append_lowrank.argtypes = [D, vp, vp, vp, vp, i32, vp, sz, vp]
+    L.jssa_score.restype = i32
+    L.jssa_score.argtypes = [D, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+    L.jssa_topk.restype = i32
+    L.jssa_topk.argtypes = [D, vp, vp, i32, vp, vp, vp, sz, vp]
+    L.jssa_select.restype = i32
+    L.jssa_select.argtypes = [D, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+    L.jssa_indexed_decode.restype = i32
+    L.jssa_indexed_decode.argtypes = [D, vp, vp, vp, vp, vp, i32, vp, f32, vp, vp, vp, sz, vp]
+    L.jssa_dense_decode.restype = i32
+    L.jssa_dense_decode.argtypes = [D, vp, vp, vp, vp, i32, f32, vp, vp, vp, sz, vp]
+    L.jssa_gather_then_dense.restype = i32
+    L.jssa_gather_then_dense.argtypes = [D, vp, vp, vp, vp, vp, i32, vp, f32, vp, sz, vp, vp, vp, sz, vp]
+    L.jssa_decode_step.restype = i32
+    L.jssa_decode_step.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, sz, vp]
+    _lib = L
+    return L
+
+
+def _check(st):
+    if st != 0:
+        raise JssaError(st, lib().jssa_last_error().decode(errors="replace"))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dt(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError("bf16 or fp32 expected, got %s" % t.dtype)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("libjssa works on CUDA tensors only (got a %s tensor)" % t.device)
+            if not t.is_contiguous():
+                raise ValueError("libjssa needs contiguous tensors")
+
+
+def make_dims(q, K, V, P=None, Kt=None, r=None):
+    """Dims from tensor shapes; V None means a latent cache (V is K)."""
+    B, Hq, d = q.shape
+    _, T_cap, Hkv, dk = K.shape
+    assert dk == d, "q and K widths differ"
+    if V is None:
+        dv = 512 if d == 576 else d
+    else:
+        dv = V.shape[3]
+    if r is None:
+        r = P.shape[2] if P is not None else (Kt.shape[3] if Kt is not None else 8)
+    kt = _dt(Kt) if Kt is not None else BF16
+    return Dims(B, Hq, Hkv, d, dv, r, T_cap, _dt(K), kt)
+
+
+def workspace_size(dims: Dims, k: int, op: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().jssa_workspace_size(ctypes.byref(dims), int(k), int(op), ctypes.byref(n)))
+    return int(n.value)
+
+
+def new_workspace(dims: Dims, k: int, op: int, device) -> torch.Tensor:
+    """Allocate (through torch) and zero a workspace for `op`."""
+    n = max(workspace_size(dims, k, op), 256)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().jssa_workspace_init(_p(ws), n, _stream(ws.device)))
+    return ws
+
+
+def workspace_init(ws: torch.Tensor):
+    _check(lib().jssa_workspace_init(_p(ws), ws.numel(), _stream(ws.device)))
+
+
+def device_status(ws: torch.Tensor) -> int:
+    """Sticky device status word (JSSA_DEV_* bits); synchronises on the copy."""
+    return int(ws[:4].view(torch.int32).item()) & 0xFFFFFFFF
+
+
+def _ws(ws, dims, k, op, device):
+    return new_workspace(dims, k, op, device) if ws is None else ws
+
+
+# ------------------------------------------------------------------- ops ---
+def append_lowrank(K, P, Kt, pos_begin, n_new, ws=None):
+    """Kt[b,h,t,:] = round(K[b,t,h,:] @ P[h]) for t in [pos_begin[b], pos_begin[b] + n_new)."""
+    _cuda(K, P, Kt, pos_begin)
+    B, T_cap, Hkv, d = K.shape
+    dims = Dims(B, 1 * Hkv, Hkv, d, 512 if d == 576 else d, P.shape[2], T_cap, _dt(K), _dt(Kt))
+    ws = _ws(ws, dims, 1, OP_APPEND, K.device)
+    _check(lib().jssa_append_lowrank(ctypes.byref(dims), _p(K), _p(P), _p(Kt), _p(pos_begin), int(n_new), _p(ws),
+                                     ws.numel(), _stream(K.device)))
+    return Kt
+
+
+def build_lowrank_cache(K, P, kt_dtype=torch.bfloat16, ws=None):
+    """Kt for all T_cap rows of K (prefix build)."""
+    B, T_cap, Hkv, d = K.shape
+    Kt = torch.empty((B, Hkv, T_cap, P.shape[2]), dtype=kt_dtype, device=K.device)
+    pos = torch.zeros(B, dtype=torch.int32, device=K.device)
+    return append_lowrank(K, P, Kt, pos, T_cap, ws=ws)
+
+
+def score(q, P, Kt, seq_lens, agg=AGG_SUM, scores=None, ws=None):
+    """Subspace scores [B, Hkv, T_cap] fp32 (t >= T_b not written)."""
+    _cuda(q, P, Kt, seq_lens, scores)
+    B, Hq, d = q.shape
+    _, Hkv, T_cap, r = Kt.shape
+    dims = Dims(B, Hq, Hkv, d, 512 if d == 576 else d, r, T_cap, _dt(q), _dt(Kt))
+    if scores is None:
+        scores = torch.full((B, Hkv, T_cap), float("nan"), dtype=torch.float32, device=q.device)
+    ws = _ws(ws, dims, 1, OP_SCORE, q.device)
+    _check(lib().jssa_score(ctypes.byref(dims), _p(q), _p(P), _p(Kt), _p(seq_lens), int(agg), _p(scores), _p(ws),
+                            ws.numel(), _stream(q.device)))
+    return scores
+
+
+def topk(scores, seq_lens, k, Hq=None, d=128, ws=None):
+    """Per-(b,h) top-k of a score array: (idx [B,Hkv,k], count [B,Hkv])."""
+    _cuda(scores, seq_lens)
+    B, Hkv, T_cap = scores.shape
+    dims = Dims(B, Hq or Hkv, Hkv, d, 512 if d == 576 else d, 8, T_cap, BF16, BF16)
+    idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=scores.device)
+    cnt = torch.empty((B, Hkv), dtype=torch.int32, device=scores.device)
+    ws = _ws(ws, dims, k, OP_TOPK, scores.device)
+    _check(lib().jssa_topk(ctypes.byref(dims), _p(scores), _p(seq_lens), int(k), _p(idx), _p(cnt), _p(ws),
+                           ws.numel(), _stream(scores.device)))
+    return idx, cnt
+
+
+def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None):
+    """Fused score + top-k: (idx [B,Hkv,k], count [B,Hkv])."""
+    _cuda(q, P, Kt, seq_lens)
+    B, Hq, d = q.shape
+    _, Hkv, T_cap, r = Kt.shape
+    dims = Dims(B, Hq, Hkv, d, 512 if d == 576 else d, r, T_cap, _dt(q), _dt(Kt))
+    if idx is None:
+        idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    ws = _ws(ws, dims, k, OP_SELECT, q.device)
+    _check(lib().jssa_select(ctypes.byref(dims), _p(q), _p(P), _p(Kt), _p(seq_lens), int(agg), int(k), _p(idx),
+                             _p(count), _p(ws), ws.numel(), _stream(q.device)))
+    return idx, count
+
+
+def indexed_decode(q, K, V, idx, count, seq_lens, scale, ws=None, out=None, lse=None):
+    """Gather-free attention over the selected rows: (out [B,Hq,dv], lse [B,Hq])."""
+    _cuda(q, K, V, idx, count, seq_lens, out, lse)
+    k = idx.shape[2]
+    dims = make_dims(q, K, V, r=8)
+    if out is None:
+        out = torch.empty((dims.B, dims.Hq, dims.dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((dims.B, dims.Hq), dtype=torch.float32, device=q.device)
+    ws = _ws(ws, dims, k, OP_INDEXED_DECODE, q.device)
+    _check(lib().jssa_indexed_decode(ctypes.byref(dims), _p(q), _p(K), _p(K if V is None else V), _p(idx),
+                                     _p(count), int(k), _p(seq_lens), float(scale), _p(out), _p(lse), _p(ws),
+                                     ws.numel(), _stream(q.device)))
+    return out, lse
+
+
+def dense_decode(q, K, V, seq_lens, scale, window=0, ws=None, out=None, lse=None):
+    """Full-KV (window 0) or sliding-window decode attention: (out, lse)."""
+    _cuda(q, K, V, seq_lens, out, lse)
+    dims = make_dims(q, K, V, r=8)
+    if out is None:
+        out = torch.empty((dims.B, dims.Hq, dims.dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((dims.B, dims.Hq), dtype=torch.float32, device=q.device)
+    ws = _ws(ws, dims, 1, OP_DENSE_DECODE, q.device)
+    _check(lib().jssa_dense_decode(ctypes.byref(dims), _p(q), _p(K), _p(K if V is None else V), _p(seq_lens),
+                                   int(window), float(scale), _p(out), _p(lse), _p(ws), ws.numel(),
+                                   _stream(q.device)))
+    return out, lse
+
+
+def gather_buffer_bytes(dims: Dims, k: int) -> int:
+    return 2 * dims.B * dims.Hkv * k * dims.d * (2 if dims.kv_dtype == BF16 else 4)
+
+
+def gather_then_dense(q, K, V, idx, count, seq_lens, scale, gather_buf=None, ws=None, out=None, lse=None):
+    """Gather the selected rows into a contiguous buffer, then dense decode over them."""
+    _cuda(q, K, V, idx, count, seq_lens, gather_buf, out, lse)
+    k = idx.shape[2]
+    dims = make_dims(q, K, V, r=8)
+    if gather_buf is None:
+        gather_buf = torch.empty(gather_buffer_bytes(dims, k), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((dims.B, dims.Hq, dims.dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((dims.B, dims.Hq), dtype=torch.float32, device=q.device)
+    ws = _ws(ws, dims, k, OP_GATHER_THEN_DENSE, q.device)
+    _check(lib().jssa_gather_then_dense(ctypes.byref(dims), _p(q), _p(K), _p(K if V is None else V), _p(idx),
+                                        _p(count), int(k), _p(seq_lens), float(scale), _p(gather_buf),
+                                        gather_buf.numel() * gather_buf.element_size(), _p(out), _p(lse), _p(ws),
+                                        ws.numel(), _stream(q.device)))
+    return out, lse
+
+
+def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=None, idx=None, count=None,
+                out=None, lse=None):
+    """Append the row at pos_begin, select, indexed decode: (out, lse, idx, count)."""
+    _cuda(q, K, V, P, Kt, seq_lens, pos_begin, idx, count, out, lse)
+    dims = make_dims(q, K, V, P=P, Kt=Kt)
+    B, Hkv = dims.B, dims.Hkv
+    if idx is None:
+        idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty((B, dims.Hq, dims.dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, dims.Hq), dtype=torch.float32, device=q.device)
+    ws = _ws(ws, dims, k, OP_DECODE_STEP, q.device)
+    _check(lib().jssa_decode_step(ctypes.byref(dims), _p(q), _p(K), _p(K if V is None else V), _p(P), _p(Kt),
+                                  _p(seq_lens), _p(pos_begin), int(k), int(agg), float(scale), _p(idx), _p(count),
+                                  _p(out), _p(lse), _p(ws), ws.numel(), _stream(q.device)))
+    return out, lse, idx, count
+
+
+class DecodeSession:
+    """Device-resident state of one attention layer's decode (the public API
+    of the end-to-end path): KV cache, low-rank key cache, basis, workspace
+    and output buffers.  ``step_from_host`` takes one step's inputs from
+    pinned host memory and returns the attention output in pinned host
+    memory."""
+
+    def __init__(self, K, V, P, seq_lens, k, scale, Kt=None, kt_dtype=torch.bfloat16, agg=AGG_SUM):
+        _cuda(K, V, P, seq_lens)
+        self.K, self.V, self.P, self.seq_lens = K, V, P, seq_lens
+        self.k, self.scale, self.agg = int(k), float(scale), int(agg)
+        dev = K.device
+        self.Kt = build_lowrank_cache(K, P, kt_dtype) if Kt is None else Kt
+        B, T_cap, Hkv, d = K.shape
+        self.B, self.Hkv, self.d = B, Hkv, d
+        self.pos = (seq_lens.to(torch.int32) - 1).clamp_min(0).contiguous()
+        self._dims = None
+        self.ws = None
+        self.q_dev = None
+        self.out = self.lse = self.idx = self.count = None
+
+    def _ensure(self, q_shape, dtype):
+        if self.q_dev is not None and tuple(self.q_dev.shape) == tuple(q_shape):
+            return
+        dev = self.K.device
+        self.q_dev = torch.empty(q_shape, dtype=dtype, device=dev)
+        dims = make_dims(self.q_dev, self.K, self.V, P=self.P, Kt=self.Kt)
+        self.ws = new_workspace(dims, self.k, OP_DECODE_STEP, dev)
+        self.idx = torch.empty((self.B, self.Hkv, self.k), dtype=torch.int32, device=dev)
+        self.count = torch.empty((self.B, self.Hkv), dtype=torch.int32, device=dev)
+        self.out = torch.empty((dims.B, dims.Hq, dims.dv), dtype=dtype, device=dev)
+        self.lse = torch.empty((dims.B, dims.Hq), dtype=torch.float32, device=dev)
+        self.out_host = torch.empty(self.out.shape, dtype=dtype, pin_memory=True)
+
+    def step(self, q):
+        """One step on a device-resident query (the new token's K/V row must
+        already be at position seq_lens-1 of the cache)."""
+        out, lse, idx, count = decode_step(q, self.K, self.V, self.P, self.Kt, self.seq_lens, self.pos, self.k,
+                                           self.scale, agg=self.agg, ws=self.ws, idx=self.idx, count=self.count,
+                                           out=self.out, lse=self.lse)
+        return out
+
+    def step_from_host(self, q_host, k_new_host, v_new_host):
+        """Copy q [B,Hq,d] and the new token's K/V rows [B,Hkv,d] from pinned host
+        memory, write the rows at position seq_lens-1, run the step, and copy the
+        output back to pinned host memory (returned; valid after a stream sync)."""
+        self._ensure(q_host.shape, q_host.dtype)
+        self.q_dev.copy_(q_host, non_blocking=True)
+        pos = int(self._host_pos())
+        self.K[:, pos].copy_(k_new_host, non_blocking=True)
+        self.V[:, pos].copy_(v_new_host, non_blocking=True)
+        self.step(self.q_dev)
+        self.out_host.copy_(self.out, non_blocking=True)
+        return self.out_host
+
+    def _host_pos(self):
+        if not hasattr(self, "_pos_cache"):
+            p = self.pos.cpu()
+            if not bool((p == p[0]).all()):
+                raise ValueError("step_from_host needs one shared position across the batch")
+            self._pos_cache = int(p[0])
+        return self._pos_cache
