@@ -241,9 +241,7 @@ def oracle_baseline(w, budget_s, n_rows, threads):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    from token_level_sparse_kv_b200.inputs import WORKLOADS
-
-    w = WORKLOADS[args.workload]
+    w = workload_of(args)
     threads = os.cpu_count() or 1
     smp = OracleSample(w, max(1, min(w.B, args.cpu_rows)), threads)
     # size the per-step sample so that warm-up + timed steps take about 2 minutes
@@ -264,6 +262,21 @@ def run_reference(args, world, rank):
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def workload_of(args):
+    from token_level_sparse_kv_b200.inputs import WORKLOADS, Workload
+
+    w = WORKLOADS[args.workload]
+    over = {}
+    if args.batch is not None and args.batch != w.B:
+        over["B"] = args.batch
+    if args.topk is not None and args.topk != w.k:
+        over["k"] = args.topk
+    if over:
+        name = w.name + "".join("_%s%d" % (("b" if k == "B" else "k"), v) for k, v in over.items())
+        w = Workload(**{**w.__dict__, **over, "name": name})
+    return w
 
 
 def config_of(w, world):
@@ -294,9 +307,9 @@ def run_jssa(args, world, rank, local):
     import torch
 
     from token_level_sparse_kv_b200 import ops
-    from token_level_sparse_kv_b200.inputs import WORKLOADS, Workload, make_inputs, make_queries
+    from token_level_sparse_kv_b200.inputs import Workload, make_inputs, make_queries
 
-    w0 = WORKLOADS[args.workload]
+    w0 = workload_of(args)
     w = Workload(**{**w0.__dict__, "seed": w0.seed + 1000 * rank})
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
@@ -436,6 +449,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="jssa", choices=["jssa", "reference"])
     ap.add_argument("--workload", default="gqa_128k_b16")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (sweeps)")
+    ap.add_argument("--topk", type=int, default=None, help="override the workload's k (sweeps)")
     ap.add_argument("--cmp-steps", type=int, default=200)
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-rows", type=int, default=2, help="batch rows in the oracle's timed sample")

@@ -1,11 +1,11 @@
 """Comparison rules between the CUDA path and the fp64 oracle.
 
 Tolerances (written here once, used by every GPU test):
-  * low-rank append: the stored value is one of the two neighbours of the
-    exact sum on the storage grid (bf16: at most one ulp away) and equals the
-    oracle's round-to-nearest-even value in all but a tiny fraction of
-    elements (fp32 accumulation can flip a rounding that lies within a few
-    fp32 ulps of a bf16 tie);
+  * low-rank append: the stored value is one rounding (<= 1 ulp of the
+    storage grid) away from a value within the fp32 accumulation bound
+    (d * 2^-24 * sum |terms|) of the exact sum, and equals the oracle's
+    round-to-nearest-even value in all but 0.1 % of the elements (fp32
+    accumulation moves sums that lie close to a bf16 tie, or close to zero);
   * scores: |gpu - exact| <= 1e-5 * (sum of |terms|) + 1e-6 (fp32 dot products
     of length r after an fp32 projection of length d);
   * selection: exact ties and near-ties may resolve differently in fp32 and
@@ -32,15 +32,6 @@ def host(t):
     return t.detach().cpu()
 
 
-def bf16_neighbours_ok(gpu_bits: np.ndarray, exact: np.ndarray) -> np.ndarray:
-    """True where the bf16 value is the floor or ceiling of `exact` on the bf16 grid."""
-    g = oracle.bf16_bits_to_f64(gpu_bits)
-    e = exact
-    ex = np.frexp(np.abs(e))[1]
-    ulp = np.ldexp(1.0, np.maximum(ex - 8, -133))
-    return np.abs(g - e) < ulp * (1 + 1e-12)
-
-
 def check_append(Kt_gpu: torch.Tensor, K_host, P_host, pos, n_new):
     """Compare GPU low-rank rows with the oracle's (exact sums and RNE values)."""
     kt_code = oracle.BF16 if Kt_gpu.dtype == torch.bfloat16 else oracle.FP32
@@ -51,14 +42,22 @@ def check_append(Kt_gpu: torch.Tensor, K_host, P_host, pos, n_new):
     for b in range(B):
         mask[b, :, pos[b]:pos[b] + n_new] = True
     g, r, e = got[mask], ref[mask], exact[mask]
+    # fp32 accumulation error bound of a length-d dot product: d * 2^-24 * sum |terms|
+    Pa = np.abs(np.asarray(P_host, np.float64))
+    d = Pa.shape[1]
+    Kf = oracle.to_f64(K_host)
+    absum = np.concatenate([np.einsum("thi,hij->htj", np.abs(Kf[b, pos[b]:pos[b] + n_new]), Pa).reshape(-1, Pa.shape[2])
+                            for b in range(B)])
+    acc_err = d * 2.0**-24 * absum
     if kt_code == oracle.BF16:
-        assert np.all(bf16_neighbours_ok(g, e)), "a bf16 value is not a neighbour of the exact sum"
+        gv = oracle.bf16_bits_to_f64(g)
+        ulp = np.ldexp(1.0, np.maximum(np.frexp(np.abs(e))[1] - 8, -133))
+        # one rounding of a value within the fp32 accumulation error of the exact sum
+        assert np.all(np.abs(gv - e) <= ulp + acc_err), "a bf16 value is further than one rounding from the sum"
         frac = np.mean(g != r)
         assert frac <= 1e-3, "%.4f%% of elements differ from round-to-nearest-even" % (100 * frac)
     else:
-        absum = np.einsum("bthi,hij->bhtj", np.abs(oracle.to_f64(K_host)), np.abs(np.asarray(P_host, np.float64)))
-        bound = 1e-6 * absum[mask] + 1e-30
-        assert np.all(np.abs(g.astype(np.float64) - e) <= bound)
+        assert np.all(np.abs(g.astype(np.float64) - e) <= acc_err + np.abs(e) * 2.0**-24)
     return got
 
 
