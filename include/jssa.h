@@ -212,6 +212,37 @@ JSSA_API int jssa_decode_step(const jssa_dims *dims, const void *q, const void *
                      int32_t *idx, int32_t *count, void *out, float *lse, void *ws,
                      size_t ws_bytes, jssa_stream_t stream);
 
+/* Allocation-free variant of jssa_indexed_decode.  The method pages have no
+ * counterpart: this is an integration entry point of this library.
+ *
+ * Some callers cannot hand the library device scratch memory, because they
+ * cannot allocate at call time: a serving engine whose allocator has already
+ * reserved the GPU's memory for its KV-cache pool, a real-time decode loop
+ * that cannot afford the implicit device synchronisation of cudaMalloc /
+ * cudaFree, or a plugin host that forbids allocation inside its hooks.  This
+ * entry point takes the same inputs and outputs as jssa_indexed_decode but no
+ * workspace: its scratch (split partials, arrival counters, status word) is a
+ * fixed 8 MiB array of device memory inside the library, which every GPU that
+ * loads the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ *  - Shapes whose scratch would exceed 8 MiB are rejected with
+ *    JSSA_ERR_WORKSPACE and a message (use jssa_indexed_decode then).
+ *  - The first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents.  The call clears the counters and the status word on `stream`
+ *    before its kernel; calls whose execution overlaps on the GPU (other
+ *    streams, concurrent threads) race on the array and must be serialised
+ *    by the caller.
+ *  - The device status word is not readable by the caller here; bad indices
+ *    are still skipped as in jssa_indexed_decode.
+ * Results equal those of jssa_indexed_decode on the same inputs. */
+JSSA_API int jssa_indexed_decode_noalloc(const jssa_dims *dims, const void *q, const void *K,
+                                         const void *V, const int32_t *idx, const int32_t *count,
+                                         int k, const int32_t *seq_lens, float softmax_scale,
+                                         void *out, float *lse, jssa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

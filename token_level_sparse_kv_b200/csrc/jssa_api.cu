@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "jssa_internal.h"
 
@@ -535,3 +536,78 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------ allocation-free ---
+// jssa_indexed_decode_noalloc: the indexed decode with its scratch (split
+// partials, arrival counters, status word) in a fixed device array owned by
+// the library instead of a caller workspace.  Each device that loads the
+// library holds kNoAllocBytes of it until the process exits.
+namespace {
+
+constexpr size_t kNoAllocBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array for the current device (looked up once
+// per device, with that device current).
+int noalloc_scratch(void **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the current device");
+    if (dev < 0 || dev >= kMaxDevices) return fail(JSSA_ERR_UNSUPPORTED, "device index %d above %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "looking up the allocation-free scratch array");
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return JSSA_OK;
+}
+
+}  // namespace
+
+extern "C" int jssa_indexed_decode_noalloc(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                                           const int32_t *idx, const int32_t *count, int k,
+                                           const int32_t *seq_lens, float softmax_scale, void *out, float *lse,
+                                           jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    if ((st = check_attn_shape(dims, sh))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(out);
+    OPTIONAL_PTR(count);
+    OPTIONAL_PTR(lse);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, L))) return st;
+    if (L.total > kNoAllocBytes)
+        return fail(JSSA_ERR_WORKSPACE,
+                    "this shape needs %zu bytes of scratch, above the %zu bytes of the allocation-free entry point; "
+                    "use jssa_indexed_decode with a caller workspace",
+                    L.total, kNoAllocBytes);
+    if (dims->B == 0) return JSSA_OK;
+    void *ws = nullptr;
+    if ((st = noalloc_scratch(&ws))) return st;
+    // the status word and the arrival counters must start at zero
+    cudaError_t e = cudaMemsetAsync(ws, 0, 256, S(stream));
+    if (e == cudaSuccess) e = cudaMemsetAsync(at<char>(ws, L.att_ctr), 0, (size_t)sh.BH * 4, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the allocation-free scratch");
+    AttnArgs a;
+    fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
+    a.idx = idx;
+    a.count = count;
+    a.k = k;
+    e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the indexed decode");
+    return JSSA_OK;
+}
