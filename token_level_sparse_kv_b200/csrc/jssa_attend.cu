@@ -13,15 +13,23 @@
 // One CTA handles all G query heads of one KV head for one split of the token
 // list, so every K/V row is read once for the whole group.  Rows are staged
 // with cp.async (16 B per request; a row of d = 128 bf16 is 256 B) straight
-// from their place in the [B, T, Hkv, d] cache, double-buffered in tiles of
-// NT rows; rows are padded in shared memory so that the logit phase reads
-// them without bank conflicts.  Logits use fp32 with the softmax scale folded
-// (times log2 e) into q; the softmax is online across tiles; the split partials
-// (unnormalised o, running max m, running sum l) go to the workspace and the
-// last CTA of each (b, h) to arrive (ticket, no waiting) combines them by
-// log-sum-exp and writes out / lse.
+// from their place in the [B, T, Hkv, d] cache, in tiles of NT rows (one
+// buffer when a split fits one tile, two for longer lists); rows are padded in
+// shared memory so that the logit phase reads them without bank conflicts.
+// Logits use fp32 with the softmax scale folded (times log2 e) into q; the
+// softmax is online across tiles.  Split partials (unnormalised o, running max
+// m, running sum l) are combined by log-sum-exp:
+//  * short lists (indexed / gathered): the splits of one (b,h) form one
+//    thread-block cluster and combine through distributed shared memory, each
+//    CTA finishing a slice of the output;
+//  * long lists (dense): partials go to the workspace and the last CTA of the
+//    (b,h) to arrive (ticket, no waiting) combines them.
+#include <cooperative_groups.h>
+
 #include "jssa_common.cuh"
 #include "jssa_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace jssa {
 
@@ -29,6 +37,7 @@ namespace {
 
 constexpr int NTH = kAttnThreads;
 constexpr float kLn2 = 0.693147180559945309417f;
+constexpr int kMaxCluster = 16;
 
 template <typename KV, int D>
 struct AttnShape {
@@ -46,27 +55,32 @@ struct AttnShape {
     static_assert(CPR % TPR == 0, "row split");
 };
 
-template <typename KV, int D, int GM>
-size_t attend_smem_bytes() {
+template <typename KV, int D, int GM, int STAGES>
+constexpr size_t attend_smem_bytes() {
     using S = AttnShape<KV, D>;
-    size_t o = 2 * (size_t)S::STAGE;           // two stages
-    o += (size_t)GM * D * 4;                   // scaled queries
-    o += (size_t)S::NT * GM * 4;               // logits / probabilities
-    o += 2 * (size_t)S::NT * 4;                // token ids per stage
-    o += 3 * (size_t)GM * 4 + 16 * 4;          // m, l, alpha, misc
+    size_t st = (size_t)STAGES * S::STAGE;
+    const size_t part = (size_t)GM * D * 4;  // cluster partial o reuses the stage buffers
+    if (st < part) st = part;
+    size_t o = st;
+    o += (size_t)GM * D * 4;          // scaled queries
+    o += (size_t)S::NT * GM * 4;      // logits / probabilities
+    o += (size_t)STAGES * S::NT * 4;  // token ids per stage
+    o += 3 * (size_t)GM * 4 + 16 * 4; // m, l, alpha, misc
     return (o + 127) / 128 * 128;
 }
 
-template <typename KV, int D, int GM, int SRC>
+template <typename KV, int D, int GM, int SRC, int STAGES, bool CLUSTER>
 __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
     using S = AttnShape<KV, D>;
     constexpr int NT = S::NT, TPR = S::TPR, CPT = S::CPT, STRIDE = S::STRIDE, EPL = S::EPL, DPT = S::DPT;
+    constexpr size_t STAGE_BYTES = ((size_t)STAGES * S::STAGE > (size_t)GM * D * 4) ? (size_t)STAGES * S::STAGE
+                                                                                    : (size_t)GM * D * 4;
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *stage0 = smem;
-    float *q_s = reinterpret_cast<float *>(smem + 2 * S::STAGE);
+    float *q_s = reinterpret_cast<float *>(smem + STAGE_BYTES);
     float *lg = q_s + GM * D;
     int *tok_s = reinterpret_cast<int *>(lg + NT * GM);
-    float *m_run = reinterpret_cast<float *>(tok_s + 2 * NT);
+    float *m_run = reinterpret_cast<float *>(tok_s + STAGES * NT);
     float *l_run = m_run + GM;
     float *alpha_s = l_run + GM;
     int *misc = reinterpret_cast<int *>(alpha_s + GM);
@@ -107,34 +121,39 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
     const int p1 = min(p0 + a.pos_per_split, npos);
     const int ntile = p1 > p0 ? (p1 - p0 + NT - 1) / NT : 0;
 
-    // token of list position p (-1 = skip)
-    auto token_of = [&](int p) -> int {
-        if (SRC == ATT_INDEXED) {
-            const int t = __ldg(a.idx + (size_t)bh * a.k + p);
-            if (t < 0 || t >= Tb) {
-                if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_INDEX);
-                return -1;
-            }
-            return t;
-        } else if (SRC == ATT_RANGE) {
-            return lo + p;
-        }
-        return p;
-    };
-
     const char *Kb = static_cast<const char *>(a.K);
     const char *Vb = static_cast<const char *>(a.V);
+    // stage the token ids of tile j (one global read per row), then its rows
     auto issue = [&](int j, int st) {
         const int pos0 = p0 + j * NT;
         const int rows = min(NT, p1 - pos0);
+        int *tk = tok_s + st * NT;
+        if (tid < NT) {
+            int t = -1;
+            if (tid < rows) {
+                const int p = pos0 + tid;
+                if (SRC == ATT_INDEXED) {
+                    t = __ldg(a.idx + (size_t)bh * a.k + p);
+                    if (t < 0 || t >= Tb) {
+                        if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_INDEX);
+                        t = -1;
+                    }
+                } else if (SRC == ATT_RANGE) {
+                    t = lo + p;
+                } else {
+                    t = p;
+                }
+            }
+            tk[tid] = t;
+        }
+        __syncthreads();
         unsigned char *ks = stage0 + (size_t)st * S::STAGE;
         constexpr int CH = NT * S::CPR;
         for (int c = tid; c < 2 * CH; c += NTH) {
             const int kv = c >= CH;
             const int rem = c - kv * CH;
             const int row = rem / S::CPR, ch = rem - row * S::CPR;
-            int t = -1;
-            if (row < rows) t = token_of(pos0 + row);
+            const int t = tk[row];
             unsigned char *dst = ks + (size_t)kv * NT * STRIDE + (size_t)row * STRIDE + ch * 16;
             if (t >= 0) {
                 const long long off = kv ? ((long long)b * a.v_sb + (long long)t * a.v_st + (long long)h * a.v_sh)
@@ -144,20 +163,19 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
                 cp_async16(dst, Kb, 0);
             }
         }
-        if (tid < NT) tok_s[st * NT + tid] = tid < rows ? token_of(pos0 + tid) : -1;
         cp_async_commit();
     };
 
-    if (ntile > 0) issue(0, 0);
-    if (ntile > 1) issue(1, 1);
-
-    // scaled queries of the group, m / l state
+    // scaled queries of the group and the m / l state (visible after the first wait + sync)
     const KV *q = static_cast<const KV *>(a.q) + ((size_t)b * a.Hq + (size_t)h * G) * D;
     for (int p = tid; p < G * D; p += NTH) q_s[p] = to_f32(q[p]) * a.scale_log2;
     if (tid < GM) {
         m_run[tid] = -INFINITY;
         l_run[tid] = 0.f;
     }
+
+    if (ntile > 0) issue(0, 0);
+    if (STAGES > 1 && ntile > 1) issue(1, 1 % STAGES);
 
     float acc[GM][DPT];
 #pragma unroll
@@ -171,12 +189,12 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
     const int lane = tid & 31, warp = tid >> 5;
 
     for (int j = 0; j < ntile; ++j) {
-        if (j + 1 < ntile)
+        if (STAGES > 1 && j + 1 < ntile)
             cp_async_wait<1>();
         else
             cp_async_wait<0>();
         __syncthreads();
-        const int st = j & 1;
+        const int st = j % STAGES;
         const unsigned char *Ks = stage0 + (size_t)st * S::STAGE;
         const unsigned char *Vs = Ks + (size_t)NT * STRIDE;
         const int rows = min(NT, p1 - (p0 + j * NT));
@@ -268,7 +286,7 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
             }
         }
         __syncthreads();
-        if (j + 2 < ntile) issue(j + 2, st);
+        if (STAGES > 1 && j + STAGES < ntile) issue(j + STAGES, st);
     }
 
     KV *out = static_cast<KV *>(a.out);
@@ -292,54 +310,91 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
         return;
     }
 
-    // split partials, then the last CTA of this (b,h) combines them
-    const size_t pbase = ((size_t)bh * a.splits + split) * G;
-    if (own) {
-#pragma unroll
-        for (int g = 0; g < GM; ++g)
-            if (g < G)
-#pragma unroll
-                for (int u = 0; u < DPT; ++u) a.part_o[(pbase + g) * D + d0 + u] = acc[g][u];
-    }
-    if (tid < G) {
-        a.part_ml[(pbase + tid) * 2 + 0] = m_run[tid];
-        a.part_ml[(pbase + tid) * 2 + 1] = l_run[tid];
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) misc[0] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(a.splits - 1);
-    __syncthreads();
-    if (!misc[0]) return;
-    __threadfence();
-    for (int g = 0; g < G; ++g) {
-        float M = -INFINITY;
-        for (int s = 0; s < a.splits; ++s)
-            M = fmaxf(M, __ldcg(a.part_ml + (((size_t)bh * a.splits + s) * G + g) * 2));
-        float L = 0.f;
-        float o[DPT];
-#pragma unroll
-        for (int u = 0; u < DPT; ++u) o[u] = 0.f;
-        for (int s = 0; s < a.splits; ++s) {
-            const size_t pb = ((size_t)bh * a.splits + s) * G + g;
-            const float ms = __ldcg(a.part_ml + pb * 2);
-            if (ms == -INFINITY) continue;
-            const float w = exp2f(ms - M);
-            L = fmaf(__ldcg(a.part_ml + pb * 2 + 1), w, L);
-            if (own) {
-#pragma unroll
-                for (int u = 0; u < DPT; ++u) o[u] = fmaf(__ldcg(a.part_o + pb * D + d0 + u), w, o[u]);
-            }
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
+    if constexpr (CLUSTER) {
+        // partial o into this CTA's shared memory (the stage buffers are free now)
+        float *po = reinterpret_cast<float *>(stage0);
         if (own) {
 #pragma unroll
-            for (int u = 0; u < DPT; ++u)
-                store_elem(out + ((size_t)b * a.Hq + (size_t)h * G + g) * D + d0 + u, o[u] * inv);
+            for (int g = 0; g < GM; ++g)
+                if (g < G)
+#pragma unroll
+                    for (int u = 0; u < DPT; ++u) po[g * D + d0 + u] = acc[g][u];
         }
-        if (a.lse && tid == 0)
-            a.lse[(size_t)b * a.Hq + (size_t)h * G + g] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        // CTA `split` combines dims [split*slice, (split+1)*slice) of every head
+        const int ns = a.splits;
+        const int slice = (D + ns - 1) / ns;
+        const int c0 = split * slice, c1 = min(D, c0 + slice);
+        const int width = c1 - c0;
+        for (int p = tid; p < G * (width > 0 ? width : 0); p += NTH) {
+            const int g = p / width, c = c0 + (p - g * width);
+            float M = -INFINITY;
+            for (int s = 0; s < ns; ++s) M = fmaxf(M, *cluster.map_shared_rank(m_run + g, s));
+            float L = 0.f, o = 0.f;
+            for (int s = 0; s < ns; ++s) {
+                const float ms = *cluster.map_shared_rank(m_run + g, s);
+                if (ms == -INFINITY) continue;
+                const float w = exp2f(ms - M);
+                L = fmaf(*cluster.map_shared_rank(l_run + g, s), w, L);
+                o = fmaf(*cluster.map_shared_rank(po + g * D + c, s), w, o);
+            }
+            store_elem(out + ((size_t)b * a.Hq + (size_t)h * G + g) * D + c, L > 0.f ? o / L : 0.f);
+            if (a.lse && split == 0 && c == c0)
+                a.lse[(size_t)b * a.Hq + (size_t)h * G + g] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        }
+        cluster.sync();  // peers keep their shared memory until every slice is read
+        return;
+    } else {
+        // split partials in the workspace; the last CTA of this (b,h) combines them
+        const size_t pbase = ((size_t)bh * a.splits + split) * G;
+        if (own) {
+#pragma unroll
+            for (int g = 0; g < GM; ++g)
+                if (g < G)
+#pragma unroll
+                    for (int u = 0; u < DPT; ++u) a.part_o[(pbase + g) * D + d0 + u] = acc[g][u];
+        }
+        if (tid < G) {
+            a.part_ml[(pbase + tid) * 2 + 0] = m_run[tid];
+            a.part_ml[(pbase + tid) * 2 + 1] = l_run[tid];
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) misc[0] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(a.splits - 1);
+        __syncthreads();
+        if (!misc[0]) return;
+        __threadfence();
+        for (int g = 0; g < G; ++g) {
+            float M = -INFINITY;
+            for (int s = 0; s < a.splits; ++s)
+                M = fmaxf(M, __ldcg(a.part_ml + (((size_t)bh * a.splits + s) * G + g) * 2));
+            float L = 0.f;
+            float o[DPT];
+#pragma unroll
+            for (int u = 0; u < DPT; ++u) o[u] = 0.f;
+            for (int s = 0; s < a.splits; ++s) {
+                const size_t pb = ((size_t)bh * a.splits + s) * G + g;
+                const float ms = __ldcg(a.part_ml + pb * 2);
+                if (ms == -INFINITY) continue;
+                const float w = exp2f(ms - M);
+                L = fmaf(__ldcg(a.part_ml + pb * 2 + 1), w, L);
+                if (own) {
+#pragma unroll
+                    for (int u = 0; u < DPT; ++u) o[u] = fmaf(__ldcg(a.part_o + pb * D + d0 + u), w, o[u]);
+                }
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            if (own) {
+#pragma unroll
+                for (int u = 0; u < DPT; ++u)
+                    store_elem(out + ((size_t)b * a.Hq + (size_t)h * G + g) * D + d0 + u, o[u] * inv);
+            }
+            if (a.lse && tid == 0)
+                a.lse[(size_t)b * a.Hq + (size_t)h * G + g] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        }
+        if (tid == 0) a.counters[bh] = 0u;
     }
-    if (tid == 0) a.counters[bh] = 0u;
 }
 
 // Copy the selected K and V rows of each (b,h) into contiguous [B,Hkv,k,d]
@@ -348,8 +403,8 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
 template <typename KV>
 __global__ void __launch_bounds__(NTH) gather_kernel(GatherArgs a) {
     extern __shared__ __align__(16) int g_sm[];
-    int *comp = g_sm;           // [k] compacted token ids
-    int *tmp = g_sm + a.k;      // [32]
+    int *comp = g_sm;       // [k] compacted token ids
+    int *tmp = g_sm + a.k;  // [32]
     const int tid = threadIdx.x;
     const int bh = blockIdx.x;
     const int b = bh / a.Hkv, h = bh - b * a.Hkv;
@@ -401,96 +456,164 @@ __global__ void __launch_bounds__(NTH) gather_kernel(GatherArgs a) {
     }
 }
 
+using AttnKernel = void (*)(AttnArgs);
+
+struct AttnPick {
+    AttnKernel kern = nullptr;
+    size_t smem = 0;
+    int nt = 0;
+};
+
+// Long lists (dense): two stages, workspace combine.  Short lists (indexed,
+// gathered): one stage when a split fits one tile, cluster combine.
 template <typename KV, int D, int GM>
-void (*pick_attend_src(int src))(AttnArgs) {
-    switch (src) {
-        case ATT_INDEXED: return attend_kernel<KV, D, GM, ATT_INDEXED>;
-        case ATT_RANGE: return attend_kernel<KV, D, GM, ATT_RANGE>;
-        default: return attend_kernel<KV, D, GM, ATT_RANGE_BH>;
+AttnPick pick_attend_g(int src, int stages) {
+    AttnPick p;
+    p.nt = AttnShape<KV, D>::NT;
+    if (src == ATT_RANGE) {
+        p.kern = attend_kernel<KV, D, GM, ATT_RANGE, 2, false>;
+        p.smem = attend_smem_bytes<KV, D, GM, 2>();
+    } else if (src == ATT_INDEXED) {
+        p.kern = stages == 1 ? attend_kernel<KV, D, GM, ATT_INDEXED, 1, true>
+                             : attend_kernel<KV, D, GM, ATT_INDEXED, 2, true>;
+        p.smem = stages == 1 ? attend_smem_bytes<KV, D, GM, 1>() : attend_smem_bytes<KV, D, GM, 2>();
+    } else {
+        p.kern = stages == 1 ? attend_kernel<KV, D, GM, ATT_RANGE_BH, 1, true>
+                             : attend_kernel<KV, D, GM, ATT_RANGE_BH, 2, true>;
+        p.smem = stages == 1 ? attend_smem_bytes<KV, D, GM, 1>() : attend_smem_bytes<KV, D, GM, 2>();
     }
+    return p;
 }
 
 template <typename KV, int D>
-void (*pick_attend_g(int src, int G, size_t *smem))(AttnArgs) {
-    if (G <= 4) {
-        *smem = attend_smem_bytes<KV, D, 4>();
-        return pick_attend_src<KV, D, 4>(src);
-    }
-    if (G <= 8) {
-        *smem = attend_smem_bytes<KV, D, 8>();
-        return pick_attend_src<KV, D, 8>(src);
-    }
-    *smem = attend_smem_bytes<KV, D, 16>();
-    return pick_attend_src<KV, D, 16>(src);
+AttnPick pick_attend_d(int src, int G, int stages) {
+    if (G <= 4) return pick_attend_g<KV, D, 4>(src, stages);
+    if (G <= 8) return pick_attend_g<KV, D, 8>(src, stages);
+    return pick_attend_g<KV, D, 16>(src, stages);
 }
 
 template <typename KV>
-void (*pick_attend_d(int src, int d, int G, size_t *smem, int *nt))(AttnArgs) {
+AttnPick pick_attend_kv(int src, int d, int G, int stages) {
     switch (d) {
-        case 64: *nt = AttnShape<KV, 64>::NT; return pick_attend_g<KV, 64>(src, G, smem);
-        case 128: *nt = AttnShape<KV, 128>::NT; return pick_attend_g<KV, 128>(src, G, smem);
-        case 256: *nt = AttnShape<KV, 256>::NT; return pick_attend_g<KV, 256>(src, G, smem);
-        default: return nullptr;
+        case 64: return pick_attend_d<KV, 64>(src, G, stages);
+        case 128: return pick_attend_d<KV, 128>(src, G, stages);
+        case 256: return pick_attend_d<KV, 256>(src, G, stages);
+        default: return AttnPick();
     }
 }
 
-void (*pick_attend(int src, int kv_dtype, int d, int G, size_t *smem, int *nt))(AttnArgs) {
-    if (G < 1 || G > kMaxG) return nullptr;
-    return kv_dtype == JSSA_BF16 ? pick_attend_d<__nv_bfloat16>(src, d, G, smem, nt)
-                                 : pick_attend_d<float>(src, d, G, smem, nt);
+AttnPick pick_attend(int src, int kv_dtype, int d, int G, int stages) {
+    if (G < 1 || G > kMaxG) return AttnPick();
+    return kv_dtype == JSSA_BF16 ? pick_attend_kv<__nv_bfloat16>(src, d, G, stages)
+                                 : pick_attend_kv<float>(src, d, G, stages);
+}
+
+int rows_per_tile(int kv_dtype, int d) {
+    const int rowb = d * (kv_dtype == JSSA_BF16 ? 2 : 4);
+    int nt = 16384 / rowb;
+    return nt > 64 ? 64 : (nt < 16 ? 16 : nt);
 }
 
 }  // namespace
 
 cudaError_t plan_attend(int src, int kv_dtype, int d, int G, int B, int Hkv, int npos, AttnPlan *p) {
-    size_t smem = 0;
-    int nt = 0;
-    auto kern = pick_attend(src, kv_dtype, d, G, &smem, &nt);
-    if (!kern) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NTH, smem);
-    if (e != cudaSuccess) return e;
-    if (occ < 1) return cudaErrorInvalidConfiguration;
+    const int nt = rows_per_tile(kv_dtype, d);
     const long long BH = (long long)B * Hkv;
     const int sms = device_sm_count();
     if (npos < 1) npos = 1;
-    int splits;
+    int splits, pps, stages;
     if (src == ATT_RANGE) {
         // long lists: ~16 tiles per CTA, many CTAs (the scheduler balances)
         splits = (npos + 16 * nt - 1) / (16 * nt);
+        if (splits < 1) splits = 1;
+        pps = (npos + splits - 1) / splits;
+        pps = (pps + nt - 1) / nt * nt;
+        splits = (npos + pps - 1) / pps;
+        stages = 2;
+        if (splits > 65535) return cudaErrorInvalidConfiguration;
     } else {
-        // short lists: enough CTAs for two per SM, at least 16 positions each
+        // short lists: one cluster of splits per (b,h); enough CTAs for about two
+        // per SM, at least 16 positions each, at most kMaxCluster splits
         long long want = (2LL * sms + BH - 1) / BH;
-        int by_tile = (npos + nt - 1) / nt;
-        int most = (npos + 15) / 16;
+        const int by_tile = (npos + nt - 1) / nt;
+        const int most = (npos + 15) / 16;
         splits = (int)(want > by_tile ? want : by_tile);
         if (splits > most) splits = most;
+        if (splits > kMaxCluster) splits = kMaxCluster;
+        if (splits < 1) splits = 1;
+        pps = (npos + splits - 1) / splits;
+        splits = (npos + pps - 1) / pps;
+        stages = pps <= nt ? 1 : 2;
     }
-    if (splits < 1) splits = 1;
-    int pps = (npos + splits - 1) / splits;
-    if (src == ATT_RANGE) pps = (pps + nt - 1) / nt * nt;
-    splits = (npos + pps - 1) / pps;
-    if (splits > 65535) return cudaErrorInvalidConfiguration;
+    AttnPick pk;
+    for (;;) {
+        pk = pick_attend(src, kv_dtype, d, G, stages);
+        if (!pk.kern) return cudaErrorInvalidValue;
+        cudaError_t e = cudaFuncSetAttribute(pk.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pk.smem);
+        if (e != cudaSuccess) return e;
+        if (src == ATT_RANGE || splits == 1) break;
+        if (splits > 8) {
+            e = cudaFuncSetAttribute(pk.kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
+        // the cluster of `splits` CTAs must fit on the device; otherwise halve it
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(splits, 1);
+        cfg.blockDim = dim3(NTH);
+        cfg.dynamicSmemBytes = pk.smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = splits;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&nclusters, pk.kern, &cfg);
+        if (e != cudaSuccess) return e;
+        if (nclusters > 0) break;
+        splits = (splits + 1) / 2;
+        pps = (npos + splits - 1) / splits;
+        splits = (npos + pps - 1) / pps;
+        stages = pps <= nt ? 1 : 2;
+    }
     p->nt = nt;
     p->splits = splits;
     p->pos_per_split = pps;
-    p->stages = 2;
-    p->smem = smem;
+    p->stages = stages;
+    p->smem = pk.smem;
     return cudaSuccess;
 }
 
 cudaError_t launch_attend(const AttnPlan &p, int src, const AttnArgs &a0, int kv_dtype, int d, cudaStream_t s,
                           bool pdl) {
-    size_t smem = 0;
-    int nt = 0;
-    auto kern = pick_attend(src, kv_dtype, d, a0.G, &smem, &nt);
-    if (!kern) return cudaErrorInvalidValue;
+    AttnPick pk = pick_attend(src, kv_dtype, d, a0.G, p.stages);
+    if (!pk.kern) return cudaErrorInvalidValue;
     AttnArgs a = a0;
     a.splits = p.splits;
     a.pos_per_split = p.pos_per_split;
-    return launch_kernel(kern, dim3(p.splits, a.B * a.Hkv), dim3(NTH), p.smem, s, pdl, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.splits, a.B * a.Hkv);
+    cfg.blockDim = dim3(NTH);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (src != ATT_RANGE && p.splits > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = p.splits;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, pk.kern, a);
 }
 
 cudaError_t launch_gather(const GatherArgs &a, int kv_dtype, cudaStream_t s, bool pdl) {

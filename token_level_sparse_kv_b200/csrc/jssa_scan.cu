@@ -8,23 +8,28 @@
 //
 // One persistent kernel streams token tiles of every (b, h):
 //  * work = the flattened list of (b,h, tile) tiles; CTA i takes the
-//    contiguous range [i*N/grid, (i+1)*N/grid), so the load is balanced to
-//    one tile whatever B*Hkv is.  A range crosses at most a few (b,h)
-//    boundaries; each (b,h) piece of it is a "segment".
-//  * low-rank key tiles (16 KiB) arrive through a ring of bulk asynchronous
-//    copies (TMA engine, mbarrier completion, evict-first L2 hint); lanes
-//    groups of r*es/16 threads reduce one token's dot product with warp
-//    shuffles.  The score array source (jssa_topk) is read with plain loads.
-//  * MODE_WRITE stores the fp32 scores.  MODE_SELECT keeps a running top-k
-//    of the segment in shared memory: a token survives only if its key beats
-//    the current k-th key, survivors are appended in token order, and when
-//    the buffer fills a radix select (4 passes of 8 bits over order-
-//    preserving uint32 keys) keeps the best k, ties to the lower index.  The
-//    segment's k candidates go to the workspace; the last CTA to finish a
-//    (b,h) (arrival ticket, no waiting) merges its segments with the same
-//    machinery and writes the ascending index list.
-// Because the order (score desc, index asc) is a strict total order, the top-k
-// of the union of per-segment top-k sets is the global top-k: the fused path
+//    contiguous range [i*N/grid, (i+1)*N/grid), so the load is balanced to one
+//    tile whatever B*Hkv is.  A range crosses at most a few (b,h) boundaries;
+//    each (b,h) piece of it is a "segment".
+//  * 32 KiB tiles of the low-rank key cache arrive through a 3-deep ring of
+//    bulk asynchronous copies (TMA engine, mbarrier completion, evict-first L2
+//    hint).  A thread scores whole tokens (up to 64 bytes of a row; wider
+//    rows are split over 2..8 lanes and reduced with shuffles), reading its
+//    16-byte chunks in a lane-rotated order so that every quarter-warp hits 8
+//    distinct bank groups.  The score-array source (jssa_topk) is read with
+//    plain coalesced loads.
+//  * MODE_WRITE stores fp32 scores.  MODE_SELECT keeps a running top-k of the
+//    segment in shared memory: a token survives only if its key beats the
+//    k-th key kept so far (tokens arrive in ascending index order within a
+//    segment, so an equal key always loses to the kept one); survivors are
+//    appended with one warp-aggregated shared atomic; when the buffer may not
+//    absorb another tile, a radix select (4 passes of 8 bits over
+//    order-preserving uint32 keys, then over inverted indices for the tie
+//    group) keeps the best k.  The segment's candidates go to the workspace;
+//    the last CTA to finish a (b,h) (arrival ticket, no waiting) merges the
+//    segments the same way and writes the selection sorted by index.
+// The order (score desc, index asc) is a strict total order, so the top-k of
+// the union of per-segment top-k sets is the global top-k: the fused path
 // returns exactly what jssa_score + jssa_topk return.
 #include <type_traits>
 
@@ -36,29 +41,32 @@ namespace jssa {
 namespace {
 
 constexpr int NT = kScanThreads;
+constexpr int kTileBytes = 2 * kScanStageBytes;  // 32 KiB per stage
+constexpr int kStages = 3;
+
+__host__ __device__ inline int next_pow2(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
 
 struct ScanSmem {
-    size_t stages, bars, tkey, tidx, qs, buf_key, buf_idx, res_key, res_idx, hist, tmp, misc, total;
+    size_t stages, bars, qs, buf_key, buf_idx, res_key, res_idx, hist, tmp, misc, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline ScanSmem scan_smem(int src, int mode, int r, int nstages, int cap, int k,
-                                              int tile) {
+__host__ __device__ inline ScanSmem scan_smem(int src, int mode, int r, int nq, int nstages, int cap, int k) {
     ScanSmem L;
     size_t o = 0;
     const bool from_kt = src != SRC_SCORES;
+    const bool sel = mode == MODE_SELECT;
     L.stages = o;
-    o += from_kt ? (size_t)nstages * kScanStageBytes : 0;
+    o += from_kt ? (size_t)nstages * kTileBytes : 0;
     L.bars = o;
     o = align_up(o + (from_kt ? (size_t)nstages * 8 : 0), 16);
-    L.tkey = o;
-    o = align_up(o + (size_t)tile * 4, 16);
-    L.tidx = o;
-    o = align_up(o + (mode == MODE_SELECT ? (size_t)tile * 4 : 0), 16);
     L.qs = o;
-    o = align_up(o + (from_kt ? (size_t)kMaxG * r * 4 : 0), 16);
-    const bool sel = mode == MODE_SELECT;
+    o = align_up(o + (from_kt ? (size_t)nq * r * 4 : 0), 16);
     L.buf_key = o;
     o = align_up(o + (sel ? (size_t)cap * 4 : 0), 16);
     L.buf_idx = o;
@@ -66,7 +74,7 @@ __host__ __device__ inline ScanSmem scan_smem(int src, int mode, int r, int nsta
     L.res_key = o;
     o = align_up(o + (sel ? (size_t)k * 4 : 0), 16);
     L.res_idx = o;
-    o = align_up(o + (sel ? (size_t)k * 4 : 0), 16);
+    o = align_up(o + (sel ? (size_t)next_pow2(k) * 4 : 0), 16);
     L.hist = o;
     o = align_up(o + 256 * 4, 16);
     L.tmp = o;
@@ -77,7 +85,8 @@ __host__ __device__ inline ScanSmem scan_smem(int src, int mode, int r, int nsta
     return L;
 }
 
-// Shared state of the running top-k buffer (all values uniform across the block).
+// Running top-k buffer in shared memory.  Entries are unordered; the count
+// lives in shared memory (misc[4]) because warps append with atomics.
 struct TopK {
     uint32_t *key;
     int32_t *idx;
@@ -85,23 +94,61 @@ struct TopK {
     int32_t *res_idx;
     uint32_t *hist;
     int *tmp;
-    int *misc;
-    int n;          // entries in the buffer
-    bool valid;     // thresh holds the k-th best key of a full reduction
+    int *misc;  // [0..1], [5] select scratch, [2] ticket flag, [3] keep counter, [4] count
+    bool valid;  // thresh holds the k-th best key of a completed reduction
     uint32_t thresh;
 };
 
-// kk-th largest key among keys[0..n) (1 <= kk <= n): returns the key value and
-// how many entries equal to it belong to the top kk.
-__device__ void radix_select(const uint32_t *keys, int n, int kk, TopK &tk, uint32_t &tau, int &need) {
+// Sum of the per-chunk partials of one thread, independent of the lane's
+// rotation of the visiting order: a rotation by one swaps the pairs {0,2} and
+// {1,3} as wholes, and each pair sum is commutative, so every lane adds the
+// same two pair sums.  Identical rows therefore score bit-identically.
+template <int CPT>
+__device__ __forceinline__ float chunk_sum(const float *p) {
+    if (CPT == 4) return (p[0] + p[2]) + (p[1] + p[3]);
+    if (CPT == 2) return p[0] + p[1];
+    return p[0];
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Warp-aggregated append of one candidate per lane (all 32 lanes call it).
+__device__ __forceinline__ void offer(TopK &tk, bool take, uint32_t key, int32_t idx, int cap) {
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (m == 0u) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(&tk.misc[4], __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (take) {
+        const int pos = base + __popc(m & lanemask_lt());
+        if (pos < cap) {
+            tk.key[pos] = key;
+            tk.idx[pos] = idx;
+        }
+    }
+}
+
+// kk-th largest value of val(j) over the entries with use(j) (1 <= kk <= their
+// count).  Returns the value, how many entries equal to it are in the top kk,
+// and (eq_total) how many used entries equal it.
+template <typename Use, typename Val>
+__device__ void radix_select(int n, int kk, TopK &tk, Use use, Val val, uint32_t &tau, int &need, int &eq_total) {
     const int tid = threadIdx.x;
     uint32_t prefix = 0u, mask = 0u;
+    int last_count = 0;
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
         tk.hist[tid] = 0u;
         __syncthreads();
         for (int j = tid; j < n; j += NT) {
-            const uint32_t u = keys[j];
+            if (!use(j)) continue;
+            const uint32_t u = val(j);
             if ((u & mask) == prefix) atomicAdd(&tk.hist[(u >> shift) & 0xffu], 1u);
         }
         __syncthreads();
@@ -111,56 +158,60 @@ __device__ void radix_select(const uint32_t *keys, int n, int kk, TopK &tk, uint
         if (ex < kk && ex + c >= kk) {
             tk.misc[0] = 255 - tid;
             tk.misc[1] = ex;
+            tk.misc[5] = c;
         }
         __syncthreads();
         prefix |= (uint32_t)tk.misc[0] << shift;
         mask |= 0xffu << shift;
         kk -= tk.misc[1];
+        last_count = tk.misc[5];
         __syncthreads();
     }
     tau = prefix;
     need = kk;
+    eq_total = last_count;
 }
 
-// Keep the best k of the buffer (requires tk.n > k), stable in buffer order.
-__device__ void reduce_topk(TopK &tk, int k) {
+// Keep the best k of the n > k buffered entries under (key desc, idx asc).
+__device__ void reduce_topk(TopK &tk, int n, int k) {
     const int tid = threadIdx.x;
-    uint32_t tau;
-    int need;
-    radix_select(tk.key, tk.n, k, tk, tau, need);
-    const int per = (tk.n + NT - 1) / NT;
-    const int j0 = min(tid * per, tk.n), j1 = min(j0 + per, tk.n);
-    int ceq = 0;
-    for (int j = j0; j < j1; ++j) ceq += tk.key[j] == tau;
-    int tot;
-    const int eq0 = block_excl_scan<NT>(ceq, tk.tmp, tot);
-    int ckeep = 0;
-    {
-        int e = eq0;
-        for (int j = j0; j < j1; ++j) {
-            const uint32_t u = tk.key[j];
-            if (u > tau) {
-                ++ckeep;
-            } else if (u == tau) {
-                ckeep += e < need;
-                ++e;
-            }
-        }
+    uint32_t tau, tau2 = 0u;
+    int need, m;
+    radix_select(
+        n, k, tk, [&](int) { return true; }, [&](int j) { return tk.key[j]; }, tau, need, m);
+    const bool all_ties = need == m;
+    if (!all_ties) {
+        // among the entries equal to tau, the `need` lowest indices
+        int need2, m2;
+        radix_select(
+            n, need, tk, [&](int j) { return tk.key[j] == tau; },
+            [&](int j) { return ~(uint32_t)tk.idx[j]; }, tau2, need2, m2);
     }
-    int w = block_excl_scan<NT>(ckeep, tk.tmp, tot);
-    {
-        int e = eq0;
-        for (int j = j0; j < j1; ++j) {
-            const uint32_t u = tk.key[j];
-            bool keep = u > tau;
-            if (u == tau) {
-                keep = e < need;
-                ++e;
-            }
-            if (keep && w < k) {
-                tk.res_key[w] = u;
-                tk.res_idx[w] = tk.idx[j];
-                ++w;
+    if (tid == 0) tk.misc[3] = 0;
+    __syncthreads();
+    const int lane = tid & 31;
+    for (int j0 = 0; j0 < n; j0 += NT) {
+        const int j = j0 + tid;
+        bool keep = false;
+        uint32_t u = 0u;
+        int32_t ix = 0;
+        if (j < n) {
+            u = tk.key[j];
+            ix = tk.idx[j];
+            keep = u > tau || (u == tau && (all_ties || ~(uint32_t)ix >= tau2));
+        }
+        const unsigned msk = __ballot_sync(0xffffffffu, keep);
+        int base = 0;
+        if (msk) {
+            const int leader = __ffs(msk) - 1;
+            if (lane == leader) base = atomicAdd(&tk.misc[3], __popc(msk));
+            base = __shfl_sync(0xffffffffu, base, leader);
+        }
+        if (keep) {
+            const int pos = base + __popc(msk & lanemask_lt());
+            if (pos < k) {
+                tk.res_key[pos] = u;
+                tk.res_idx[pos] = ix;
             }
         }
     }
@@ -169,36 +220,34 @@ __device__ void reduce_topk(TopK &tk, int k) {
         tk.key[j] = tk.res_key[j];
         tk.idx[j] = tk.res_idx[j];
     }
+    if (tid == 0) tk.misc[4] = k;
     __syncthreads();
-    tk.n = k;
     tk.valid = true;
     tk.thresh = tau;
 }
 
-// Append the survivors among keys[0..n) (indices t0 + j, or ids[j]) in order,
-// then shrink the buffer if the next chunk of `chunk` entries might not fit.
-template <int CHUNK>
-__device__ void append_chunk(TopK &tk, const uint32_t *keys, const int32_t *ids, int t0, int n, int k, int cap) {
-    constexpr int PER = (CHUNK + NT - 1) / NT;
+// Sort a[0..n) ascending in place (bitonic network over the next power of two,
+// padded with INT_MAX; a has room for next_pow2(n) entries).
+__device__ void sort_ascending(int32_t *a, int n) {
     const int tid = threadIdx.x;
-    const int j0 = min(tid * PER, n), j1 = min(j0 + PER, n);
-    const bool all = !tk.valid;
-    const uint32_t th = tk.thresh;
-    int c = 0;
-    for (int j = j0; j < j1; ++j) c += all || keys[j] > th;
-    int tot;
-    int w = tk.n + block_excl_scan<NT>(c, tk.tmp, tot);
-    for (int j = j0; j < j1; ++j) {
-        const uint32_t u = keys[j];
-        if ((all || u > th) && w < cap) {
-            tk.key[w] = u;
-            tk.idx[w] = ids ? ids[j] : t0 + j;
-            ++w;
+    const int P = next_pow2(n < 1 ? 1 : n);
+    for (int j = n + tid; j < P; j += NT) a[j] = 0x7fffffff;
+    __syncthreads();
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = tid; i < P / 2; i += NT) {
+                const int lo = 2 * stride * (i / stride) + (i % stride);
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const int32_t x = a[lo], y = a[hi];
+                if ((x > y) == up) {
+                    a[lo] = y;
+                    a[hi] = x;
+                }
+            }
+            __syncthreads();
         }
     }
-    tk.n += tot;
-    __syncthreads();
-    if (tk.n > cap - CHUNK) reduce_topk(tk, k);
 }
 
 template <int SRC, int MODE, int R, int AGG>
@@ -206,17 +255,22 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
     constexpr bool FROM_KT = SRC != SRC_SCORES;
     using KT = typename std::conditional<SRC == SRC_KT_FP32, float, __nv_bfloat16>::type;
     constexpr int ES = SRC == SRC_KT_FP32 ? 4 : 2;
-    constexpr int ROWB = FROM_KT ? R * ES : 4;
-    constexpr int LPT = FROM_KT ? ROWB / 16 : 1;  // lanes per token
-    constexpr int EPL = 16 / ES;                  // elements per lane
-    constexpr int TILE = FROM_KT ? kScanStageBytes / ROWB : kScoreTileTokens;
-    static_assert(!FROM_KT || (LPT >= 1 && LPT <= 32 && (LPT & (LPT - 1)) == 0), "bad lanes per token");
+    constexpr int ROWB = FROM_KT ? R * ES : 4;  // bytes per token
+    constexpr int TPB = ROWB > 64 ? 64 : ROWB;  // bytes of a token per thread
+    constexpr int LPT = ROWB / TPB;             // lanes per token
+    constexpr int CPT = FROM_KT ? TPB / 16 : 1;  // 16-byte chunks per thread
+    constexpr int EPL = 16 / ES;                // elements per chunk
+    constexpr int TILE = FROM_KT ? kTileBytes / ROWB : kScoreTileTokens;
+    constexpr int TPP = NT / LPT;  // tokens per pass
+    constexpr int PASSES = FROM_KT ? TILE / TPP : TILE / NT;
+    constexpr int QN = FROM_KT ? CPT * EPL : 1;
+    static_assert(!FROM_KT || (LPT >= 1 && LPT <= 32 && (LPT & (LPT - 1)) == 0), "lanes per token");
+    static_assert(!FROM_KT || (CPT >= 1 && CPT <= 4), "chunks per thread");
+    static_assert(!FROM_KT || TILE % TPP == 0, "tile / pass");
 
     extern __shared__ __align__(128) unsigned char smem[];
-    const ScanSmem L = scan_smem(SRC, MODE, FROM_KT ? R : 0, a.nstages, a.cap, a.k, TILE);
+    const ScanSmem L = scan_smem(SRC, MODE, FROM_KT ? R : 0, a.nq, kStages, a.cap, a.k);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
-    uint32_t *tkey = reinterpret_cast<uint32_t *>(smem + L.tkey);
-    int32_t *tidx = reinterpret_cast<int32_t *>(smem + L.tidx);
     float *qs = reinterpret_cast<float *>(smem + L.qs);
 
     TopK tk;
@@ -227,11 +281,10 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
     tk.hist = reinterpret_cast<uint32_t *>(smem + L.hist);
     tk.tmp = reinterpret_cast<int *>(smem + L.tmp);
     tk.misc = reinterpret_cast<int *>(smem + L.misc);
-    tk.n = 0;
     tk.valid = false;
     tk.thresh = 0u;
 
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const long long cta = blockIdx.x;
     const long long x_begin = cta * a.total_tiles / a.grid;
     const long long x_end = (cta + 1) * a.total_tiles / a.grid;
@@ -239,124 +292,158 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
     const int tpb = a.tiles_per_bh;
 
     if (FROM_KT && tid == 0) {
-        for (int s = 0; s < a.nstages; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
         fence_barrier_init();
     }
+    if (tid == 0) tk.misc[4] = 0;
     __syncthreads();
     pdl_trigger();
     pdl_wait();
 
-    auto tile_info = [&](long long x, int &bh, int &t0, int &n) {
-        bh = (int)(x / tpb);
-        t0 = (int)(x - (long long)bh * tpb) * TILE;
-        const int b = bh / a.Hkv;
-        const int Tb = clamp_seq(__ldg(a.seq_lens + b), a.T_cap, a.status);
-        n = min(TILE, Tb - t0);
-        if (n < 0) n = 0;
-    };
+    auto seq_len_of = [&](int bh) { return clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, a.status); };
 
+    // producer cursor (thread 0): (bh, tile within bh) of the next copy to issue
+    int p_bh = (int)(x_begin / tpb), p_t = (int)(x_begin - (long long)p_bh * tpb);
     uint64_t pol = 0;
-    auto issue = [&](int i) {  // thread 0 only
-        int bh, t0, n;
-        tile_info(x_begin + i, bh, t0, n);
-        const int s = i % a.nstages;
+    auto issue_next = [&](int s) {
+        const int Tb = seq_len_of(p_bh);
+        const int t0 = p_t * TILE;
+        const int n = min(TILE, Tb - t0);
         if (n > 0) {
             const uint32_t bytes = (uint32_t)n * ROWB;
             mbar_arrive_expect_tx(&bars[s], bytes);
-            const char *src = static_cast<const char *>(a.src) + ((size_t)bh * a.T_cap + t0) * ROWB;
-            bulk_g2s(smem + L.stages + (size_t)s * kScanStageBytes, src, bytes, &bars[s], pol);
+            const char *src = static_cast<const char *>(a.src) + ((size_t)p_bh * a.T_cap + t0) * ROWB;
+            bulk_g2s(smem + L.stages + (size_t)s * kTileBytes, src, bytes, &bars[s], pol);
         } else {
             mbar_arrive(&bars[s]);
+        }
+        if (++p_t == tpb) {
+            p_t = 0;
+            ++p_bh;
         }
     };
 
     int issued = 0;
     if (FROM_KT && tid == 0) {
         pol = policy_evict_first();
-        issued = min(a.nstages, ntiles);
-        for (int i = 0; i < issued; ++i) issue(i);
+        issued = min(kStages, ntiles);
+        for (int i = 0; i < issued; ++i) issue_next(i);
     }
 
-    // per-thread query slice (SUM: one folded query kept in registers)
-    const int chunk = tid % LPT;
-    float qreg[EPL];
+    // lane-rotated chunk order: each quarter-warp reads 8 distinct 16-byte bank groups
+    const int sub = tid % LPT;
+    const int rot = CPT == 4 ? (lane >> 1) & 3 : (CPT == 2 ? (lane >> 2) & 1 : 0);
+    float qreg[QN];  // SUM: this thread's slice of the folded query, in chunk-visit order
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) qreg[e] = 0.f;
+    for (int e = 0; e < QN; ++e) qreg[e] = 0.f;
 
     auto begin_segment = [&](int bh) {
         if (FROM_KT) {
-            const int nq = a.nq;
-            for (int p = tid; p < nq * R; p += NT) qs[p] = a.qproj[(size_t)bh * nq * R + p];
+            for (int p = tid; p < a.nq * R; p += NT) qs[p] = a.qproj[(size_t)bh * a.nq * R + p];
         }
-        tk.n = 0;
+        if (tid == 0) tk.misc[4] = 0;
         tk.valid = false;
         __syncthreads();
         if (FROM_KT && AGG == JSSA_AGG_SUM) {
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) qreg[e] = qs[chunk * EPL + e];
+            for (int c = 0; c < CPT; ++c) {
+                const int ch = sub * CPT + ((c + rot) % CPT);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) qreg[(c * EPL + e) % QN] = qs[ch * EPL + e];
+            }
         }
     };
 
     auto cta_of = [&](long long x) -> long long { return ((x + 1) * a.grid - 1) / a.total_tiles; };
 
     auto finish_segment = [&](int bh) {
-        if (tk.n > a.k) reduce_topk(tk, a.k);
+        int n = tk.misc[4];
+        __syncthreads();
+        if (n > a.k) {
+            reduce_topk(tk, n, a.k);
+            n = a.k;
+        }
         const long long first = (long long)bh * tpb;
         const long long c_first = cta_of(first), c_last = cta_of(first + tpb - 1);
         const int slot = (int)(cta - c_first), nseg = (int)(c_last - c_first + 1);
         const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
-        for (int j = tid; j < tk.n; j += NT) {
+        for (int j = tid; j < n; j += NT) {
             a.cand_key[cb + j] = tk.key[j];
             a.cand_idx[cb + j] = tk.idx[j];
         }
-        if (tid == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = tk.n;
+        if (tid == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
         __threadfence();
         __syncthreads();
         if (tid == 0) tk.misc[2] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
         __syncthreads();
         const bool last = tk.misc[2] != 0;
-        __syncthreads();
         if (!last) return;
         __threadfence();
-        tk.n = 0;
+        // merge the segments in ascending token order; inside one segment the
+        // order is arbitrary, so keys equal to the threshold stay candidates
+        if (tid == 0) tk.misc[4] = 0;
         tk.valid = false;
+        __syncthreads();
+        constexpr int MCH = FROM_KT ? (TILE > 1024 ? TILE : 1024) : TILE;  // cap >= k + MCH
         for (int s = 0; s < nseg; ++s) {
             const int cnt = __ldcg(a.cand_cnt + (size_t)bh * a.max_seg + s);
             const size_t base = ((size_t)bh * a.max_seg + s) * a.k;
-            for (int off = 0; off < cnt; off += TILE) {
-                const int m = min(TILE, cnt - off);
-                for (int j = tid; j < m; j += NT) {
-                    tkey[j] = __ldcg(a.cand_key + base + off + j);
-                    tidx[j] = __ldcg(a.cand_idx + base + off + j);
+            for (int off = 0; off < cnt; off += MCH) {
+                const int m = min(MCH, cnt - off);
+                for (int j0 = 0; j0 < m; j0 += NT) {
+                    const int j = j0 + tid;
+                    uint32_t u = 0u;
+                    int32_t ix = 0;
+                    if (j < m) {
+                        u = __ldcg(a.cand_key + base + off + j);
+                        ix = __ldcg(a.cand_idx + base + off + j);
+                    }
+                    offer(tk, j < m && (!tk.valid || u >= tk.thresh), u, ix, a.cap);
                 }
                 __syncthreads();
-                append_chunk<TILE>(tk, tkey, tidx, 0, m, a.k, a.cap);
+                const int nb = tk.misc[4];
                 __syncthreads();
+                if (nb > a.cap - MCH) reduce_topk(tk, nb, a.k);
             }
         }
-        if (tk.n > a.k) reduce_topk(tk, a.k);
-        for (int j = tid; j < a.k; j += NT) a.idx_out[(size_t)bh * a.k + j] = j < tk.n ? tk.idx[j] : -1;
+        n = tk.misc[4];
+        __syncthreads();
+        if (n > a.k) {
+            reduce_topk(tk, n, a.k);
+            n = a.k;
+        }
+        int32_t *srt = tk.res_idx;
+        for (int j = tid; j < n; j += NT) srt[j] = tk.idx[j];
+        __syncthreads();
+        sort_ascending(srt, n);
+        for (int j = tid; j < a.k; j += NT) a.idx_out[(size_t)bh * a.k + j] = j < n ? srt[j] : -1;
         if (tid == 0) {
-            if (a.count_out) a.count_out[bh] = tk.n;
+            if (a.count_out) a.count_out[bh] = n;
             a.counters[bh] = 0u;
         }
         __syncthreads();
     };
 
-    int cur_bh = -1;
+    int c_bh = (int)(x_begin / tpb), c_t = (int)(x_begin - (long long)c_bh * tpb);
+    int cur_bh = -1, Tb = 0;
     bool timed_out = false;
     int consumed = 0;
     for (int i = 0; i < ntiles; ++i) {
-        int bh, t0, n;
-        tile_info(x_begin + i, bh, t0, n);
+        const int bh = c_bh, t0 = c_t * TILE;
+        if (++c_t == tpb) {
+            c_t = 0;
+            ++c_bh;
+        }
         if (bh != cur_bh) {
             if (MODE == MODE_SELECT && cur_bh >= 0) finish_segment(cur_bh);
             cur_bh = bh;
+            Tb = seq_len_of(bh);
             begin_segment(bh);
         }
+        const int n = max(0, min(TILE, Tb - t0));
         if constexpr (FROM_KT) {
-            const int s = i % a.nstages;
-            const uint32_t par = (uint32_t)(i / a.nstages) & 1u;
+            const int s = i % kStages;
+            const uint32_t par = (uint32_t)(i / kStages) & 1u;
             const bool ok = __syncthreads_and(mbar_wait_bounded(&bars[s], par) ? 1 : 0) != 0;
             if (!ok) {
                 timed_out = true;
@@ -364,69 +451,94 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
             }
             consumed = i + 1;
             if (n > 0) {
-                const uint4 *sv = reinterpret_cast<const uint4 *>(smem + L.stages + (size_t)s * kScanStageBytes);
+                const unsigned char *st = smem + L.stages + (size_t)s * kTileBytes;
 #pragma unroll
-                for (int tt = tid / LPT; tt < TILE; tt += NT / LPT) {
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (tt < n) v = sv[tt * LPT + chunk];
-                    float kf[EPL];
-                    Vec16<KT>::unpack(v, kf);
+                for (int ps = 0; ps < PASSES; ++ps) {
+                    const int tt = ps * TPP + tid / LPT;
+                    const bool live = tt < n;
                     float sc;
                     if (AGG == JSSA_AGG_SUM) {
-                        float acc = 0.f;
+                        float pc[CPT];
 #pragma unroll
-                        for (int e = 0; e < EPL; ++e) acc = fmaf(kf[e], qreg[e], acc);
+                        for (int c = 0; c < CPT; ++c) {
+                            const int ch = sub * CPT + ((c + rot) % CPT);
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (live) v = *reinterpret_cast<const uint4 *>(st + (size_t)tt * ROWB + ch * 16);
+                            float kf[EPL];
+                            Vec16<KT>::unpack(v, kf);
+                            float acc = 0.f;
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e) acc = fmaf(kf[e], qreg[(c * EPL + e) % QN], acc);
+                            pc[c] = acc;
+                        }
+                        float acc = chunk_sum<CPT>(pc);
 #pragma unroll
                         for (int off = 1; off < LPT; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
                         sc = acc;
                     } else {
+                        float kf[CPT][EPL];
+#pragma unroll
+                        for (int c = 0; c < CPT; ++c) {
+                            const int ch = sub * CPT + ((c + rot) % CPT);
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (live) v = *reinterpret_cast<const uint4 *>(st + (size_t)tt * ROWB + ch * 16);
+                            Vec16<KT>::unpack(v, kf[c]);
+                        }
                         float best = -INFINITY;
                         for (int g = 0; g < a.nq; ++g) {
-                            const float *qg = qs + g * R + chunk * EPL;
-                            float acc = 0.f;
+                            float pc[CPT];
 #pragma unroll
-                            for (int e = 0; e < EPL; ++e) acc = fmaf(kf[e], qg[e], acc);
+                            for (int c = 0; c < CPT; ++c) {
+                                const int ch = sub * CPT + ((c + rot) % CPT);
+                                const float *qg = qs + g * R + ch * EPL;
+                                float acc = 0.f;
+#pragma unroll
+                                for (int e = 0; e < EPL; ++e) acc = fmaf(kf[c][e], qg[e], acc);
+                                pc[c] = acc;
+                            }
+                            float acc = chunk_sum<CPT>(pc);
 #pragma unroll
                             for (int off = 1; off < LPT; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
                             best = fmaxf(best, acc);
                         }
                         sc = best;
                     }
-                    if (chunk == 0 && tt < n) tkey[tt] = MODE == MODE_WRITE ? __float_as_uint(sc) : score_key(sc);
+                    if (MODE == MODE_WRITE) {
+                        if (live && sub == 0) a.scores_out[(size_t)bh * a.T_cap + t0 + tt] = sc;
+                    } else {
+                        const uint32_t u = score_key(sc);
+                        offer(tk, live && sub == 0 && (!tk.valid || u > tk.thresh), u, t0 + tt, a.cap);
+                    }
                 }
             }
-            __syncthreads();  // stage s consumed; tkey complete
+            __syncthreads();  // stage s consumed; buffer count final for this tile
             if (tid == 0 && issued < ntiles) {
-                issue(issued);
+                issue_next(issued % kStages);
                 ++issued;
             }
         } else {
             if (n > 0) {
-                constexpr int PERT = (TILE + NT - 1) / NT;
                 const float *srow = static_cast<const float *>(a.src) + (size_t)bh * a.T_cap + t0;
-                float v[PERT];
+                float v[PASSES];
 #pragma unroll
-                for (int u = 0; u < PERT; ++u) {
+                for (int u = 0; u < PASSES; ++u) {
                     const int j = tid + u * NT;
                     v[u] = j < n ? __ldcs(srow + j) : 0.f;
                 }
 #pragma unroll
-                for (int u = 0; u < PERT; ++u) {
+                for (int u = 0; u < PASSES; ++u) {
                     const int j = tid + u * NT;
-                    if (j < n) tkey[j] = score_key(v[u]);
+                    const uint32_t key = score_key(v[u]);
+                    offer(tk, j < n && (!tk.valid || key > tk.thresh), key, t0 + j, a.cap);
                 }
             }
             __syncthreads();
         }
-        if (n > 0) {
-            if (MODE == MODE_WRITE) {
-                float *dst = a.scores_out + (size_t)bh * a.T_cap + t0;
-                for (int j = tid; j < n; j += NT) dst[j] = __uint_as_float(tkey[j]);
-            } else {
-                append_chunk<TILE>(tk, tkey, nullptr, t0, n, a.k, a.cap);
-            }
+        if (MODE == MODE_SELECT) {
+            const int nb = tk.misc[4];
+            __syncthreads();
+            if (nb > a.cap - TILE) reduce_topk(tk, nb, a.k);
         }
-        __syncthreads();
     }
 
     if (timed_out) {
@@ -434,7 +546,7 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
             if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
             // let the copies already in flight land before the CTA exits
             for (int i = consumed; i < issued; ++i)
-                (void)mbar_wait_bounded(&bars[i % a.nstages], (uint32_t)(i / a.nstages) & 1u);
+                (void)mbar_wait_bounded(&bars[i % kStages], (uint32_t)(i / kStages) & 1u);
         }
         __syncthreads();
         return;
@@ -468,13 +580,12 @@ void (*pick_scan(int src, int mode, int r, int agg))(ScanArgs) {
 
 int scan_tile_tokens(int src, int r) {
     if (src == SRC_SCORES) return kScoreTileTokens;
-    return kScanStageBytes / (r * (src == SRC_KT_FP32 ? 4 : 2));
+    return kTileBytes / (r * (src == SRC_KT_FP32 ? 4 : 2));
 }
 
 }  // namespace
 
 cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, ScanPlan *p) {
-    (void)nq;
     auto kern = pick_scan(src, mode, r, agg);
     if (!kern) return cudaErrorInvalidValue;
     ScanPlan P;
@@ -483,11 +594,13 @@ cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int
     P.tile_tokens = scan_tile_tokens(src, r);
     P.tiles_per_bh = (T_cap + P.tile_tokens - 1) / P.tile_tokens;
     P.total_tiles = (long long)B * Hkv * P.tiles_per_bh;
-    P.nstages = src == SRC_SCORES ? 0 : 3;
-    P.cap = mode == MODE_SELECT ? k + (P.tile_tokens > 1024 ? P.tile_tokens : 1024) : 0;
-    P.smem = scan_smem(src, mode, src == SRC_SCORES ? 0 : r, P.nstages, P.cap, mode == MODE_SELECT ? k : 0,
-                       P.tile_tokens)
-                 .total;
+    P.nstages = src == SRC_SCORES ? 0 : kStages;
+    // capacity: k kept entries, one tile (or one merge chunk) of new survivors,
+    // and slack so that a reduction is needed only every few tiles
+    const int chunk = src == SRC_SCORES ? P.tile_tokens : (P.tile_tokens > 1024 ? P.tile_tokens : 1024);
+    const int slack = src == SRC_SCORES ? P.tile_tokens : 256;
+    P.cap = mode == MODE_SELECT ? k + chunk + slack : 0;
+    P.smem = scan_smem(src, mode, src == SRC_SCORES ? 0 : r, nq, kStages, P.cap, mode == MODE_SELECT ? k : 0).total;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
