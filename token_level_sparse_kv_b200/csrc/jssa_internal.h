@@ -16,7 +16,7 @@ constexpr int kMaxK = 2048;
 constexpr int kMaxG = 16;
 constexpr int kScanThreads = 256;
 constexpr int kScanStageBytes = 16384;
-constexpr int kScoreTileTokens = 4096;  // tokens per tile when the source is a score array
+constexpr int kScoreTileTokens = 2048;  // tokens per tile when the source is a score array
 constexpr int kAttnThreads = 128;
 
 // ------------------------------------------------------------------ scan ---

@@ -40,9 +40,21 @@ namespace jssa {
 
 namespace {
 
-constexpr int NT = kScanThreads;
-constexpr int kTileBytes = 2 * kScanStageBytes;  // 32 KiB per stage
-constexpr int kStages = 3;
+// Tile size, ring depth and block size of the streaming pass (compile-time;
+// the defaults are the measured best on B200 for r*2 = 64-byte rows).
+#ifndef JSSA_SCAN_TILE_BYTES
+#define JSSA_SCAN_TILE_BYTES 32768
+#endif
+#ifndef JSSA_SCAN_STAGES
+#define JSSA_SCAN_STAGES 3
+#endif
+#ifndef JSSA_SCAN_THREADS
+#define JSSA_SCAN_THREADS 256
+#endif
+constexpr int NT = JSSA_SCAN_THREADS;
+constexpr int kTileBytes = JSSA_SCAN_TILE_BYTES;
+constexpr int kStages = JSSA_SCAN_STAGES;
+static_assert(NT >= 256 && NT % 256 == 0, "the radix select uses one thread per digit");
 
 __host__ __device__ inline int next_pow2(int x) {
     int p = 1;
@@ -85,8 +97,9 @@ __host__ __device__ inline ScanSmem scan_smem(int src, int mode, int r, int nq, 
     return L;
 }
 
-// Running top-k buffer in shared memory.  Entries are unordered; the count
-// lives in shared memory (misc[4]) because warps append with atomics.
+// Running top-k buffer in shared memory (pointers only; passed by value so that
+// nothing of the hot loop lives in local memory).  Entries are unordered; the
+// count lives in shared memory (misc[4]) because warps append with atomics.
 struct TopK {
     uint32_t *key;
     int32_t *idx;
@@ -94,9 +107,8 @@ struct TopK {
     int32_t *res_idx;
     uint32_t *hist;
     int *tmp;
-    int *misc;  // [0..1], [5] select scratch, [2] ticket flag, [3] keep counter, [4] count
-    bool valid;  // thresh holds the k-th best key of a completed reduction
-    uint32_t thresh;
+    int *misc;  // [0..1], [5] select scratch, [2] ticket flag, [3] keep counter, [4] count,
+                // [6] timeout flag, [8..9] shrink decisions
 };
 
 // Sum of the per-chunk partials of one thread, independent of the lane's
@@ -104,9 +116,9 @@ struct TopK {
 // {1,3} as wholes, and each pair sum is commutative, so every lane adds the
 // same two pair sums.  Identical rows therefore score bit-identically.
 template <int CPT>
-__device__ __forceinline__ float chunk_sum(const float *p) {
-    if (CPT == 4) return (p[0] + p[2]) + (p[1] + p[3]);
-    if (CPT == 2) return p[0] + p[1];
+__device__ __forceinline__ float chunk_sum(const float (&p)[CPT]) {
+    if constexpr (CPT == 4) return (p[0] + p[2]) + (p[1] + p[3]);
+    if constexpr (CPT == 2) return p[0] + p[1];
     return p[0];
 }
 
@@ -117,19 +129,20 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 // Warp-aggregated append of one candidate per lane (all 32 lanes call it).
-__device__ __forceinline__ void offer(TopK &tk, bool take, uint32_t key, int32_t idx, int cap) {
+__device__ __forceinline__ void offer(uint32_t *bkey, int32_t *bidx, int *count, bool take, uint32_t key,
+                                      int32_t idx, int cap) {
     const unsigned m = __ballot_sync(0xffffffffu, take);
     if (m == 0u) return;
     const int lane = threadIdx.x & 31;
     const int leader = __ffs(m) - 1;
     int base = 0;
-    if (lane == leader) base = atomicAdd(&tk.misc[4], __popc(m));
+    if (lane == leader) base = atomicAdd(count, __popc(m));
     base = __shfl_sync(0xffffffffu, base, leader);
     if (take) {
         const int pos = base + __popc(m & lanemask_lt());
         if (pos < cap) {
-            tk.key[pos] = key;
-            tk.idx[pos] = idx;
+            bkey[pos] = key;
+            bidx[pos] = idx;
         }
     }
 }
@@ -138,13 +151,14 @@ __device__ __forceinline__ void offer(TopK &tk, bool take, uint32_t key, int32_t
 // count).  Returns the value, how many entries equal to it are in the top kk,
 // and (eq_total) how many used entries equal it.
 template <typename Use, typename Val>
-__device__ void radix_select(int n, int kk, TopK &tk, Use use, Val val, uint32_t &tau, int &need, int &eq_total) {
+__device__ __forceinline__ void radix_select(int n, int kk, const TopK tk, Use use, Val val, uint32_t &tau,
+                                             int &need, int &eq_total) {
     const int tid = threadIdx.x;
     uint32_t prefix = 0u, mask = 0u;
     int last_count = 0;
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
-        tk.hist[tid] = 0u;
+        if (tid < 256) tk.hist[tid] = 0u;
         __syncthreads();
         for (int j = tid; j < n; j += NT) {
             if (!use(j)) continue;
@@ -152,7 +166,7 @@ __device__ void radix_select(int n, int kk, TopK &tk, Use use, Val val, uint32_t
             if ((u & mask) == prefix) atomicAdd(&tk.hist[(u >> shift) & 0xffu], 1u);
         }
         __syncthreads();
-        const int c = (int)tk.hist[255 - tid];
+        const int c = tid < 256 ? (int)tk.hist[255 - tid] : 0;
         int tot;
         const int ex = block_excl_scan<NT>(c, tk.tmp, tot);
         if (ex < kk && ex + c >= kk) {
@@ -172,8 +186,9 @@ __device__ void radix_select(int n, int kk, TopK &tk, Use use, Val val, uint32_t
     eq_total = last_count;
 }
 
-// Keep the best k of the n > k buffered entries under (key desc, idx asc).
-__device__ void reduce_topk(TopK &tk, int n, int k) {
+// Keep the best k of the n > k buffered entries under (key desc, idx asc);
+// returns the key of the k-th kept entry (the new survival threshold).
+__device__ __forceinline__ uint32_t reduce_topk(const TopK tk, int n, int k) {
     const int tid = threadIdx.x;
     uint32_t tau, tau2 = 0u;
     int need, m;
@@ -222,8 +237,7 @@ __device__ void reduce_topk(TopK &tk, int n, int k) {
     }
     if (tid == 0) tk.misc[4] = k;
     __syncthreads();
-    tk.valid = true;
-    tk.thresh = tau;
+    return tau;
 }
 
 // Sort a[0..n) ascending in place (bitonic network over the next power of two,
@@ -250,29 +264,107 @@ __device__ void sort_ascending(int32_t *a, int n) {
     }
 }
 
+// End of a segment: publish its candidates; the last CTA of the (b,h) merges
+// all segments (ascending token order; inside one segment the order is
+// arbitrary, so keys equal to the threshold stay candidates) and writes the
+// selection sorted by index.
+template <int MCH>
+__device__ __forceinline__ void finish_segment(const ScanArgs &a, const TopK tk, int bh, long long cta) {
+    const int tid = threadIdx.x;
+    int n = tk.misc[4];
+    __syncthreads();
+    if (n > a.k) {
+        reduce_topk(tk, n, a.k);
+        n = a.k;
+    }
+    const int tpb = a.tiles_per_bh;
+    const long long first = (long long)bh * tpb;
+    const long long c_first = ((first + 1) * a.grid - 1) / a.total_tiles;
+    const long long c_last = ((first + tpb) * a.grid - 1) / a.total_tiles;
+    const int slot = (int)(cta - c_first), nseg = (int)(c_last - c_first + 1);
+    const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
+    for (int j = tid; j < n; j += NT) {
+        a.cand_key[cb + j] = tk.key[j];
+        a.cand_idx[cb + j] = tk.idx[j];
+    }
+    if (tid == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) tk.misc[2] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
+    __syncthreads();
+    const bool last = tk.misc[2] != 0;
+    if (!last) return;
+    __threadfence();
+    if (tid == 0) tk.misc[4] = 0;
+    __syncthreads();
+    bool valid = false;
+    uint32_t thresh = 0u;
+    for (int s = 0; s < nseg; ++s) {
+        const int cnt = __ldcg(a.cand_cnt + (size_t)bh * a.max_seg + s);
+        const size_t base = ((size_t)bh * a.max_seg + s) * a.k;
+        for (int off = 0; off < cnt; off += MCH) {
+            const int m = min(MCH, cnt - off);
+            for (int j0 = 0; j0 < m; j0 += NT) {
+                const int j = j0 + tid;
+                uint32_t u = 0u;
+                int32_t ix = 0;
+                if (j < m) {
+                    u = __ldcg(a.cand_key + base + off + j);
+                    ix = __ldcg(a.cand_idx + base + off + j);
+                }
+                offer(tk.key, tk.idx, &tk.misc[4], j < m && (!valid || u >= thresh), u, ix, a.cap);
+            }
+            __syncthreads();
+            const int nb = tk.misc[4];
+            __syncthreads();
+            if (nb > a.cap - MCH) {
+                thresh = reduce_topk(tk, nb, a.k);
+                valid = true;
+            }
+        }
+    }
+    n = tk.misc[4];
+    __syncthreads();
+    if (n > a.k) {
+        reduce_topk(tk, n, a.k);
+        n = a.k;
+    }
+    int32_t *srt = tk.res_idx;
+    for (int j = tid; j < n; j += NT) srt[j] = tk.idx[j];
+    __syncthreads();
+    sort_ascending(srt, n);
+    for (int j = tid; j < a.k; j += NT) a.idx_out[(size_t)bh * a.k + j] = j < n ? srt[j] : -1;
+    if (tid == 0) {
+        if (a.count_out) a.count_out[bh] = n;
+        a.counters[bh] = 0u;
+    }
+    __syncthreads();
+}
+
 template <int SRC, int MODE, int R, int AGG>
-__global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
+__global__ void __launch_bounds__(NT, 2) scan_kernel(ScanArgs a) {
     constexpr bool FROM_KT = SRC != SRC_SCORES;
     using KT = typename std::conditional<SRC == SRC_KT_FP32, float, __nv_bfloat16>::type;
     constexpr int ES = SRC == SRC_KT_FP32 ? 4 : 2;
-    constexpr int ROWB = FROM_KT ? R * ES : 4;  // bytes per token
-    constexpr int TPB = ROWB > 64 ? 64 : ROWB;  // bytes of a token per thread
-    constexpr int LPT = ROWB / TPB;             // lanes per token
+    constexpr int ROWB = FROM_KT ? R * ES : 4;   // bytes per token
+    constexpr int TPB = ROWB > 64 ? 64 : ROWB;   // bytes of a token per thread
+    constexpr int LPT = ROWB / TPB;              // lanes per token
     constexpr int CPT = FROM_KT ? TPB / 16 : 1;  // 16-byte chunks per thread
-    constexpr int EPL = 16 / ES;                // elements per chunk
+    constexpr int EPL = 16 / ES;                 // elements per chunk
     constexpr int TILE = FROM_KT ? kTileBytes / ROWB : kScoreTileTokens;
     constexpr int TPP = NT / LPT;  // tokens per pass
     constexpr int PASSES = FROM_KT ? TILE / TPP : TILE / NT;
     constexpr int QN = FROM_KT ? CPT * EPL : 1;
+    constexpr int MCH = FROM_KT ? (TILE > 1024 ? TILE : 1024) : TILE;  // merge chunk; cap >= k + MCH
     static_assert(!FROM_KT || (LPT >= 1 && LPT <= 32 && (LPT & (LPT - 1)) == 0), "lanes per token");
     static_assert(!FROM_KT || (CPT >= 1 && CPT <= 4), "chunks per thread");
     static_assert(!FROM_KT || TILE % TPP == 0, "tile / pass");
 
     extern __shared__ __align__(128) unsigned char smem[];
-    const ScanSmem L = scan_smem(SRC, MODE, FROM_KT ? R : 0, a.nq, kStages, a.cap, a.k);
+    const int nstages = a.nstages;  // ring depth chosen by the planner (<= kStages)
+    const ScanSmem L = scan_smem(SRC, MODE, FROM_KT ? R : 0, a.nq, nstages, a.cap, a.k);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
     float *qs = reinterpret_cast<float *>(smem + L.qs);
-
     TopK tk;
     tk.key = reinterpret_cast<uint32_t *>(smem + L.buf_key);
     tk.idx = reinterpret_cast<int32_t *>(smem + L.buf_idx);
@@ -281,8 +373,10 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
     tk.hist = reinterpret_cast<uint32_t *>(smem + L.hist);
     tk.tmp = reinterpret_cast<int *>(smem + L.tmp);
     tk.misc = reinterpret_cast<int *>(smem + L.misc);
-    tk.valid = false;
-    tk.thresh = 0u;
+    uint32_t *const bkey = tk.key;
+    int32_t *const bidx = tk.idx;
+    int *const bcount = tk.misc + 4;
+    volatile int *const flags = tk.misc;
 
     const int tid = threadIdx.x, lane = tid & 31;
     const long long cta = blockIdx.x;
@@ -292,42 +386,42 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
     const int tpb = a.tiles_per_bh;
 
     if (FROM_KT && tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
         fence_barrier_init();
     }
-    if (tid == 0) tk.misc[4] = 0;
+    if (tid == 0) {
+        tk.misc[4] = 0;
+        tk.misc[6] = 0;
+        tk.misc[8] = 0;
+        tk.misc[9] = 0;
+    }
     __syncthreads();
     pdl_trigger();
     pdl_wait();
 
-    auto seq_len_of = [&](int bh) { return clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, a.status); };
-
-    // producer cursor (thread 0): (bh, tile within bh) of the next copy to issue
-    int p_bh = (int)(x_begin / tpb), p_t = (int)(x_begin - (long long)p_bh * tpb);
+    // producer state (thread 0): next tile to copy and its ring slot
+    int p_bh = (int)(x_begin / tpb), p_t = (int)(x_begin - (long long)p_bh * tpb), p_s = 0, issued = 0;
     uint64_t pol = 0;
-    auto issue_next = [&](int s) {
-        const int Tb = seq_len_of(p_bh);
-        const int t0 = p_t * TILE;
-        const int n = min(TILE, Tb - t0);
-        if (n > 0) {
-            const uint32_t bytes = (uint32_t)n * ROWB;
-            mbar_arrive_expect_tx(&bars[s], bytes);
-            const char *src = static_cast<const char *>(a.src) + ((size_t)p_bh * a.T_cap + t0) * ROWB;
-            bulk_g2s(smem + L.stages + (size_t)s * kTileBytes, src, bytes, &bars[s], pol);
-        } else {
-            mbar_arrive(&bars[s]);
-        }
-        if (++p_t == tpb) {
-            p_t = 0;
-            ++p_bh;
-        }
-    };
-
-    int issued = 0;
+    const char *const src_base = static_cast<const char *>(a.src);
     if (FROM_KT && tid == 0) {
         pol = policy_evict_first();
-        issued = min(kStages, ntiles);
-        for (int i = 0; i < issued; ++i) issue_next(i);
+        const int first = min(nstages, ntiles);
+        for (; issued < first; ++issued) {
+            const int Tb_p = clamp_seq(__ldg(a.seq_lens + p_bh / a.Hkv), a.T_cap, a.status);
+            const int t0 = p_t * TILE, n = min(TILE, Tb_p - t0);
+            if (n > 0) {
+                mbar_arrive_expect_tx(&bars[p_s], (uint32_t)n * ROWB);
+                bulk_g2s(smem + L.stages + (size_t)p_s * kTileBytes, src_base + ((size_t)p_bh * a.T_cap + t0) * ROWB,
+                         (uint32_t)n * ROWB, &bars[p_s], pol);
+            } else {
+                mbar_arrive(&bars[p_s]);
+            }
+            if (++p_t == tpb) {
+                p_t = 0;
+                ++p_bh;
+            }
+            if (++p_s == nstages) p_s = 0;
+        }
     }
 
     // lane-rotated chunk order: each quarter-warp reads 8 distinct 16-byte bank groups
@@ -337,97 +431,11 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
 #pragma unroll
     for (int e = 0; e < QN; ++e) qreg[e] = 0.f;
 
-    auto begin_segment = [&](int bh) {
-        if (FROM_KT) {
-            for (int p = tid; p < a.nq * R; p += NT) qs[p] = a.qproj[(size_t)bh * a.nq * R + p];
-        }
-        if (tid == 0) tk.misc[4] = 0;
-        tk.valid = false;
-        __syncthreads();
-        if (FROM_KT && AGG == JSSA_AGG_SUM) {
-#pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-                const int ch = sub * CPT + ((c + rot) % CPT);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) qreg[(c * EPL + e) % QN] = qs[ch * EPL + e];
-            }
-        }
-    };
-
-    auto cta_of = [&](long long x) -> long long { return ((x + 1) * a.grid - 1) / a.total_tiles; };
-
-    auto finish_segment = [&](int bh) {
-        int n = tk.misc[4];
-        __syncthreads();
-        if (n > a.k) {
-            reduce_topk(tk, n, a.k);
-            n = a.k;
-        }
-        const long long first = (long long)bh * tpb;
-        const long long c_first = cta_of(first), c_last = cta_of(first + tpb - 1);
-        const int slot = (int)(cta - c_first), nseg = (int)(c_last - c_first + 1);
-        const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
-        for (int j = tid; j < n; j += NT) {
-            a.cand_key[cb + j] = tk.key[j];
-            a.cand_idx[cb + j] = tk.idx[j];
-        }
-        if (tid == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) tk.misc[2] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
-        __syncthreads();
-        const bool last = tk.misc[2] != 0;
-        if (!last) return;
-        __threadfence();
-        // merge the segments in ascending token order; inside one segment the
-        // order is arbitrary, so keys equal to the threshold stay candidates
-        if (tid == 0) tk.misc[4] = 0;
-        tk.valid = false;
-        __syncthreads();
-        constexpr int MCH = FROM_KT ? (TILE > 1024 ? TILE : 1024) : TILE;  // cap >= k + MCH
-        for (int s = 0; s < nseg; ++s) {
-            const int cnt = __ldcg(a.cand_cnt + (size_t)bh * a.max_seg + s);
-            const size_t base = ((size_t)bh * a.max_seg + s) * a.k;
-            for (int off = 0; off < cnt; off += MCH) {
-                const int m = min(MCH, cnt - off);
-                for (int j0 = 0; j0 < m; j0 += NT) {
-                    const int j = j0 + tid;
-                    uint32_t u = 0u;
-                    int32_t ix = 0;
-                    if (j < m) {
-                        u = __ldcg(a.cand_key + base + off + j);
-                        ix = __ldcg(a.cand_idx + base + off + j);
-                    }
-                    offer(tk, j < m && (!tk.valid || u >= tk.thresh), u, ix, a.cap);
-                }
-                __syncthreads();
-                const int nb = tk.misc[4];
-                __syncthreads();
-                if (nb > a.cap - MCH) reduce_topk(tk, nb, a.k);
-            }
-        }
-        n = tk.misc[4];
-        __syncthreads();
-        if (n > a.k) {
-            reduce_topk(tk, n, a.k);
-            n = a.k;
-        }
-        int32_t *srt = tk.res_idx;
-        for (int j = tid; j < n; j += NT) srt[j] = tk.idx[j];
-        __syncthreads();
-        sort_ascending(srt, n);
-        for (int j = tid; j < a.k; j += NT) a.idx_out[(size_t)bh * a.k + j] = j < n ? srt[j] : -1;
-        if (tid == 0) {
-            if (a.count_out) a.count_out[bh] = n;
-            a.counters[bh] = 0u;
-        }
-        __syncthreads();
-    };
-
-    int c_bh = (int)(x_begin / tpb), c_t = (int)(x_begin - (long long)c_bh * tpb);
-    int cur_bh = -1, Tb = 0;
-    bool timed_out = false;
-    int consumed = 0;
+    int c_bh = (int)(x_begin / tpb), c_t = (int)(x_begin - (long long)c_bh * tpb), c_s = 0;
+    uint32_t c_par = 0u;
+    int cur_bh = -1, Tb = 0, consumed = 0;
+    bool valid = false, timed_out = false;
+    uint32_t thresh = 0u;
     for (int i = 0; i < ntiles; ++i) {
         const int bh = c_bh, t0 = c_t * TILE;
         if (++c_t == tpb) {
@@ -435,40 +443,50 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
             ++c_bh;
         }
         if (bh != cur_bh) {
-            if (MODE == MODE_SELECT && cur_bh >= 0) finish_segment(cur_bh);
+            if (MODE == MODE_SELECT && cur_bh >= 0) finish_segment<MCH>(a, tk, cur_bh, cta);
             cur_bh = bh;
-            Tb = seq_len_of(bh);
-            begin_segment(bh);
+            Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, a.status);
+            if (FROM_KT) {
+                for (int p = tid; p < a.nq * R; p += NT) qs[p] = a.qproj[(size_t)bh * a.nq * R + p];
+            }
+            if (tid == 0) {
+                tk.misc[4] = 0;
+                tk.misc[8] = 0;
+                tk.misc[9] = 0;
+            }
+            valid = false;
+            __syncthreads();
+            if (FROM_KT && AGG == JSSA_AGG_SUM) {
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    const int ch = sub * CPT + ((c + rot) % CPT);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) qreg[(c * EPL + e) % QN] = qs[ch * EPL + e];
+                }
+            }
         }
         const int n = max(0, min(TILE, Tb - t0));
         if constexpr (FROM_KT) {
-            const int s = i % kStages;
-            const uint32_t par = (uint32_t)(i / kStages) & 1u;
-            const bool ok = __syncthreads_and(mbar_wait_bounded(&bars[s], par) ? 1 : 0) != 0;
-            if (!ok) {
-                timed_out = true;
-                break;
-            }
-            consumed = i + 1;
+            if (!mbar_wait_bounded(&bars[c_s], c_par)) flags[6] = 1;  // seen by all after the tile barrier
             if (n > 0) {
-                const unsigned char *st = smem + L.stages + (size_t)s * kTileBytes;
+                const unsigned char *st = smem + L.stages + (size_t)c_s * kTileBytes;
 #pragma unroll
                 for (int ps = 0; ps < PASSES; ++ps) {
                     const int tt = ps * TPP + tid / LPT;
                     const bool live = tt < n;
+                    const unsigned char *row = st + (size_t)tt * ROWB + sub * TPB;
                     float sc;
-                    if (AGG == JSSA_AGG_SUM) {
+                    if constexpr (AGG == JSSA_AGG_SUM) {
                         float pc[CPT];
 #pragma unroll
                         for (int c = 0; c < CPT; ++c) {
-                            const int ch = sub * CPT + ((c + rot) % CPT);
                             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                            if (live) v = *reinterpret_cast<const uint4 *>(st + (size_t)tt * ROWB + ch * 16);
+                            if (live) v = *reinterpret_cast<const uint4 *>(row + ((c + rot) % CPT) * 16);
                             float kf[EPL];
                             Vec16<KT>::unpack(v, kf);
                             float acc = 0.f;
 #pragma unroll
-                            for (int e = 0; e < EPL; ++e) acc = fmaf(kf[e], qreg[(c * EPL + e) % QN], acc);
+                            for (int e = 0; e < EPL; ++e) acc = fmaf(kf[e], qreg[c * EPL + e], acc);
                             pc[c] = acc;
                         }
                         float acc = chunk_sum<CPT>(pc);
@@ -479,9 +497,8 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
                         float kf[CPT][EPL];
 #pragma unroll
                         for (int c = 0; c < CPT; ++c) {
-                            const int ch = sub * CPT + ((c + rot) % CPT);
                             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                            if (live) v = *reinterpret_cast<const uint4 *>(st + (size_t)tt * ROWB + ch * 16);
+                            if (live) v = *reinterpret_cast<const uint4 *>(row + ((c + rot) % CPT) * 16);
                             Vec16<KT>::unpack(v, kf[c]);
                         }
                         float best = -INFINITY;
@@ -503,22 +520,44 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
                         }
                         sc = best;
                     }
-                    if (MODE == MODE_WRITE) {
+                    if constexpr (MODE == MODE_WRITE) {
                         if (live && sub == 0) a.scores_out[(size_t)bh * a.T_cap + t0 + tt] = sc;
                     } else {
                         const uint32_t u = score_key(sc);
-                        offer(tk, live && sub == 0 && (!tk.valid || u > tk.thresh), u, t0 + tt, a.cap);
+                        offer(bkey, bidx, bcount, live && sub == 0 && (!valid || u > thresh), u, t0 + tt, a.cap);
                     }
                 }
             }
-            __syncthreads();  // stage s consumed; buffer count final for this tile
+            if (++c_s == nstages) {
+                c_s = 0;
+                c_par ^= 1u;
+            }
+            __syncthreads();  // this stage is consumed; every append of the tile is done
+            if (flags[6]) {   // a copy never landed: stop (uniform after the barrier)
+                timed_out = true;
+                break;
+            }
+            consumed = i + 1;
             if (tid == 0 && issued < ntiles) {
-                issue_next(issued % kStages);
+                const int Tb_p = clamp_seq(__ldg(a.seq_lens + p_bh / a.Hkv), a.T_cap, a.status);
+                const int tp0 = p_t * TILE, np = min(TILE, Tb_p - tp0);
+                if (np > 0) {
+                    mbar_arrive_expect_tx(&bars[p_s], (uint32_t)np * ROWB);
+                    bulk_g2s(smem + L.stages + (size_t)p_s * kTileBytes,
+                             src_base + ((size_t)p_bh * a.T_cap + tp0) * ROWB, (uint32_t)np * ROWB, &bars[p_s], pol);
+                } else {
+                    mbar_arrive(&bars[p_s]);
+                }
+                if (++p_t == tpb) {
+                    p_t = 0;
+                    ++p_bh;
+                }
+                if (++p_s == nstages) p_s = 0;
                 ++issued;
             }
         } else {
             if (n > 0) {
-                const float *srow = static_cast<const float *>(a.src) + (size_t)bh * a.T_cap + t0;
+                const float *srow = reinterpret_cast<const float *>(src_base) + (size_t)bh * a.T_cap + t0;
                 float v[PASSES];
 #pragma unroll
                 for (int u = 0; u < PASSES; ++u) {
@@ -529,15 +568,25 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
                 for (int u = 0; u < PASSES; ++u) {
                     const int j = tid + u * NT;
                     const uint32_t key = score_key(v[u]);
-                    offer(tk, j < n && (!tk.valid || key > tk.thresh), key, t0 + j, a.cap);
+                    offer(bkey, bidx, bcount, j < n && (!valid || key > thresh), key, t0 + j, a.cap);
                 }
             }
             __syncthreads();
         }
-        if (MODE == MODE_SELECT) {
-            const int nb = tk.misc[4];
-            __syncthreads();
-            if (nb > a.cap - TILE) reduce_topk(tk, nb, a.k);
+        if constexpr (MODE == MODE_SELECT) {
+            // The buffer is shrunk one tile late, on a decision that thread 0 took
+            // after the previous tile's barrier, so that no second barrier per tile
+            // is needed; the capacity holds k + slack + two tiles.
+            if (flags[8 + ((i + 1) & 1)]) {
+                __syncthreads();
+                const int nb = tk.misc[4];
+                __syncthreads();
+                if (nb > a.k) {
+                    thresh = reduce_topk(tk, nb, a.k);
+                    valid = true;
+                }
+            }
+            if (tid == 0) flags[8 + (i & 1)] = tk.misc[4] > a.cap - 2 * TILE;
         }
     }
 
@@ -546,12 +595,12 @@ __global__ void __launch_bounds__(NT) scan_kernel(ScanArgs a) {
             if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
             // let the copies already in flight land before the CTA exits
             for (int i = consumed; i < issued; ++i)
-                (void)mbar_wait_bounded(&bars[i % kStages], (uint32_t)(i / kStages) & 1u);
+                (void)mbar_wait_bounded(&bars[i % nstages], (uint32_t)(i / nstages) & 1u);
         }
         __syncthreads();
         return;
     }
-    if (MODE == MODE_SELECT && cur_bh >= 0) finish_segment(cur_bh);
+    if (MODE == MODE_SELECT && cur_bh >= 0) finish_segment<MCH>(a, tk, cur_bh, cta);
 }
 
 template <int SRC, int MODE, int R, int AGG>
@@ -594,18 +643,24 @@ cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int
     P.tile_tokens = scan_tile_tokens(src, r);
     P.tiles_per_bh = (T_cap + P.tile_tokens - 1) / P.tile_tokens;
     P.total_tiles = (long long)B * Hkv * P.tiles_per_bh;
-    P.nstages = src == SRC_SCORES ? 0 : kStages;
+    P.nstages = src == SRC_SCORES ? 0 : kStages;  // may drop to 2 below to keep two CTAs per SM
     // capacity: k kept entries, one tile (or one merge chunk) of new survivors,
     // and slack so that a reduction is needed only every few tiles
+    const int tiles2 = 2 * P.tile_tokens;
     const int chunk = src == SRC_SCORES ? P.tile_tokens : (P.tile_tokens > 1024 ? P.tile_tokens : 1024);
     const int slack = src == SRC_SCORES ? P.tile_tokens : 256;
-    P.cap = mode == MODE_SELECT ? k + chunk + slack : 0;
-    P.smem = scan_smem(src, mode, src == SRC_SCORES ? 0 : r, nq, kStages, P.cap, mode == MODE_SELECT ? k : 0).total;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
-    if (e != cudaSuccess) return e;
+    P.cap = mode == MODE_SELECT ? k + (tiles2 > chunk ? tiles2 : chunk) + slack : 0;
     int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, P.smem);
-    if (e != cudaSuccess) return e;
+    for (;;) {
+        P.smem = scan_smem(src, mode, src == SRC_SCORES ? 0 : r, nq, P.nstages, P.cap, mode == MODE_SELECT ? k : 0)
+                     .total;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, P.smem);
+        if (e != cudaSuccess) return e;
+        if (occ >= 2 || P.nstages <= 2) break;
+        --P.nstages;
+    }
     if (occ < 1) return cudaErrorInvalidConfiguration;
     long long g = (long long)device_sm_count() * occ;
     if (g > P.total_tiles) g = P.total_tiles;
