@@ -55,6 +55,8 @@ constexpr int NT = JSSA_SCAN_THREADS;
 constexpr int kTileBytes = JSSA_SCAN_TILE_BYTES;
 constexpr int kStages = JSSA_SCAN_STAGES;
 static_assert(NT >= 256 && NT % 256 == 0, "the radix select uses one thread per digit");
+constexpr int kHistBins = 2048;  // 11-bit digits of the one-pass select
+constexpr int kBoundaryMax = 64;  // boundary-group entries resolved by exact ranking
 
 __host__ __device__ inline int next_pow2(int x) {
     int p = 1;
@@ -88,7 +90,7 @@ __host__ __device__ inline ScanSmem scan_smem(int src, int mode, int r, int nq, 
     L.res_idx = o;
     o = align_up(o + (sel ? (size_t)next_pow2(k) * 4 : 0), 16);
     L.hist = o;
-    o = align_up(o + 256 * 4, 16);
+    o = align_up(o + (size_t)kHistBins * 4, 16);
     L.tmp = o;
     o = align_up(o + 32 * 4, 16);
     L.misc = o;
@@ -128,6 +130,12 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     return m;
 }
 
+// Histogram increment (measured: aggregating equal bins across a warp with
+// match.any costs more than the shared-memory atomic contention it saves).
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t bin, bool active) {
+    if (active) atomicAdd(&hist[bin], 1u);
+}
+
 // Warp-aggregated append of one candidate per lane (all 32 lanes call it).
 __device__ __forceinline__ void offer(uint32_t *bkey, int32_t *bidx, int *count, bool take, uint32_t key,
                                       int32_t idx, int cap) {
@@ -160,10 +168,15 @@ __device__ __forceinline__ void radix_select(int n, int kk, const TopK tk, Use u
     for (int shift = 24; shift >= 0; shift -= 8) {
         if (tid < 256) tk.hist[tid] = 0u;
         __syncthreads();
-        for (int j = tid; j < n; j += NT) {
-            if (!use(j)) continue;
-            const uint32_t u = val(j);
-            if ((u & mask) == prefix) atomicAdd(&tk.hist[(u >> shift) & 0xffu], 1u);
+        for (int j0 = 0; j0 < n; j0 += NT) {
+            const int j = j0 + tid;
+            bool on = false;
+            uint32_t u = 0u;
+            if (j < n && use(j)) {
+                u = val(j);
+                on = (u & mask) == prefix;
+            }
+            hist_add(tk.hist, (u >> shift) & 0xffu, on);
         }
         __syncthreads();
         const int c = tid < 256 ? (int)tk.hist[255 - tid] : 0;
@@ -188,7 +201,9 @@ __device__ __forceinline__ void radix_select(int n, int kk, const TopK tk, Use u
 
 // Keep the best k of the n > k buffered entries under (key desc, idx asc);
 // returns the key of the k-th kept entry (the new survival threshold).
-__device__ __forceinline__ uint32_t reduce_topk(const TopK tk, int n, int k) {
+// General form: 8-bit radix passes, then the same over inverted indices for
+// the tie group.  Used when the one-pass form below cannot separate the keys.
+__device__ __noinline__ uint32_t reduce_topk_radix(const TopK tk, int n, int k) {
     const int tid = threadIdx.x;
     uint32_t tau, tau2 = 0u;
     int need, m;
@@ -240,6 +255,170 @@ __device__ __forceinline__ uint32_t reduce_topk(const TopK tk, int n, int k) {
     return tau;
 }
 
+__device__ __forceinline__ bool ranks_before(uint32_t ka, int32_t ia, uint32_t kb, int32_t ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+// Adaptive-digit form of the same reduction.  The keys of the buffer share all
+// bits above the highest bit where its minimum and maximum differ, so the 11
+// bits below that point give a monotone 2048-bin histogram; one scan finds
+// the bin of the k-th key.  While that bin is large, the next 11 bits of its
+// keys are histogrammed the same way; its last few entries are then ranked
+// exactly by (key desc, index asc).  Usually one or two levels instead of the
+// four fixed 8-bit passes of the radix form.
+__device__ __noinline__ uint32_t reduce_topk(const TopK tk, int n, int k) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    unsigned *um = reinterpret_cast<unsigned *>(tk.misc);
+    if (tid == 0) {
+        um[10] = 0u;           // max key
+        um[11] = 0xffffffffu;  // min key
+    }
+    __syncthreads();
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int j = tid; j < n; j += NT) {
+        const uint32_t u = tk.key[j];
+        lo = min(lo, u);
+        hi = max(hi, u);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        atomicMin(&um[11], lo);
+        atomicMax(&um[10], hi);
+    }
+    __syncthreads();
+    hi = um[10];
+    lo = um[11];
+    if (hi == lo) return reduce_topk_radix(tk, n, k);  // every key equal: order by index alone
+    int top = 31 - __clz((int)(hi ^ lo));           // highest bit where keys differ
+    uint32_t pmask = top == 31 ? 0u : ~((2u << top) - 1u), pval = hi & pmask;
+    int kk = k, mb = 0;
+    for (;;) {
+        const int width = top + 1 < 11 ? top + 1 : 11;
+        const int shift = top + 1 - width;
+        const uint32_t dmask = (1u << width) - 1u;
+        for (int d = tid; d < kHistBins; d += NT) tk.hist[d] = 0u;
+        __syncthreads();
+        for (int j0 = 0; j0 < n; j0 += NT) {
+            const int j = j0 + tid;
+            const uint32_t u = j < n ? tk.key[j] : 0u;
+            hist_add(tk.hist, (u >> shift) & dmask, j < n && (u & pmask) == pval);
+        }
+        __syncthreads();
+        // descending scan: thread t owns bins [kHistBins - BPT (t+1), kHistBins - BPT t)
+        constexpr int BPT = kHistBins / NT;
+        const int base_bin = kHistBins - BPT * (tid + 1);
+        int cnt[BPT];
+        int sum = 0;
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) {
+            cnt[q] = (int)tk.hist[base_bin + BPT - 1 - q];
+            sum += cnt[q];
+        }
+        int tot;
+        int ex = block_excl_scan<NT>(sum, tk.tmp, tot);
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) {
+            if (ex < kk && ex + cnt[q] >= kk) {
+                tk.misc[0] = base_bin + BPT - 1 - q;
+                tk.misc[1] = ex;
+                tk.misc[5] = cnt[q];
+            }
+            ex += cnt[q];
+        }
+        __syncthreads();
+        const uint32_t D = (uint32_t)tk.misc[0];
+        kk -= tk.misc[1];
+        mb = tk.misc[5];
+        pmask |= dmask << shift;
+        pval |= D << shift;
+        __syncthreads();
+        if (kk == mb || mb <= kBoundaryMax || shift == 0) break;
+        top = shift - 1;
+    }
+    // kk entries of the boundary group (keys matching pval under pmask) are kept
+    uint32_t kstar = 0u;
+    int32_t istar = 0x7fffffff;
+    const bool whole = kk == mb;
+    if (!whole) {
+        if (mb > kBoundaryMax) return reduce_topk_radix(tk, n, k);  // a large group of equal keys
+        if (tid == 0) tk.misc[3] = 0;
+        __syncthreads();
+        uint32_t *bk = tk.hist;
+        int32_t *bi = reinterpret_cast<int32_t *>(tk.hist + kBoundaryMax);
+        for (int j = tid; j < n; j += NT) {
+            const uint32_t u = tk.key[j];
+            if ((u & pmask) == pval) {
+                const int p = atomicAdd(&tk.misc[3], 1);
+                bk[p] = u;
+                bi[p] = tk.idx[j];
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < mb; i += NT) {
+            const uint32_t ki = bk[i];
+            const int32_t ii = bi[i];
+            int r = 0;
+            for (int j = 0; j < mb; ++j) r += ranks_before(bk[j], bi[j], ki, ii);
+            if (r == kk - 1) {
+                um[12] = ki;
+                tk.misc[13] = ii;
+            }
+        }
+        __syncthreads();
+        kstar = um[12];
+        istar = tk.misc[13];
+    }
+    if (tid == 0) {
+        tk.misc[3] = 0;
+        um[14] = 0xffffffffu;
+    }
+    __syncthreads();
+    uint32_t kept_min = 0xffffffffu;
+    for (int j0 = 0; j0 < n; j0 += NT) {
+        const int j = j0 + tid;
+        bool keep = false;
+        uint32_t u = 0u;
+        int32_t ix = 0;
+        if (j < n) {
+            u = tk.key[j];
+            ix = tk.idx[j];
+            const uint32_t um_ = u & pmask;
+            keep = um_ > pval || (um_ == pval && (whole || !ranks_before(kstar, istar, u, ix)));
+        }
+        if (keep) kept_min = min(kept_min, u);
+        const unsigned msk = __ballot_sync(0xffffffffu, keep);
+        int base = 0;
+        if (msk) {
+            const int leader = __ffs(msk) - 1;
+            if (lane == leader) base = atomicAdd(&tk.misc[3], __popc(msk));
+            base = __shfl_sync(0xffffffffu, base, leader);
+        }
+        if (keep) {
+            const int pos = base + __popc(msk & lanemask_lt());
+            if (pos < k) {
+                tk.res_key[pos] = u;
+                tk.res_idx[pos] = ix;
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kept_min = min(kept_min, __shfl_xor_sync(0xffffffffu, kept_min, off));
+    if (lane == 0) atomicMin(&um[14], kept_min);
+    __syncthreads();
+    for (int j = tid; j < k; j += NT) {
+        tk.key[j] = tk.res_key[j];
+        tk.idx[j] = tk.res_idx[j];
+    }
+    const uint32_t tau = um[14];
+    if (tid == 0) tk.misc[4] = k;
+    __syncthreads();
+    return tau;
+}
+
 // Sort a[0..n) ascending in place (bitonic network over the next power of two,
 // padded with INT_MAX; a has room for next_pow2(n) entries).
 __device__ void sort_ascending(int32_t *a, int n) {
@@ -269,7 +448,7 @@ __device__ void sort_ascending(int32_t *a, int n) {
 // arbitrary, so keys equal to the threshold stay candidates) and writes the
 // selection sorted by index.
 template <int MCH>
-__device__ __forceinline__ void finish_segment(const ScanArgs &a, const TopK tk, int bh, long long cta) {
+__device__ __noinline__ void finish_segment(const ScanArgs &a, const TopK tk, int bh, long long cta) {
     const int tid = threadIdx.x;
     int n = tk.misc[4];
     __syncthreads();
@@ -643,23 +822,26 @@ cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int
     P.tile_tokens = scan_tile_tokens(src, r);
     P.tiles_per_bh = (T_cap + P.tile_tokens - 1) / P.tile_tokens;
     P.total_tiles = (long long)B * Hkv * P.tiles_per_bh;
-    P.nstages = src == SRC_SCORES ? 0 : kStages;  // may drop to 2 below to keep two CTAs per SM
-    // capacity: k kept entries, one tile (or one merge chunk) of new survivors,
-    // and slack so that a reduction is needed only every few tiles
+    // two 32 KiB stages keep the copy engine saturated (measured: the pure
+    // stream reaches the copy-bandwidth peak with 2 or 3 stages)
+    P.nstages = src == SRC_SCORES ? 0 : (kStages < 2 ? kStages : 2);
+    // capacity: k kept entries, two tiles (or one merge chunk) of new survivors,
+    // and slack so that the buffer is shrunk only every few tiles; the slack is
+    // the largest that still leaves two CTAs per SM
     const int tiles2 = 2 * P.tile_tokens;
     const int chunk = src == SRC_SCORES ? P.tile_tokens : (P.tile_tokens > 1024 ? P.tile_tokens : 1024);
-    const int slack = src == SRC_SCORES ? P.tile_tokens : 256;
-    P.cap = mode == MODE_SELECT ? k + (tiles2 > chunk ? tiles2 : chunk) + slack : 0;
     int occ = 0;
-    for (;;) {
+    const int slacks[4] = {1024, 512, 256, 0};
+    for (int si = 0; si < 4; ++si) {
+        const int slack = src == SRC_SCORES ? (si == 0 ? P.tile_tokens : slacks[si]) : slacks[si];
+        P.cap = mode == MODE_SELECT ? k + (tiles2 > chunk ? tiles2 : chunk) + slack : 0;
         P.smem = scan_smem(src, mode, src == SRC_SCORES ? 0 : r, nq, P.nstages, P.cap, mode == MODE_SELECT ? k : 0)
                      .total;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
         if (e != cudaSuccess) return e;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, P.smem);
         if (e != cudaSuccess) return e;
-        if (occ >= 2 || P.nstages <= 2) break;
-        --P.nstages;
+        if (occ >= 2 || mode != MODE_SELECT) break;
     }
     if (occ < 1) return cudaErrorInvalidConfiguration;
     long long g = (long long)device_sm_count() * occ;
