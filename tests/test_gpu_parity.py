@@ -410,3 +410,67 @@ def test_full_size_hybrid_global_sampled():
 
 def test_full_size_gqa_4k_b1_all_heads():
     _full_size_sampled("gqa_4k_b1", [(0, h) for h in range(8)])
+
+
+# ------------------------------------------------------- latent cache (MLA)
+def MW(**kw):
+    base = dict(name="mla", B=2, Hq=128, Hkv=1, d=576, dv=512, T=3000, r=64, k=300, latent=True, seed=60)
+    base.update(kw)
+    return Workload(**base)
+
+
+@pytest.mark.parametrize("k,sl", [(100, [3000, 77]), (300, [3000, 2999]), (2048, [3000, 2500]), (128, [128, 0])])
+def test_mla_indexed_decode_parity(k, sl):
+    w = MW(k=k, seed=61 + k)
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    assert V is None
+    g = torch.Generator().manual_seed(7)
+    idx = torch.full((w.B, 1, k), -1, dtype=torch.int32)
+    cnt = torch.zeros((w.B, 1), dtype=torch.int32)
+    for b in range(w.B):
+        c = min(k, int(slh[b]))
+        cnt[b, 0] = c
+        idx[b, 0, :c] = torch.sort(torch.randperm(int(slh[b]), generator=g)[:c])[0].to(torch.int32)
+    out, lse = ops.indexed_decode(qd, Kd, None, idx.to(DEV), cnt.to(DEV), sld, w.scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attend(q, K, None, idx, cnt, slh, w.scale, dv=512, v_aliases_k=True)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
+def test_mla_decode_step_end_to_end():
+    w = MW(T=5000, k=512, kind="spiked", seed=70)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[5000, 4321])
+    pos = (sl - 1).clamp_min(0)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    out, lse, idx, cnt = ops.decode_step(qd, Kd, None, Pd, Kt, sld, pos.to(DEV), w.k, w.scale)
+    torch.cuda.synchronize()
+    check_append(Kt, K, P, pos.tolist(), 1)
+    ref_s = oracle.score(q, P, host(Kt), sl)
+    check_selection(host(idx).numpy(), host(cnt).numpy(), ref_s, sl.numpy(), w.k)
+    ref_o, ref_l = oracle.attend(q, K, None, host(idx), host(cnt), sl, w.scale, dv=512, v_aliases_k=True)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
+def test_full_size_mla_64k_b8_sampled():
+    from token_level_sparse_kv_b200.inputs import WORKLOADS
+
+    w = WORKLOADS["mla_64k_b8"]
+    q, K, V, P, sl = make_inputs(w, device=DEV)
+    Kt = ops.build_lowrank_cache(K, P)
+    pos = (sl - 1).clamp_min(0)
+    out, lse, idx, cnt = ops.decode_step(q, K, None, P, Kt, sl, pos, w.k, w.scale)
+    s = ops.score(q, P, Kt, sl)
+    idx2, cnt2 = ops.topk(s, sl, w.k, Hq=w.Hq, d=w.d)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(cnt, cnt2)
+    for b in (0, 5):
+        qs = host(q[b:b + 1])
+        Ks = host(K[b:b + 1])
+        slh = sl[b:b + 1].cpu()
+        ref_s = oracle.score(qs, host(P), host(Kt[b:b + 1]), slh)
+        check_selection(host(idx[b:b + 1]).numpy(), host(cnt[b:b + 1]).numpy(), ref_s, slh.numpy(), w.k)
+        ref_o, ref_l = oracle.attend(qs, Ks, None, host(idx[b:b + 1]), host(cnt[b:b + 1]), slh, w.scale, dv=512,
+                                     v_aliases_k=True)
+        check_attention(out[b:b + 1], lse[b:b + 1], ref_o, ref_l, torch.bfloat16)
+    del q, K, Kt, s
+    torch.cuda.empty_cache()

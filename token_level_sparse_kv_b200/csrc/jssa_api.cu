@@ -86,10 +86,16 @@ int check_k(int k) {
     return JSSA_OK;
 }
 
-int check_attn_shape(const jssa_dims *d, const Shape &sh) {
-    if (sh.latent) return fail(JSSA_ERR_UNSUPPORTED, "latent-cache attention (d=576) has no kernel in this build");
+// Attention kernels exist for GQA (G <= 16, bf16 or fp32) and, for the indexed
+// path, for the latent cache with 128 heads in bf16.
+int check_attn_shape(const jssa_dims *d, const Shape &sh, bool indexed) {
+    if (sh.latent) {
+        if (!indexed) return fail(JSSA_ERR_UNSUPPORTED, "dense / gathered latent-cache attention has no kernel in this build");
+        if (d->Hq != 128 || d->kv_dtype != JSSA_BF16)
+            return fail(JSSA_ERR_UNSUPPORTED, "latent-cache attention needs Hq = 128 and bf16 (got Hq=%d)", d->Hq);
+        return JSSA_OK;
+    }
     if (sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "G=%d query heads per KV head above %d", sh.G, kMaxG);
-    (void)d;
     return JSSA_OK;
 }
 
@@ -131,6 +137,14 @@ int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, 
 }
 
 int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout &L) {
+    if (sh.latent) {
+        L.ap = AttnPlan();
+        L.ap.splits = mla_splits(npos);
+        L.part_o = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * d->dv * 4);
+        L.part_ml = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * 2 * 4);
+        L.att_ctr = take(L.total, (size_t)sh.BH * 4);
+        return JSSA_OK;
+    }
     cudaError_t e = plan_attend(src, d->kv_dtype, d->d, sh.G, d->B, d->Hkv, npos, &L.ap);
     if (e != cudaSuccess) return cuda_fail(e, "planning the attention pass");
     L.part_o = take(L.total, (size_t)sh.BH * L.ap.splits * sh.G * d->dv * 4);
@@ -249,6 +263,30 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
     return JSSA_OK;
 }
 
+int run_mla(const jssa_dims *d, const void *q, const void *K, const int32_t *idx, const int32_t *count, int k,
+            const int32_t *seq_lens, float scale, void *out, float *lse, void *ws, const Layout &L, cudaStream_t s) {
+    MlaArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q;
+    a.K = K;
+    a.idx = idx;
+    a.count = count;
+    a.seq_lens = seq_lens;
+    a.k = k;
+    a.T_cap = d->T_cap;
+    a.B = d->B;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.splits = L.ap.splits;
+    a.part_o = at<float>(ws, L.part_o);
+    a.part_ml = at<float>(ws, L.part_ml);
+    a.out = out;
+    a.lse = lse;
+    a.status = at<uint32_t>(ws, 0);
+    cudaError_t e = launch_mla(a, true, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the latent-cache indexed decode");
+    return JSSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -278,7 +316,7 @@ int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes) {
     if (needs_k && (st = check_k(k))) return st;
     if ((op == JSSA_OP_INDEXED_DECODE || op == JSSA_OP_DENSE_DECODE || op == JSSA_OP_GATHER_THEN_DENSE ||
          op == JSSA_OP_DECODE_STEP) &&
-        (st = check_attn_shape(dims, sh)))
+        (st = check_attn_shape(dims, sh, op == JSSA_OP_INDEXED_DECODE || op == JSSA_OP_DECODE_STEP)))
         return st;
     size_t best = 0;
     for (int agg = 0; agg < 2; ++agg) {
@@ -402,7 +440,7 @@ int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, con
     int st = check_dims(dims, &sh);
     if (st) return st;
     if ((st = check_k(k))) return st;
-    if ((st = check_attn_shape(dims, sh))) return st;
+    if ((st = check_attn_shape(dims, sh, true))) return st;
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
     REQUIRE_PTR(V);
@@ -415,6 +453,7 @@ int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, con
     if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
+    if (sh.latent) return run_mla(dims, q, K, idx, count, k, seq_lens, softmax_scale, out, lse, ws, L, S(stream));
     AttnArgs a;
     fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
     a.idx = idx;
@@ -431,7 +470,7 @@ int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const
     Shape sh;
     int st = check_dims(dims, &sh);
     if (st) return st;
-    if ((st = check_attn_shape(dims, sh))) return st;
+    if ((st = check_attn_shape(dims, sh, false))) return st;
     if (window < 0) return fail(JSSA_ERR_INVALID_ARG, "window=%d is negative", window);
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
@@ -459,7 +498,7 @@ int jssa_gather_then_dense(const jssa_dims *dims, const void *q, const void *K, 
     int st = check_dims(dims, &sh);
     if (st) return st;
     if ((st = check_k(k))) return st;
-    if ((st = check_attn_shape(dims, sh))) return st;
+    if ((st = check_attn_shape(dims, sh, false))) return st;
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
     REQUIRE_PTR(V);
@@ -503,7 +542,7 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
     int st = check_dims(dims, &sh);
     if (st) return st;
     if ((st = check_k(k))) return st;
-    if ((st = check_attn_shape(dims, sh))) return st;
+    if ((st = check_attn_shape(dims, sh, true))) return st;
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
     REQUIRE_PTR(V);
@@ -525,6 +564,7 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
     cudaError_t e = launch_prep(ap, pj, S(stream), true, dims->kv_dtype, dims->kt_dtype);
     if (e != cudaSuccess) return cuda_fail(e, "launching the append + projection prologue");
     if ((st = run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), false))) return st;
+    if (sh.latent) return run_mla(dims, q, K, idx, count, k, seq_lens, softmax_scale, out, lse, ws, L, S(stream));
     AttnArgs a;
     fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
     a.idx = idx;
@@ -579,7 +619,7 @@ extern "C" int jssa_indexed_decode_noalloc(const jssa_dims *dims, const void *q,
     int st = check_dims(dims, &sh);
     if (st) return st;
     if ((st = check_k(k))) return st;
-    if ((st = check_attn_shape(dims, sh))) return st;
+    if ((st = check_attn_shape(dims, sh, true))) return st;
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
     REQUIRE_PTR(V);

@@ -108,6 +108,27 @@ struct GatherArgs {
     int B, Hkv, T_cap, d, k;
 };
 
+// ------------------------------------------------------------------- MLA ---
+// Latent-cache attention: 128 query heads, 576-wide latent rows, the value is
+// the first 512 columns of the row.
+struct MlaArgs {
+    const void *q;            // [B, 128, 576] bf16
+    const void *K;            // [B, T_cap, 1, 576] bf16 (also the values)
+    const int32_t *idx;       // [B, k] selected tokens (indexed form)
+    const int32_t *count;     // [B] or null
+    const int32_t *seq_lens;  // [B]
+    int k, T_cap, B;
+    float scale_log2;
+    int splits;               // CTAs per batch row (128 tokens each)
+    float *part_o;            // [B, splits, 128, 512]
+    float *part_ml;           // [B, splits, 128, 2]
+    void *out;                // [B, 128, 512] bf16
+    float *lse;               // [B, 128] or null
+    uint32_t *status;
+};
+int mla_splits(int npos);
+cudaError_t launch_mla(const MlaArgs &a, bool indexed, cudaStream_t s, bool pdl);
+
 // --------------------------------------------------------------- helpers ---
 int device_sm_count();
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype);

@@ -1,0 +1,381 @@
+// Indexed decode attention over a shared latent cache (multi-head latent
+// attention), on the 5th-generation tensor cores.
+//
+// Method: news item "JSSA makes token-level sparse decoding gather-free",
+// Perspective para 1 (for MLA models the selection runs over the shared latent
+// cache); "Joint Subspace Sparse Attention for Efficient Long-Context
+// Decoding", Abstract (token-level indexed attention).  One latent row of 576
+// bf16 per token is both the key (all 576 dims) and the value (its first 512
+// dims); all 128 query heads attend over the selected rows of their batch row.
+//
+// With 128 heads the per-token work is a dense contraction (~228 flop per
+// byte of selected rows), so it runs as two tcgen05 matrix products per CTA:
+//   S[128 heads x 128 tokens] = Q[128 x 576] . K_sel^T      (fp32 in TMEM)
+//   O[128 x 512]             = softmax(S) (bf16) . V_sel     (fp32 in TMEM)
+// A CTA takes one batch row and one split of up to 128 selected tokens.  The
+// selected rows are gathered in place from the [B, T, 1, 576] cache with
+// cp.async into nine 128-byte-swizzled K-major blocks (the same bytes serve as
+// the MN-major V operand of the second product); Q streams through four
+// swizzled 16 KiB buffers; P is written to shared memory in the A-operand
+// layout.  TMEM holds S in columns 0..127, then O in columns 0..511.  Splits
+// write (unnormalised O, row max, row sum) and a combine kernel merges them by
+// log-sum-exp.
+#include "jssa_common.cuh"
+#include "jssa_internal.h"
+
+namespace jssa {
+
+namespace {
+
+constexpr int kD = 576, kDv = 512, kH = 128, kTok = 128, kThr = 128;
+constexpr int kKB = 9;          // 64-column blocks of a latent row
+constexpr int kQBuf = 4;        // Q block buffers
+constexpr int kBlk = 16384;     // one block: 128 rows x 128 bytes
+constexpr size_t kSmemK = (size_t)kKB * kBlk;
+constexpr size_t kSmemQ = (size_t)kQBuf * kBlk;
+constexpr size_t kSmemMisc = 2048;
+constexpr size_t kSmemBytes = kSmemK + kSmemQ + kSmemMisc;
+
+// Shared-memory matrix descriptor of a 128-byte-swizzled canonical layout
+// (start address, leading / stride byte offsets, descriptor version 1 for
+// this architecture, swizzle mode 128B).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor: bf16 x bf16 -> fp32, M x N, operand majorness.
+__host__ __device__ constexpr uint32_t mma_idesc(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(addr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+template <int N>
+__device__ __forceinline__ void cp_wait_dyn(int n) {
+    if (n >= N) {
+        cp_async_wait<N>();
+    } else if constexpr (N > 0) {
+        cp_wait_dyn<N - 1>(n);
+    }
+}
+
+template <bool INDEXED>
+__global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    unsigned char *sK = smem;
+    unsigned char *sQ = smem + kSmemK;
+    unsigned char *sP = sQ;  // P reuses Q buffers 0-1 once S is complete
+    uint64_t *qfree = reinterpret_cast<uint64_t *>(smem + kSmemK + kSmemQ);  // [kQBuf]
+    uint64_t *sdone = qfree + kQBuf;
+    uint64_t *odone = qfree + kQBuf + 1;
+    uint32_t *tptr = reinterpret_cast<uint32_t *>(qfree + kQBuf + 2);
+    int *flag = reinterpret_cast<int *>(tptr + 1);
+    int *tok = reinterpret_cast<int *>(qfree + 8);  // [kTok]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x, b = blockIdx.y;
+
+    pdl_trigger();
+    pdl_wait();
+
+    const int Tb = clamp_seq(a.seq_lens[b], a.T_cap, a.status);
+    int npos;
+    if (INDEXED) {
+        if (a.count) {
+            npos = a.count[b];
+            if (npos < 0 || npos > a.k) {
+                if (tid == 0 && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_INDEX);
+                npos = npos < 0 ? 0 : a.k;
+            }
+        } else {
+            npos = 0;
+            const int32_t *lst = a.idx + (size_t)b * a.k;
+            for (int j0 = 0; j0 < a.k; j0 += kThr) npos += __syncthreads_count(j0 + tid < a.k && lst[j0 + tid] >= 0);
+        }
+    } else {
+        npos = Tb;
+    }
+    const int p0 = split * kTok;
+    const int rows = max(0, min(kTok, npos - p0));
+
+    if (tid == 0) {
+        for (int i = 0; i < kQBuf + 2; ++i) mbar_init(&qfree[i], 1);
+        fence_barrier_init();
+        *flag = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tptr)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+    }
+    {
+        int t = -1;
+        if (tid < rows) {
+            t = INDEXED ? __ldg(a.idx + (size_t)b * a.k + p0 + tid) : p0 + tid;
+            if (t < 0 || t >= Tb) {
+                if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_INDEX);
+                t = -1;
+            }
+        }
+        tok[tid] = t;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tptr;
+
+    // ---- loads: selected latent rows (9 blocks) and Q blocks 0..3 --------------
+    const char *Kg = static_cast<const char *>(a.K);
+    const char *Qg = static_cast<const char *>(a.q) + (size_t)b * kH * kD * 2;
+    auto load_k_block = [&](int kb) {
+        for (int c = tid; c < kTok * 8; c += kThr) {
+            const int j = c >> 3, ch = c & 7;
+            const int t = tok[j];
+            unsigned char *dst = sK + (size_t)kb * kBlk + j * 128 + ((ch ^ (j & 7)) << 4);
+            if (t >= 0)
+                cp_async16(dst, Kg + ((size_t)b * a.T_cap + t) * (kD * 2) + kb * 128 + ch * 16, 16);
+            else
+                cp_async16(dst, Kg, 0);
+        }
+    };
+    auto load_q_block = [&](int kb, int buf) {
+        for (int c = tid; c < kH * 8; c += kThr) {
+            const int hh = c >> 3, ch = c & 7;
+            cp_async16(sQ + (size_t)buf * kBlk + hh * 128 + ((ch ^ (hh & 7)) << 4), Qg + (size_t)hh * (kD * 2) + kb * 128 + ch * 16,
+                       16);
+        }
+    };
+    for (int g = 0; g < kQBuf; ++g) {
+        load_k_block(g);
+        load_q_block(g, g);
+        cp_async_commit();
+    }
+    for (int kb = kQBuf; kb < kKB; ++kb) load_k_block(kb);
+    cp_async_commit();
+
+    // ---- S = Q K^T over the nine 64-column blocks -------------------------------
+    constexpr uint32_t idS = mma_idesc(128, kTok, 0, 0);
+    bool ok = true;
+    for (int kb = 0; kb < kKB; ++kb) {
+        // groups committed after the one holding block kb (see the load order)
+        const int after = kb < kQBuf ? kQBuf : min(kQBuf - 1, kKB - 1 - kb);
+        cp_wait_dyn<kQBuf>(after);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && ok) {
+            const uint32_t qa = smem_u32(sQ + (size_t)(kb % kQBuf) * kBlk), ka = smem_u32(sK + (size_t)kb * kBlk);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem, sw128_desc(qa + kk * 32, 16, 1024), sw128_desc(ka + kk * 32, 16, 1024), idS,
+                         (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&qfree[kb % kQBuf]);
+        }
+        if (kb + kQBuf < kKB) {
+            // refill this Q buffer with block kb+4 once the products reading it are done
+            if (ok && !mbar_wait_bounded(&qfree[kb % kQBuf], (uint32_t)(kb / kQBuf) & 1u)) atomicOr(flag, 1);
+            fence_async_smem();
+            if (*flag == 0) load_q_block(kb + kQBuf, kb % kQBuf);
+            cp_async_commit();
+        }
+        __syncthreads();
+        ok = *flag == 0;
+    }
+    if (tid == 0 && ok) mma_commit(sdone);
+    if (ok && !mbar_wait_bounded(sdone, 0u)) atomicOr(flag, 1);
+    tc_fence_after();
+    __syncthreads();
+    ok = *flag == 0;
+
+    // ---- softmax over the tile's tokens, one head per thread (TMEM lane) --------
+    const int h = warp * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float m = -INFINITY, l = 0.f;
+    if (ok) {
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTok; c0 += 32) {
+            float v[32];
+            tmem_ld32(lane_base + c0, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (c0 + j < rows && tok[c0 + j] >= 0) mx = fmaxf(mx, v[j]);
+        }
+        m = mx == -INFINITY ? -INFINITY : mx * a.scale_log2;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTok; c0 += 32) {
+            float v[32];
+            tmem_ld32(lane_base + c0, v);
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float pr[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = c0 + g8 * 8 + e * 2 + u;
+                        const bool live = col < rows && tok[col] >= 0;
+                        const float p = live ? exp2f(v[g8 * 8 + e * 2 + u] * a.scale_log2 - m) : 0.f;
+                        l += p;
+                        pr[u] = p;
+                    }
+                    const __nv_bfloat162 pk = __floats2bfloat162_rn(pr[0], pr[1]);
+                    w[e] = *reinterpret_cast<const uint32_t *>(&pk);
+                }
+                const int col8 = (c0 + g8 * 8) & 63, blk = (c0 + g8 * 8) >> 6;
+                *reinterpret_cast<uint4 *>(sP + (size_t)blk * kBlk + h * 128 + (((col8 >> 3) ^ (h & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- O = P V: V is the first 512 columns of the same rows (MN-major) --------
+    constexpr uint32_t idO = mma_idesc(128, 256, 0, 1);
+    if (tid == 0 && ok) {
+        const uint32_t pa = smem_u32(sP), ka = smem_u32(sK);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int kk = 0; kk < kTok / 16; ++kk)
+                mma_bf16(tmem + half * 256, sw128_desc(pa + (kk >> 2) * kBlk + (kk & 3) * 32, 16, 1024),
+                         sw128_desc(ka + half * 4 * kBlk + kk * 2048, kBlk, 1024), idO, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(odone);
+    }
+    if (ok && !mbar_wait_bounded(odone, 0u)) atomicOr(flag, 1);
+    tc_fence_after();
+    __syncthreads();
+    ok = *flag == 0;
+    if (!ok && tid == 0 && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+
+    // ---- epilogue --------------------------------------------------------------
+    if (ok) {
+        if (a.splits == 1) {
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * kH + h) * kDv;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kDv; c0 += 32) {
+                float v[32];
+                tmem_ld32(lane_base + c0, v);
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 pk = __floats2bfloat162_rn(v[j + 2 * e] * inv, v[j + 2 * e + 1] * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&pk);
+                    }
+                    *reinterpret_cast<uint4 *>(orow + c0 + j) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            if (a.lse) a.lse[(size_t)b * kH + h] = l > 0.f ? (m + log2f(l)) * 0.693147180559945309417f : -INFINITY;
+        } else {
+            float *po = a.part_o + (((size_t)b * a.splits + split) * kH + h) * kDv;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kDv; c0 += 32) {
+                float v[32];
+                tmem_ld32(lane_base + c0, v);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(po + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+            float *pml = a.part_ml + (((size_t)b * a.splits + split) * kH + h) * 2;
+            pml[0] = m;
+            pml[1] = l;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+}
+
+// Log-sum-exp merge of the splits: CTA (b, 4 heads), 16 output dims per thread.
+__global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x, h = blockIdx.y * 4 + (threadIdx.x >> 5), c0 = (threadIdx.x & 31) * 16;
+    const int ns = a.splits;
+    float M = -INFINITY;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, a.part_ml[(((size_t)b * ns + s) * kH + h) * 2]);
+    float L = 0.f, o[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) o[j] = 0.f;
+    for (int s = 0; s < ns; ++s) {
+        const float *pml = a.part_ml + (((size_t)b * ns + s) * kH + h) * 2;
+        const float ms = pml[0];
+        if (ms == -INFINITY) continue;
+        const float w = exp2f(ms - M);
+        L = fmaf(pml[1], w, L);
+        const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (((size_t)b * ns + s) * kH + h) * kDv + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = po[q];
+            o[4 * q] = fmaf(v.x, w, o[4 * q]);
+            o[4 * q + 1] = fmaf(v.y, w, o[4 * q + 1]);
+            o[4 * q + 2] = fmaf(v.z, w, o[4 * q + 2]);
+            o[4 * q + 3] = fmaf(v.w, w, o[4 * q + 3]);
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * kH + h) * kDv + c0;
+    uint32_t w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const __nv_bfloat162 pk = __floats2bfloat162_rn(o[2 * e] * inv, o[2 * e + 1] * inv);
+        w[e] = *reinterpret_cast<const uint32_t *>(&pk);
+    }
+    reinterpret_cast<uint4 *>(orow)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4 *>(orow)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    if (a.lse && (threadIdx.x & 31) == 0)
+        a.lse[(size_t)b * kH + h] = L > 0.f ? (M + log2f(L)) * 0.693147180559945309417f : -INFINITY;
+}
+
+}  // namespace
+
+int mla_splits(int npos) { return npos <= kTok ? 1 : (npos + kTok - 1) / kTok; }
+
+cudaError_t launch_mla(const MlaArgs &a0, bool indexed, cudaStream_t s, bool pdl) {
+    MlaArgs a = a0;
+    void (*k)(MlaArgs) = indexed ? mla_kernel<true> : mla_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(k, dim3(a.splits, a.B), dim3(kThr), kSmemBytes, s, pdl, a);
+    if (e != cudaSuccess || a.splits == 1) return e;
+    return launch_kernel(mla_combine_kernel, dim3(a.B, kH / 4), dim3(128), 0, s, pdl, a);
+}
+
+}  // namespace jssa
