@@ -57,7 +57,8 @@ def algorithmic_bytes(w):
     selected K and V rows per (b, h), the queries and the outputs."""
     es = 2
     kt = w.B * w.Hkv * w.T * w.r * es
-    sel = w.B * w.Hkv * min(w.k, w.T) * (w.d + w.Dv) * es
+    row = w.d if w.latent else w.d + w.Dv  # a latent row is key and value at once
+    sel = w.B * w.Hkv * min(w.k, w.T) * row * es
     qo = w.B * w.Hq * (w.d + w.Dv) * es
     return kt + sel + qo, kt
 
@@ -360,6 +361,7 @@ def run_jssa(args, world, rank, local):
 
     peak, peak_kind = measured_peaks()
     step_bytes, kt_bytes = algorithmic_bytes(w)
+    step_flops = 2 * w.B * w.Hq * min(w.k, w.T) * (w.d + w.Dv)  # q.k and p.v of the selected rows
     sbytes = select_bytes(w)
     sel_s = sel_secs / sel_steps
     achieved = sbytes / sel_s / 1e9
@@ -373,12 +375,13 @@ def run_jssa(args, world, rank, local):
                          "peak_kind": peak_kind + " (burst copy)", "traffic": traffic,
                          "algorithmic_bytes_per_launch": sbytes, "us_per_launch": sel_s * 1e6},
             "step_hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms / 1e3) / 1e9,
-                         "frac_of_peak": step_bytes / (ms / 1e3) / 1e9 / peak, "peak_gbs": peak},
+                         "frac_of_peak": step_bytes / (ms / 1e3) / 1e9 / peak, "peak_gbs": peak,
+                         "attention_flops_per_step": step_flops},
             "gpu_launches": 3 * args.steps}
     if clocks:
         line["clocks"] = clocks
 
-    if not args.quick:
+    if not args.quick and not w.latent:
         # comparison paths from the same build, same inputs
         ws_d = ops.new_workspace(dims, 1, ops.OP_DENSE_DECODE, dev)
         ws_a = ops.new_workspace(dims, 1, ops.OP_APPEND, dev)
@@ -387,6 +390,9 @@ def run_jssa(args, world, rank, local):
         cmp_steps = max(5, min(args.steps, args.cmp_steps))
 
         def dense(i):
+            ops.dense_decode(qs[i & 3], K, Vv, sl, w.scale, window=0, ws=ws_d, out=out, lse=lse)
+
+        def local(i):  # the sliding-window layer of a hybrid global/local pair
             ops.dense_decode(qs[i & 3], K, Vv, sl, w.scale, window=w.window, ws=ws_d, out=out, lse=lse)
 
         def gather(i):
@@ -401,7 +407,10 @@ def run_jssa(args, world, rank, local):
             ops.indexed_decode(qs[i & 3], K, Vv, idx, cnt, sl, w.scale, ws=ws_g, out=out, lse=lse)
 
         res = {}
-        for name, fn in (("dense_full_kv", dense), ("gather_then_dense", gather), ("split_calls_gather_free", split)):
+        paths = [("dense_full_kv", dense), ("gather_then_dense", gather), ("split_calls_gather_free", split)]
+        if w.window:
+            paths.append(("local_window_layer", local))
+        for name, fn in paths:
             for i in range(3):
                 fn(i)
             t = max_over_ranks(time_loop(fn, cmp_steps, stream), world)
@@ -409,14 +418,20 @@ def run_jssa(args, world, rank, local):
         res["speedup_vs_dense"] = value / res["dense_full_kv"]["steps_per_s"]
         res["speedup_vs_gather_then_dense"] = value / res["gather_then_dense"]["steps_per_s"]
         if w.window:
-            res["dense_full_kv"]["note"] = "sliding window %d (the local layer of the hybrid pair)" % w.window
+            res["local_window_layer"]["note"] = "dense sliding window %d over the same cache shape" % w.window
+            pair_ms = ms + res["local_window_layer"]["ms_per_step"]
+            res["hybrid_pair"] = {"steps_per_s": world * 1e3 / pair_ms, "ms_per_step": pair_ms,
+                                  "note": "sparse global layer (the timed step) + dense sliding-window local layer"}
         line["comparison"] = res
+    elif not args.quick:
+        line["comparison"] = {"note": "dense and gather-then-dense latent-cache kernels are not built"}
 
+    if not args.quick:
         # end to end through the session API with host buffers
         sess = ops.DecodeSession(K, Vv, P, sl, w.k, w.scale, Kt=Kt)
         qh = [x.cpu().pin_memory() for x in qs]
         kh = torch.randn((w.B, w.Hkv, w.d), dtype=torch.float32).to(q.dtype).pin_memory()
-        vh = torch.randn((w.B, w.Hkv, w.Dv), dtype=torch.float32).to(q.dtype).pin_memory()
+        vh = None if w.latent else torch.randn((w.B, w.Hkv, w.Dv), dtype=torch.float32).to(q.dtype).pin_memory()
         e2e_steps = max(5, min(args.steps, args.e2e_steps))
         for i in range(3):
             sess.step_from_host(qh[i & 3], kh, vh)
@@ -427,7 +442,8 @@ def run_jssa(args, world, rank, local):
             o = sess.step_from_host(qh[i & 3], kh, vh)
             stream.synchronize()  # the host reads the output every step
         te = max_over_ranks(time.perf_counter() - t0, world)
-        h2d = qh[0].numel() * qh[0].element_size() + kh.numel() * kh.element_size() + vh.numel() * vh.element_size()
+        h2d = qh[0].numel() * qh[0].element_size() + kh.numel() * kh.element_size() + (
+            0 if vh is None else vh.numel() * vh.element_size())
         d2h = o.numel() * o.element_size()
         line["e2e"] = {"value": world * e2e_steps / te, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "api": "DecodeSession.step_from_host (pinned host in/out)"}

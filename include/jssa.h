@@ -57,6 +57,15 @@
  * Word 0 of the workspace is a sticky status word: kernels OR in
  * JSSA_DEV_* bits for bad data they meet (and skip that item); read it back
  * with a device-to-host copy of 4 bytes; jssa_workspace_init() clears it.
+ *
+ * Host state: launch plans of the selection pass are cached per device and
+ * shape in host memory (mutex-protected).  The selection (jssa_topk,
+ * jssa_select, jssa_decode_step) has two forms with identical results: one
+ * thread-block cluster per (b, h) holding the keys of its rows in shared
+ * memory, taken when all B*Hkv clusters fit on the GPU at once, and a
+ * persistent streaming pass with a segment merge otherwise.  The environment
+ * variable JSSA_SELECT_FORM = "cluster" or "stream" forces one form at
+ * planning time (tests and measurement); size the workspace after setting it.
  */
 #ifndef JSSA_H
 #define JSSA_H

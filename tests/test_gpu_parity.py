@@ -94,8 +94,23 @@ def test_score_parity(agg, kt):
     assert np.all(np.isnan(sg[1, :, 700:])), "entries past T_b were written"
 
 
+# Both selection forms (one cluster per (b,h) holding its keys in shared
+# memory, and the persistent streaming pass with a segment merge) must return
+# the same indices; JSSA_SELECT_FORM forces one at planning time.
+FORMS = ["auto", "cluster", "stream"]
+
+
+@pytest.fixture(params=FORMS)
+def form(request, monkeypatch):
+    if request.param == "auto":
+        monkeypatch.delenv("JSSA_SELECT_FORM", raising=False)
+    else:
+        monkeypatch.setenv("JSSA_SELECT_FORM", request.param)
+    return request.param
+
+
 # -------------------------------------------------------------------- topk
-def test_topk_is_exact_on_the_same_scores():
+def test_topk_is_exact_on_the_same_scores(form):
     w = W(B=3, Hkv=2, Hq=4, T=9000)
     g = torch.Generator().manual_seed(3)
     s = torch.randn(w.B, w.Hkv, w.T, generator=g)
@@ -112,7 +127,7 @@ def test_topk_is_exact_on_the_same_scores():
         np.testing.assert_array_equal(host(cnt).numpy(), ref_cnt)
 
 
-def test_topk_ragged_and_empty():
+def test_topk_ragged_and_empty(form):
     g = torch.Generator().manual_seed(4)
     s = torch.randn(4, 1, 5000, generator=g)
     sl = torch.tensor([0, 1, 255, 5000], dtype=torch.int32)
@@ -125,7 +140,7 @@ def test_topk_ragged_and_empty():
 
 # ------------------------------------------------------------------ select
 @pytest.mark.parametrize("case", ["small", "multi_segment", "r64", "fp32", "max"])
-def test_select_equals_score_then_topk_and_matches_oracle(case):
+def test_select_equals_score_then_topk_and_matches_oracle(case, form):
     kt = torch.bfloat16
     agg = ops.AGG_SUM
     if case == "small":
@@ -151,7 +166,7 @@ def test_select_equals_score_then_topk_and_matches_oracle(case):
     check_selection(host(idx).numpy(), host(cnt).numpy(), ref, slh.numpy(), w.k)
 
 
-def test_select_exact_ties_take_lowest_index():
+def test_select_exact_ties_take_lowest_index(form):
     w = W(B=1, Hkv=2, Hq=4, T=3000, k=50, kind="plain", seed=16)
     (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
     # head 0: every row equal -> every score equal -> the first k tokens
@@ -473,4 +488,23 @@ def test_full_size_mla_64k_b8_sampled():
                                      v_aliases_k=True)
         check_attention(out[b:b + 1], lse[b:b + 1], ref_o, ref_l, torch.bfloat16)
     del q, K, Kt, s
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("wname", ["gqa_4k_b1", "gqa_32k_b4", "mla_64k_b8"])
+def test_select_forms_agree_full_size(wname, monkeypatch):
+    """The cluster and the streaming selection give identical index lists on
+    the full-size workloads (the shapes where the automatic choice flips)."""
+    from token_level_sparse_kv_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[wname]
+    q, K, V, P, sl = make_inputs(w, device=DEV)
+    Kt = ops.build_lowrank_cache(K, P)
+    res = []
+    for f in ("cluster", "stream"):
+        monkeypatch.setenv("JSSA_SELECT_FORM", f)
+        res.append(ops.select(q, P, Kt, sl, w.k))
+    torch.cuda.synchronize()
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    del q, K, V, Kt
     torch.cuda.empty_cache()

@@ -116,6 +116,8 @@ struct Layout {
     size_t total = 256;  // [0, 256): status word
     ScanPlan sp{};
     AttnPlan ap{};
+    bool csel = false;  // selection by one cluster per (b,h) (else the streaming form)
+    CSelPlan cp{};
 };
 
 size_t take(size_t &off, size_t bytes) {
@@ -126,7 +128,14 @@ size_t take(size_t &off, size_t bytes) {
 
 int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, Layout &L) {
     const int nq = (src != SRC_SCORES && agg == JSSA_AGG_MAX) ? sh.G : 1;
-    cudaError_t e = plan_scan(src, MODE_SELECT, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.sp);
+    cudaError_t e = plan_csel(src, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.cp);
+    if (e == cudaSuccess) {
+        L.csel = true;
+        return JSSA_OK;
+    }
+    cudaGetLastError();
+    if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the cluster selection");
+    e = plan_scan(src, MODE_SELECT, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.sp);
     if (e != cudaSuccess) return cuda_fail(e, "planning the selection pass");
     const size_t nc = (size_t)sh.BH * L.sp.max_seg * k;
     L.cand_key = take(L.total, nc * 4);
@@ -239,6 +248,27 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
         ProjArgs pj{q, P, at<float>(ws, L.qproj), d->B, d->Hq, d->Hkv, d->d, d->r, agg};
         cudaError_t e = launch_project(pj, s, true, d->kv_dtype);
         if (e != cudaSuccess) return cuda_fail(e, "launching the query projection");
+    }
+    if (L.csel) {
+        CSelArgs ca;
+        memset(&ca, 0, sizeof ca);
+        ca.src = Kt;
+        ca.qproj = at<float>(ws, L.qproj);
+        ca.seq_lens = seq_lens;
+        ca.idx_out = idx;
+        ca.count_out = count;
+        ca.status = at<uint32_t>(ws, 0);
+        ca.B = d->B;
+        ca.Hkv = d->Hkv;
+        ca.T_cap = d->T_cap;
+        ca.r = d->r;
+        ca.nq = nq;
+        ca.k = k;
+        // a null query means the source is a score array (jssa_topk)
+        const int src = q == nullptr ? SRC_SCORES : (d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32);
+        cudaError_t e = launch_csel(L.cp, ca, src, q == nullptr ? JSSA_AGG_SUM : agg, s, true);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the cluster selection");
+        return JSSA_OK;
     }
     ScanArgs sa;
     memset(&sa, 0, sizeof sa);

@@ -108,6 +108,24 @@ struct GatherArgs {
     int B, Hkv, T_cap, d, k;
 };
 
+// --------------------------------------------------------- cluster select ---
+// Top-k of one (b,h) by a cluster of CTAs holding the keys in shared memory.
+struct CSelArgs {
+    const void *src;          // Kt [B,Hkv,T_cap,r] or scores [B,Hkv,T_cap]
+    const float *qproj;       // [B*Hkv, nq, r]
+    const int32_t *seq_lens;  // [B]
+    int32_t *idx_out;         // [BH, k]
+    int32_t *count_out;       // [BH] or null
+    uint32_t *status;
+    int B, Hkv, T_cap, r, nq, k, csize, slice;
+};
+struct CSelPlan {
+    int csize, slice, grid_y;
+    size_t smem;
+};
+cudaError_t plan_csel(int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p);
+cudaError_t launch_csel(const CSelPlan &p, const CSelArgs &a, int src, int agg, cudaStream_t s, bool pdl);
+
 // ------------------------------------------------------------------- MLA ---
 // Latent-cache attention: 128 query heads, 576-wide latent rows, the value is
 // the first 512 columns of the row.

@@ -30,15 +30,16 @@ constexpr int kChunk = 16;  // d is a multiple of 16 for every supported shape
 __device__ __forceinline__ void chunked_dots(const float *x, const float *__restrict__ P, int d, int r, int n_out,
                                              float *part) {
     const int nch = d / kChunk;
+    // consecutive threads take consecutive outputs (columns of P): coalesced P reads
     for (int p = threadIdx.x; p < n_out * nch; p += blockDim.x) {
-        const int o = p / nch, c = p - o * nch;
+        const int c = p / n_out, o = p - c * n_out;
         const int row = o / r, j = o - row * r;
         const float *xr = x + (size_t)row * d + c * kChunk;
         const float *pc = P + (size_t)(c * kChunk) * r + j;
         float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < kChunk; ++i) acc = fmaf(xr[i], __ldg(pc + (size_t)i * r), acc);
-        part[p] = acc;
+        part[(size_t)o * nch + c] = acc;
     }
     __syncthreads();
 }
@@ -86,11 +87,20 @@ __device__ void project_bh(const ProjArgs &a, int bh, float *xs, float *part) {
     const KV *q = static_cast<const KV *>(a.q) + ((size_t)b * a.Hq + (size_t)h * G) * d;
     const int nrow = a.agg == JSSA_AGG_SUM ? 1 : G;
     if (a.agg == JSSA_AGG_SUM) {
+        // stage the group's queries in shared memory (every load in flight at
+        // once), then sum over the group in head order
+        KV *qsm = reinterpret_cast<KV *>(part + (size_t)r * (d / kChunk));
+        const int nvec = G * d * (int)sizeof(KV) / 16;
+        for (int v = threadIdx.x; v < nvec; v += blockDim.x) cp_async16(qsm + (size_t)v * (16 / sizeof(KV)), q + (size_t)v * (16 / sizeof(KV)), 16);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
         for (int i = threadIdx.x; i < d; i += blockDim.x) {
             float s = 0.f;
-            for (int g = 0; g < G; ++g) s += to_f32(q[(size_t)g * d + i]);
+            for (int g = 0; g < G; ++g) s += to_f32(qsm[(size_t)g * d + i]);
             xs[i] = s;
         }
+        __syncthreads();
     } else {
         for (int p = threadIdx.x; p < G * d; p += blockDim.x) xs[p] = to_f32(q[p]);
     }
@@ -173,7 +183,9 @@ cudaError_t launch_append(const AppendArgs &a0, cudaStream_t s, bool pdl, int kv
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype) {
     const int G = a.Hq / a.Hkv;
     const int nrow = a.agg == JSSA_AGG_SUM ? 1 : G;
-    const size_t smem = ((size_t)nrow * a.d + (size_t)nrow * a.r * (a.d / kChunk)) * sizeof(float);
+    const size_t es = kv_dtype == JSSA_BF16 ? 2 : 4;
+    const size_t stage = a.agg == JSSA_AGG_SUM ? (size_t)G * a.d * es : 0;
+    const size_t smem = ((size_t)nrow * a.d + (size_t)nrow * a.r * (a.d / kChunk)) * sizeof(float) + stage;
     void (*k)(ProjArgs) = kv_dtype == JSSA_BF16 ? project_kernel<__nv_bfloat16> : project_kernel<float>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
@@ -189,7 +201,9 @@ cudaError_t launch_prep(const AppendArgs &ap0, const ProjArgs &pj, cudaStream_t 
     const int nrow = pj.agg == JSSA_AGG_SUM ? 1 : G;
     size_t xs = (size_t)nrow * pj.d;
     size_t part = (size_t)(nrow > 1 ? nrow : 1) * pj.r * (pj.d / kChunk);
-    const size_t smem = (xs + part) * sizeof(float);
+    const size_t es = kv_dtype == JSSA_BF16 ? 2 : 4;
+    const size_t stage = pj.agg == JSSA_AGG_SUM ? (size_t)G * pj.d * es : 0;
+    const size_t smem = (xs + part) * sizeof(float) + stage;
     void (*k)(AppendArgs, ProjArgs);
     if (kv_dtype == JSSA_BF16)
         k = kt_dtype == JSSA_BF16 ? prep_kernel<__nv_bfloat16, __nv_bfloat16> : prep_kernel<__nv_bfloat16, float>;

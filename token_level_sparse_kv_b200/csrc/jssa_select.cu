@@ -1,0 +1,572 @@
+// Per-(batch, KV head) top-k selection by one thread-block cluster per (b, h).
+//
+// Method: news item "JSSA makes token-level sparse decoding gather-free",
+// Synopsis (tokens scored in a shared low-dimensional query-key subspace; a
+// distinct selected token set for each KV head); "Joint Subspace Sparse
+// Attention for Efficient Long-Context Decoding", Abstract (distinct
+// per-KV-head selections).
+//
+// The C CTAs of a cluster split the token range of one (b, h) into C
+// contiguous slices.  Each CTA streams its slice of the low-rank key cache
+// through a two-deep ring of 32 KiB bulk asynchronous copies (or reads its
+// slice of a score array), computes the fp32 scores exactly as the score pass
+// does, and keeps their order-preserving uint32 keys in shared memory.  The
+// cluster then finds the k-th key together: three radix levels of 11, 11 and
+// 10 bits; at each level every CTA histograms its keys that match the prefix
+// found so far, each CTA sums one slice of the bins across the cluster through
+// distributed shared memory, and every CTA scans the summed histogram.  Keys
+// equal to the k-th key are taken lowest token index first (CTAs hold
+// ascending token ranges, so an exclusive scan of their tie counts orders
+// them).  Each CTA finally writes its selected tokens, already ascending, at
+// its offset in the index list: no merge and no sort.  The result is the same
+// set, in the same order, as jssa_score + jssa_topk.
+#include <cooperative_groups.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include "jssa_common.cuh"
+#include "jssa_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace jssa {
+
+namespace {
+
+constexpr int NT = 256;
+constexpr int kTileB = 32768;   // bytes per ring stage
+constexpr int kStagesC = 2;
+constexpr int kBins = 2048;
+constexpr int kMaxSlice = 16384;  // tokens per CTA kept in shared memory
+
+struct CSmem {
+    size_t stages, bars, qs, keys, hist, gsum, gall, misc, total;
+};
+
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) / 16 * 16; }
+
+__host__ __device__ inline CSmem csel_smem(bool from_kt, int r, int nq, int slice) {
+    CSmem L;
+    size_t o = 0;
+    L.stages = o;
+    o += from_kt ? (size_t)kStagesC * kTileB : 0;
+    L.bars = o;
+    o = align16(o + 64);
+    L.qs = o;
+    o = align16(o + (from_kt ? (size_t)nq * r * 4 : 0));
+    L.keys = o;
+    o = align16(o + (size_t)slice * 4);
+    L.hist = o;
+    o = align16(o + (size_t)kBins * 4);
+    L.gsum = o;
+    o = align16(o + (size_t)kBins * 4 / 2);  // one slice of summed bins (C >= 2)
+    L.gall = o;
+    o = align16(o + (size_t)kBins * 4);
+    L.misc = o;
+    o = align16(o + 64 * 4);
+    L.total = (o + 127) / 128 * 128;
+    return L;
+}
+
+template <int CPT>
+__device__ __forceinline__ float chunk_sum(const float (&p)[CPT]) {
+    if constexpr (CPT == 4) return (p[0] + p[2]) + (p[1] + p[3]);
+    if constexpr (CPT == 2) return p[0] + p[1];
+    return p[0];
+}
+
+template <int SRC, int R, int AGG>
+__global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
+    constexpr bool FROM_KT = SRC != SRC_SCORES;
+    using KT = typename std::conditional<SRC == SRC_KT_FP32, float, __nv_bfloat16>::type;
+    constexpr int ES = SRC == SRC_KT_FP32 ? 4 : 2;
+    constexpr int ROWB = FROM_KT ? R * ES : 4;
+    constexpr int TPB = ROWB > 64 ? 64 : ROWB;
+    constexpr int LPT = ROWB / TPB;
+    constexpr int CPT = FROM_KT ? TPB / 16 : 1;
+    constexpr int EPL = 16 / ES;
+    constexpr int TILE = FROM_KT ? kTileB / ROWB : 2048;
+    constexpr int TPP = NT / LPT;
+    constexpr int PASSES = FROM_KT ? TILE / TPP : TILE / NT;
+    constexpr int QN = FROM_KT ? CPT * EPL : 1;
+    static_assert(!FROM_KT || TILE % TPP == 0, "tile / pass");
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    const CSmem L = csel_smem(FROM_KT, FROM_KT ? R : 0, a.nq, a.slice);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+    float *qs = reinterpret_cast<float *>(smem + L.qs);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem + L.keys);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + L.hist);
+    uint32_t *gsum = reinterpret_cast<uint32_t *>(smem + L.gsum);
+    uint32_t *gall = reinterpret_cast<uint32_t *>(smem + L.gall);
+    int *misc = reinterpret_cast<int *>(smem + L.misc);
+    int *tmp = misc + 16;
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = a.csize;
+    const int c = (int)cluster.block_rank();
+    const int bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31;
+
+    if (FROM_KT && tid == 0) {
+        for (int s = 0; s < kStagesC; ++s) mbar_init(&bars[s], 1);
+        fence_barrier_init();
+    }
+    if (tid == 0) misc[6] = 0;
+    __syncthreads();
+    pdl_trigger();
+    pdl_wait();
+
+    const int Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, a.status);
+    const int kb = min(a.k, Tb);
+    const int lo = c * a.slice;
+    const int n_loc = max(0, min(a.slice, Tb - lo));  // valid tokens of this CTA
+    const int ntiles = (n_loc + TILE - 1) / TILE;
+
+    // ---- scores of this slice into shared memory ---------------------------
+    if constexpr (FROM_KT) {
+        const char *src = static_cast<const char *>(a.src) + ((size_t)bh * a.T_cap + lo) * ROWB;
+        uint64_t pol = 0;
+        if (tid == 0) {
+            pol = policy_evict_first();
+            for (int i = 0; i < min(kStagesC, ntiles); ++i) {
+                const int n = min(TILE, n_loc - i * TILE);
+                mbar_arrive_expect_tx(&bars[i], (uint32_t)n * ROWB);
+                bulk_g2s(smem + L.stages + (size_t)i * kTileB, src + (size_t)i * TILE * ROWB, (uint32_t)n * ROWB, &bars[i],
+                         pol);
+            }
+        }
+        for (int p = tid; p < a.nq * R; p += NT) qs[p] = a.qproj[(size_t)bh * a.nq * R + p];
+        __syncthreads();
+        const int sub = tid % LPT;
+        const int rot = CPT == 4 ? (lane >> 1) & 3 : (CPT == 2 ? (lane >> 2) & 1 : 0);
+        float qreg[QN];
+        if (AGG == JSSA_AGG_SUM) {
+#pragma unroll
+            for (int cc = 0; cc < CPT; ++cc) {
+                const int ch = sub * CPT + ((cc + rot) % CPT);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) qreg[(cc * EPL + e) % QN] = qs[ch * EPL + e];
+            }
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % kStagesC;
+            const int t0 = i * TILE, n = min(TILE, n_loc - t0);
+            if (!mbar_wait_bounded(&bars[s], (uint32_t)(i / kStagesC) & 1u)) misc[6] = 1;
+            const unsigned char *st = smem + L.stages + (size_t)s * kTileB;
+#pragma unroll
+            for (int ps = 0; ps < PASSES; ++ps) {
+                const int tt = ps * TPP + tid / LPT;
+                const bool live = tt < n;
+                const unsigned char *row = st + (size_t)tt * ROWB + sub * TPB;
+                float sc;
+                if constexpr (AGG == JSSA_AGG_SUM) {
+                    float pc[CPT];
+#pragma unroll
+                    for (int cc = 0; cc < CPT; ++cc) {
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (live) v = *reinterpret_cast<const uint4 *>(row + ((cc + rot) % CPT) * 16);
+                        float kf[EPL];
+                        Vec16<KT>::unpack(v, kf);
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) acc = fmaf(kf[e], qreg[cc * EPL + e], acc);
+                        pc[cc] = acc;
+                    }
+                    float acc = chunk_sum<CPT>(pc);
+#pragma unroll
+                    for (int off = 1; off < LPT; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                    sc = acc;
+                } else {
+                    float kf[CPT][EPL];
+#pragma unroll
+                    for (int cc = 0; cc < CPT; ++cc) {
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (live) v = *reinterpret_cast<const uint4 *>(row + ((cc + rot) % CPT) * 16);
+                        Vec16<KT>::unpack(v, kf[cc]);
+                    }
+                    float best = -INFINITY;
+                    for (int g = 0; g < a.nq; ++g) {
+                        float pc[CPT];
+#pragma unroll
+                        for (int cc = 0; cc < CPT; ++cc) {
+                            const int ch = sub * CPT + ((cc + rot) % CPT);
+                            const float *qg = qs + g * R + ch * EPL;
+                            float acc = 0.f;
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e) acc = fmaf(kf[cc][e], qg[e], acc);
+                            pc[cc] = acc;
+                        }
+                        float acc = chunk_sum<CPT>(pc);
+#pragma unroll
+                        for (int off = 1; off < LPT; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                        best = fmaxf(best, acc);
+                    }
+                    sc = best;
+                }
+                if (live && sub == 0) keys[t0 + tt] = score_key(sc);
+            }
+            __syncthreads();  // stage s consumed
+            if (tid == 0 && i + kStagesC < ntiles) {
+                const int n2 = min(TILE, n_loc - (i + kStagesC) * TILE);
+                mbar_arrive_expect_tx(&bars[s], (uint32_t)n2 * ROWB);
+                bulk_g2s(smem + L.stages + (size_t)s * kTileB, src + (size_t)(i + kStagesC) * TILE * ROWB,
+                         (uint32_t)n2 * ROWB, &bars[s], pol);
+            }
+        }
+    } else {
+        const float *srow = static_cast<const float *>(a.src) + (size_t)bh * a.T_cap + lo;
+        for (int j0 = 0; j0 < n_loc; j0 += NT * 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u * NT + tid;
+                v[u] = j < n_loc ? __ldcs(srow + j) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u * NT + tid;
+                if (j < n_loc) keys[j] = score_key(v[u]);
+            }
+        }
+    }
+    __syncthreads();
+    const bool local_timeout = misc[6] != 0;
+
+    // ---- cluster radix select of the k-th key ------------------------------
+    uint32_t prefix = 0u, mask = 0u;
+    int kk = kb, grp = 0;
+    bool whole = true;
+    const int bins_per_cta = kBins / C;
+    if (kb > 0 && kb < Tb) {
+        const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+        for (int lev = 0; lev < 3; ++lev) {
+            const int shift = shifts[lev];
+            const uint32_t dmask = (1u << widths[lev]) - 1u;
+            for (int d = tid; d < kBins; d += NT) hist[d] = 0u;
+            __syncthreads();
+            for (int j = tid; j < n_loc; j += NT) {
+                const uint32_t u = keys[j];
+                if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+            }
+            cluster.sync();
+            // this CTA sums bins [c * bins_per_cta, (c+1) * bins_per_cta) over the cluster
+            for (int q = tid; q < bins_per_cta; q += NT) {
+                uint32_t v[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) v[r] = r < C ? *cluster.map_shared_rank(hist + c * bins_per_cta + q, r) : 0u;
+                uint32_t sum = 0u;
+#pragma unroll
+                for (int r = 0; r < 16; ++r) sum += v[r];
+                gsum[q] = sum;
+            }
+            cluster.sync();
+            {
+                uint32_t v[kBins / NT];
+#pragma unroll
+                for (int u = 0; u < kBins / NT; ++u) {
+                    const int d = tid + u * NT;
+                    v[u] = *cluster.map_shared_rank(gsum + (d % bins_per_cta), d / bins_per_cta);
+                }
+#pragma unroll
+                for (int u = 0; u < kBins / NT; ++u) gall[tid + u * NT] = v[u];
+            }
+            __syncthreads();
+            // descending scan over all bins: thread t owns 8 bins from the top
+            constexpr int BPT = kBins / NT;
+            const int base_bin = kBins - BPT * (tid + 1);
+            int cnt[BPT];
+            int s = 0;
+#pragma unroll
+            for (int q = 0; q < BPT; ++q) {
+                cnt[q] = (int)gall[base_bin + BPT - 1 - q];
+                s += cnt[q];
+            }
+            int tot;
+            int ex = block_excl_scan<NT>(s, tmp, tot);
+#pragma unroll
+            for (int q = 0; q < BPT; ++q) {
+                if (ex < kk && ex + cnt[q] >= kk) {
+                    misc[0] = base_bin + BPT - 1 - q;
+                    misc[1] = ex;
+                    misc[2] = cnt[q];
+                }
+                ex += cnt[q];
+            }
+            __syncthreads();
+            prefix |= (uint32_t)misc[0] << shift;
+            mask |= dmask << shift;
+            kk -= misc[1];
+            grp = misc[2];
+            __syncthreads();
+            if (kk == grp) break;
+        }
+        whole = kk == grp;
+    }
+
+    // ---- ties: equal keys go to the lowest token indices, CTA by CTA --------
+    int take_ties = 0;
+    if (!whole) {
+        int e = 0;
+        for (int j = tid; j < n_loc; j += NT) e += (keys[j] & mask) == prefix;
+        int tot;
+        (void)block_excl_scan<NT>(e, tmp, tot);
+        if (tid == 0) misc[3] = tot;
+        cluster.sync();
+        int before = 0;
+        for (int r = 0; r < c; ++r) before += *cluster.map_shared_rank(misc + 3, r);
+        take_ties = max(0, min(tot, kk - before));
+    }
+
+    // ---- emit the selection in ascending token order -----------------------
+    const bool take_all = kb >= Tb;
+    const int per = (n_loc + NT - 1) / NT;
+    const int j0 = min(tid * per, n_loc), j1 = min(j0 + per, n_loc);
+    auto above = [&](uint32_t u) { return (u & mask) > prefix; };
+    auto in_group = [&](uint32_t u) { return (u & mask) == prefix; };
+    int cs = 0, ce = 0;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t u = keys[j];
+        cs += take_all || (kb > 0 && (above(u) || (in_group(u) && whole)));
+        ce += !take_all && kb > 0 && !whole && in_group(u);
+    }
+    int tot_e;
+    const int e0 = block_excl_scan<NT>(ce, tmp, tot_e);  // tie rank of this thread's first tie
+    {
+        int e = e0;
+        for (int j = j0; j < j1; ++j) {
+            const uint32_t u = keys[j];
+            if (!take_all && kb > 0 && !whole && in_group(u)) {
+                cs += e < take_ties;
+                ++e;
+            }
+        }
+    }
+    int tot_s;
+    int w = block_excl_scan<NT>(cs, tmp, tot_s);
+    if (tid == 0) misc[4] = tot_s;
+    cluster.sync();
+    int base = 0;
+    for (int r = 0; r < c; ++r) base += *cluster.map_shared_rank(misc + 4, r);
+    int32_t *out = a.idx_out + (size_t)bh * a.k;
+    {
+        int e = e0;
+        w += base;
+        for (int j = j0; j < j1; ++j) {
+            const uint32_t u = keys[j];
+            bool sel = take_all || (kb > 0 && (above(u) || (in_group(u) && whole)));
+            if (!take_all && kb > 0 && !whole && in_group(u)) {
+                sel = e < take_ties;
+                ++e;
+            }
+            if (sel) {
+                if (w < a.k) out[w] = lo + j;
+                ++w;
+            }
+        }
+    }
+    if (c == C - 1) {
+        const int total = base + tot_s;  // = k_b
+        for (int j = total + tid; j < a.k; j += NT) out[j] = -1;
+        if (tid == 0 && a.count_out) a.count_out[bh] = total;
+    }
+    if (local_timeout && tid == 0 && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+    cluster.sync();  // peers may still read this CTA's shared memory until here
+}
+
+template <int SRC, int R, int AGG>
+void (*pick_c3())(CSelArgs) {
+    return select_cluster_kernel<SRC, R, AGG>;
+}
+
+template <int SRC>
+void (*pick_cr(int r, int agg))(CSelArgs) {
+    switch (r) {
+        case 8: return agg ? pick_c3<SRC, 8, 1>() : pick_c3<SRC, 8, 0>();
+        case 16: return agg ? pick_c3<SRC, 16, 1>() : pick_c3<SRC, 16, 0>();
+        case 32: return agg ? pick_c3<SRC, 32, 1>() : pick_c3<SRC, 32, 0>();
+        case 64: return agg ? pick_c3<SRC, 64, 1>() : pick_c3<SRC, 64, 0>();
+        case 128: return agg ? pick_c3<SRC, 128, 1>() : pick_c3<SRC, 128, 0>();
+        default: return nullptr;
+    }
+}
+
+void (*pick_csel(int src, int r, int agg))(CSelArgs) {
+    if (src == SRC_SCORES) return select_cluster_kernel<SRC_SCORES, 8, 0>;
+    return src == SRC_KT_BF16 ? pick_cr<SRC_KT_BF16>(r, agg) : pick_cr<SRC_KT_FP32>(r, agg);
+}
+
+int csel_tile(int src, int r) {
+    if (src == SRC_SCORES) return 2048;
+    return kTileB / (r * (src == SRC_KT_FP32 ? 4 : 2));
+}
+
+}  // namespace
+
+// Which selection form a shape uses.  The cluster form is taken when every
+// (b,h) gets its own cluster, all resident at once, with the keys of its slice
+// in shared memory: it has no segment merge and no second wave.  Otherwise
+// (many (b,h) rows or rows too long for shared memory) the persistent
+// streaming pass is taken.  Both return the same indices.  The environment
+// variable JSSA_SELECT_FORM overrides the choice at planning time: "cluster"
+// takes the cluster form wherever its slices fit in shared memory (several
+// waves allowed), "stream" always takes the streaming form.
+static int select_form_override() {
+    const char *v = getenv("JSSA_SELECT_FORM");
+    if (!v) return 0;
+    if (!strcmp(v, "cluster")) return 1;
+    if (!strcmp(v, "stream")) return 2;
+    return 0;
+}
+
+namespace {
+
+// Resident clusters of size C for this kernel and shared-memory size (0 on error).
+int resident_clusters(void (*kern)(CSelArgs), int C, size_t smem) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, 1);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return ncl;
+}
+
+// Plans are cached per device and shape: the occupancy queries cost far more
+// host time than a decode step's launches.
+struct CSelKey {
+    int dev, form, src, agg, B, Hkv, T_cap, r, nq, k;
+    bool operator==(const CSelKey &o) const { return !memcmp(this, &o, sizeof *this); }
+};
+struct CSelEntry {
+    CSelKey key;
+    cudaError_t err;
+    CSelPlan plan;
+};
+constexpr int kPlanCache = 64;
+CSelEntry g_cache[kPlanCache];
+int g_cache_n = 0, g_cache_next = 0;
+std::mutex g_cache_mu;
+
+cudaError_t plan_csel_uncached(int form, int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k,
+                               CSelPlan *p) {
+    if (form == 2) return cudaErrorNotSupported;
+    auto kern = pick_csel(src, r, agg);
+    if (!kern) return cudaErrorNotSupported;
+    const int tile = csel_tile(src, r);
+    const int tiles = (T_cap + tile - 1) / tile;
+    const int BH = B * Hkv;
+    // The largest power-of-two cluster (the summed histogram is split evenly
+    // over its CTAs) whose slices fit in shared memory and whose B*Hkv
+    // clusters are all resident at once (one wave).  "cluster" relaxes the
+    // one-wave condition.
+    for (int C = 16; C >= 2; C >>= 1) {
+        if (C > tiles && C > 2) continue;
+        int slice = (T_cap + C - 1) / C;
+        slice = (slice + tile - 1) / tile * tile;
+        if (slice > kMaxSlice) break;  // smaller clusters only lengthen the slices
+        const size_t smem = csel_smem(src != SRC_SCORES, src == SRC_SCORES ? 0 : r, nq, slice).total;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        const int ncl = resident_clusters(kern, C, smem);
+        if (ncl < 1) continue;
+        if (form == 0 && ncl < BH) continue;
+        p->csize = C;
+        p->slice = slice;
+        p->smem = smem;
+        p->grid_y = BH;
+        return cudaSuccess;
+    }
+    return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+cudaError_t plan_csel(int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    CSelKey key;
+    memset(&key, 0, sizeof key);
+    key.dev = dev;
+    key.form = select_form_override();
+    key.src = src;
+    key.agg = agg;
+    key.B = B;
+    key.Hkv = Hkv;
+    key.T_cap = T_cap;
+    key.r = r;
+    key.nq = nq;
+    key.k = k;
+    {
+        std::lock_guard<std::mutex> lk(g_cache_mu);
+        for (int i = 0; i < g_cache_n; ++i)
+            if (g_cache[i].key == key) {
+                if (g_cache[i].err == cudaSuccess) {
+                    // the attributes are per device and function: set them again
+                    // in case this thread planned nothing on the device yet
+                    auto kern = pick_csel(src, r, agg);
+                    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)g_cache[i].plan.smem);
+                    cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+                    *p = g_cache[i].plan;
+                }
+                return g_cache[i].err;
+            }
+    }
+    CSelPlan P{};
+    e = plan_csel_uncached(key.form, src, agg, B, Hkv, T_cap, r, nq, k, &P);
+    if (e != cudaSuccess && e != cudaErrorNotSupported) return e;  // not cached: a real failure
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    CSelEntry &slot = g_cache[g_cache_n < kPlanCache ? g_cache_n++ : (g_cache_next++ % kPlanCache)];
+    slot.key = key;
+    slot.err = e;
+    slot.plan = P;
+    if (e == cudaSuccess) *p = P;
+    return e;
+}
+
+cudaError_t launch_csel(const CSelPlan &p, const CSelArgs &a0, int src, int agg, cudaStream_t s, bool pdl) {
+    auto kern = pick_csel(src, a0.r, agg);
+    if (!kern) return cudaErrorInvalidValue;
+    CSelArgs a = a0;
+    a.csize = p.csize;
+    a.slice = p.slice;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.csize, p.grid_y);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p.csize;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace jssa

@@ -305,7 +305,7 @@ class DecodeSession:
 
     def __init__(self, K, V, P, seq_lens, k, scale, Kt=None, kt_dtype=torch.bfloat16, agg=AGG_SUM):
         _cuda(K, V, P, seq_lens)
-        self.K, self.V, self.P, self.seq_lens = K, V, P, seq_lens
+        self.K, self.V, self.P, self.seq_lens = K, V, P, seq_lens  # V None: latent cache
         self.k, self.scale, self.agg = int(k), float(scale), int(agg)
         dev = K.device
         self.Kt = build_lowrank_cache(K, P, kt_dtype) if Kt is None else Kt
@@ -346,7 +346,8 @@ class DecodeSession:
         self.q_dev.copy_(q_host, non_blocking=True)
         pos = int(self._host_pos())
         self.K[:, pos].copy_(k_new_host, non_blocking=True)
-        self.V[:, pos].copy_(v_new_host, non_blocking=True)
+        if self.V is not None:
+            self.V[:, pos].copy_(v_new_host, non_blocking=True)
         self.step(self.q_dev)
         self.out_host.copy_(self.out, non_blocking=True)
         return self.out_host
