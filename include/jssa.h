@@ -60,12 +60,14 @@
  *
  * Host state: launch plans of the selection pass are cached per device and
  * shape in host memory (mutex-protected).  The selection (jssa_topk,
- * jssa_select, jssa_decode_step) has two forms with identical results: one
- * thread-block cluster per (b, h) holding the keys of its rows in shared
- * memory, taken when all B*Hkv clusters fit on the GPU at once, and a
- * persistent streaming pass with a segment merge otherwise.  The environment
- * variable JSSA_SELECT_FORM = "cluster" or "stream" forces one form at
- * planning time (tests and measurement); size the workspace after setting it.
+ * jssa_select, jssa_decode_step) has three forms with identical results:
+ * one thread-block cluster per (b, h) holding the keys of its rows in shared
+ * memory, taken when all B*Hkv clusters fit on the GPU at once; otherwise a
+ * persistent streaming pass with a segment merge, warp-specialised for SUM
+ * over the low-rank cache, block-synchronous for the other cases.  The
+ * environment variable JSSA_SELECT_FORM = "cluster", "stream" or "scan"
+ * forces one form at planning time where it has a kernel (tests and
+ * measurement); size the workspace after setting it.
  */
 #ifndef JSSA_H
 #define JSSA_H

@@ -94,10 +94,11 @@ def test_score_parity(agg, kt):
     assert np.all(np.isnan(sg[1, :, 700:])), "entries past T_b were written"
 
 
-# Both selection forms (one cluster per (b,h) holding its keys in shared
-# memory, and the persistent streaming pass with a segment merge) must return
-# the same indices; JSSA_SELECT_FORM forces one at planning time.
-FORMS = ["auto", "cluster", "stream"]
+# Every selection form (one cluster per (b,h) holding its keys in shared
+# memory; the warp-specialised streaming pass; the block-synchronous streaming
+# pass) must return the same indices; JSSA_SELECT_FORM forces one at planning
+# time.
+FORMS = ["auto", "cluster", "stream", "scan"]
 
 
 @pytest.fixture(params=FORMS)
@@ -491,7 +492,7 @@ def test_full_size_mla_64k_b8_sampled():
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("wname", ["gqa_4k_b1", "gqa_32k_b4", "mla_64k_b8"])
+@pytest.mark.parametrize("wname", ["gqa_4k_b1", "gqa_32k_b4", "mla_64k_b8", "hybrid_global_128k_b8", "gqa_128k_b16"])
 def test_select_forms_agree_full_size(wname, monkeypatch):
     """The cluster and the streaming selection give identical index lists on
     the full-size workloads (the shapes where the automatic choice flips)."""
@@ -501,10 +502,11 @@ def test_select_forms_agree_full_size(wname, monkeypatch):
     q, K, V, P, sl = make_inputs(w, device=DEV)
     Kt = ops.build_lowrank_cache(K, P)
     res = []
-    for f in ("cluster", "stream"):
+    for f in ("cluster", "stream", "scan"):
         monkeypatch.setenv("JSSA_SELECT_FORM", f)
         res.append(ops.select(q, P, Kt, sl, w.k))
     torch.cuda.synchronize()
-    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    for r in res[1:]:
+        assert torch.equal(res[0][0], r[0]) and torch.equal(res[0][1], r[1])
     del q, K, V, Kt
     torch.cuda.empty_cache()

@@ -116,7 +116,8 @@ struct Layout {
     size_t total = 256;  // [0, 256): status word
     ScanPlan sp{};
     AttnPlan ap{};
-    bool csel = false;  // selection by one cluster per (b,h) (else the streaming form)
+    bool csel = false;   // selection by one cluster per (b,h)
+    bool wspec = false;  // warp-specialised streaming selection (else block-synchronous)
     CSelPlan cp{};
 };
 
@@ -135,8 +136,16 @@ int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, 
     }
     cudaGetLastError();
     if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the cluster selection");
-    e = plan_scan(src, MODE_SELECT, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.sp);
-    if (e != cudaSuccess) return cuda_fail(e, "planning the selection pass");
+    e = select_form_override() == 3 ? cudaErrorNotSupported
+                                    : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
+    if (e == cudaSuccess) {
+        L.wspec = true;
+    } else {
+        cudaGetLastError();
+        if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the streaming selection");
+        e = plan_scan(src, MODE_SELECT, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.sp);
+        if (e != cudaSuccess) return cuda_fail(e, "planning the selection pass");
+    }
     const size_t nc = (size_t)sh.BH * L.sp.max_seg * k;
     L.cand_key = take(L.total, nc * 4);
     L.cand_idx = take(L.total, nc * 4);
@@ -288,7 +297,7 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
     sa.r = d->r;
     sa.nq = nq;
     sa.k = k;
-    cudaError_t e = launch_scan(L.sp, sa, agg, s, true);
+    cudaError_t e = L.wspec ? launch_stream(L.sp, sa, s, true) : launch_scan(L.sp, sa, agg, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the selection pass");
     return JSSA_OK;
 }

@@ -155,6 +155,13 @@ cudaError_t launch_prep(const AppendArgs &ap, const ProjArgs &pj, cudaStream_t s
                         int kt_dtype);
 cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, ScanPlan *p);
 cudaError_t launch_scan(const ScanPlan &p, const ScanArgs &a, int agg, cudaStream_t s, bool pdl);
+// Warp-specialised streaming select (SUM over the low-rank key cache):
+// cudaErrorNotSupported where it has no kernel.
+cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int k, ScanPlan *p);
+cudaError_t launch_stream(const ScanPlan &p, const ScanArgs &a, cudaStream_t s, bool pdl);
+// Selection form forced by the environment (JSSA_SELECT_FORM): 0 automatic,
+// 1 "cluster", 2 "stream", 3 "scan".
+int select_form_override();
 cudaError_t plan_attend(int src, int kv_dtype, int d, int G, int B, int Hkv, int npos, AttnPlan *p);
 cudaError_t launch_attend(const AttnPlan &p, int src, const AttnArgs &a, int kv_dtype, int d, cudaStream_t s,
                           bool pdl);

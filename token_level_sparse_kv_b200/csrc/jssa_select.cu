@@ -409,16 +409,20 @@ int csel_tile(int src, int r) {
 // Which selection form a shape uses.  The cluster form is taken when every
 // (b,h) gets its own cluster, all resident at once, with the keys of its slice
 // in shared memory: it has no segment merge and no second wave.  Otherwise
-// (many (b,h) rows or rows too long for shared memory) the persistent
-// streaming pass is taken.  Both return the same indices.  The environment
-// variable JSSA_SELECT_FORM overrides the choice at planning time: "cluster"
-// takes the cluster form wherever its slices fit in shared memory (several
-// waves allowed), "stream" always takes the streaming form.
-static int select_form_override() {
+// (many (b,h) rows or rows too long for shared memory) a persistent streaming
+// pass is taken: the warp-specialised one for SUM over the low-rank cache,
+// the block-synchronous one for the other sources and aggregations.  All
+// return the same indices.  The environment variable JSSA_SELECT_FORM
+// overrides the choice at planning time: "cluster" takes the cluster form
+// wherever its slices fit in shared memory (several waves allowed), "stream"
+// the warp-specialised pass where it has a kernel, "scan" the
+// block-synchronous pass.
+int select_form_override() {
     const char *v = getenv("JSSA_SELECT_FORM");
     if (!v) return 0;
     if (!strcmp(v, "cluster")) return 1;
     if (!strcmp(v, "stream")) return 2;
+    if (!strcmp(v, "scan")) return 3;
     return 0;
 }
 
@@ -463,7 +467,7 @@ std::mutex g_cache_mu;
 
 cudaError_t plan_csel_uncached(int form, int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k,
                                CSelPlan *p) {
-    if (form == 2) return cudaErrorNotSupported;
+    if (form == 2 || form == 3) return cudaErrorNotSupported;
     auto kern = pick_csel(src, r, agg);
     if (!kern) return cudaErrorNotSupported;
     const int tile = csel_tile(src, r);

@@ -1,0 +1,1164 @@
+// Per-(batch, KV head) top-k selection fused with subspace scoring: the
+// warp-specialised persistent streaming form.
+//
+// Method: news item "JSSA makes token-level sparse decoding gather-free",
+// Synopsis (tokens scored in a shared low-dimensional query-key subspace, a
+// distinct selected token set per KV head) and Interpretation para 2; "Joint
+// Subspace Sparse Attention for Efficient Long-Context Decoding", Abstract
+// (distinct per-KV-head selections).
+//
+// One CTA per SM streams a contiguous range of the flattened (b,h, tile) list
+// of the low-rank key cache.  Three roles share the CTA:
+//  * a producer thread keeps a ring of 32 KiB bulk asynchronous copies in
+//    flight (full / empty mbarriers per stage, evict-first L2 hint);
+//  * 16 consumer warps score every token of a tile (the same fp32 arithmetic,
+//    lane rotation and chunk order as the score pass, so scores are
+//    bit-identical) and append the tokens whose order-preserving key beats the
+//    current threshold to an epoch buffer (two buffers, alternating epochs of
+//    >= 1024 tokens);
+//  * 4 selector warps fold each finished epoch into the running candidate set
+//    of the segment, cut it back to the best k with a radix select when it
+//    fills, and publish the k-th key (tagged with the segment) as the new
+//    threshold.  At the end of a segment they write its candidates to the
+//    workspace; the last CTA of a (b,h) to finish (arrival ticket, no waiting)
+//    merges the segments and writes the selection sorted by token index.
+// The consumers never wait for a selection: only for data, and for an epoch
+// buffer two epochs back.  Tokens of a segment arrive in ascending index order
+// and a threshold is only ever computed from finished epochs, so a token whose
+// key equals the threshold always loses to the kept entry (strict filter).
+// The order (score desc, index asc) is strict and total, so the top-k of the
+// union of per-segment top-k sets is the global top-k: the result is exactly
+// that of the score pass followed by the top-k pass.
+#include <type_traits>
+
+#include "jssa_common.cuh"
+#include "jssa_internal.h"
+
+namespace jssa {
+
+namespace {
+
+constexpr int kConsWarps = 16;
+constexpr int kCons = kConsWarps * 32;            // consumer threads
+constexpr int kSelWarps = 8;
+constexpr int kSelT = kSelWarps * 32;             // selector threads
+// Warp roles, selector first: the schedulers favour lower warp ids when
+// several warps are ready, and the selector's latency-bound steps are the
+// ones that must not wait behind the consumers' streaming work.
+constexpr int kSelBase = 0;                       // first selector thread
+constexpr int kProdBase = kSelT;                  // producer warp
+constexpr int kConsBase = kSelT + 32;             // first consumer thread
+constexpr int kThreads = kConsBase + kCons;       // 800
+constexpr int kEB = 3;                            // epoch buffers
+constexpr int kTile = 32768;                      // bytes per ring stage
+constexpr int kMaxStages = 8;
+constexpr int kBins = 2048;                       // 11-bit digits
+constexpr int kBoundary = 64;                     // boundary group ranked exactly
+constexpr int kEpochTokens = 1024;                // minimum tokens per epoch
+
+__host__ __device__ inline int npow2(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+__host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct StreamSmem {
+    size_t ring, bars, ek, ei, rk, ri, sk, si, hist, misc, total;
+};
+
+// misc words (int): [0] abort, [3] candidate count, [4..6] select results,
+// [7] boundary counter, [8] selector go/stop, [9] ticket, [10..15] select
+// scratch, [16..23] scan partials, [24] copies issued, [32..33] threshold
+// (u64), [40..42] epoch buffer counts, [44..45] smallest / largest key
+// appended to the segment's candidates, [48..63] reduction scratch.
+__host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k) {
+    StreamSmem L;
+    size_t o = 0;
+    L.ring = o;
+    o += (size_t)nstages * kTile;
+    L.bars = o;
+    o = al(o + (size_t)(2 * nstages + 2 * kEB) * 8, 16);
+    L.ek = o;
+    o = al(o + (size_t)kEB * ept * 4, 16);
+    L.ei = o;
+    o = al(o + (size_t)kEB * ept * 4, 16);
+    L.rk = o;
+    o = al(o + (size_t)cap * 4, 16);
+    L.ri = o;
+    o = al(o + (size_t)cap * 4, 16);
+    L.sk = o;
+    o = al(o + (size_t)k * 4, 16);
+    L.si = o;
+    o = al(o + (size_t)npow2(k) * 4, 16);
+    L.hist = o;
+    o = al(o + (size_t)kBins * 4, 16);
+    L.misc = o;
+    o = al(o + 64 * 4, 128);
+    L.total = o;
+    return L;
+}
+
+// ------------------------------------------------------------- selector ---
+__device__ __forceinline__ void sel_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSelT) : "memory"); }
+
+__device__ __forceinline__ unsigned lane_lt() {
+    unsigned m;
+    asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive scan over the selector threads (two selector barriers).
+__device__ __forceinline__ int sel_scan(int v, int *tmp, int st, int &total) {
+    const int lane = st & 31, w = st >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) tmp[w] = x;
+    sel_sync();
+    int pre = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < kSelWarps; ++i) {
+        const int t = tmp[i];
+        pre += i < w ? t : 0;
+        tot += t;
+    }
+    sel_sync();
+    total = tot;
+    return pre + x - v;
+}
+
+// Candidate set and scratch of the selector, in shared memory.
+struct Sel {
+    uint32_t *rk;  // candidate keys [cap]
+    int32_t *ri;   // candidate token indices [cap]
+    uint32_t *sk;  // kept keys [k]
+    int32_t *si;   // kept indices / sort scratch [npow2(k)]
+    uint32_t *hist;
+    int *misc;
+    int st;
+};
+
+__device__ __forceinline__ bool before(uint32_t ka, int32_t ia, uint32_t kb, int32_t ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+// kk-th largest of val(j) over the entries with use(j), by 8-bit radix
+// passes: returns the value, the number of entries equal to it inside the
+// top kk, and how many used entries equal it.
+template <typename Use, typename Val>
+__device__ void sel_radix(const Sel &S, int n, int kk, Use use, Val val, uint32_t &tau, int &need, int &eq) {
+    uint32_t prefix = 0u, mask = 0u;
+    int last = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int d = S.st; d < 256; d += kSelT) S.hist[d] = 0u;
+        sel_sync();
+        for (int j = S.st; j < n; j += kSelT) {
+            if (!use(j)) continue;
+            const uint32_t u = val(j);
+            if ((u & mask) == prefix) atomicAdd(&S.hist[(u >> shift) & 0xffu], 1u);
+        }
+        sel_sync();
+        // thread st owns bin 255 - st (descending)
+        static_assert(kSelT == 256, "one radix bin per selector thread");
+        const int c0 = (int)S.hist[255 - S.st];
+        int tot;
+        const int ex = sel_scan(c0, S.misc + 16, S.st, tot);
+        if (ex < kk && ex + c0 >= kk) {
+            S.misc[4] = 255 - S.st;
+            S.misc[5] = ex;
+            S.misc[6] = c0;
+        }
+        sel_sync();
+        prefix |= (uint32_t)S.misc[4] << shift;
+        mask |= 0xffu << shift;
+        kk -= S.misc[5];
+        last = S.misc[6];
+        sel_sync();
+    }
+    tau = prefix;
+    need = kk;
+    eq = last;
+}
+
+// Compact the kept entries (keep(j)) of rk/ri[0..n) into rk/ri[0..k) through
+// sk/si; returns the smallest kept key.
+template <typename Keep>
+__device__ uint32_t sel_compact(const Sel &S, int n, int k, Keep keep) {
+    unsigned *um = reinterpret_cast<unsigned *>(S.misc);
+    if (S.st == 0) {
+        S.misc[10] = 0;
+        um[11] = 0xffffffffu;
+    }
+    sel_sync();
+    const int lane = S.st & 31;
+    uint32_t kmin = 0xffffffffu;
+    for (int j0 = 0; j0 < n; j0 += kSelT) {
+        const int j = j0 + S.st;
+        uint32_t u = 0u;
+        int32_t ix = 0;
+        bool kp = false;
+        if (j < n) {
+            u = S.rk[j];
+            ix = S.ri[j];
+            kp = keep(u, ix);
+        }
+        if (kp) kmin = min(kmin, u);
+        const unsigned m = __ballot_sync(0xffffffffu, kp);
+        int base = 0;
+        if (m) {
+            const int ld = __ffs(m) - 1;
+            if (lane == ld) base = atomicAdd(&S.misc[10], __popc(m));
+            base = __shfl_sync(0xffffffffu, base, ld);
+        }
+        if (kp) {
+            const int p = base + __popc(m & lane_lt());
+            if (p < k) {
+                S.sk[p] = u;
+                S.si[p] = ix;
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+    if (lane == 0) atomicMin(&um[11], kmin);
+    sel_sync();
+    for (int j = S.st; j < k; j += kSelT) {
+        S.rk[j] = S.sk[j];
+        S.ri[j] = S.si[j];
+    }
+    const uint32_t t = um[11];
+    sel_sync();
+    return t;
+}
+
+// Keep the best k of the n > k candidates under (key desc, index asc), with
+// the candidates read from shared memory on every pass (any n).
+// Adaptive digits: the keys share every bit above the highest bit where
+// their minimum and maximum differ, so 11 bits below it give a monotone
+// histogram; the bin of the k-th key is refined by the next 11 bits while it
+// holds many entries, and a small boundary group is ranked exactly.  Large
+// groups of equal keys fall back to 8-bit passes over keys, then over
+// inverted indices.  Returns the k-th kept key (the new threshold).
+__device__ __noinline__ uint32_t sel_reduce_smem(const Sel &S, int n, int k) {
+    unsigned *um = reinterpret_cast<unsigned *>(S.misc);
+    if (S.st == 0) {
+        um[12] = 0u;
+        um[13] = 0xffffffffu;
+    }
+    sel_sync();
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int j = S.st; j < n; j += kSelT) {
+        const uint32_t u = S.rk[j];
+        lo = min(lo, u);
+        hi = max(hi, u);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if ((S.st & 31) == 0) {
+        atomicMax(&um[12], hi);
+        atomicMin(&um[13], lo);
+    }
+    sel_sync();
+    hi = um[12];
+    lo = um[13];
+    sel_sync();
+    bool general = hi == lo;
+    uint32_t pmask = 0u, pval = 0u;
+    int kk = k, mb = 0;
+    if (!general) {
+        int top = 31 - __clz((int)(hi ^ lo));
+        pmask = top == 31 ? 0u : ~((2u << top) - 1u);
+        pval = hi & pmask;
+        for (;;) {
+            const int width = top + 1 < 11 ? top + 1 : 11;
+            const int shift = top + 1 - width;
+            const uint32_t dmask = (1u << width) - 1u;
+            for (int d = S.st; d < kBins; d += kSelT) S.hist[d] = 0u;
+            sel_sync();
+            for (int j = S.st; j < n; j += kSelT) {
+                const uint32_t u = S.rk[j];
+                if ((u & pmask) == pval) atomicAdd(&S.hist[(u >> shift) & dmask], 1u);
+            }
+            sel_sync();
+            constexpr int BPT = kBins / kSelT;  // bins per thread, descending
+            const int bb = kBins - BPT * (S.st + 1);
+            int cnt[BPT];
+            int sum = 0;
+#pragma unroll
+            for (int q = 0; q < BPT; ++q) {
+                cnt[q] = (int)S.hist[bb + BPT - 1 - q];
+                sum += cnt[q];
+            }
+            int tot;
+            int ex = sel_scan(sum, S.misc + 16, S.st, tot);
+#pragma unroll
+            for (int q = 0; q < BPT; ++q) {
+                if (ex < kk && ex + cnt[q] >= kk) {
+                    S.misc[4] = bb + BPT - 1 - q;
+                    S.misc[5] = ex;
+                    S.misc[6] = cnt[q];
+                }
+                ex += cnt[q];
+            }
+            sel_sync();
+            pmask |= dmask << shift;
+            pval |= (uint32_t)S.misc[4] << shift;
+            kk -= S.misc[5];
+            mb = S.misc[6];
+            sel_sync();
+            if (kk == mb || mb <= kBoundary || shift == 0) break;
+            top = shift - 1;
+        }
+        general = kk != mb && mb > kBoundary;
+    }
+    if (general) {
+        uint32_t tau, tau2 = 0u;
+        int need, eq;
+        sel_radix(
+            S, n, k, [&](int) { return true; }, [&](int j) { return S.rk[j]; }, tau, need, eq);
+        const bool all = need == eq;
+        if (!all) {
+            int need2, eq2;
+            sel_radix(
+                S, n, need, [&](int j) { return S.rk[j] == tau; }, [&](int j) { return ~(uint32_t)S.ri[j]; },
+                tau2, need2, eq2);
+        }
+        return sel_compact(S, n, k, [&](uint32_t u, int32_t ix) {
+            return u > tau || (u == tau && (all || ~(uint32_t)ix >= tau2));
+        });
+    }
+    // boundary group: kk of its mb entries are kept, ranked exactly
+    uint32_t kstar = 0u;
+    int32_t istar = 0x7fffffff;
+    const bool whole = kk == mb;
+    if (!whole) {
+        uint32_t *bk = S.hist;
+        int32_t *bi = reinterpret_cast<int32_t *>(S.hist + kBoundary);
+        if (S.st == 0) S.misc[7] = 0;
+        sel_sync();
+        for (int j = S.st; j < n; j += kSelT) {
+            const uint32_t u = S.rk[j];
+            if ((u & pmask) == pval) {
+                const int p = atomicAdd(&S.misc[7], 1);
+                bk[p] = u;
+                bi[p] = S.ri[j];
+            }
+        }
+        sel_sync();
+        for (int i = S.st; i < mb; i += kSelT) {
+            const uint32_t ki = bk[i];
+            const int32_t ii = bi[i];
+            int r = 0;
+            for (int j = 0; j < mb; ++j) r += before(bk[j], bi[j], ki, ii);
+            if (r == kk - 1) {
+                um[14] = ki;
+                S.misc[15] = ii;
+            }
+        }
+        sel_sync();
+        kstar = um[14];
+        istar = S.misc[15];
+        sel_sync();
+    }
+    return sel_compact(S, n, k, [&](uint32_t u, int32_t ix) {
+        const uint32_t m = u & pmask;
+        return m > pval || (m == pval && (whole || !before(kstar, istar, u, ix)));
+    });
+}
+
+// The same reduction with the keys held in registers (n <= kRegKeys *
+// kSelT): one shared-memory read of the candidates, one histogram pass per
+// level, and the survivors written back in place after all reads are done.
+constexpr int kRegKeys = 8;
+__device__ uint32_t sel_reduce(const Sel &S, int n, int k) {
+    if (n > kRegKeys * kSelT) return sel_reduce_smem(S, n, k);
+    const int st = S.st, lane = st & 31, w = st >> 5;
+    unsigned *um = reinterpret_cast<unsigned *>(S.misc);
+    uint32_t u[kRegKeys];
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+        const int j = st + q * kSelT;
+        u[q] = j < n ? S.rk[j] : 0u;
+        if (j < n) {
+            lo = min(lo, u[q]);
+            hi = max(hi, u[q]);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        um[48 + w] = lo;
+        um[56 + w] = hi;
+    }
+    if (st == 0) S.misc[7] = 0;  // boundary-group counter
+    sel_sync();
+#pragma unroll
+    for (int i = 0; i < kSelWarps; ++i) {
+        lo = min(lo, um[48 + i]);
+        hi = max(hi, um[56 + i]);
+    }
+    if (hi == lo) return sel_reduce_smem(S, n, k);  // every key equal: order by index alone
+    int top = 31 - __clz((int)(hi ^ lo));
+    uint32_t pmask = top == 31 ? 0u : ~((2u << top) - 1u), pval = hi & pmask;
+    int kk = k, mb = 0;
+    for (;;) {
+        const int width = top + 1 < 11 ? top + 1 : 11;
+        const int shift = top + 1 - width;
+        const uint32_t dmask = (1u << width) - 1u;
+        constexpr int BPT = kBins / kSelT;
+        uint4 *h4 = reinterpret_cast<uint4 *>(S.hist);
+#pragma unroll
+        for (int q = 0; q < BPT / 4; ++q) h4[st * (BPT / 4) + q] = make_uint4(0u, 0u, 0u, 0u);
+        sel_sync();
+#pragma unroll
+        for (int q = 0; q < kRegKeys; ++q)
+            if (st + q * kSelT < n && (u[q] & pmask) == pval) atomicAdd(&S.hist[(u[q] >> shift) & dmask], 1u);
+        sel_sync();
+        // descending scan: thread st owns bins [kBins - BPT (st+1), kBins - BPT st)
+        const int bb = kBins - BPT * (st + 1);
+        int cnt[BPT];
+        int sum = 0;
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) {
+            cnt[q] = (int)S.hist[bb + BPT - 1 - q];
+            sum += cnt[q];
+        }
+        int tot;
+        int ex = sel_scan(sum, S.misc + 16, st, tot);
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) {
+            if (ex < kk && ex + cnt[q] >= kk) {
+                S.misc[4] = bb + BPT - 1 - q;
+                S.misc[5] = ex;
+                S.misc[6] = cnt[q];
+            }
+            ex += cnt[q];
+        }
+        sel_sync();
+        pmask |= dmask << shift;
+        pval |= (uint32_t)S.misc[4] << shift;
+        kk -= S.misc[5];
+        mb = S.misc[6];
+        if (kk == mb || mb <= kBoundary || shift == 0) break;
+        top = shift - 1;
+    }
+    const bool whole = kk == mb;
+    if (!whole && mb > kBoundary) return sel_reduce_smem(S, n, k);  // a large group of equal keys
+    uint32_t kstar = 0u;
+    int32_t istar = 0x7fffffff;
+    if (!whole) {
+        // boundary group: gather it (keys from registers) and rank it exactly
+        uint32_t *bk = S.hist;
+        int32_t *bi = reinterpret_cast<int32_t *>(S.hist + kBoundary);
+#pragma unroll
+        for (int q = 0; q < kRegKeys; ++q) {
+            const int j = st + q * kSelT;
+            if (j < n && (u[q] & pmask) == pval) {
+                const int p = atomicAdd(&S.misc[7], 1);
+                bk[p] = u[q];
+                bi[p] = S.ri[j];
+            }
+        }
+        sel_sync();
+        if (st < mb) {
+            const uint32_t ki = bk[st];
+            const int32_t ii = bi[st];
+            int r = 0;
+            for (int j = 0; j < mb; ++j) r += before(bk[j], bi[j], ki, ii);
+            if (r == kk - 1) {
+                um[14] = ki;
+                S.misc[15] = ii;
+            }
+        }
+        sel_sync();
+        kstar = um[14];
+        istar = S.misc[15];
+    }
+    // compaction: read the kept indices, scan the counts, write in place
+    int32_t ix[kRegKeys];
+    unsigned keep = 0u;
+    int c = 0;
+    uint32_t kmin = 0xffffffffu;
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+        const int j = st + q * kSelT;
+        ix[q] = 0;
+        if (j < n) {
+            const uint32_t m = u[q] & pmask;
+            bool kp = m > pval;
+            if (m == pval) {
+                ix[q] = S.ri[j];
+                kp = whole || !before(kstar, istar, u[q], ix[q]);
+            } else if (kp) {
+                ix[q] = S.ri[j];
+            }
+            if (kp) {
+                keep |= 1u << q;
+                ++c;
+                kmin = min(kmin, u[q]);
+            }
+        }
+    }
+    int tot;
+    int pos = sel_scan(c, S.misc + 16, st, tot);  // its barriers also end every read above
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+        if (keep & (1u << q)) {
+            S.rk[pos] = u[q];
+            S.ri[pos] = ix[q];
+            ++pos;
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+    if (lane == 0) um[48 + w] = kmin;
+    sel_sync();
+#pragma unroll
+    for (int i = 0; i < kSelWarps; ++i) kmin = min(kmin, um[48 + i]);
+    sel_sync();
+    return kmin;
+}
+
+// Mid-segment cut (n <= kRegKeys * kSelT): one histogram of the keys over
+// [lo, hi] (the range the appends tracked) in 2048 equal bins, then keep the
+// bins at and above the one holding the k-th key.  At least k kept keys are
+// strictly above the returned threshold-1 edge, so a later token (higher
+// index) whose key is at or below the threshold can never enter the top k;
+// the kept set exceeds k by at most the population of one fine bin.  Returns
+// the threshold (keys > it survive) and sets `kept`.
+__device__ uint32_t sel_trim(const Sel &S, int n, int k, uint32_t lo, uint32_t hi, int &kept) {
+    const int st = S.st, lane = st & 31;
+    uint32_t u[kRegKeys];
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+        const int j = st + q * kSelT;
+        u[q] = j < n ? S.rk[j] : 0u;
+    }
+    const uint32_t span = hi - lo;
+    const int bits = span == 0u ? 0 : 32 - __clz((int)span);
+    const int sh = bits > 11 ? bits - 11 : 0;
+    constexpr int BPT = kBins / kSelT;
+    uint4 *h4 = reinterpret_cast<uint4 *>(S.hist);
+#pragma unroll
+    for (int q = 0; q < BPT / 4; ++q) h4[st * (BPT / 4) + q] = make_uint4(0u, 0u, 0u, 0u);
+    sel_sync();
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q)
+        if (st + q * kSelT < n && u[q] >= lo) atomicAdd(&S.hist[min((u[q] - lo) >> sh, (uint32_t)(kBins - 1))], 1u);
+    sel_sync();
+    const int bb = kBins - BPT * (st + 1);
+    int cnt[BPT];
+    int sum = 0;
+#pragma unroll
+    for (int q = 0; q < BPT; ++q) {
+        cnt[q] = (int)S.hist[bb + BPT - 1 - q];
+        sum += cnt[q];
+    }
+    int tot;
+    int ex = sel_scan(sum, S.misc + 16, st, tot);
+#pragma unroll
+    for (int q = 0; q < BPT; ++q) {
+        if (ex < k && ex + cnt[q] >= k) S.misc[4] = bb + BPT - 1 - q;
+        ex += cnt[q];
+    }
+    sel_sync();
+    const uint32_t edge = lo + ((uint32_t)S.misc[4] << sh);  // lowest key of the k-th key's bin
+    if (tot < k || edge == 0u) {  // fewer than k keys in range, or nothing below key 0 to cut
+        kept = n;
+        sel_sync();
+        return 0u;
+    }
+    const uint32_t thr = edge - 1u;
+    int32_t ix[kRegKeys];
+    unsigned keep = 0u;
+    int c = 0;
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+        const int j = st + q * kSelT;
+        ix[q] = 0;
+        if (j < n && u[q] > thr) {
+            ix[q] = S.ri[j];
+            keep |= 1u << q;
+            ++c;
+        }
+    }
+    int pos = sel_scan(c, S.misc + 16, st, tot);  // its barriers also end every read above
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+        if (keep & (1u << q)) {
+            S.rk[pos] = u[q];
+            S.ri[pos] = ix[q];
+            ++pos;
+        }
+    }
+    (void)lane;
+    kept = tot;
+    sel_sync();
+    return thr;
+}
+
+// Sort a[0..n) ascending (bitonic over npow2(n), padded with INT_MAX).
+__device__ void sel_sort(int32_t *a, int n, int st) {
+    const int P = npow2(n < 1 ? 1 : n);
+    for (int j = n + st; j < P; j += kSelT) a[j] = 0x7fffffff;
+    sel_sync();
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = st; i < P / 2; i += kSelT) {
+                const int lo = 2 * stride * (i / stride) + (i % stride);
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const int32_t x = a[lo], y = a[hi];
+                if ((x > y) == up) {
+                    a[lo] = y;
+                    a[hi] = x;
+                }
+            }
+            sel_sync();
+        }
+    }
+}
+
+// Bounded wait that also gives up when another role raised the abort flag.
+// The thread is parked in the hardware between polls (up to 20 us per poll),
+// so waiting warps do not take issue slots from the working ones.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0; it < (1u << 20); ++it) {
+        if (mbar_try_wait_for(bar, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > 2000000000ull) return false;
+    }
+    return false;
+}
+
+// Tile cursor over a CTA's range: (b,h) row and tile index within the row of
+// the current tile, advanced without divisions.  An epoch ends after E tiles
+// of one segment, at a segment end, or at the end of the range; consumers and
+// selector walk the range identically.
+struct Cursor {
+    int bh, t, tpb;
+    __device__ void next() {
+        if (++t == tpb) {
+            t = 0;
+            ++bh;
+        }
+    }
+    __device__ bool seg_last(int i, int ntiles) const { return i == ntiles - 1 || t + 1 == tpb; }
+};
+
+// Ring position: stage of the current tile and the parity of its phase.
+struct RingPos {
+    int s = 0, n;
+    uint32_t ph = 0u;
+    __device__ explicit RingPos(int stages) : n(stages) {}
+    __device__ void next() {
+        if (++s == n) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+};
+
+// End of a segment (selector): cut to k, publish, and merge if this CTA is
+// the last of the (b,h) to finish.
+__device__ void sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long long cta, int ept, int cap) {
+    if (n > a.k) {
+        sel_reduce(S, n, a.k);
+        n = a.k;
+    }
+    const int tpb = a.tiles_per_bh;
+    const long long first = (long long)bh * tpb;
+    const long long c_first = ((first + 1) * a.grid - 1) / a.total_tiles;
+    const long long c_last = ((first + tpb) * a.grid - 1) / a.total_tiles;
+    const int slot = (int)(cta - c_first), nseg = (int)(c_last - c_first + 1);
+    const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
+    for (int j = S.st; j < n; j += kSelT) {
+        a.cand_key[cb + j] = S.rk[j];
+        a.cand_idx[cb + j] = S.ri[j];
+    }
+    if (S.st == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
+    __threadfence();
+    sel_sync();
+    if (S.st == 0) S.misc[9] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
+    sel_sync();
+    const bool last = S.misc[9] != 0;
+    sel_sync();
+    if (!last) return;
+    __threadfence();
+    // merge: segments in ascending token order, chunks of at most ept entries;
+    // equal keys stay candidates (order inside a segment is arbitrary)
+    if (S.st == 0) S.misc[3] = 0;
+    sel_sync();
+    int m = 0;
+    bool valid = false;
+    uint32_t thr = 0u;
+    const int lane = S.st & 31;
+    for (int s = 0; s < nseg; ++s) {
+        const int cnt = __ldcg(a.cand_cnt + (size_t)bh * a.max_seg + s);
+        const size_t base = ((size_t)bh * a.max_seg + s) * a.k;
+        for (int off = 0; off < cnt; off += ept) {
+            if (m > cap - ept) {
+                thr = sel_reduce(S, m, a.k);
+                valid = true;
+                m = a.k;
+                if (S.st == 0) S.misc[3] = m;
+                sel_sync();
+            }
+            const int c = min(ept, cnt - off);
+            for (int j0 = 0; j0 < c; j0 += kSelT) {
+                const int j = j0 + S.st;
+                uint32_t u = 0u;
+                int32_t ix = 0;
+                if (j < c) {
+                    u = __ldcg(a.cand_key + base + off + j);
+                    ix = __ldcg(a.cand_idx + base + off + j);
+                }
+                const bool take = j < c && (!valid || u >= thr);
+                const unsigned msk = __ballot_sync(0xffffffffu, take);
+                int b0 = 0;
+                if (msk) {
+                    const int ld = __ffs(msk) - 1;
+                    if (lane == ld) b0 = atomicAdd(&S.misc[3], __popc(msk));
+                    b0 = __shfl_sync(0xffffffffu, b0, ld);
+                }
+                if (take) {
+                    const int p = b0 + __popc(msk & lane_lt());
+                    S.rk[p] = u;
+                    S.ri[p] = ix;
+                }
+            }
+            sel_sync();
+            m = S.misc[3];
+            sel_sync();
+        }
+    }
+    if (m > a.k) {
+        sel_reduce(S, m, a.k);
+        m = a.k;
+    }
+    for (int j = S.st; j < m; j += kSelT) S.si[j] = S.ri[j];
+    sel_sync();
+    sel_sort(S.si, m, S.st);
+    for (int j = S.st; j < a.k; j += kSelT) a.idx_out[(size_t)bh * a.k + j] = j < m ? S.si[j] : -1;
+    if (S.st == 0) {
+        if (a.count_out) a.count_out[bh] = m;
+        a.counters[bh] = 0u;
+    }
+    sel_sync();
+}
+
+template <int SRC, int R>
+__global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) {
+    using KT = typename std::conditional<SRC == SRC_KT_FP32, float, __nv_bfloat16>::type;
+    constexpr int ES = SRC == SRC_KT_FP32 ? 4 : 2;
+    constexpr int ROWB = R * ES;                  // bytes per token
+    constexpr int TPB = ROWB > 64 ? 64 : ROWB;    // bytes of a token per thread
+    constexpr int LPT = ROWB / TPB;               // lanes per token
+    constexpr int CPT = TPB / 16;                 // 16-byte chunks per thread
+    constexpr int EPL = 16 / ES;                  // elements per chunk
+    constexpr int TILE = kTile / ROWB;            // tokens per tile
+    constexpr int TPP = kCons / LPT;              // tokens per pass
+    constexpr int PASSES = TILE / TPP;
+    constexpr int QN = CPT * EPL;
+    constexpr int E = TILE >= kEpochTokens ? 1 : kEpochTokens / TILE;  // tiles per epoch
+    constexpr int EPT = E * TILE;                                      // tokens per epoch
+    static_assert(LPT >= 1 && LPT <= 32 && (LPT & (LPT - 1)) == 0, "lanes per token");
+    static_assert(CPT >= 1 && CPT <= 4, "chunks per thread");
+    static_assert(PASSES >= 1 && TILE % TPP == 0, "tile / pass");
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int S_ = a.nstages;
+    const StreamSmem L = stream_smem(S_, EPT, a.cap, a.k);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
+    uint64_t *empty = full + S_;
+    uint64_t *efull = empty + S_;  // [kEB]
+    uint64_t *efree = efull + kEB; // [kEB]
+    uint32_t *ek = reinterpret_cast<uint32_t *>(smem + L.ek);
+    int32_t *ei = reinterpret_cast<int32_t *>(smem + L.ei);
+    int *misc = reinterpret_cast<int *>(smem + L.misc);
+    volatile int *abort_flag = misc;
+    volatile unsigned long long *thr_word = reinterpret_cast<volatile unsigned long long *>(misc + 32);
+
+    const int tid = threadIdx.x, lane = tid & 31;
+    const long long cta = blockIdx.x;
+    const long long x_begin = cta * a.total_tiles / a.grid;
+    const long long x_end = (cta + 1) * a.total_tiles / a.grid;
+    const int ntiles = (int)(x_end - x_begin);
+    Cursor c0;
+    c0.tpb = a.tiles_per_bh;
+    c0.bh = (int)(x_begin / c0.tpb);
+    c0.t = (int)(x_begin - (long long)c0.bh * c0.tpb);
+
+    if (tid == 0) {
+        for (int s = 0; s < S_; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsWarps);
+        }
+        for (int p = 0; p < kEB; ++p) {
+            mbar_init(&efull[p], kConsWarps);
+            mbar_init(&efree[p], 1);
+            misc[40 + p] = 0;
+        }
+        fence_barrier_init();
+        misc[0] = 0;
+        misc[3] = 0;
+        misc[44] = (int)0xffffffffu;
+        misc[45] = 0;
+        *thr_word = 0ull;
+    }
+    __syncthreads();
+    pdl_trigger();
+    pdl_wait();
+
+    if (tid >= kProdBase && tid < kConsBase) {
+        // ------------------------------------------------------ producer
+        if (tid == kProdBase) {
+            const char *src = static_cast<const char *>(a.src);
+            const uint64_t pol = policy_evict_first();
+            int issued = 0;
+            Cursor cur = c0;
+            RingPos rp(S_);
+            int Tb = 0;
+            for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
+                const int s = rp.s;
+                if (i >= S_ && !wait_or_abort(&empty[s], rp.ph ^ 1u, abort_flag)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int bh = cur.bh, t0 = cur.t * TILE;
+                if (i == 0 || cur.t == 0) Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, nullptr);
+                const int n = min(TILE, Tb - t0);
+                if (n > 0) {
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)n * ROWB);
+                    bulk_g2s(smem + L.ring + (size_t)s * kTile, src + ((size_t)bh * a.T_cap + t0) * ROWB,
+                             (uint32_t)n * ROWB, &full[s], pol);
+                } else {
+                    mbar_arrive(&full[s]);
+                }
+                issued = i + 1;
+            }
+            misc[24] = issued;
+        }
+    } else if (tid >= kConsBase) {
+        // ------------------------------------------------------ consumers
+        const int ct = tid - kConsBase;  // consumer thread index
+        const int sub = ct % LPT;
+        const int rot = CPT == 4 ? (lane >> 1) & 3 : (CPT == 2 ? (lane >> 2) & 1 : 0);
+        float qreg[QN];
+#pragma unroll
+        for (int e = 0; e < QN; ++e) qreg[e] = 0.f;
+        int Tb = 0, e = 0, epos = 0, p = 0;
+        uint32_t eph = 0u;  // use parity of epoch buffer p
+        uint32_t tag = 0u;
+        Cursor cur = c0;
+        RingPos rp(S_);
+        for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
+            const int bh = cur.bh, t = cur.t, s = rp.s;
+            if (i == 0 || t == 0) {
+                Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, ct == 0 ? a.status : nullptr);
+                tag = (uint32_t)bh + 1u;
+                const float *qp = a.qproj + (size_t)bh * R;  // written by the preceding kernel: read through L2
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    const int ch = sub * CPT + ((c + rot) % CPT);
+#pragma unroll
+                    for (int x = 0; x < EPL; ++x) qreg[c * EPL + x] = __ldcg(qp + ch * EPL + x);
+                }
+            }
+            if (epos == 0 && e >= kEB) {
+                bool ok = wait_or_abort(&efree[p], eph ^ 1u, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+            {
+                bool ok = wait_or_abort(&full[s], rp.ph, abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+            const int t0 = t * TILE;
+            const int n = max(0, min(TILE, Tb - t0));
+            const unsigned long long tw = *thr_word;
+            const bool use = (uint32_t)(tw >> 32) == tag;
+            const uint32_t tk = (uint32_t)tw;
+            const unsigned char *st = smem + L.ring + (size_t)s * kTile;
+#pragma unroll
+            for (int ps = 0; ps < PASSES; ++ps) {
+                const int tt = ps * TPP + ct / LPT;
+                const bool live = tt < n;
+                const unsigned char *row = st + (size_t)tt * ROWB + sub * TPB;
+                float pc[CPT];
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (live) v = *reinterpret_cast<const uint4 *>(row + ((c + rot) % CPT) * 16);
+                    float kf[EPL];
+                    Vec16<KT>::unpack(v, kf);
+                    float acc = 0.f;
+#pragma unroll
+                    for (int x = 0; x < EPL; ++x) acc = fmaf(kf[x], qreg[c * EPL + x], acc);
+                    pc[c] = acc;
+                }
+                float sc;
+                if constexpr (CPT == 4) sc = (pc[0] + pc[2]) + (pc[1] + pc[3]);
+                else if constexpr (CPT == 2) sc = pc[0] + pc[1];
+                else sc = pc[0];
+#pragma unroll
+                for (int off = 1; off < LPT; off <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, off);
+                const uint32_t key = score_key(sc);
+                const bool take = live && sub == 0 && (!use || key > tk);
+                const unsigned msk = __ballot_sync(0xffffffffu, take);
+                if (msk) {
+                    const int ld = __ffs(msk) - 1;
+                    int b0 = 0;
+                    if (lane == ld) b0 = atomicAdd(&misc[40 + p], __popc(msk));
+                    b0 = __shfl_sync(0xffffffffu, b0, ld);
+                    if (take) {
+                        const int q = b0 + __popc(msk & lane_lt());
+                        ek[p * EPT + q] = key;
+                        ei[p * EPT + q] = t0 + tt;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            if (epos == E - 1 || cur.seg_last(i, ntiles)) {
+                if (lane == 0) mbar_arrive(&efull[p]);
+                ++e;
+                epos = 0;
+                if (++p == kEB) {
+                    p = 0;
+                    eph ^= 1u;
+                }
+            } else {
+                ++epos;
+            }
+        }
+    } else {
+        // ------------------------------------------------------ selector
+        Sel S;
+        S.rk = reinterpret_cast<uint32_t *>(smem + L.rk);
+        S.ri = reinterpret_cast<int32_t *>(smem + L.ri);
+        S.sk = reinterpret_cast<uint32_t *>(smem + L.sk);
+        S.si = reinterpret_cast<int32_t *>(smem + L.si);
+        S.hist = reinterpret_cast<uint32_t *>(smem + L.hist);
+        S.misc = misc;
+        S.st = tid - kSelBase;
+        const int slane = S.st & 31;
+        int epos = 0, m = 0, p = 0;
+        uint32_t eph = 0u;
+        bool valid = false;
+        uint32_t thr = 0u;
+        Cursor cur = c0;
+        for (int i = 0; i < ntiles; ++i, cur.next()) {
+            const bool send = cur.seg_last(i, ntiles);
+            if (!(epos == E - 1 || send)) {
+                ++epos;
+                continue;
+            }
+            epos = 0;
+            if (S.st == 0) {
+                // one thread waits; the others are parked at the barrier
+                const bool ok = wait_or_abort(&efull[p], eph, abort_flag);
+                if (!ok) *abort_flag = 1;
+                misc[8] = *abort_flag;
+            }
+            sel_sync();
+            if (misc[8]) break;
+            const int ne = misc[40 + p];
+            for (int j0 = 0; j0 < ne; j0 += kSelT) {
+                const int j = j0 + S.st;
+                uint32_t u = 0u;
+                int32_t ix = 0;
+                if (j < ne) {
+                    u = ek[p * EPT + j];
+                    ix = ei[p * EPT + j];
+                }
+                const bool take = j < ne && (!valid || u > thr);
+                const unsigned msk = __ballot_sync(0xffffffffu, take);
+                int b0 = 0;
+                if (msk) {
+                    const int ld = __ffs(msk) - 1;
+                    uint32_t mn = take ? u : 0xffffffffu, mx = take ? u : 0u;
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) {
+                        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                    }
+                    if (slane == ld) {
+                        b0 = atomicAdd(&misc[3], __popc(msk));
+                        atomicMin(reinterpret_cast<unsigned *>(&misc[44]), mn);
+                        atomicMax(reinterpret_cast<unsigned *>(&misc[45]), mx);
+                    }
+                    b0 = __shfl_sync(0xffffffffu, b0, ld);
+                }
+                if (take) {
+                    const int q = b0 + __popc(msk & lane_lt());
+                    S.rk[q] = u;
+                    S.ri[q] = ix;
+                }
+            }
+            sel_sync();
+            m = misc[3];
+            if (S.st == 0) {
+                misc[40 + p] = 0;
+                mbar_arrive(&efree[p]);  // the epoch buffer may be refilled
+            }
+            if (++p == kEB) {
+                p = 0;
+                eph ^= 1u;
+            }
+            const int bh = cur.bh;
+            if (send) {
+                sel_finish(a, S, m, bh, cta, EPT, a.cap);
+                m = 0;
+                valid = false;
+                if (S.st == 0) {
+                    misc[3] = 0;
+                    misc[44] = (int)0xffffffffu;
+                    misc[45] = 0;
+                }
+                sel_sync();
+            } else if ((!valid && m > a.k) || m > a.cap - EPT) {
+                const uint32_t lo = valid ? thr + 1u : (uint32_t)misc[44], hi = (uint32_t)misc[45];
+                uint32_t t = thr;
+                int kept = m;
+                bool done = false;
+                if (m <= kRegKeys * kSelT) {
+                    t = sel_trim(S, m, a.k, lo, hi, kept);
+                    done = kept <= a.cap - EPT;
+                }
+                if (!done) {  // too many keys for registers, or one bin too full to make room
+                    t = sel_reduce(S, kept, a.k);
+                    kept = a.k;
+                }
+                m = kept;
+                if (t > thr || !valid) {
+                    thr = t;
+                    valid = true;
+                }
+                if (S.st == 0) {
+                    misc[3] = m;
+                    misc[44] = (int)(thr + 1u);
+                    *thr_word = ((unsigned long long)((uint32_t)bh + 1u) << 32) | thr;
+                }
+                sel_sync();
+            }
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        if (tid == kProdBase) {
+            if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+            // let the copies already in flight land before the CTA exits
+            const int issued = misc[24];
+            for (int i = issued - S_ > 0 ? issued - S_ : 0; i < issued; ++i)
+                (void)mbar_wait_bounded(&full[i % S_], (uint32_t)(i / S_) & 1u);
+        }
+        __syncthreads();
+    }
+}
+
+template <int SRC>
+void (*pick_r(int r))(ScanArgs) {
+    switch (r) {
+        case 8: return stream_select_kernel<SRC, 8>;
+        case 16: return stream_select_kernel<SRC, 16>;
+        case 32: return stream_select_kernel<SRC, 32>;
+        case 64: return stream_select_kernel<SRC, 64>;
+        case 128: return stream_select_kernel<SRC, 128>;
+        default: return nullptr;
+    }
+}
+
+void (*pick_stream(int src, int r))(ScanArgs) {
+    if (src == SRC_KT_BF16) return pick_r<SRC_KT_BF16>(r);
+    if (src == SRC_KT_FP32) return pick_r<SRC_KT_FP32>(r);
+    return nullptr;
+}
+
+}  // namespace
+
+// Plan of the warp-specialised form: SUM aggregation over the low-rank key
+// cache (the decode-step path).  cudaErrorNotSupported for other forms.
+cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int k, ScanPlan *p) {
+    if (agg != JSSA_AGG_SUM) return cudaErrorNotSupported;
+    auto kern = pick_stream(src, r);
+    if (!kern) return cudaErrorNotSupported;
+    const int rowb = r * (src == SRC_KT_FP32 ? 4 : 2);
+    const int tile = kTile / rowb;
+    const int ept = tile >= kEpochTokens ? tile : kEpochTokens;
+    ScanPlan P;
+    P.src = src;
+    P.mode = MODE_SELECT;
+    P.tile_tokens = tile;
+    P.tiles_per_bh = (T_cap + tile - 1) / tile;
+    P.total_tiles = (long long)B * Hkv * P.tiles_per_bh;
+    P.cap = k + 2 * ept;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int optin = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    int ns = kMaxStages;
+    while (ns >= 3 && stream_smem(ns, ept, P.cap, k).total > (size_t)optin) --ns;
+    if (ns < 3) return cudaErrorNotSupported;
+    P.nstages = ns;
+    P.smem = stream_smem(ns, ept, P.cap, k).total;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, P.smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorNotSupported;
+    long long g = device_sm_count();
+    if (g > P.total_tiles) g = P.total_tiles;
+    if (g < 1) g = 1;
+    P.grid = (int)g;
+    int ms = 1;
+    const long long BH = (long long)B * Hkv;
+    for (long long bh = 0; bh < BH; ++bh) {
+        const long long f = bh * P.tiles_per_bh, l = f + P.tiles_per_bh - 1;
+        const long long cf = ((f + 1) * P.grid - 1) / P.total_tiles;
+        const long long cl = ((l + 1) * P.grid - 1) / P.total_tiles;
+        if (cl - cf + 1 > ms) ms = (int)(cl - cf + 1);
+    }
+    P.max_seg = ms;
+    *p = P;
+    return cudaSuccess;
+}
+
+cudaError_t launch_stream(const ScanPlan &p, const ScanArgs &a0, cudaStream_t s, bool pdl) {
+    auto kern = pick_stream(p.src, a0.r);
+    if (!kern) return cudaErrorInvalidValue;
+    if (p.total_tiles <= 0) return cudaSuccess;
+    ScanArgs a = a0;
+    a.tile_tokens = p.tile_tokens;
+    a.tiles_per_bh = p.tiles_per_bh;
+    a.total_tiles = p.total_tiles;
+    a.grid = p.grid;
+    a.max_seg = p.max_seg;
+    a.cap = p.cap;
+    a.nstages = p.nstages;
+    return launch_kernel(kern, dim3(p.grid), dim3(kThreads), p.smem, s, pdl, a);
+}
+
+}  // namespace jssa
