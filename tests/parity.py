@@ -54,8 +54,10 @@ def check_append(Kt_gpu: torch.Tensor, K_host, P_host, pos, n_new):
         ulp = np.ldexp(1.0, np.maximum(np.frexp(np.abs(e))[1] - 8, -133))
         # one rounding of a value within the fp32 accumulation error of the exact sum
         assert np.all(np.abs(gv - e) <= ulp + acc_err), "a bf16 value is further than one rounding from the sum"
-        frac = np.mean(g != r)
-        assert frac <= 1e-3, "%.4f%% of elements differ from round-to-nearest-even" % (100 * frac)
+        # the rate of rounding-boundary cases is a statistical bound: a
+        # sample of a few hundred elements may hold one
+        ndiff = int(np.sum(g != r))
+        assert ndiff <= max(1, 1e-3 * g.size), "%d of %d elements differ from round-to-nearest-even" % (ndiff, g.size)
     else:
         assert np.all(np.abs(g.astype(np.float64) - e) <= acc_err + np.abs(e) * 2.0**-24)
     return got

@@ -296,6 +296,46 @@ def test_decode_step_end_to_end(agg):
                 assert np.abs(o[b, h * G:(h + 1) * G] - out_or[b, h * G:(h + 1) * G]).max() <= 2e-2
 
 
+@pytest.mark.parametrize("shape", ["d128_g4", "d256_g8_r64", "d128_g16", "d128_g1", "ragged"])
+def test_fused_decode_step_matches_three_launch_and_oracle(shape, monkeypatch):
+    """The one-launch decode step (append and folded query in the streaming
+    kernel's prologue, attention in its epilogue) against the three-launch
+    step and the oracle: same appended rows and selections bit for bit, outputs
+    within the bf16 tolerance."""
+    monkeypatch.setenv("JSSA_SELECT_FORM", "stream")
+    if shape == "d128_g4":
+        w, sl = W(B=3, T=20000, k=256, seed=80), [20000, 19999, 7000]
+    elif shape == "d256_g8_r64":
+        w, sl = W(B=2, Hq=16, Hkv=2, d=256, r=64, T=9000, k=256, seed=81), [9000, 4321]
+    elif shape == "d128_g16":
+        w, sl = W(B=2, Hq=32, Hkv=2, T=5000, k=300, seed=82), [5000, 100]
+    elif shape == "d128_g1":
+        w, sl = W(B=2, Hq=4, Hkv=4, T=3000, k=64, seed=83), [3000, 1]
+    else:
+        w, sl = W(B=4, T=12000, k=128, seed=84), [12000, 0, 1, 6001]
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    pos = (slh - 1).clamp_min(0)
+    Kt0 = ops.build_lowrank_cache(Kd, Pd)
+    for b in range(w.B):
+        Kt0[b, :, int(pos[b])] = 0
+    Kt1 = Kt0.clone()
+    monkeypatch.delenv("JSSA_FUSED_STEP", raising=False)
+    out1, lse1, idx1, cnt1 = ops.decode_step(qd, Kd, Vd, Pd, Kt0, sld, pos.to(DEV), w.k, w.scale)
+    monkeypatch.setenv("JSSA_FUSED_STEP", "0")
+    out2, lse2, idx2, cnt2 = ops.decode_step(qd, Kd, Vd, Pd, Kt1, sld, pos.to(DEV), w.k, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(Kt0, Kt1)
+    assert torch.equal(idx1, idx2) and torch.equal(cnt1, cnt2)
+    assert (out1.float() - out2.float()).abs().max().item() <= 2e-2
+    l1, l2 = host(lse1).double().numpy(), host(lse2).double().numpy()
+    assert np.array_equal(np.isinf(l1), np.isinf(l2))
+    fin = np.isfinite(l1)
+    assert np.abs(l1[fin] - l2[fin]).max(initial=0.0) <= 1e-3
+    check_append(Kt0, K, P, pos.tolist(), 1)
+    ref_o, ref_l = oracle.attend(q, K, V, host(idx1), host(cnt1), slh, w.scale)
+    check_attention(out1, lse1, ref_o, ref_l, torch.bfloat16)
+
+
 # -------------------------------------------------------------- edge cases
 def test_empty_and_short_sequences():
     w = W(B=3, T=300, k=64, seed=50)

@@ -2,6 +2,7 @@
 // workspace layout and kernel launches.  No allocation, no synchronisation.
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -118,6 +119,8 @@ struct Layout {
     AttnPlan ap{};
     bool csel = false;   // selection by one cluster per (b,h)
     bool wspec = false;  // warp-specialised streaming selection (else block-synchronous)
+    bool fused = false;  // decode step in one launch of the streaming kernel
+    ScanPlan fp{};
     CSelPlan cp{};
 };
 
@@ -171,6 +174,13 @@ int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout
     return JSSA_OK;
 }
 
+// The fused decode step can be switched off with JSSA_FUSED_STEP=0 (tests of
+// the three-launch form and measurement).
+bool fused_step_allowed() {
+    const char *v = getenv("JSSA_FUSED_STEP");
+    return !(v && v[0] == '0');
+}
+
 int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L) {
     L = Layout();
     int st = JSSA_OK;
@@ -201,6 +211,16 @@ int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, in
             L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
             st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L);
             if (st == JSSA_OK) st = layout_attend(d, sh, ATT_INDEXED, k, L);
+            if (st == JSSA_OK && L.wspec && !sh.latent && agg == JSSA_AGG_SUM && d->kv_dtype == JSSA_BF16 &&
+                d->kt_dtype == JSSA_BF16 && fused_step_allowed()) {
+                cudaError_t e = plan_step_fused(d->B, d->Hkv, d->Hq, d->d, d->T_cap, d->r, k, &L.fp);
+                if (e == cudaSuccess && L.fp.max_seg <= L.sp.max_seg) {
+                    L.fused = true;
+                } else {
+                    cudaGetLastError();
+                    if (e != cudaSuccess && e != cudaErrorNotSupported) return cuda_fail(e, "planning the fused step");
+                }
+            }
             break;
         default: return fail(JSSA_ERR_INVALID_ARG, "unknown op %d", op);
     }
@@ -598,6 +618,40 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
     if ((st = build_layout(dims, sh, k, JSSA_OP_DECODE_STEP, agg, 0, L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
+    if (L.fused) {
+        ScanArgs sa;
+        memset(&sa, 0, sizeof sa);
+        sa.src = Kt;
+        sa.seq_lens = seq_lens;
+        sa.cand_key = at<uint32_t>(ws, L.cand_key);
+        sa.cand_idx = at<int32_t>(ws, L.cand_idx);
+        sa.cand_cnt = at<int32_t>(ws, L.cand_cnt);
+        sa.counters = at<uint32_t>(ws, L.sel_ctr);
+        sa.idx_out = idx;
+        sa.count_out = count;
+        sa.status = at<uint32_t>(ws, 0);
+        sa.B = dims->B;
+        sa.Hkv = dims->Hkv;
+        sa.T_cap = dims->T_cap;
+        sa.r = dims->r;
+        sa.nq = 1;
+        sa.k = k;
+        StepExtra x;
+        x.q = q;
+        x.P = P;
+        x.K = K;
+        x.V = V;
+        x.pos_begin = pos_begin;
+        x.out = out;
+        x.lse = lse;
+        x.scale_log2 = softmax_scale * 1.4426950408889634f;
+        x.Hq = dims->Hq;
+        x.G = sh.G;
+        x.d = dims->d;
+        cudaError_t e = launch_step_fused(L.fp, sa, x, S(stream), true);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the fused decode step");
+        return JSSA_OK;
+    }
     AppendArgs ap{K, P, Kt, pos_begin, at<uint32_t>(ws, 0), dims->B, dims->T_cap, dims->Hkv, dims->d, dims->r, 1, 1};
     ProjArgs pj{q, P, at<float>(ws, L.qproj), dims->B, dims->Hq, dims->Hkv, dims->d, dims->r, agg};
     cudaError_t e = launch_prep(ap, pj, S(stream), true, dims->kv_dtype, dims->kt_dtype);

@@ -159,6 +159,25 @@ cudaError_t launch_scan(const ScanPlan &p, const ScanArgs &a, int agg, cudaStrea
 // cudaErrorNotSupported where it has no kernel.
 cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int k, ScanPlan *p);
 cudaError_t launch_stream(const ScanPlan &p, const ScanArgs &a, cudaStream_t s, bool pdl);
+
+// The whole decode step in the streaming kernel: the new row of the low-rank
+// cache and the folded query are computed in its prologue, the attention of
+// each (b,h) by the CTA that completes its selection, in its epilogue.
+struct StepExtra {
+    const void *q;            // [B, Hq, d] bf16
+    const float *P;           // [Hkv, d, r]
+    const void *K;            // [B, T_cap, Hkv, d] bf16
+    const void *V;            // [B, T_cap, Hkv, d] bf16
+    const int32_t *pos_begin; // [B] position of the appended token
+    void *out;                // [B, Hq, d] bf16
+    float *lse;               // [B, Hq] or null
+    float scale_log2;         // softmax_scale * log2(e)
+    int Hq, G, d;
+};
+// Fused plan for this shape (bf16 K/V and low-rank cache, SUM, d in {128, 256},
+// r in {32, 64}, G a power of two <= 16); cudaErrorNotSupported otherwise.
+cudaError_t plan_step_fused(int B, int Hkv, int Hq, int d, int T_cap, int r, int k, ScanPlan *p);
+cudaError_t launch_step_fused(const ScanPlan &p, const ScanArgs &a, const StepExtra &x, cudaStream_t s, bool pdl);
 // Selection form forced by the environment (JSSA_SELECT_FORM): 0 automatic,
 // 1 "cluster", 2 "stream", 3 "scan".
 int select_form_override();

@@ -29,6 +29,7 @@
 // The order (score desc, index asc) is strict and total, so the top-k of the
 // union of per-segment top-k sets is the global top-k: the result is exactly
 // that of the score pass followed by the top-k pass.
+#include <cstring>
 #include <type_traits>
 
 #include "jssa_common.cuh"
@@ -55,6 +56,8 @@ constexpr int kMaxStages = 8;
 constexpr int kBins = 2048;                       // 11-bit digits
 constexpr int kBoundary = 64;                     // boundary group ranked exactly
 constexpr int kEpochTokens = 1024;                // minimum tokens per epoch
+constexpr int kMaxRows = 8;                       // (b,h) rows per CTA range on the fused step
+constexpr int kChunkD = 16;                       // inputs per partial sum of a projection
 
 __host__ __device__ inline int npow2(int x) {
     int p = 1;
@@ -64,7 +67,7 @@ __host__ __device__ inline int npow2(int x) {
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct StreamSmem {
-    size_t ring, bars, ek, ei, rk, ri, sk, si, hist, misc, total;
+    size_t ring, bars, ek, ei, rk, ri, sk, si, hist, misc, qb, xs, total;
 };
 
 // misc words (int): [0] abort, [3] candidate count, [4..6] select results,
@@ -72,13 +75,16 @@ struct StreamSmem {
 // scratch, [16..23] scan partials, [24] copies issued, [32..33] threshold
 // (u64), [40..42] epoch buffer counts, [44..45] smallest / largest key
 // appended to the segment's candidates, [48..63] reduction scratch.
-__host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k) {
+// misc words, fused step: [46] rows to attend, [64..71] their (b,h), [72..79]
+// their token counts.  qb: folded queries of the range's rows [kMaxRows][r];
+// xs: one input row of a projection [256].
+__host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k, int fused_r = 0) {
     StreamSmem L;
     size_t o = 0;
     L.ring = o;
     o += (size_t)nstages * kTile;
     L.bars = o;
-    o = al(o + (size_t)(2 * nstages + 2 * kEB) * 8, 16);
+    o = al(o + (size_t)(2 * nstages + 2 * kEB + 2) * 8, 16);
     L.ek = o;
     o = al(o + (size_t)kEB * ept * 4, 16);
     L.ei = o;
@@ -94,7 +100,11 @@ __host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap,
     L.hist = o;
     o = al(o + (size_t)kBins * 4, 16);
     L.misc = o;
-    o = al(o + 64 * 4, 128);
+    o = al(o + 96 * 4, 16);
+    L.qb = o;
+    o = al(o + (size_t)kMaxRows * fused_r * 4, 16);
+    L.xs = o;
+    o = al(o + (fused_r ? 256 * 4 : 0), 128);
     L.total = o;
     return L;
 }
@@ -673,8 +683,9 @@ struct RingPos {
 };
 
 // End of a segment (selector): cut to k, publish, and merge if this CTA is
-// the last of the (b,h) to finish.
-__device__ void sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long long cta, int ept, int cap) {
+// the last of the (b,h) to finish.  Returns the selection's size when this
+// CTA merged it, else -1.
+__device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long long cta, int ept, int cap) {
     if (n > a.k) {
         sel_reduce(S, n, a.k);
         n = a.k;
@@ -696,7 +707,7 @@ __device__ void sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long 
     sel_sync();
     const bool last = S.misc[9] != 0;
     sel_sync();
-    if (!last) return;
+    if (!last) return -1;
     __threadfence();
     // merge: segments in ascending token order, chunks of at most ept entries;
     // equal keys stay candidates (order inside a segment is arbitrary)
@@ -758,10 +769,187 @@ __device__ void sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long 
         a.counters[bh] = 0u;
     }
     sel_sync();
+    return m;
 }
 
-template <int SRC, int R>
-__global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) {
+// ------------------------------------------------------ fused decode step ---
+struct StreamArgs {
+    ScanArgs s;
+    StepExtra x;
+};
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Barrier of the consumer warps alone.
+__device__ __forceinline__ void cons_sync() { asm volatile("bar.sync 2, %0;" ::"n"(kCons) : "memory"); }
+
+// part[j][c] = sum over the c-th chunk of kChunkD inputs of xs[i] * P[i][j]
+// (an fma chain from 0), the fixed order of the projection and append
+// kernels, so every path yields bit-identical rows.
+template <int R>
+__device__ void sel_dots(const float *xs, const float *P, int d, float *part, int st) {
+    const int nch = d / kChunkD;
+    for (int p = st; p < R * nch; p += kSelT) {
+        const int c = p / R, j = p - c * R;
+        const float *xr = xs + c * kChunkD;
+        const float *pc = P + (size_t)(c * kChunkD) * R + j;
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kChunkD; ++i) acc = fmaf(xr[i], __ldg(pc + (size_t)i * R), acc);
+        part[(size_t)j * nch + c] = acc;
+    }
+    sel_sync();
+}
+
+__device__ __forceinline__ float sum_parts(const float *part, int j, int nch) {
+    float s = part[(size_t)j * nch];
+    for (int c = 1; c < nch; ++c) s += part[(size_t)j * nch + c];
+    return s;
+}
+
+// Folded query of row bh: qb = P_h^T (sum of the group's queries, in head order).
+template <int R>
+__device__ void sel_project(const StepExtra &x, int Hkv, int bh, float *qb, float *xs, float *part, int st) {
+    const int b = bh / Hkv, h = bh - b * Hkv, G = x.G, d = x.d;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(x.q) + ((size_t)b * x.Hq + (size_t)h * G) * d;
+    for (int i = st; i < d; i += kSelT) {
+        float sum = 0.f;
+        for (int g = 0; g < G; ++g) sum += __bfloat162float(q[(size_t)g * d + i]);
+        xs[i] = sum;
+    }
+    sel_sync();
+    sel_dots<R>(xs, x.P + (size_t)h * d * R, d, part, st);
+    for (int j = st; j < R; j += kSelT) qb[j] = sum_parts(part, j, d / kChunkD);
+    sel_sync();
+}
+
+// New row of the low-rank cache: Kt[b,h,pos,:] = bf16(K[b,pos,h,:] . P_h),
+// stored to global memory and fenced for the bulk copies that read it.
+template <int R>
+__device__ void sel_append(const ScanArgs &a, const StepExtra &x, int bh, int pos, float *xs, float *part, int st) {
+    const int b = bh / a.Hkv, h = bh - b * a.Hkv, d = x.d;
+    const __nv_bfloat16 *K = static_cast<const __nv_bfloat16 *>(x.K);
+    for (int i = st; i < d; i += kSelT) xs[i] = __bfloat162float(K[(((size_t)b * a.T_cap + pos) * a.Hkv + h) * d + i]);
+    sel_sync();
+    sel_dots<R>(xs, x.P + (size_t)h * d * R, d, part, st);
+    __nv_bfloat16 *Kt = static_cast<__nv_bfloat16 *>(const_cast<void *>(a.src));
+    for (int j = st; j < R; j += kSelT)
+        Kt[((size_t)bh * a.T_cap + pos) * R + j] = __float2bfloat16_rn(sum_parts(part, j, d / kChunkD));
+    fence_proxy_async_global();
+    sel_sync();
+}
+
+// Attention of the G query heads of row bh over its kb selected tokens, by
+// the consumer warps (ct = consumer thread index).  Warps are split over the
+// heads (16 / G warps per head, each taking every (16/G)-th token); the K and
+// V rows of a chunk of tokens are staged in `buf` with 16-byte asynchronous
+// copies straight from the cache; fp32 online softmax in the log2 domain;
+// the warps of a head are combined by log-sum-exp.
+template <int D>
+__device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int kb, unsigned char *buf,
+                             size_t buf_bytes, int ct) {
+    constexpr int EPLD = D / 32;      // dims per lane
+    constexpr int ROW2 = 2 * D * 2;   // a K row and its V row, bf16
+    constexpr int CPR = D * 2 / 16;   // 16-byte chunks of one row
+    const int w = ct >> 5, lane = ct & 31;
+    const int G = x.G, wph = kConsWarps / G, g = w / wph, wi = w - g * wph;
+    const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+    float *comb = reinterpret_cast<float *>(buf);  // [kConsWarps][D + 2]
+    unsigned char *stage = buf + al((size_t)kConsWarps * (D + 2) * 4, 128);
+    const int CH = (int)((buf_bytes - (size_t)(stage - buf)) / ROW2);
+    float qv[EPLD], o[EPLD];
+    const __nv_bfloat16 *qp =
+        static_cast<const __nv_bfloat16 *>(x.q) + ((size_t)b * x.Hq + (size_t)h * G + g) * D + lane * EPLD;
+#pragma unroll
+    for (int e = 0; e < EPLD; ++e) {
+        qv[e] = __bfloat162float(qp[e]) * x.scale_log2;
+        o[e] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    const int32_t *idx = a.idx_out + (size_t)bh * a.k;
+    const __nv_bfloat16 *Kc = static_cast<const __nv_bfloat16 *>(x.K);
+    const __nv_bfloat16 *Vc = static_cast<const __nv_bfloat16 *>(x.V);
+    for (int c0 = 0; c0 < kb; c0 += CH) {
+        const int n = min(CH, kb - c0);
+        for (int p = ct; p < n * 2 * CPR; p += kCons) {
+            const int row = p / (2 * CPR), rem = p - row * 2 * CPR;
+            const int isv = rem >= CPR, ch = rem - isv * CPR;
+            const int t = idx[c0 + row];
+            const bool ok = (unsigned)t < (unsigned)a.T_cap;
+            const __nv_bfloat16 *src =
+                (isv ? Vc : Kc) + (((size_t)b * a.T_cap + (ok ? t : 0)) * a.Hkv + h) * D + ch * 8;
+            cp_async16(stage + (size_t)row * ROW2 + isv * D * 2 + ch * 16, src, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        cons_sync();
+        for (int j = wi; j < n; j += wph) {
+            const unsigned char *kr = stage + (size_t)j * ROW2 + lane * EPLD * 2;
+            float kf[EPLD], vf[EPLD];
+            if constexpr (EPLD == 4) {
+                const uint2 kk = *reinterpret_cast<const uint2 *>(kr);
+                const uint2 vv = *reinterpret_cast<const uint2 *>(kr + D * 2);
+                kf[0] = bf16_lo(kk.x); kf[1] = bf16_hi(kk.x); kf[2] = bf16_lo(kk.y); kf[3] = bf16_hi(kk.y);
+                vf[0] = bf16_lo(vv.x); vf[1] = bf16_hi(vv.x); vf[2] = bf16_lo(vv.y); vf[3] = bf16_hi(vv.y);
+            } else {
+                const uint4 kk = *reinterpret_cast<const uint4 *>(kr);
+                const uint4 vv = *reinterpret_cast<const uint4 *>(kr + D * 2);
+                Vec16<__nv_bfloat16>::unpack(kk, kf);
+                Vec16<__nv_bfloat16>::unpack(vv, vf);
+            }
+            float dot = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPLD; ++e) dot = fmaf(qv[e], kf[e], dot);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+            const float mn = fmaxf(m, dot);
+            const float corr = exp2f(m - mn), pw = exp2f(dot - mn);
+            l = l * corr + pw;
+#pragma unroll
+            for (int e = 0; e < EPLD; ++e) o[e] = fmaf(pw, vf[e], o[e] * corr);
+            m = mn;
+        }
+        cons_sync();
+    }
+    // log-sum-exp combine of the warps of head g
+    float *cw = comb + (size_t)w * (D + 2);
+#pragma unroll
+    for (int e = 0; e < EPLD; ++e) cw[lane * EPLD + e] = o[e];
+    if (lane == 0) {
+        cw[D] = m;
+        cw[D + 1] = l;
+    }
+    cons_sync();
+    if (wi == 0) {
+        float M = -INFINITY;
+        for (int i = 0; i < wph; ++i) M = fmaxf(M, comb[(size_t)(w + i) * (D + 2) + D]);
+        float Ls = 0.f, O[EPLD];
+#pragma unroll
+        for (int e = 0; e < EPLD; ++e) O[e] = 0.f;
+        for (int i = 0; i < wph; ++i) {
+            const float *ci = comb + (size_t)(w + i) * (D + 2);
+            const float mi = ci[D];
+            const float f = mi == -INFINITY ? 0.f : exp2f(mi - M);
+            Ls = fmaf(ci[D + 1], f, Ls);
+#pragma unroll
+            for (int e = 0; e < EPLD; ++e) O[e] = fmaf(ci[lane * EPLD + e], f, O[e]);
+        }
+        const size_t row_out = (size_t)b * x.Hq + (size_t)h * G + g;
+        __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(x.out) + row_out * D + lane * EPLD;
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+        for (int e = 0; e < EPLD; ++e) op[e] = __float2bfloat16_rn(O[e] * inv);
+        if (lane == 0 && x.lse) x.lse[row_out] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+    }
+    cons_sync();
+}
+
+// D = 0: the selection alone.  D > 0: the fused decode step with head width D.
+template <int SRC, int R, int D>
+__global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A) {
+    const ScanArgs &a = A.s;
+    constexpr bool FUSED = D > 0;
     using KT = typename std::conditional<SRC == SRC_KT_FP32, float, __nv_bfloat16>::type;
     constexpr int ES = SRC == SRC_KT_FP32 ? 4 : 2;
     constexpr int ROWB = R * ES;                  // bytes per token
@@ -781,11 +969,13 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
 
     extern __shared__ __align__(128) unsigned char smem[];
     const int S_ = a.nstages;
-    const StreamSmem L = stream_smem(S_, EPT, a.cap, a.k);
+    const StreamSmem L = stream_smem(S_, EPT, a.cap, a.k, FUSED ? R : 0);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + S_;
     uint64_t *efull = empty + S_;  // [kEB]
     uint64_t *efree = efull + kEB; // [kEB]
+    uint64_t *qready = efree + kEB;  // fused: folded queries in shared memory
+    uint64_t *aready = qready + 1;   // fused: new low-rank rows stored
     uint32_t *ek = reinterpret_cast<uint32_t *>(smem + L.ek);
     int32_t *ei = reinterpret_cast<int32_t *>(smem + L.ei);
     int *misc = reinterpret_cast<int *>(smem + L.misc);
@@ -801,6 +991,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
     c0.tpb = a.tiles_per_bh;
     c0.bh = (int)(x_begin / c0.tpb);
     c0.t = (int)(x_begin - (long long)c0.bh * c0.tpb);
+    const int row0 = c0.bh;
+    const int nrows = ntiles > 0 ? (int)((x_end - 1) / c0.tpb) - row0 + 1 : 0;
+    float *qb = reinterpret_cast<float *>(smem + L.qb);
 
     if (tid == 0) {
         for (int s = 0; s < S_; ++s) {
@@ -812,6 +1005,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
             mbar_init(&efree[p], 1);
             misc[40 + p] = 0;
         }
+        mbar_init(qready, 1);
+        mbar_init(aready, 1);
+        misc[46] = 0;
         fence_barrier_init();
         misc[0] = 0;
         misc[3] = 0;
@@ -831,7 +1027,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
             int issued = 0;
             Cursor cur = c0;
             RingPos rp(S_);
-            int Tb = 0;
+            int Tb = 0, atile = -1;
+            bool appended = false;
             for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
                 const int s = rp.s;
                 if (i >= S_ && !wait_or_abort(&empty[s], rp.ph ^ 1u, abort_flag)) {
@@ -839,7 +1036,21 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
                     break;
                 }
                 const int bh = cur.bh, t0 = cur.t * TILE;
-                if (i == 0 || cur.t == 0) Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, nullptr);
+                if (i == 0 || cur.t == 0) {
+                    Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, nullptr);
+                    if constexpr (FUSED) {
+                        const int pos = __ldg(A.x.pos_begin + bh / a.Hkv);
+                        atile = (pos >= 0 && pos < a.T_cap) ? pos / TILE : -1;
+                    }
+                }
+                if (FUSED && !appended && cur.t == atile) {
+                    // this tile holds the row appended in the prologue
+                    if (!wait_or_abort(aready, 0u, abort_flag)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    appended = true;
+                }
                 const int n = min(TILE, Tb - t0);
                 if (n > 0) {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)n * ROWB);
@@ -863,19 +1074,34 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
         int Tb = 0, e = 0, epos = 0, p = 0;
         uint32_t eph = 0u;  // use parity of epoch buffer p
         uint32_t tag = 0u;
+        bool qok = true;
+        if (FUSED && ntiles > 0) {  // the folded queries come from the selector's prologue
+            qok = __all_sync(0xffffffffu, wait_or_abort(qready, 0u, abort_flag));
+            if (!qok) *abort_flag = 1;
+        }
         Cursor cur = c0;
         RingPos rp(S_);
-        for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
+        for (int i = 0; qok && i < ntiles; ++i, cur.next(), rp.next()) {
             const int bh = cur.bh, t = cur.t, s = rp.s;
             if (i == 0 || t == 0) {
                 Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, ct == 0 ? a.status : nullptr);
                 tag = (uint32_t)bh + 1u;
-                const float *qp = a.qproj + (size_t)bh * R;  // written by the preceding kernel: read through L2
+                if constexpr (FUSED) {
+                    const float *qp = qb + (size_t)(bh - row0) * R;
 #pragma unroll
-                for (int c = 0; c < CPT; ++c) {
-                    const int ch = sub * CPT + ((c + rot) % CPT);
+                    for (int c = 0; c < CPT; ++c) {
+                        const int ch = sub * CPT + ((c + rot) % CPT);
 #pragma unroll
-                    for (int x = 0; x < EPL; ++x) qreg[c * EPL + x] = __ldcg(qp + ch * EPL + x);
+                        for (int x = 0; x < EPL; ++x) qreg[c * EPL + x] = qp[ch * EPL + x];
+                    }
+                } else {
+                    const float *qp = a.qproj + (size_t)bh * R;  // written by the preceding kernel: read through L2
+#pragma unroll
+                    for (int c = 0; c < CPT; ++c) {
+                        const int ch = sub * CPT + ((c + rot) % CPT);
+#pragma unroll
+                        for (int x = 0; x < EPL; ++x) qreg[c * EPL + x] = __ldcg(qp + ch * EPL + x);
+                    }
                 }
             }
             if (epos == 0 && e >= kEB) {
@@ -965,6 +1191,26 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
         uint32_t eph = 0u;
         bool valid = false;
         uint32_t thr = 0u;
+        if constexpr (FUSED) {
+            // prologue: folded queries of the range's rows, then the new rows of
+            // the low-rank cache whose tiles this CTA streams
+            float *xs = reinterpret_cast<float *>(smem + L.xs);
+            float *part = reinterpret_cast<float *>(S.hist);
+            for (int rl = 0; rl < nrows; ++rl)
+                sel_project<R>(A.x, a.Hkv, row0 + rl, qb + (size_t)rl * R, xs, part, S.st);
+            if (S.st == 0) mbar_arrive(qready);
+            for (int rl = 0; rl < nrows; ++rl) {
+                const int bh = row0 + rl;
+                const int pos = __ldg(A.x.pos_begin + bh / a.Hkv);
+                if (pos < 0 || pos >= a.T_cap) {
+                    if (S.st == 0 && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_POS);
+                    continue;
+                }
+                const long long xt = (long long)bh * a.tiles_per_bh + pos / TILE;
+                if (xt >= x_begin && xt < x_end) sel_append<R>(a, A.x, bh, pos, xs, part, S.st);
+            }
+            if (S.st == 0) mbar_arrive(aready);
+        }
         Cursor cur = c0;
         for (int i = 0; i < ntiles; ++i, cur.next()) {
             const bool send = cur.seg_last(i, ntiles);
@@ -1026,7 +1272,13 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
             }
             const int bh = cur.bh;
             if (send) {
-                sel_finish(a, S, m, bh, cta, EPT, a.cap);
+                const int fin = sel_finish(a, S, m, bh, cta, EPT, a.cap);
+                if (FUSED && fin >= 0 && S.st == 0) {  // this CTA attends over the row at the end
+                    const int na = misc[46];
+                    misc[64 + na] = bh;
+                    misc[72 + na] = fin;
+                    misc[46] = na + 1;
+                }
                 m = 0;
                 valid = false;
                 if (S.st == 0) {
@@ -1073,35 +1325,48 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(ScanArgs a) 
                 (void)mbar_wait_bounded(&full[i % S_], (uint32_t)(i / S_) & 1u);
         }
         __syncthreads();
+        return;
+    }
+    if constexpr (FUSED) {
+        // epilogue: attention of the rows whose selection this CTA completed,
+        // in the (now idle) ring buffer
+        if (tid >= kConsBase) {
+            const int na = misc[46];
+            for (int i = 0; i < na; ++i)
+                fused_attend<D>(a, A.x, misc[64 + i], misc[72 + i], smem + L.ring, (size_t)S_ * kTile, tid - kConsBase);
+        }
     }
 }
 
 template <int SRC>
-void (*pick_r(int r))(ScanArgs) {
+void (*pick_r(int r))(StreamArgs) {
     switch (r) {
-        case 8: return stream_select_kernel<SRC, 8>;
-        case 16: return stream_select_kernel<SRC, 16>;
-        case 32: return stream_select_kernel<SRC, 32>;
-        case 64: return stream_select_kernel<SRC, 64>;
-        case 128: return stream_select_kernel<SRC, 128>;
+        case 8: return stream_select_kernel<SRC, 8, 0>;
+        case 16: return stream_select_kernel<SRC, 16, 0>;
+        case 32: return stream_select_kernel<SRC, 32, 0>;
+        case 64: return stream_select_kernel<SRC, 64, 0>;
+        case 128: return stream_select_kernel<SRC, 128, 0>;
         default: return nullptr;
     }
 }
 
-void (*pick_stream(int src, int r))(ScanArgs) {
+void (*pick_stream(int src, int r))(StreamArgs) {
     if (src == SRC_KT_BF16) return pick_r<SRC_KT_BF16>(r);
     if (src == SRC_KT_FP32) return pick_r<SRC_KT_FP32>(r);
     return nullptr;
 }
 
-}  // namespace
+void (*pick_fused(int r, int d))(StreamArgs) {
+    if (r == 32 && d == 128) return stream_select_kernel<SRC_KT_BF16, 32, 128>;
+    if (r == 32 && d == 256) return stream_select_kernel<SRC_KT_BF16, 32, 256>;
+    if (r == 64 && d == 128) return stream_select_kernel<SRC_KT_BF16, 64, 128>;
+    if (r == 64 && d == 256) return stream_select_kernel<SRC_KT_BF16, 64, 256>;
+    return nullptr;
+}
 
-// Plan of the warp-specialised form: SUM aggregation over the low-rank key
-// cache (the decode-step path).  cudaErrorNotSupported for other forms.
-cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int k, ScanPlan *p) {
-    if (agg != JSSA_AGG_SUM) return cudaErrorNotSupported;
-    auto kern = pick_stream(src, r);
-    if (!kern) return cudaErrorNotSupported;
+// Shared planning of both forms: tiles, epochs, ring depth, grid, segments.
+cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T_cap, int r, int k, int fused_r,
+                        ScanPlan *p) {
     const int rowb = r * (src == SRC_KT_FP32 ? 4 : 2);
     const int tile = kTile / rowb;
     const int ept = tile >= kEpochTokens ? tile : kEpochTokens;
@@ -1119,10 +1384,10 @@ cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int 
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
     int ns = kMaxStages;
-    while (ns >= 3 && stream_smem(ns, ept, P.cap, k).total > (size_t)optin) --ns;
+    while (ns >= 3 && stream_smem(ns, ept, P.cap, k, fused_r).total > (size_t)optin) --ns;
     if (ns < 3) return cudaErrorNotSupported;
     P.nstages = ns;
-    P.smem = stream_smem(ns, ept, P.cap, k).total;
+    P.smem = stream_smem(ns, ept, P.cap, k, fused_r).total;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
@@ -1146,19 +1411,68 @@ cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int 
     return cudaSuccess;
 }
 
+}  // namespace
+
+// Plan of the warp-specialised form: SUM aggregation over the low-rank key
+// cache (the decode-step path).  cudaErrorNotSupported for other forms.
+cudaError_t plan_stream(int src, int agg, int B, int Hkv, int T_cap, int r, int k, ScanPlan *p) {
+    if (agg != JSSA_AGG_SUM) return cudaErrorNotSupported;
+    auto kern = pick_stream(src, r);
+    if (!kern) return cudaErrorNotSupported;
+    return plan_common(kern, src, B, Hkv, T_cap, r, k, 0, p);
+}
+
+namespace {
+void fill_plan(StreamArgs &A, const ScanPlan &p) {
+    A.s.tile_tokens = p.tile_tokens;
+    A.s.tiles_per_bh = p.tiles_per_bh;
+    A.s.total_tiles = p.total_tiles;
+    A.s.grid = p.grid;
+    A.s.max_seg = p.max_seg;
+    A.s.cap = p.cap;
+    A.s.nstages = p.nstages;
+}
+}  // namespace
+
 cudaError_t launch_stream(const ScanPlan &p, const ScanArgs &a0, cudaStream_t s, bool pdl) {
     auto kern = pick_stream(p.src, a0.r);
     if (!kern) return cudaErrorInvalidValue;
     if (p.total_tiles <= 0) return cudaSuccess;
-    ScanArgs a = a0;
-    a.tile_tokens = p.tile_tokens;
-    a.tiles_per_bh = p.tiles_per_bh;
-    a.total_tiles = p.total_tiles;
-    a.grid = p.grid;
-    a.max_seg = p.max_seg;
-    a.cap = p.cap;
-    a.nstages = p.nstages;
-    return launch_kernel(kern, dim3(p.grid), dim3(kThreads), p.smem, s, pdl, a);
+    StreamArgs A;
+    memset(&A, 0, sizeof A);
+    A.s = a0;
+    fill_plan(A, p);
+    return launch_kernel(kern, dim3(p.grid), dim3(kThreads), p.smem, s, pdl, A);
+}
+
+cudaError_t plan_step_fused(int B, int Hkv, int Hq, int d, int T_cap, int r, int k, ScanPlan *p) {
+    auto kern = pick_fused(r, d);
+    if (!kern || Hkv < 1 || Hq % Hkv) return cudaErrorNotSupported;
+    const int G = Hq / Hkv;
+    if (G < 1 || G > kConsWarps || (G & (G - 1))) return cudaErrorNotSupported;
+    cudaError_t e = plan_common(kern, SRC_KT_BF16, B, Hkv, T_cap, r, k, r, p);
+    if (e != cudaSuccess) return e;
+    // every CTA range spans at most kMaxRows (b,h) rows, and the ring holds
+    // the attention's combine area plus one staged K/V row pair
+    for (long long c = 0; c < p->grid; ++c) {
+        const long long xb = c * p->total_tiles / p->grid, xe = (c + 1) * p->total_tiles / p->grid;
+        if (xe > xb && (xe - 1) / p->tiles_per_bh - xb / p->tiles_per_bh + 1 > kMaxRows) return cudaErrorNotSupported;
+    }
+    const size_t need = al((size_t)kConsWarps * (d + 2) * 4, 128) + (size_t)4 * d;
+    if ((size_t)p->nstages * kTile < need) return cudaErrorNotSupported;
+    return cudaSuccess;
+}
+
+cudaError_t launch_step_fused(const ScanPlan &p, const ScanArgs &a0, const StepExtra &x, cudaStream_t s, bool pdl) {
+    auto kern = pick_fused(a0.r, x.d);
+    if (!kern) return cudaErrorInvalidValue;
+    if (p.total_tiles <= 0) return cudaSuccess;
+    StreamArgs A;
+    memset(&A, 0, sizeof A);
+    A.s = a0;
+    A.x = x;
+    fill_plan(A, p);
+    return launch_kernel(kern, dim3(p.grid), dim3(kThreads), p.smem, s, pdl, A);
 }
 
 }  // namespace jssa
