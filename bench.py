@@ -5,8 +5,10 @@
 A step is one decode step of one attention layer at the workload's shape:
 append the new token's low-rank key row, score the low-rank cache, select a
 top-k token set per (batch, KV head), and run gather-free indexed attention
-(jssa_decode_step: three kernels).  The default workload is the 128K-context,
-batch-16 GQA layer (B=16, Hq=32, Hkv=8, d=128, T=131072, r=32, k=256).
+(jssa_decode_step: one launch of the fused streaming kernel where that form
+applies, else three or four kernels).  The default workload is the
+128K-context, batch-16 GQA layer (B=16, Hq=32, Hkv=8, d=128, T=131072, r=32,
+k=256).
 
 value  = steps/s of the whole job (N replicas, one per GPU, each running the
          full workload: weak scaling, no collective on the data path), timed
@@ -14,9 +16,10 @@ value  = steps/s of the whole job (N replicas, one per GPU, each running the
 e2e    = the same metric through the public session API with host buffers:
          every step copies q and the new K/V rows from pinned host memory and
          reads the output back (synchronising per step).
-roofline = the dominant kernel (the fused score + top-k pass, jssa_select)
-         timed alone, algorithmic bytes / duration against the measured HBM copy
-         bandwidth.
+roofline = the dominant kernel against the measured HBM copy bandwidth: the
+         fused step kernel itself when the step is one launch (algorithmic bytes
+         of the step / its duration in the timed loop), else the selection pass
+         (jssa_select) timed alone.
 cpu_baseline / --impl reference = the fp64 C oracle on the host cores over a
          bounded sample of (batch, KV head) pairs, scaled to a whole step.
 """
@@ -69,10 +72,11 @@ def select_bytes(w):
     return w.B * w.Hkv * w.T * w.r * 2 + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * (w.k + 1) * 4
 
 
-def profile_traffic(kernel_file, workload):
-    """DRAM bytes per launch from a committed ncu summary, if the summary's
-    source hash matches the kernel source as it is now (else None)."""
-    path = os.path.join(ROOT, "profiles", "scan_select_%s.txt" % workload)
+def profile_traffic(kernel_file, summary):
+    """DRAM bytes per launch from a committed ncu summary (profiles/<summary>),
+    if the summary's source hash matches the kernel source as it is now (else
+    None)."""
+    path = os.path.join(ROOT, "profiles", summary)
     src = os.path.join(ROOT, "token_level_sparse_kv_b200", "csrc", kernel_file)
     if not (os.path.exists(path) and os.path.exists(src)):
         return None
@@ -321,6 +325,8 @@ def run_jssa(args, world, rank, local):
     pos = (sl - 1).clamp_min(0).contiguous()
     dims = ops.make_dims(q, K, V, P=P, Kt=Kt)
     ws = ops.new_workspace(dims, w.k, ops.OP_DECODE_STEP, dev)
+    launches, step_form = ops.plan_info(dims, w.k, ops.OP_DECODE_STEP)
+    sel_form = ops.plan_info(dims, w.k, ops.OP_SELECT)[1]
     idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
     cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
     out = torch.empty((w.B, w.Hq, w.Dv), dtype=q.dtype, device=dev)
@@ -362,22 +368,32 @@ def run_jssa(args, world, rank, local):
     peak, peak_kind = measured_peaks()
     step_bytes, kt_bytes = algorithmic_bytes(w)
     step_flops = 2 * w.B * w.Hq * min(w.k, w.T) * (w.d + w.Dv)  # q.k and p.v of the selected rows
-    sbytes = select_bytes(w)
     sel_s = sel_secs / sel_steps
-    achieved = sbytes / sel_s / 1e9
-    traffic = profile_traffic("jssa_scan.cu", w.name)
+    if launches == 1:
+        # the step is one launch of the fused streaming kernel: it is the dominant kernel
+        kname = "stream_select_kernel (fused decode step: append, projection, score, top-k, attention)"
+        kbytes, k_s = step_bytes, ms / 1e3
+        traffic = profile_traffic("jssa_stream.cu", "stream_step_%s.txt" % w.name)
+    else:
+        kname = "selection pass (jssa_select: %s)" % sel_form
+        kbytes, k_s = select_bytes(w), sel_s
+        traffic = None
+    achieved = kbytes / k_s / 1e9
 
     line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
-            "roofline": {"bound": "hbm", "kernel": "scan_kernel (jssa_select: fused score + top-k)",
+            "roofline": {"bound": "hbm", "kernel": kname,
                          "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind + " (burst copy)", "traffic": traffic,
-                         "algorithmic_bytes_per_launch": sbytes, "us_per_launch": sel_s * 1e6},
+                         "algorithmic_bytes_per_launch": kbytes, "us_per_launch": k_s * 1e6},
+            "select_alone": {"us_per_call": sel_s * 1e6, "algorithmic_bytes": select_bytes(w),
+                             "achieved_gbs": select_bytes(w) / sel_s / 1e9, "form": sel_form},
             "step_hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms / 1e3) / 1e9,
                          "frac_of_peak": step_bytes / (ms / 1e3) / 1e9 / peak, "peak_gbs": peak,
                          "attention_flops_per_step": step_flops},
-            "gpu_launches": 3 * args.steps}
+            "step_form": step_form,
+            "gpu_launches": launches * args.steps}
     if clocks:
         line["clocks"] = clocks
 

@@ -144,6 +144,16 @@ JSSA_API const char *jssa_last_error(void);
  * returns a status. */
 JSSA_API int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes);
 
+/* How one call of `op` (JSSA_OP_*) with these dims, k and aggregation is
+ * carried out on the current device: *launches = the kernels it enqueues
+ * (the decode step is a single launch when its fused streaming form applies,
+ * else three or four), and, when desc is not NULL, a NUL-terminated
+ * description of the forms chosen (at most desc_len bytes written).  Host
+ * planning only: nothing is enqueued.  The pages have no counterpart; this
+ * is a measurement aid (launch counts of a timed region). */
+JSSA_API int jssa_plan_info(const jssa_dims *dims, int k, int op, int agg, int *launches, char *desc,
+                            size_t desc_len);
+
 /* Zero `ws_bytes` bytes of workspace on `stream` (clears the status word and
  * the arrival counters).  Needed once per workspace before first use. */
 JSSA_API int jssa_workspace_init(void *ws, size_t ws_bytes, jssa_stream_t stream);

@@ -389,6 +389,48 @@ int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes) {
     return JSSA_OK;
 }
 
+int jssa_plan_info(const jssa_dims *dims, int k, int op, int agg, int *launches, char *desc, size_t desc_len) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if (!launches) return fail(JSSA_ERR_INVALID_ARG, "launches is NULL");
+    if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
+    const bool needs_k = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_INDEXED_DECODE ||
+                         op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP;
+    if (needs_k && (st = check_k(k))) return st;
+    Layout L;
+    if ((st = build_layout(dims, sh, k, op, agg, 0, L))) return st;
+    const char *sel = L.csel ? "cluster" : (L.wspec ? "stream" : "scan");
+    const int att = sh.latent ? 1 + (L.ap.splits > 1 ? 1 : 0) : 1;
+    int n = 0;
+    char text[160];
+    switch (op) {
+        case JSSA_OP_APPEND: n = 1; snprintf(text, sizeof text, "append"); break;
+        case JSSA_OP_SCORE: n = 2; snprintf(text, sizeof text, "projection + score pass"); break;
+        case JSSA_OP_TOPK: n = 1; snprintf(text, sizeof text, "top-k (%s form)", sel); break;
+        case JSSA_OP_SELECT: n = 2; snprintf(text, sizeof text, "projection + selection (%s form)", sel); break;
+        case JSSA_OP_INDEXED_DECODE: n = att; snprintf(text, sizeof text, "indexed attention"); break;
+        case JSSA_OP_DENSE_DECODE: n = 1; snprintf(text, sizeof text, "dense attention"); break;
+        case JSSA_OP_GATHER_THEN_DENSE: n = 2; snprintf(text, sizeof text, "gather + dense attention"); break;
+        case JSSA_OP_DECODE_STEP:
+            if (L.fused) {
+                n = 1;
+                snprintf(text, sizeof text, "fused step (stream form: append, projection, selection, attention)");
+            } else {
+                n = 2 + att;
+                snprintf(text, sizeof text, "append + projection, selection (%s form), attention", sel);
+            }
+            break;
+        default: return fail(JSSA_ERR_INVALID_ARG, "unknown op %d", op);
+    }
+    *launches = n;
+    if (desc && desc_len) {
+        strncpy(desc, text, desc_len - 1);
+        desc[desc_len - 1] = 0;
+    }
+    return JSSA_OK;
+}
+
 int jssa_workspace_init(void *ws, size_t ws_bytes, jssa_stream_t stream) {
     if (!ws) return fail(JSSA_ERR_INVALID_ARG, "ws is NULL");
     cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, S(stream));

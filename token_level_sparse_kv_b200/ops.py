@@ -64,6 +64,8 @@ def lib():
     L.jssa_last_error.restype = ctypes.c_char_p
     L.jssa_workspace_size.restype = i32
     L.jssa_workspace_size.argtypes = [D, i32, i32, ctypes.POINTER(sz)]
+    L.jssa_plan_info.restype = i32
+    L.jssa_plan_info.argtypes = [D, i32, i32, i32, ctypes.POINTER(i32), ctypes.c_char_p, sz]
     L.jssa_workspace_init.restype = i32
     L.jssa_workspace_init.argtypes = [vp, sz, vp]
     L.jssa_append_lowrank.restype = i32
@@ -129,6 +131,14 @@ def make_dims(q, K, V, P=None, Kt=None, r=None):
         r = P.shape[2] if P is not None else (Kt.shape[3] if Kt is not None else 8)
     kt = _dt(Kt) if Kt is not None else BF16
     return Dims(B, Hq, Hkv, d, dv, r, T_cap, _dt(K), kt)
+
+
+def plan_info(dims: Dims, k: int, op: int, agg: int = 0):
+    """(kernel launches per call, description of the forms chosen) for op."""
+    n = ctypes.c_int32(0)
+    buf = ctypes.create_string_buffer(160)
+    _check(lib().jssa_plan_info(ctypes.byref(dims), int(k), int(op), int(agg), ctypes.byref(n), buf, 160))
+    return int(n.value), buf.value.decode()
 
 
 def workspace_size(dims: Dims, k: int, op: int) -> int:
