@@ -12,7 +12,9 @@ k=256).
 
 value  = steps/s of the whole job (N replicas, one per GPU, each running the
          full workload: weak scaling, no collective on the data path), timed
-         on the device with CUDA events over exactly K steps, max over ranks.
+         on the device with CUDA events over exactly K steps, max over ranks;
+         each step is a replay of a CUDA graph of jssa_decode_step (one graph
+         per rotating query; --eager times the plain call loop instead).
 e2e    = the same metric through the public session API with host buffers:
          every step copies q and the new K/V rows from pinned host memory and
          reads the output back (synchronising per step).
@@ -344,12 +346,33 @@ def run_jssa(args, world, rank, local):
     status = ops.device_status(ws)
     if status:
         raise RuntimeError("device status 0x%x after warm-up" % status)
+    # the timed loop replays one CUDA graph per rotating query (the step's
+    # launches without host planning), as a serving decode loop would
+    graphs, launch_mode = None, "eager"
+    if not args.eager:
+        try:
+            graphs = [ops.StepGraph(lambda j=j: step(j), dev) for j in range(4)]
+            launch_mode = "cuda graph (one replay per step)"
+        except Exception as e:  # capture unsupported: time the eager loop
+            log("graph capture failed (%s); timing the eager loop" % e)
+            graphs = None
+    if graphs:
+        def timed(i):
+            graphs[i & 3].replay()
+
+        for i in range(max(3, args.warmup)):
+            timed(i)
+        torch.cuda.synchronize()
+    else:
+        timed = step
 
     sampler = ClockSampler(local)
     with sampler:
         barrier(world)
-        secs = time_loop(step, args.steps, stream)
+        secs = time_loop(timed, args.steps, stream)
         barrier(world)
+        eager_steps = max(5, min(args.steps, 200))
+        eager_secs = time_loop(step, eager_steps, stream) if graphs else None
         # dominant kernel alone: the fused score + top-k pass (jssa_select)
         ws_sel = ops.new_workspace(dims, w.k, ops.OP_SELECT, dev)
         sel_steps = max(args.steps, 20)
@@ -393,6 +416,8 @@ def run_jssa(args, world, rank, local):
                          "frac_of_peak": step_bytes / (ms / 1e3) / 1e9 / peak, "peak_gbs": peak,
                          "attention_flops_per_step": step_flops},
             "step_form": step_form,
+            "launch": launch_mode,
+            "eager_ms_per_step": (max_over_ranks(eager_secs, world) / eager_steps * 1e3) if graphs else ms,
             "gpu_launches": launches * args.steps}
     if clocks:
         line["clocks"] = clocks
@@ -449,20 +474,22 @@ def run_jssa(args, world, rank, local):
         kh = torch.randn((w.B, w.Hkv, w.d), dtype=torch.float32).to(q.dtype).pin_memory()
         vh = None if w.latent else torch.randn((w.B, w.Hkv, w.Dv), dtype=torch.float32).to(q.dtype).pin_memory()
         e2e_steps = max(5, min(args.steps, args.e2e_steps))
+        use_graph = graphs is not None
         for i in range(3):
-            sess.step_from_host(qh[i & 3], kh, vh)
+            sess.step_from_host(qh[i & 3], kh, vh, graph=use_graph)
             stream.synchronize()
         barrier(world)
         t0 = time.perf_counter()
         for i in range(e2e_steps):
-            o = sess.step_from_host(qh[i & 3], kh, vh)
+            o = sess.step_from_host(qh[i & 3], kh, vh, graph=use_graph)
             stream.synchronize()  # the host reads the output every step
         te = max_over_ranks(time.perf_counter() - t0, world)
         h2d = qh[0].numel() * qh[0].element_size() + kh.numel() * kh.element_size() + (
             0 if vh is None else vh.numel() * vh.element_size())
         d2h = o.numel() * o.element_size()
         line["e2e"] = {"value": world * e2e_steps / te, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h, "api": "DecodeSession.step_from_host (pinned host in/out)"}
+                       "d2h_bytes_per_step": d2h,
+                       "api": "DecodeSession.step_from_host (pinned host in/out%s)" % (", graph=True" if use_graph else "")}
 
     if rank == 0 and not args.no_cpu:
         v, desc, thr = oracle_baseline(w0, args.cpu_seconds, max(1, min(w0.B, args.cpu_rows)), os.cpu_count() or 1)
@@ -488,6 +515,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=2, help="batch rows in the oracle's timed sample")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host seconds of oracle work to time")
     ap.add_argument("--quick", action="store_true", help="skip the comparison and end-to-end passes")
+    ap.add_argument("--eager", action="store_true", help="time the eager call loop instead of CUDA graph replays")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     args = ap.parse_args()
     if args.warmup < 3:

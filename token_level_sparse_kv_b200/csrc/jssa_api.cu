@@ -10,6 +10,32 @@
 
 namespace jssa {
 
+cudaError_t ensure_smem(const void *kern, size_t smem) {
+    if (smem <= 48 * 1024) return cudaSuccess;
+    struct Entry {
+        const void *kern;
+        int dev;
+        size_t smem;
+    };
+    static Entry table[256];
+    static int n = 0;
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n; ++i)
+        if (table[i].kern == kern && table[i].dev == dev) {
+            if (table[i].smem >= smem) return cudaSuccess;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess) table[i].smem = smem;
+            return e;
+        }
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && n < 256) table[n++] = Entry{kern, dev, smem};
+    return e;
+}
+
 int device_sm_count() {
     static int cache[64] = {0};
     int dev = 0;
@@ -181,7 +207,57 @@ bool fused_step_allowed() {
     return !(v && v[0] == '0');
 }
 
+int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L);
+
+// Layouts (workspace offsets and kernel plans) are cached per device, dims,
+// op and settings: planning costs occupancy queries and attribute calls that
+// would otherwise dominate the host time of a decode step.  The kernels'
+// shared-memory attributes set by the first planning stay set for the
+// process, so a cached plan can be launched directly.
+struct LayoutKey {
+    int dev, op, k, agg, window, form, fused;
+    jssa_dims dims;
+    bool operator==(const LayoutKey &o) const { return !memcmp(this, &o, sizeof *this); }
+};
+struct LayoutEntry {
+    LayoutKey key;
+    Layout L;
+};
+constexpr int kLayoutCache = 64;
+LayoutEntry g_layouts[kLayoutCache];
+int g_layouts_n = 0, g_layouts_next = 0;
+std::mutex g_layouts_mu;
+
 int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L) {
+    LayoutKey key;
+    memset(&key, 0, sizeof key);
+    cudaError_t e = cudaGetDevice(&key.dev);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the current device");
+    key.op = op;
+    key.k = k;
+    key.agg = agg;
+    key.window = window;
+    key.form = select_form_override();
+    key.fused = fused_step_allowed() ? 1 : 0;
+    key.dims = *d;
+    {
+        std::lock_guard<std::mutex> lk(g_layouts_mu);
+        for (int i = 0; i < g_layouts_n; ++i)
+            if (g_layouts[i].key == key) {
+                L = g_layouts[i].L;
+                return JSSA_OK;
+            }
+    }
+    const int st = build_layout_uncached(d, sh, k, op, agg, window, L);
+    if (st != JSSA_OK) return st;
+    std::lock_guard<std::mutex> lk(g_layouts_mu);
+    LayoutEntry &slot = g_layouts[g_layouts_n < kLayoutCache ? g_layouts_n++ : (g_layouts_next++ % kLayoutCache)];
+    slot.key = key;
+    slot.L = L;
+    return JSSA_OK;
+}
+
+int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L) {
     L = Layout();
     int st = JSSA_OK;
     const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;

@@ -149,6 +149,10 @@ cudaError_t launch_mla(const MlaArgs &a, bool indexed, cudaStream_t s, bool pdl)
 
 // --------------------------------------------------------------- helpers ---
 int device_sm_count();
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device
+// (launch paths call it on every launch; the runtime call is made only when
+// the requested size grows).
+cudaError_t ensure_smem(const void *kern, size_t smem);
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype);
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s, bool pdl, int kv_dtype, int kt_dtype);
 cudaError_t launch_prep(const AppendArgs &ap, const ProjArgs &pj, cudaStream_t s, bool pdl, int kv_dtype,

@@ -371,7 +371,7 @@ int mla_splits(int npos) { return npos <= kTok ? 1 : (npos + kTok - 1) / kTok; }
 cudaError_t launch_mla(const MlaArgs &a0, bool indexed, cudaStream_t s, bool pdl) {
     MlaArgs a = a0;
     void (*k)(MlaArgs) = indexed ? mla_kernel<true> : mla_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(k), kSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_kernel(k, dim3(a.splits, a.B), dim3(kThr), kSmemBytes, s, pdl, a);
     if (e != cudaSuccess || a.splits == 1) return e;

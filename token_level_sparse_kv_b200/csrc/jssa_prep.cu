@@ -155,8 +155,7 @@ size_t prep_smem(int rows, int d, int r) {
 
 template <typename Kern>
 cudaError_t allow_smem(Kern k, size_t smem) {
-    if (smem <= 48 * 1024) return cudaSuccess;
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    return ensure_smem(reinterpret_cast<const void *>(k), smem);
 }
 
 }  // namespace

@@ -51,6 +51,7 @@ constexpr int kProdBase = kSelT;                  // producer warp
 constexpr int kConsBase = kSelT + 32;             // first consumer thread
 constexpr int kThreads = kConsBase + kCons;       // 800
 constexpr int kEB = 3;                            // epoch buffers
+static_assert(kEB <= 4, "epoch buffer counts live in misc[40..43]");
 constexpr int kTile = 32768;                      // bytes per ring stage
 constexpr int kMaxStages = 8;
 constexpr int kBins = 2048;                       // 11-bit digits
@@ -84,7 +85,7 @@ __host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap,
     L.ring = o;
     o += (size_t)nstages * kTile;
     L.bars = o;
-    o = al(o + (size_t)(2 * nstages + 2 * kEB + 2) * 8, 16);
+    o = al(o + (size_t)(2 * nstages + 2 * kEB + kMaxRows + 1) * 8, 16);
     L.ek = o;
     o = al(o + (size_t)kEB * ept * 4, 16);
     L.ei = o;
@@ -760,9 +761,21 @@ __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long l
         sel_reduce(S, m, a.k);
         m = a.k;
     }
-    for (int j = S.st; j < m; j += kSelT) S.si[j] = S.ri[j];
-    sel_sync();
-    sel_sort(S.si, m, S.st);
+    if (m <= 2 * kSelT) {
+        // ascending order by rank: the indices are distinct, so each entry's
+        // place is the number of smaller ones (broadcast reads, one barrier)
+        for (int j = S.st; j < m; j += kSelT) {
+            const int32_t v = S.ri[j];
+            int rank = 0;
+            for (int i = 0; i < m; ++i) rank += S.ri[i] < v;
+            S.si[rank] = v;
+        }
+        sel_sync();
+    } else {
+        for (int j = S.st; j < m; j += kSelT) S.si[j] = S.ri[j];
+        sel_sync();
+        sel_sort(S.si, m, S.st);
+    }
     for (int j = S.st; j < a.k; j += kSelT) a.idx_out[(size_t)bh * a.k + j] = j < m ? S.si[j] : -1;
     if (S.st == 0) {
         if (a.count_out) a.count_out[bh] = m;
@@ -840,107 +853,215 @@ __device__ void sel_append(const ScanArgs &a, const StepExtra &x, int bh, int po
     sel_sync();
 }
 
+// ---- attention epilogue on the tensor cores (mma.sync m16n8k16, bf16) ----
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t &r0, uint32_t &r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// D(16x8, f32) += A(16x16, bf16, row) * B(16x8, bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
 // Attention of the G query heads of row bh over its kb selected tokens, by
-// the consumer warps (ct = consumer thread index).  Warps are split over the
-// heads (16 / G warps per head, each taking every (16/G)-th token); the K and
-// V rows of a chunk of tokens are staged in `buf` with 16-byte asynchronous
-// copies straight from the cache; fp32 online softmax in the log2 domain;
-// the warps of a head are combined by log-sum-exp.
+// the 16 consumer warps (ct = consumer thread index), as two small matrix
+// products on the tensor cores with the heads padded to 16 rows:
+//   S[16 x n] = Q[16 x D] . K_sel^T      (fp32 accumulation of bf16 products)
+//   O[16 x D] = P[16 x n] . V_sel        (P = softmax weights rounded to bf16)
+// The selected K and V rows of a chunk of tokens are staged by 16-byte
+// asynchronous copies straight from the cache into `buf` (16-byte chunks
+// XOR-swizzled by token so that ldmatrix reads are conflict-free); the
+// softmax runs in fp32 in the log2 domain across the warps, online across
+// chunks; the normaliser sums the bf16 weights the second product uses.
 template <int D>
 __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int kb, unsigned char *buf,
                              size_t buf_bytes, int ct) {
-    constexpr int EPLD = D / 32;      // dims per lane
-    constexpr int ROW2 = 2 * D * 2;   // a K row and its V row, bf16
-    constexpr int CPR = D * 2 / 16;   // 16-byte chunks of one row
-    const int w = ct >> 5, lane = ct & 31;
-    const int G = x.G, wph = kConsWarps / G, g = w / wph, wi = w - g * wph;
+    constexpr int ROWB = D * 2;         // bytes of a K (or V) row
+    constexpr int CPR = ROWB / 16;      // 16-byte chunks per row
+    constexpr int ROW2 = 2 * ROWB;      // staged K row then V row
+    constexpr int QSTR = ROWB + 16;     // padded row stride of Q (bytes)
+    constexpr int NTD = D / 8;          // 8-wide output tiles
+    constexpr int TPW = NTD / kConsWarps;  // output tiles per warp (1 or 2)
+    static_assert(NTD % kConsWarps == 0, "head width");
+    const int w = ct >> 5, lane = ct & 31, gid = lane >> 2, tig = lane & 3;
+    const int G = x.G;
     const int b = bh / a.Hkv, h = bh - b * a.Hkv;
-    float *comb = reinterpret_cast<float *>(buf);  // [kConsWarps][D + 2]
-    unsigned char *stage = buf + al((size_t)kConsWarps * (D + 2) * 4, 128);
-    const int CH = (int)((buf_bytes - (size_t)(stage - buf)) / ROW2);
-    float qv[EPLD], o[EPLD];
-    const __nv_bfloat16 *qp =
-        static_cast<const __nv_bfloat16 *>(x.q) + ((size_t)b * x.Hq + (size_t)h * G + g) * D + lane * EPLD;
-#pragma unroll
-    for (int e = 0; e < EPLD; ++e) {
-        qv[e] = __bfloat162float(qp[e]) * x.scale_log2;
-        o[e] = 0.f;
+    // shared memory carve-up
+    unsigned char *q_s = buf;                                  // [16][QSTR]
+    float *red = reinterpret_cast<float *>(buf + 16 * QSTR);   // [kConsWarps][16] partial max / sum
+    float *mlc = red + kConsWarps * 16;                        // m[16], l[16], corr[16]
+    unsigned char *p_s = reinterpret_cast<unsigned char *>(mlc + 48);
+    const size_t fixed = 16 * QSTR + (size_t)kConsWarps * 16 * 4 + 48 * 4;
+    // chunk of CH tokens (a multiple of 16): P [16][CH] bf16 (+16 B per row),
+    // CH staged rows, and the chunk's logits [16][CH] fp32 after them
+    int CH = (int)((buf_bytes - fixed - 16 * 16 - 256) / (ROW2 + 32 + 64)) & ~15;
+    const int need = (kb + 15) & ~15;
+    if (CH > need) CH = need;
+    if (CH < 16) CH = 16;
+    const int PSTR = CH * 2 + 16;  // padded row stride of P (bytes)
+    unsigned char *stage = p_s + (((size_t)16 * PSTR + 127) & ~(size_t)127);
+    const uint32_t q_a = smem_u32(q_s), p_a = smem_u32(p_s), st_a = smem_u32(stage);
+
+    // Q: the G heads' queries as bf16 rows, zero rows up to 16
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(x.q) + ((size_t)b * x.Hq + (size_t)h * G) * D;
+    for (int i = ct; i < 16 * CPR; i += kCons) {
+        const int g = i / CPR, c = i - g * CPR;
+        cp_async16(q_s + g * QSTR + c * 16, g < G ? qg + (size_t)g * D + c * 8 : qg, g < G ? 16u : 0u);
     }
-    float m = -INFINITY, l = 0.f;
+    if (ct < 16) {
+        mlc[ct] = -INFINITY;  // running max (log2 domain)
+        mlc[16 + ct] = 0.f;   // running sum of weights
+    }
+    float o[TPW][4];
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
     const int32_t *idx = a.idx_out + (size_t)bh * a.k;
     const __nv_bfloat16 *Kc = static_cast<const __nv_bfloat16 *>(x.K);
     const __nv_bfloat16 *Vc = static_cast<const __nv_bfloat16 *>(x.V);
+
     for (int c0 = 0; c0 < kb; c0 += CH) {
-        const int n = min(CH, kb - c0);
-        for (int p = ct; p < n * 2 * CPR; p += kCons) {
-            const int row = p / (2 * CPR), rem = p - row * 2 * CPR;
-            const int isv = rem >= CPR, ch = rem - isv * CPR;
-            const int t = idx[c0 + row];
-            const bool ok = (unsigned)t < (unsigned)a.T_cap;
+        const int n = min(CH, kb - c0), n16 = (n + 15) & ~15;
+        // stage K and V rows (zero rows past n), chunk c of token t at c ^ (t & 7)
+        for (int p = ct; p < n16 * 2 * CPR; p += kCons) {
+            const int t = p / (2 * CPR), rem = p - t * 2 * CPR;
+            const int isv = rem >= CPR, c = rem - isv * CPR;
+            int tok = 0;
+            bool ok = false;
+            if (t < n) {
+                tok = idx[c0 + t];
+                ok = (unsigned)tok < (unsigned)a.T_cap;
+            }
             const __nv_bfloat16 *src =
-                (isv ? Vc : Kc) + (((size_t)b * a.T_cap + (ok ? t : 0)) * a.Hkv + h) * D + ch * 8;
-            cp_async16(stage + (size_t)row * ROW2 + isv * D * 2 + ch * 16, src, ok ? 16u : 0u);
+                (isv ? Vc : Kc) + (((size_t)b * a.T_cap + (ok ? tok : 0)) * a.Hkv + h) * D + c * 8;
+            cp_async16(stage + (size_t)t * ROW2 + isv * ROWB + ((c ^ (t & 7)) * 16), src, ok ? 16u : 0u);
         }
         cp_async_commit();
         cp_async_wait<0>();
         cons_sync();
-        for (int j = wi; j < n; j += wph) {
-            const unsigned char *kr = stage + (size_t)j * ROW2 + lane * EPLD * 2;
-            float kf[EPLD], vf[EPLD];
-            if constexpr (EPLD == 4) {
-                const uint2 kk = *reinterpret_cast<const uint2 *>(kr);
-                const uint2 vv = *reinterpret_cast<const uint2 *>(kr + D * 2);
-                kf[0] = bf16_lo(kk.x); kf[1] = bf16_hi(kk.x); kf[2] = bf16_lo(kk.y); kf[3] = bf16_hi(kk.y);
-                vf[0] = bf16_lo(vv.x); vf[1] = bf16_hi(vv.x); vf[2] = bf16_lo(vv.y); vf[3] = bf16_hi(vv.y);
-            } else {
-                const uint4 kk = *reinterpret_cast<const uint4 *>(kr);
-                const uint4 vv = *reinterpret_cast<const uint4 *>(kr + D * 2);
-                Vec16<__nv_bfloat16>::unpack(kk, kf);
-                Vec16<__nv_bfloat16>::unpack(vv, vf);
+
+        // S = Q K^T: warp w takes 8-token tiles w, w + 16, ...
+        const int ntt = n16 / 8;
+        float wmax[2] = {-INFINITY, -INFINITY};
+        for (int nt = w; nt < ntt; nt += kConsWarps) {
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t a0, a1, a2, a3, b0, b1;
+                // A: rows (lane % 16), k chunk 2*ks + lane / 16
+                ldsm_x4(q_a + (lane & 15) * QSTR + (2 * ks + (lane >> 4)) * 16, a0, a1, a2, a3);
+                // B: token rows nt*8 + lane % 8, k chunk 2*ks + (lane / 8) % 2
+                const int t = nt * 8 + (lane & 7), c = 2 * ks + ((lane >> 3) & 1);
+                ldsm_x2(st_a + t * ROW2 + ((c ^ (t & 7)) * 16), b0, b1);
+                mma_bf16_16816(sc, a0, a1, a2, a3, b0, b1);
             }
-            float dot = 0.f;
+            // scaled logits to P (as fp32 bits for now: rows gid, gid + 8; cols 2 tig, +1)
+            const int tc = nt * 8 + 2 * tig;
+            float v[4];
 #pragma unroll
-            for (int e = 0; e < EPLD; ++e) dot = fmaf(qv[e], kf[e], dot);
+            for (int e = 0; e < 4; ++e) {
+                const int row = e < 2 ? gid : gid + 8, col = tc + (e & 1);
+                v[e] = (row < G && col < n) ? sc[e] * x.scale_log2 : -INFINITY;
+            }
+            wmax[0] = fmaxf(wmax[0], fmaxf(v[0], v[1]));
+            wmax[1] = fmaxf(wmax[1], fmaxf(v[2], v[3]));
+            float *srow0 = reinterpret_cast<float *>(stage + (size_t)CH * ROW2);  // [16][CH] fp32 logits
+            srow0[gid * CH + tc] = v[0];
+            srow0[gid * CH + tc + 1] = v[1];
+            srow0[(gid + 8) * CH + tc] = v[2];
+            srow0[(gid + 8) * CH + tc + 1] = v[3];
+        }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-            const float mn = fmaxf(m, dot);
-            const float corr = exp2f(m - mn), pw = exp2f(dot - mn);
-            l = l * corr + pw;
-#pragma unroll
-            for (int e = 0; e < EPLD; ++e) o[e] = fmaf(pw, vf[e], o[e] * corr);
-            m = mn;
+        for (int r = 0; r < 2; ++r) {
+            wmax[r] = fmaxf(wmax[r], __shfl_xor_sync(0xffffffffu, wmax[r], 1));
+            wmax[r] = fmaxf(wmax[r], __shfl_xor_sync(0xffffffffu, wmax[r], 2));
+        }
+        if (tig == 0) {
+            red[w * 16 + gid] = wmax[0];
+            red[w * 16 + gid + 8] = wmax[1];
         }
         cons_sync();
-    }
-    // log-sum-exp combine of the warps of head g
-    float *cw = comb + (size_t)w * (D + 2);
-#pragma unroll
-    for (int e = 0; e < EPLD; ++e) cw[lane * EPLD + e] = o[e];
-    if (lane == 0) {
-        cw[D] = m;
-        cw[D + 1] = l;
-    }
-    cons_sync();
-    if (wi == 0) {
-        float M = -INFINITY;
-        for (int i = 0; i < wph; ++i) M = fmaxf(M, comb[(size_t)(w + i) * (D + 2) + D]);
-        float Ls = 0.f, O[EPLD];
-#pragma unroll
-        for (int e = 0; e < EPLD; ++e) O[e] = 0.f;
-        for (int i = 0; i < wph; ++i) {
-            const float *ci = comb + (size_t)(w + i) * (D + 2);
-            const float mi = ci[D];
-            const float f = mi == -INFINITY ? 0.f : exp2f(mi - M);
-            Ls = fmaf(ci[D + 1], f, Ls);
-#pragma unroll
-            for (int e = 0; e < EPLD; ++e) O[e] = fmaf(ci[lane * EPLD + e], f, O[e]);
+        // running max and correction per row
+        if (ct < 16) {
+            float mx = mlc[ct];
+            for (int i = 0; i < kConsWarps; ++i) mx = fmaxf(mx, red[i * 16 + ct]);
+            const float old = mlc[ct];
+            mlc[32 + ct] = old == -INFINITY ? 0.f : exp2f(old - mx);
+            mlc[ct] = mx;
         }
-        const size_t row_out = (size_t)b * x.Hq + (size_t)h * G + g;
-        __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(x.out) + row_out * D + lane * EPLD;
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        cons_sync();
+        // weights: P = bf16(exp2(s - m)), row sums of the rounded weights
+        {
+            const float *srow0 = reinterpret_cast<const float *>(stage + (size_t)CH * ROW2);
+            for (int i = ct; i < 16 * n16; i += kCons) {
+                const int row = i / n16, col = i - row * n16;
+                const float sv = srow0[row * CH + col];
+                const float mrow = mlc[row];
+                const float pw = (sv == -INFINITY || mrow == -INFINITY) ? 0.f : exp2f(sv - mrow);
+                reinterpret_cast<__nv_bfloat16 *>(p_s + row * PSTR)[col] = __float2bfloat16_rn(pw);
+            }
+        }
+        cons_sync();
+        if (ct < 16 * 16) {  // 16 threads per row sum the row's rounded weights
+            const int row = ct >> 4, sub = ct & 15;
+            float sum = 0.f;
+            const __nv_bfloat16 *pr = reinterpret_cast<const __nv_bfloat16 *>(p_s + row * PSTR);
+            for (int col = sub; col < n16; col += 16) sum += __bfloat162float(pr[col]);
 #pragma unroll
-        for (int e = 0; e < EPLD; ++e) op[e] = __float2bfloat16_rn(O[e] * inv);
-        if (lane == 0 && x.lse) x.lse[row_out] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
+            for (int off = 8; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (sub == 0) mlc[16 + row] = mlc[16 + row] * mlc[32 + row] + sum;
+        }
+        // O = O * corr + P V: warp w takes output tiles w, w + 16
+        const float cr0 = mlc[32 + gid], cr1 = mlc[32 + gid + 8];
+#pragma unroll
+        for (int u = 0; u < TPW; ++u) {
+            o[u][0] *= cr0;
+            o[u][1] *= cr0;
+            o[u][2] *= cr1;
+            o[u][3] *= cr1;
+            const int dt = w + u * kConsWarps;  // 8-dim tile = one 16-byte chunk of the V row
+            for (int ks = 0; ks < n16 / 16; ++ks) {
+                uint32_t a0, a1, a2, a3, b0, b1;
+                ldsm_x4(p_a + (lane & 15) * PSTR + (2 * ks + (lane >> 4)) * 16, a0, a1, a2, a3);
+                const int t = ks * 16 + (lane & 15);
+                ldsm_x2_t(st_a + t * ROW2 + ROWB + ((dt ^ (t & 7)) * 16), b0, b1);
+                mma_bf16_16816(o[u], a0, a1, a2, a3, b0, b1);
+            }
+        }
+        cons_sync();  // before the next chunk overwrites the stage
+    }
+    // out = O / l, lse = (m + log2 l) ln 2, rows g < G
+    const size_t row0 = (size_t)b * x.Hq + (size_t)h * G;
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int g = gid + 8 * hr;
+        if (g >= G) continue;
+        const float l = mlc[16 + g];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(x.out) + (row0 + g) * D;
+#pragma unroll
+        for (int u = 0; u < TPW; ++u) {
+            const int col = (w + u * kConsWarps) * 8 + 2 * tig;
+            *reinterpret_cast<__nv_bfloat162 *>(op + col) =
+                __floats2bfloat162_rn(o[u][2 * hr] * inv, o[u][2 * hr + 1] * inv);
+        }
+        if (w == 0 && tig == 0 && x.lse)
+            x.lse[row0 + g] = l > 0.f ? (mlc[g] + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
     cons_sync();
 }
@@ -974,8 +1095,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
     uint64_t *empty = full + S_;
     uint64_t *efull = empty + S_;  // [kEB]
     uint64_t *efree = efull + kEB; // [kEB]
-    uint64_t *qready = efree + kEB;  // fused: folded queries in shared memory
-    uint64_t *aready = qready + 1;   // fused: new low-rank rows stored
+    uint64_t *qready = efree + kEB;       // fused: folded query of row i in shared memory [kMaxRows]
+    uint64_t *aready = qready + kMaxRows;  // fused: new low-rank rows stored
     uint32_t *ek = reinterpret_cast<uint32_t *>(smem + L.ek);
     int32_t *ei = reinterpret_cast<int32_t *>(smem + L.ei);
     int *misc = reinterpret_cast<int *>(smem + L.misc);
@@ -1005,7 +1126,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             mbar_init(&efree[p], 1);
             misc[40 + p] = 0;
         }
-        mbar_init(qready, 1);
+        for (int i = 0; i < kMaxRows; ++i) mbar_init(&qready[i], 1);
         mbar_init(aready, 1);
         misc[46] = 0;
         fence_barrier_init();
@@ -1074,19 +1195,20 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
         int Tb = 0, e = 0, epos = 0, p = 0;
         uint32_t eph = 0u;  // use parity of epoch buffer p
         uint32_t tag = 0u;
-        bool qok = true;
-        if (FUSED && ntiles > 0) {  // the folded queries come from the selector's prologue
-            qok = __all_sync(0xffffffffu, wait_or_abort(qready, 0u, abort_flag));
-            if (!qok) *abort_flag = 1;
-        }
         Cursor cur = c0;
         RingPos rp(S_);
-        for (int i = 0; qok && i < ntiles; ++i, cur.next(), rp.next()) {
+        for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
             const int bh = cur.bh, t = cur.t, s = rp.s;
             if (i == 0 || t == 0) {
                 Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, ct == 0 ? a.status : nullptr);
                 tag = (uint32_t)bh + 1u;
                 if constexpr (FUSED) {
+                    // the folded query of this row comes from the selector's prologue
+                    const bool qok = __all_sync(0xffffffffu, wait_or_abort(&qready[bh - row0], 0u, abort_flag));
+                    if (!qok) {
+                        *abort_flag = 1;
+                        break;
+                    }
                     const float *qp = qb + (size_t)(bh - row0) * R;
 #pragma unroll
                     for (int c = 0; c < CPT; ++c) {
@@ -1196,9 +1318,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             // the low-rank cache whose tiles this CTA streams
             float *xs = reinterpret_cast<float *>(smem + L.xs);
             float *part = reinterpret_cast<float *>(S.hist);
-            for (int rl = 0; rl < nrows; ++rl)
+            for (int rl = 0; rl < nrows; ++rl) {
                 sel_project<R>(A.x, a.Hkv, row0 + rl, qb + (size_t)rl * R, xs, part, S.st);
-            if (S.st == 0) mbar_arrive(qready);
+                if (S.st == 0) mbar_arrive(&qready[rl]);  // consumers of row rl may start
+            }
             for (int rl = 0; rl < nrows; ++rl) {
                 const int bh = row0 + rl;
                 const int pos = __ldg(A.x.pos_begin + bh / a.Hkv);
@@ -1458,7 +1581,9 @@ cudaError_t plan_step_fused(int B, int Hkv, int Hq, int d, int T_cap, int r, int
         const long long xb = c * p->total_tiles / p->grid, xe = (c + 1) * p->total_tiles / p->grid;
         if (xe > xb && (xe - 1) / p->tiles_per_bh - xb / p->tiles_per_bh + 1 > kMaxRows) return cudaErrorNotSupported;
     }
-    const size_t need = al((size_t)kConsWarps * (d + 2) * 4, 128) + (size_t)4 * d;
+    // attention epilogue: Q, partials, and at least one 16-token chunk
+    const size_t need = 16 * (size_t)(2 * d + 16) + kConsWarps * 16 * 4 + 48 * 4 + 16 * 16 + 256 +
+                        16 * (size_t)(4 * d + 96);
     if ((size_t)p->nstages * kTile < need) return cudaErrorNotSupported;
     return cudaSuccess;
 }

@@ -306,6 +306,29 @@ def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=N
     return out, lse, idx, count
 
 
+class StepGraph:
+    """A call sequence on fixed device buffers (e.g. one jssa_decode_step)
+    captured in a CUDA graph: replay() re-launches the same kernels without
+    host planning or argument marshalling.  The buffers the calls use must
+    stay alive and are updated in place between replays.  One call runs
+    before the capture (on a side stream) so that every plan is made and
+    cached outside it."""
+
+    def __init__(self, fn, device):
+        self.fn = fn
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream(device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            fn()
+
+    def replay(self):
+        self.graph.replay()
+
+
 class DecodeSession:
     """Device-resident state of one attention layer's decode (the public API
     of the end-to-end path): KV cache, low-rank key cache, basis, workspace
@@ -348,17 +371,23 @@ class DecodeSession:
                                            out=self.out, lse=self.lse)
         return out
 
-    def step_from_host(self, q_host, k_new_host, v_new_host):
+    def step_from_host(self, q_host, k_new_host, v_new_host, graph=False):
         """Copy q [B,Hq,d] and the new token's K/V rows [B,Hkv,d] from pinned host
         memory, write the rows at position seq_lens-1, run the step, and copy the
-        output back to pinned host memory (returned; valid after a stream sync)."""
+        output back to pinned host memory (returned; valid after a stream sync).
+        graph=True replays the step from a CUDA graph captured on first use."""
         self._ensure(q_host.shape, q_host.dtype)
         self.q_dev.copy_(q_host, non_blocking=True)
         pos = int(self._host_pos())
         self.K[:, pos].copy_(k_new_host, non_blocking=True)
         if self.V is not None:
             self.V[:, pos].copy_(v_new_host, non_blocking=True)
-        self.step(self.q_dev)
+        if graph:
+            if getattr(self, "_graph", None) is None:
+                self._graph = StepGraph(lambda: self.step(self.q_dev), self.K.device)
+            self._graph.replay()
+        else:
+            self.step(self.q_dev)
         self.out_host.copy_(self.out, non_blocking=True)
         return self.out_host
 
