@@ -179,7 +179,7 @@ int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, 
     L.cand_key = take(L.total, nc * 4);
     L.cand_idx = take(L.total, nc * 4);
     L.cand_cnt = take(L.total, (size_t)sh.BH * L.sp.max_seg * 4);
-    L.sel_ctr = take(L.total, (size_t)sh.BH * 4);
+    L.sel_ctr = take(L.total, (size_t)sh.BH * 2 * 4);  // tickets and publish counts
     return JSSA_OK;
 }
 

@@ -683,42 +683,65 @@ struct RingPos {
     }
 };
 
-// End of a segment (selector): cut to k, publish, and merge if this CTA is
-// the last of the (b,h) to finish.  Returns the selection's size when this
-// CTA merged it, else -1.
+// End of a segment (selector).  The segment takes its arrival ticket first:
+// the last segment of the (b,h) to arrive merges the other segments'
+// published candidates straight into its own uncut candidate set (one exact
+// cut, nothing published); every other segment cuts to k, publishes, and
+// counts itself published.  The last one waits (bounded) for the publish
+// counts of segments that took their tickets before it, which are running
+// and publish without waiting on anything.  Returns the selection's size when
+// this CTA merged it, else -1.  counters[bh] = tickets, counters[BH + bh] =
+// published segments; the merger resets both.
 __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long long cta, int ept, int cap) {
-    if (n > a.k) {
-        sel_reduce(S, n, a.k);
-        n = a.k;
-    }
+    const int BH = a.B * a.Hkv;
     const int tpb = a.tiles_per_bh;
     const long long first = (long long)bh * tpb;
     const long long c_first = ((first + 1) * a.grid - 1) / a.total_tiles;
     const long long c_last = ((first + tpb) * a.grid - 1) / a.total_tiles;
     const int slot = (int)(cta - c_first), nseg = (int)(c_last - c_first + 1);
-    const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
-    for (int j = S.st; j < n; j += kSelT) {
-        a.cand_key[cb + j] = S.rk[j];
-        a.cand_idx[cb + j] = S.ri[j];
-    }
-    if (S.st == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
-    __threadfence();
-    sel_sync();
     if (S.st == 0) S.misc[9] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
     sel_sync();
     const bool last = S.misc[9] != 0;
     sel_sync();
-    if (!last) return -1;
+    if (!last) {
+        if (n > a.k) {
+            sel_reduce(S, n, a.k);
+            n = a.k;
+        }
+        const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
+        for (int j = S.st; j < n; j += kSelT) {
+            a.cand_key[cb + j] = S.rk[j];
+            a.cand_idx[cb + j] = S.ri[j];
+        }
+        if (S.st == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
+        __threadfence();
+        sel_sync();
+        if (S.st == 0) atomicAdd(&a.counters[BH + bh], 1u);
+        return -1;
+    }
+    if (S.st == 0 && nseg > 1) {
+        volatile unsigned *pub = a.counters + BH + bh;
+        const uint64_t t0 = global_timer_ns();
+        while (*pub < (unsigned)(nseg - 1)) {
+            if (global_timer_ns() - t0 > 2000000000ull) {
+                if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
     __threadfence();
-    // merge: segments in ascending token order, chunks of at most ept entries;
-    // equal keys stay candidates (order inside a segment is arbitrary)
-    if (S.st == 0) S.misc[3] = 0;
     sel_sync();
-    int m = 0;
+    // merge the other segments into this one's candidates, in chunks of at
+    // most ept entries; equal keys stay candidates (order is arbitrary)
+    if (S.st == 0) S.misc[3] = n;
+    sel_sync();
+    int m = n;
     bool valid = false;
     uint32_t thr = 0u;
     const int lane = S.st & 31;
     for (int s = 0; s < nseg; ++s) {
+        if (s == slot) continue;
         const int cnt = __ldcg(a.cand_cnt + (size_t)bh * a.max_seg + s);
         const size_t base = ((size_t)bh * a.max_seg + s) * a.k;
         for (int off = 0; off < cnt; off += ept) {
@@ -780,6 +803,7 @@ __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long l
     if (S.st == 0) {
         if (a.count_out) a.count_out[bh] = m;
         a.counters[bh] = 0u;
+        a.counters[BH + bh] = 0u;
     }
     sel_sync();
     return m;
