@@ -117,10 +117,10 @@ struct CSelArgs {
     int32_t *idx_out;         // [BH, k]
     int32_t *count_out;       // [BH] or null
     uint32_t *status;
-    int B, Hkv, T_cap, r, nq, k, csize, slice;
+    int B, Hkv, T_cap, r, nq, k, csize, slice, nstages;
 };
 struct CSelPlan {
-    int csize, slice, grid_y;
+    int csize, slice, grid_y, nstages;
     size_t smem;
 };
 cudaError_t plan_csel(int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p);

@@ -22,6 +22,10 @@ namespace jssa {
 namespace {
 
 constexpr int kPrepThreads = 256;
+constexpr int kPrepThreadsWide = 1024;  // latent rows: 128-head folds and 576-wide dot products
+
+// Threads per CTA for a head width: wide rows get four times the threads.
+inline int prep_threads(int d) { return d > 256 ? kPrepThreadsWide : kPrepThreads; }
 constexpr int kChunk = 16;  // d is a multiple of 16 for every supported shape
 
 // out[o] for o < n_out, with out[o] = sum_i x[row(o)][i] * P[i][col(o)], x in
@@ -96,8 +100,17 @@ __device__ void project_bh(const ProjArgs &a, int bh, float *xs, float *part) {
         cp_async_wait<0>();
         __syncthreads();
         for (int i = threadIdx.x; i < d; i += blockDim.x) {
+            // head order kept; the loads of eight heads are issued together
             float s = 0.f;
-            for (int g = 0; g < G; ++g) s += to_f32(qsm[(size_t)g * d + i]);
+            int g = 0;
+            for (; g + 8 <= G; g += 8) {
+                float v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = to_f32(qsm[(size_t)(g + u) * d + i]);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) s += v[u];
+            }
+            for (; g < G; ++g) s += to_f32(qsm[(size_t)g * d + i]);
             xs[i] = s;
         }
         __syncthreads();
@@ -112,7 +125,7 @@ __device__ void project_bh(const ProjArgs &a, int bh, float *xs, float *part) {
 }
 
 template <typename KV, typename KT>
-__global__ void __launch_bounds__(kPrepThreads) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(kPrepThreadsWide) append_kernel(AppendArgs a) {
     extern __shared__ __align__(16) float sm_prep[];
     pdl_trigger();
     pdl_wait();
@@ -124,7 +137,7 @@ __global__ void __launch_bounds__(kPrepThreads) append_kernel(AppendArgs a) {
 }
 
 template <typename KV>
-__global__ void __launch_bounds__(kPrepThreads) project_kernel(ProjArgs a) {
+__global__ void __launch_bounds__(kPrepThreadsWide) project_kernel(ProjArgs a) {
     extern __shared__ __align__(16) float sm_prep[];
     pdl_trigger();
     pdl_wait();
@@ -136,7 +149,7 @@ __global__ void __launch_bounds__(kPrepThreads) project_kernel(ProjArgs a) {
 // Decode-step prologue: one CTA per (b, h) appends the new row and projects
 // the queries; equal to append_kernel (n_new = 1) followed by project_kernel.
 template <typename KV, typename KT>
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(AppendArgs ap, ProjArgs pj) {
+__global__ void __launch_bounds__(kPrepThreadsWide) prep_kernel(AppendArgs ap, ProjArgs pj) {
     extern __shared__ __align__(16) float sm_prep[];
     pdl_trigger();
     pdl_wait();
@@ -176,7 +189,7 @@ cudaError_t launch_append(const AppendArgs &a0, cudaStream_t s, bool pdl, int kv
         k = kt_dtype == JSSA_BF16 ? append_kernel<float, __nv_bfloat16> : append_kernel<float, float>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(k, grid, dim3(kPrepThreads), smem, s, pdl, a);
+    return launch_kernel(k, grid, dim3(prep_threads(a.d)), smem, s, pdl, a);
 }
 
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype) {
@@ -188,7 +201,7 @@ cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_d
     void (*k)(ProjArgs) = kv_dtype == JSSA_BF16 ? project_kernel<__nv_bfloat16> : project_kernel<float>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(k, dim3(a.B * a.Hkv), dim3(kPrepThreads), smem, s, pdl, a);
+    return launch_kernel(k, dim3(a.B * a.Hkv), dim3(prep_threads(a.d)), smem, s, pdl, a);
 }
 
 cudaError_t launch_prep(const AppendArgs &ap0, const ProjArgs &pj, cudaStream_t s, bool pdl, int kv_dtype,
@@ -210,7 +223,7 @@ cudaError_t launch_prep(const AppendArgs &ap0, const ProjArgs &pj, cudaStream_t 
         k = kt_dtype == JSSA_BF16 ? prep_kernel<float, __nv_bfloat16> : prep_kernel<float, float>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(k, dim3(pj.B * pj.Hkv), dim3(kPrepThreads), smem, s, pdl, ap, pj);
+    return launch_kernel(k, dim3(pj.B * pj.Hkv), dim3(prep_threads(pj.d)), smem, s, pdl, ap, pj);
 }
 
 }  // namespace jssa

@@ -38,7 +38,7 @@ namespace {
 
 constexpr int NT = 256;
 constexpr int kTileB = 32768;   // bytes per ring stage
-constexpr int kStagesC = 2;
+constexpr int kMaxStagesC = 6;  // ring depth: chosen by the planner (2 .. 6)
 constexpr int kBins = 2048;
 constexpr int kMaxSlice = 16384;  // tokens per CTA kept in shared memory
 
@@ -48,13 +48,13 @@ struct CSmem {
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) / 16 * 16; }
 
-__host__ __device__ inline CSmem csel_smem(bool from_kt, int r, int nq, int slice) {
+__host__ __device__ inline CSmem csel_smem(bool from_kt, int r, int nq, int slice, int nstages) {
     CSmem L;
     size_t o = 0;
     L.stages = o;
-    o += from_kt ? (size_t)kStagesC * kTileB : 0;
+    o += from_kt ? (size_t)nstages * kTileB : 0;
     L.bars = o;
-    o = align16(o + 64);
+    o = align16(o + 8 * kMaxStagesC);
     L.qs = o;
     o = align16(o + (from_kt ? (size_t)nq * r * 4 : 0));
     L.keys = o;
@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
     static_assert(!FROM_KT || TILE % TPP == 0, "tile / pass");
 
     extern __shared__ __align__(128) unsigned char smem[];
-    const CSmem L = csel_smem(FROM_KT, FROM_KT ? R : 0, a.nq, a.slice);
+    const int NS = a.nstages;
+    const CSmem L = csel_smem(FROM_KT, FROM_KT ? R : 0, a.nq, a.slice, NS);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
     float *qs = reinterpret_cast<float *>(smem + L.qs);
     uint32_t *keys = reinterpret_cast<uint32_t *>(smem + L.keys);
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
     const int tid = threadIdx.x, lane = tid & 31;
 
     if (FROM_KT && tid == 0) {
-        for (int s = 0; s < kStagesC; ++s) mbar_init(&bars[s], 1);
+        for (int s = 0; s < NS; ++s) mbar_init(&bars[s], 1);
         fence_barrier_init();
     }
     if (tid == 0) misc[6] = 0;
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
         uint64_t pol = 0;
         if (tid == 0) {
             pol = policy_evict_first();
-            for (int i = 0; i < min(kStagesC, ntiles); ++i) {
+            for (int i = 0; i < min(NS, ntiles); ++i) {
                 const int n = min(TILE, n_loc - i * TILE);
                 mbar_arrive_expect_tx(&bars[i], (uint32_t)n * ROWB);
                 bulk_g2s(smem + L.stages + (size_t)i * kTileB, src + (size_t)i * TILE * ROWB, (uint32_t)n * ROWB, &bars[i],
@@ -153,9 +154,9 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
             }
         }
         for (int i = 0; i < ntiles; ++i) {
-            const int s = i % kStagesC;
+            const int s = i % NS;
             const int t0 = i * TILE, n = min(TILE, n_loc - t0);
-            if (!mbar_wait_bounded(&bars[s], (uint32_t)(i / kStagesC) & 1u)) misc[6] = 1;
+            if (!mbar_wait_bounded(&bars[s], (uint32_t)(i / NS) & 1u)) misc[6] = 1;
             const unsigned char *st = smem + L.stages + (size_t)s * kTileB;
 #pragma unroll
             for (int ps = 0; ps < PASSES; ++ps) {
@@ -210,10 +211,10 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
                 if (live && sub == 0) keys[t0 + tt] = score_key(sc);
             }
             __syncthreads();  // stage s consumed
-            if (tid == 0 && i + kStagesC < ntiles) {
-                const int n2 = min(TILE, n_loc - (i + kStagesC) * TILE);
+            if (tid == 0 && i + NS < ntiles) {
+                const int n2 = min(TILE, n_loc - (i + NS) * TILE);
                 mbar_arrive_expect_tx(&bars[s], (uint32_t)n2 * ROWB);
-                bulk_g2s(smem + L.stages + (size_t)s * kTileB, src + (size_t)(i + kStagesC) * TILE * ROWB,
+                bulk_g2s(smem + L.stages + (size_t)s * kTileB, src + (size_t)(i + NS) * TILE * ROWB,
                          (uint32_t)n2 * ROWB, &bars[s], pol);
             }
         }
@@ -482,19 +483,29 @@ cudaError_t plan_csel_uncached(int form, int src, int agg, int B, int Hkv, int T
         int slice = (T_cap + C - 1) / C;
         slice = (slice + tile - 1) / tile * tile;
         if (slice > kMaxSlice) break;  // smaller clusters only lengthen the slices
-        const size_t smem = csel_smem(src != SRC_SCORES, src == SRC_SCORES ? 0 : r, nq, slice).total;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        const int ncl = resident_clusters(kern, C, smem);
-        if (ncl < 1) continue;
-        if (form == 0 && ncl < BH) continue;
-        p->csize = C;
-        p->slice = slice;
-        p->smem = smem;
-        p->grid_y = BH;
-        return cudaSuccess;
+        // deepest ring (most bytes in flight per CTA) that keeps the wave resident
+        for (int ns = kMaxStagesC; ns >= 2; --ns) {
+            if (src == SRC_SCORES && ns != 2) continue;  // no ring for a score source
+            const size_t smem = csel_smem(src != SRC_SCORES, src == SRC_SCORES ? 0 : r, nq, slice, ns).total;
+            int optin = 0, dev = 0;
+            cudaError_t e = cudaGetDevice(&dev);
+            if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+            if (e != cudaSuccess) return e;
+            if (smem > (size_t)optin) continue;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            const int ncl = resident_clusters(kern, C, smem);
+            if (ncl < 1) continue;
+            if (form == 0 && ncl < BH) continue;
+            p->csize = C;
+            p->slice = slice;
+            p->smem = smem;
+            p->grid_y = BH;
+            p->nstages = ns;
+            return cudaSuccess;
+        }
     }
     return cudaErrorNotSupported;
 }
@@ -551,6 +562,7 @@ cudaError_t launch_csel(const CSelPlan &p, const CSelArgs &a0, int src, int agg,
     CSelArgs a = a0;
     a.csize = p.csize;
     a.slice = p.slice;
+    a.nstages = p.nstages;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.csize, p.grid_y);
     cfg.blockDim = dim3(NT);

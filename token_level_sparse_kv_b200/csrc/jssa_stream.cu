@@ -14,8 +14,8 @@
 //  * 16 consumer warps score every token of a tile (the same fp32 arithmetic,
 //    lane rotation and chunk order as the score pass, so scores are
 //    bit-identical) and append the tokens whose order-preserving key beats the
-//    current threshold to an epoch buffer (two buffers, alternating epochs of
-//    >= 1024 tokens);
+//    current threshold to an epoch buffer (three buffers, rotating epochs of
+//    >= 2048 tokens);
 //  * 4 selector warps fold each finished epoch into the running candidate set
 //    of the segment, cut it back to the best k with a radix select when it
 //    fills, and publish the k-th key (tagged with the segment) as the new
@@ -56,7 +56,7 @@ constexpr int kTile = 32768;                      // bytes per ring stage
 constexpr int kMaxStages = 8;
 constexpr int kBins = 2048;                       // 11-bit digits
 constexpr int kBoundary = 64;                     // boundary group ranked exactly
-constexpr int kEpochTokens = 1024;                // minimum tokens per epoch
+constexpr int kEpochTokens = 2048;                // minimum tokens per epoch
 constexpr int kMaxRows = 8;                       // (b,h) rows per CTA range on the fused step
 constexpr int kChunkD = 16;                       // inputs per partial sum of a projection
 
@@ -1523,7 +1523,9 @@ cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T
     P.tile_tokens = tile;
     P.tiles_per_bh = (T_cap + tile - 1) / tile;
     P.total_tiles = (long long)B * Hkv * P.tiles_per_bh;
-    P.cap = k + 2 * ept;
+    // candidate capacity: the kept set after a cut (k plus up to 1024 more
+    // before the next cut) and one epoch of new survivors
+    P.cap = k + ept + 1024;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
