@@ -310,6 +310,43 @@ def time_loop(fn, steps, stream, events_inside=None):
     return start.elapsed_time(end) / 1e3
 
 
+def measure_decode_loop(dev, n_layers, steps, stream):
+    """Steady-state steps/s of an n_layers attention stack at the 4K/B1 GQA
+    layer shape (each layer's output is the next layer's query), eager calls
+    vs one CUDA graph per step (every layer plus the position advance)."""
+    import torch
+
+    from token_level_sparse_kv_b200 import ops
+    from token_level_sparse_kv_b200.inputs import WORKLOADS, Workload, make_inputs
+
+    w0 = WORKLOADS["gqa_4k_b1"]
+    room = 2 * steps + 16
+    layers = []
+    for l in range(n_layers):
+        w = Workload(**{**w0.__dict__, "seed": w0.seed + 7000 + l})
+        q, K, V, P, sl = make_inputs(w, device=dev)
+        layers.append((K, V, P, ops.build_lowrank_cache(K, P)))
+    res = {"layers": n_layers, "shape": "GQA layer B=1, Hq=32, Hkv=8, d=128, T=4096, r=32, k=256"}
+    for mode in ("eager", "graph"):
+        sl = torch.full((w0.B,), w0.T - room, dtype=torch.int32, device=dev)
+        pos = sl - 1
+        loop = ops.DecodeLoop(layers, sl, pos, w0.k, w0.scale)
+        loop.set_query(q)
+        g = mode == "graph"
+        for _ in range(3):
+            loop.step(graph=g)
+        torch.cuda.synchronize()
+        secs = time_loop(lambda i: loop.step(graph=g), steps, stream)
+        res[mode] = {"steps_per_s": steps / secs, "us_per_step": secs / steps * 1e6,
+                     "us_per_layer": secs / steps / n_layers * 1e6}
+    res["launches_per_step"] = n_layers * ops.plan_info(ops.make_dims(q, layers[0][0], layers[0][1], P=layers[0][2],
+                                                                       Kt=layers[0][3]), w0.k,
+                                                        ops.OP_DECODE_STEP)[0] + 2
+    del layers
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_jssa(args, world, rank, local):
     import torch
 
@@ -490,6 +527,9 @@ def run_jssa(args, world, rank, local):
         line["e2e"] = {"value": world * e2e_steps / te, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h,
                        "api": "DecodeSession.step_from_host (pinned host in/out%s)" % (", graph=True" if use_graph else "")}
+
+    if not args.quick and world == 1:
+        line["decode_loop"] = measure_decode_loop(dev, 32, 20, stream)
 
     if rank == 0 and not args.no_cpu:
         v, desc, thr = oracle_baseline(w0, args.cpu_seconds, max(1, min(w0.B, args.cpu_rows)), os.cpu_count() or 1)

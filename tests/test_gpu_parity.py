@@ -550,3 +550,54 @@ def test_select_forms_agree_full_size(wname, monkeypatch):
         assert torch.equal(res[0][0], r[0]) and torch.equal(res[0][1], r[1])
     del q, K, V, Kt
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------- multi-layer decode loop
+def _loop_layers(w, L, seed0):
+    layers, cpu = [], []
+    for l in range(L):
+        wl = Workload(**{**w.__dict__, "seed": seed0 + l})
+        (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(wl, seq_lens=[w.T - 8] * w.B)
+        Kt = ops.build_lowrank_cache(Kd, Pd)
+        layers.append((Kd, Vd, Pd, Kt))
+        cpu.append((q, K, V, P))
+    return layers, cpu
+
+
+def test_decode_loop_graph_matches_eager_and_oracle():
+    """An L-layer stack stepped three times eagerly and by CUDA-graph replay
+    (the graph holds every layer and the device-side position advance) gives
+    bit-identical selections, low-rank rows and outputs; the last step's first
+    layer matches the oracle."""
+    w = W(B=2, Hq=8, Hkv=2, T=3000, k=64, seed=90)
+    L = 3
+    layers_a, cpu = _loop_layers(w, L, 900)
+    layers_b = [tuple(t.clone() for t in lay) for lay in layers_a]
+    q0 = cpu[0][0].to(DEV)
+    sl_a = torch.full((w.B,), w.T - 8, dtype=torch.int32, device=DEV)
+    pos_a = sl_a - 1
+    sl_b, pos_b = sl_a.clone(), pos_a.clone()
+    loop_a = ops.DecodeLoop(layers_a, sl_a, pos_a, w.k, w.scale)
+    loop_b = ops.DecodeLoop(layers_b, sl_b, pos_b, w.k, w.scale)
+    loop_a.set_query(q0)
+    loop_b.set_query(q0)
+    for _ in range(3):
+        loop_a.step()
+    loop_b.capture()  # runs one step
+    for _ in range(2):
+        loop_b.step(graph=True)
+    torch.cuda.synchronize()
+    assert torch.equal(sl_a, sl_b) and int(sl_a[0]) == w.T - 8 + 3
+    for l in range(L):
+        assert torch.equal(loop_a.idx[l], loop_b.idx[l])
+        assert torch.equal(loop_a.out[l], loop_b.out[l])
+        assert torch.equal(layers_a[l][3], layers_b[l][3])
+    # oracle: layer 0 of the last step (sequence length T-8+2, position T-8+1)
+    q, K, V, P = cpu[0]
+    slh = torch.full((w.B,), w.T - 8 + 2, dtype=torch.int32)
+    Kt0 = layers_a[0][3]
+    check_append(Kt0, K, P, [w.T - 8 + 1] * w.B, 1)
+    ref_s = oracle.score(q, P, host(Kt0), slh)
+    check_selection(host(loop_a.idx[0]).numpy(), host(loop_a.count[0]).numpy(), ref_s, slh.numpy(), w.k)
+    ref_o, ref_l = oracle.attend(q, K, V, host(loop_a.idx[0]), host(loop_a.count[0]), slh, w.scale)
+    check_attention(loop_a.out[0], loop_a.lse[0], ref_o, ref_l, torch.bfloat16)

@@ -398,3 +398,76 @@ class DecodeSession:
                 raise ValueError("step_from_host needs one shared position across the batch")
             self._pos_cache = int(p[0])
         return self._pos_cache
+
+
+class DecodeLoop:
+    """Multi-layer, multi-step decode of an attention stack (the loop around
+    the hot path): each step runs jssa_decode_step on every layer in turn,
+    layer l + 1 taking layer l's output as its query (d == dv), then advances
+    the shared sequence position on the device (seq_lens += 1, pos += 1).
+    The new token's K/V rows are expected at position pos of each layer's
+    cache before a step (a model writes them; this loop does not).
+
+    layers: list of (K, V, P, Kt) per layer, all of one shape; seq_lens,
+    pos: [B] int32 device tensors shared by the layers (advanced in place).
+    step() runs eagerly; capture() records one whole step (every layer and
+    the position advance) as a CUDA graph, replayed by step(graph=True)."""
+
+    def __init__(self, layers, seq_lens, pos, k, scale, agg=AGG_SUM):
+        if not layers:
+            raise ValueError("DecodeLoop needs at least one layer")
+        self.layers = layers
+        self.seq_lens, self.pos = seq_lens, pos
+        self.k, self.scale, self.agg = int(k), float(scale), int(agg)
+        K0, V0, P0, Kt0 = layers[0]
+        B, T_cap, Hkv, d = K0.shape
+        self.T_cap = T_cap
+        self._graph = None
+        self.q = None
+
+    def _ensure(self, q):
+        if self.q is not None and tuple(self.q.shape) == tuple(q.shape):
+            return
+        K0, V0, P0, Kt0 = self.layers[0]
+        dims = make_dims(q, K0, V0, P=P0, Kt=Kt0)
+        if dims.dv != dims.d:
+            raise ValueError("a chained stack needs dv == d")
+        dev = q.device
+        self.q = torch.empty_like(q)
+        self.ws = new_workspace(dims, self.k, OP_DECODE_STEP, dev)
+        self.idx = [torch.empty((dims.B, dims.Hkv, self.k), dtype=torch.int32, device=dev) for _ in self.layers]
+        self.count = [torch.empty((dims.B, dims.Hkv), dtype=torch.int32, device=dev) for _ in self.layers]
+        self.out = [torch.empty((dims.B, dims.Hq, dims.dv), dtype=q.dtype, device=dev) for _ in self.layers]
+        self.lse = [torch.empty((dims.B, dims.Hq), dtype=torch.float32, device=dev) for _ in self.layers]
+
+    def _run(self):
+        x = self.q
+        for l, (K, V, P, Kt) in enumerate(self.layers):
+            decode_step(x, K, V, P, Kt, self.seq_lens, self.pos, self.k, self.scale, agg=self.agg, ws=self.ws,
+                        idx=self.idx[l], count=self.count[l], out=self.out[l], lse=self.lse[l])
+            x = self.out[l]
+        self.seq_lens.add_(1)
+        self.pos.add_(1)
+
+    def set_query(self, q):
+        """Copy the first layer's query for the next step (device tensor)."""
+        self._ensure(q)
+        self.q.copy_(q)
+
+    def capture(self):
+        """Record one whole step as a CUDA graph (runs one eager step first, on
+        a side stream, which also advances the position once)."""
+        if self.q is None:
+            raise RuntimeError("set_query() before capture()")
+        self._graph = StepGraph(self._run, self.q.device)
+        return self._graph
+
+    def step(self, graph=False):
+        """One decode step of the whole stack; returns the last layer's output."""
+        if graph:
+            if self._graph is None:
+                self.capture()
+            self._graph.replay()
+        else:
+            self._run()
+        return self.out[-1]
