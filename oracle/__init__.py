@@ -64,6 +64,8 @@ def lib():
         L.oracle_score.argtypes = [i32] * 6 + [vp, i32, vp, vp, i32, vp, i32, vp, i32, vp]
         L.oracle_topk.restype = i32
         L.oracle_topk.argtypes = [i32, i32, i32, vp, vp, i32, vp, i32, vp, vp]
+        L.oracle_topk_forced.restype = i32
+        L.oracle_topk_forced.argtypes = [i32, i32, i32, vp, vp, i32, i32, i32, vp, i32, vp, vp]
         L.oracle_attend.restype = i32
         L.oracle_attend.argtypes = [i32] * 6 + [vp, i32, vp, vp, i32, i32, vp, vp, i32, vp, dbl, vp, i32, vp, vp]
         L.oracle_dense.restype = i32
@@ -198,15 +200,21 @@ def score(q, P, Kt, seq_lens, agg=AGG_SUM, bh_list=None):
     return out
 
 
-def topk(scores, seq_lens, k, bh_list=None):
-    """Per-(b,h) top-k by (score desc, index asc); ascending indices, -1 padded."""
+def topk(scores, seq_lens, k, bh_list=None, n_sink=0, n_recent=0):
+    """Per-(b,h) top-k by (score desc, index asc); ascending indices, -1 padded.
+    n_sink / n_recent: tokens [0, n_sink) and [T_b - n_recent, T_b) are always
+    selected (smallest indices first when they alone exceed k_b)."""
     s = np.ascontiguousarray(np.asarray(scores, dtype=np.float64))
     B, Hkv, T_cap = s.shape
     sl = _i32(seq_lens)
     bh, nbh = _bh(bh_list)
     idx = np.full((B, Hkv, k), -1, dtype=np.int32)
     cnt = np.zeros((B, Hkv), dtype=np.int32)
-    rc = lib().oracle_topk(B, Hkv, T_cap, _p(s), _p(sl), int(k), _p(bh), nbh, _p(idx), _p(cnt))
+    if n_sink or n_recent:
+        rc = lib().oracle_topk_forced(B, Hkv, T_cap, _p(s), _p(sl), int(k), int(n_sink), int(n_recent), _p(bh), nbh,
+                                      _p(idx), _p(cnt))
+    else:
+        rc = lib().oracle_topk(B, Hkv, T_cap, _p(s), _p(sl), int(k), _p(bh), nbh, _p(idx), _p(cnt))
     if rc != 0:
         raise ValueError("oracle_topk: bad arguments (rc=%d)" % rc)
     return idx, cnt
@@ -270,7 +278,7 @@ def dense(q, K, V, seq_lens, scale, window=0, dv=None, bh_list=None, v_aliases_k
 
 
 def step(q, K, V, P, Kt, seq_lens, k, scale, pos_begin=None, n_new=1, agg=AGG_SUM, dv=None,
-         bh_list=None, v_aliases_k=False, kt_dtype=None):
+         bh_list=None, v_aliases_k=False, kt_dtype=None, n_sink=0, n_recent=0):
     """One decode step: append n_new rows at pos_begin, score, select, attend.
 
     Kt (numpy bits / fp32, or torch CPU tensor) holds the prefix low-rank cache and
@@ -283,7 +291,7 @@ def step(q, K, V, P, Kt, seq_lens, k, scale, pos_begin=None, n_new=1, agg=AGG_SU
     if pos_begin is not None and n_new > 0:
         Ktr = append_lowrank(K, P, pos_begin, n_new, kt_dtype=code, Kt=Ktr)
     s = score(q, P, Ktr, seq_lens, agg=agg, bh_list=bh_list)
-    idx, cnt = topk(s, seq_lens, k, bh_list=bh_list)
+    idx, cnt = topk(s, seq_lens, k, bh_list=bh_list, n_sink=n_sink, n_recent=n_recent)
     out, lse = attend(q, K, V, idx, cnt, seq_lens, scale, dv=dv, bh_list=bh_list, v_aliases_k=v_aliases_k)
     return Ktr, s, idx, cnt, out, lse
 

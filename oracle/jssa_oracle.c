@@ -249,6 +249,57 @@ int oracle_topk(int B, int Hkv, int T_cap, const double *scores,
     return 0;
 }
 
+/* Top-k with forced tokens [selection variant; the pages are silent on it: a
+ * reading of "sink" and "recent-window" tokens that sparse decoders keep].
+ * F = {t < n_sink} U {t >= T_b - n_recent}, t in [0, T_b).  If |F| >= k_b
+ * the selection is the k_b smallest indices of F; otherwise it is F plus the
+ * k_b - |F| tokens outside F that come first under (s desc, t asc).  Emitted
+ * in ascending t, -1 padded.  n_sink = n_recent = 0 is oracle_topk. */
+int oracle_topk_forced(int B, int Hkv, int T_cap, const double *scores,
+                       const int32_t *seq_lens, int k, int n_sink, int n_recent,
+                       const int32_t *bh_list, int n_bh, int32_t *idx, int32_t *count)
+{
+    if (k < 1 || n_sink < 0 || n_recent < 0)
+        return -1;
+    int n = bh_list ? n_bh : B * Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int w = 0; w < n; ++w) {
+        int bh = bh_list ? bh_list[w] : w;
+        int b = bh / Hkv;
+        int Tb = clamp_len(seq_lens[b], T_cap);
+        int kb = k < Tb ? k : Tb;
+        int32_t *out = idx + (size_t)bh * k;
+        int nf = 0;
+        for (int t = 0; t < Tb; ++t) {
+            int forced = t < n_sink || t >= Tb - n_recent;
+            if (forced && nf < kb)
+                out[nf++] = t; /* ascending, the smallest indices first */
+        }
+        int rest = kb - nf;
+        if (rest > 0) {
+            or_pair *pr = (or_pair *)malloc(sizeof(or_pair) * (size_t)(Tb > 0 ? Tb : 1));
+            int m = 0;
+            for (int t = 0; t < Tb; ++t) {
+                if (t < n_sink || t >= Tb - n_recent)
+                    continue;
+                pr[m].s = scores[(size_t)bh * T_cap + t];
+                pr[m].t = t;
+                ++m;
+            }
+            qsort(pr, (size_t)m, sizeof(or_pair), cmp_pair);
+            for (int j = 0; j < rest; ++j)
+                out[nf + j] = pr[j].t;
+            free(pr);
+        }
+        qsort(out, (size_t)kb, sizeof(int32_t), cmp_i32);
+        for (int j = kb; j < k; ++j)
+            out[j] = -1;
+        if (count)
+            count[bh] = kb;
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- attend ---
  * Attention over a given token list per (b, h) [NEWS Interpretation para 3:
  * the selected key-value entries are read in place and attended as usual;

@@ -386,3 +386,51 @@ def test_basis_is_orthonormal():
     eye = torch.eye(16, dtype=torch.float64)
     for h in range(3):
         torch.testing.assert_close(P[h].T @ P[h], eye, rtol=0, atol=1e-6)
+
+
+# ------------------------------------------------ forced sink / recent tokens
+def _forced_by_lexsort(s, Tb, k, n_sink, n_recent):
+    """Independent statement of the forced selection: order the tokens by
+    (forced first; among forced tokens by index; among the others by score
+    desc, then index) with numpy's lexsort, keep k_b."""
+    t = np.arange(Tb)
+    forced = (t < n_sink) | (t >= Tb - n_recent)
+    kb = min(k, Tb)
+    order = np.lexsort((t, np.where(forced, 0.0, -s[:Tb]), ~forced))
+    return np.sort(order[:kb])
+
+
+@pytest.mark.parametrize("n_sink,n_recent", [(0, 0), (4, 0), (0, 16), (4, 16), (30, 30), (200, 0)])
+def test_topk_forced_matches_lexsort_statement(n_sink, n_recent):
+    rng = np.random.default_rng(100 + n_sink + n_recent)
+    B, Hkv, T = 3, 2, 300
+    s = rng.normal(size=(B, Hkv, T))
+    s[0, 1] = np.round(s[0, 1] * 2) / 2  # heavy exact ties
+    sl = np.array([300, 57, 5], dtype=np.int32)
+    for k in (1, 16, 64, 400):
+        idx, cnt = oracle.topk(s, sl, k, n_sink=n_sink, n_recent=n_recent)
+        for b in range(B):
+            for h in range(Hkv):
+                ref = _forced_by_lexsort(s[b, h], int(sl[b]), k, n_sink, n_recent)
+                assert cnt[b, h] == len(ref)
+                np.testing.assert_array_equal(idx[b, h, :len(ref)], ref)
+                assert np.all(idx[b, h, len(ref):] == -1)
+
+
+def test_topk_forced_plain_case_and_invariants():
+    rng = np.random.default_rng(7)
+    s = rng.normal(size=(1, 1, 500))
+    sl = np.array([500], dtype=np.int32)
+    i0, c0 = oracle.topk(s, sl, 64)
+    i1, c1 = oracle.topk(s, sl, 64, n_sink=0, n_recent=0)
+    np.testing.assert_array_equal(i0, i1)
+    idx, cnt = oracle.topk(s, sl, 64, n_sink=4, n_recent=8)
+    sel = set(idx[0, 0].tolist())
+    forced = set(range(4)) | set(range(492, 500))
+    assert forced <= sel and cnt[0, 0] == 64
+    rest = sorted(sel - forced)
+    outside = [t for t in range(500) if t not in sel and t not in forced]
+    assert min(s[0, 0, rest]) >= max(s[0, 0, outside])  # the free slots hold the best of the rest
+    # forced tokens alone exceed k: the smallest forced indices
+    idx, cnt = oracle.topk(s, sl, 6, n_sink=4, n_recent=8)
+    assert idx[0, 0].tolist() == [0, 1, 2, 3, 492, 493]
