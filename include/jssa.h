@@ -192,6 +192,28 @@ JSSA_API int jssa_select(const jssa_dims *dims, const void *q, const float *P, c
                 const int32_t *seq_lens, int agg, int k, int32_t *idx, int32_t *count,
                 void *ws, size_t ws_bytes, jssa_stream_t stream);
 
+/* Selection options: tokens that are always selected.  A variant the pages
+ * do not describe (their selection is a pure top-k); the reading is the usual
+ * one of sparse decoders that keep "sink" tokens and a recent window.  With
+ * F = {t < n_sink} U {t >= T_b - n_recent} (t < T_b): if |F| >= k_b the
+ * selection is the k_b smallest indices of F, otherwise F plus the k_b - |F|
+ * best other tokens under (score desc, t asc).  NULL or zeros: plain top-k. */
+typedef struct {
+    int32_t n_sink;   /* >= 0 */
+    int32_t n_recent; /* >= 0 */
+} jssa_select_opts;
+
+/* jssa_topk, jssa_select and jssa_decode_step with selection options (NULL
+ * = the plain calls).  jssa_select_ex stays bit-identical to jssa_score +
+ * jssa_topk_ex with the same options.  Errors: JSSA_ERR_INVALID_ARG for a
+ * negative count. */
+JSSA_API int jssa_topk_ex(const jssa_dims *dims, const float *scores, const int32_t *seq_lens, int k,
+                 const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
+                 jssa_stream_t stream);
+JSSA_API int jssa_select_ex(const jssa_dims *dims, const void *q, const float *P, const void *Kt,
+                   const int32_t *seq_lens, int agg, int k, const jssa_select_opts *opts, int32_t *idx,
+                   int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream);
+
 /* Gather-free indexed attention [ABS: token-level indexed-attention kernel
  * with distinct per-KV-head selections under the standard GQA cache layout;
  * NEWS Interpretation para 3: selected tokens are read in place through their
@@ -232,6 +254,13 @@ JSSA_API int jssa_decode_step(const jssa_dims *dims, const void *q, const void *
                      const int32_t *pos_begin, int k, int agg, float softmax_scale,
                      int32_t *idx, int32_t *count, void *out, float *lse, void *ws,
                      size_t ws_bytes, jssa_stream_t stream);
+
+/* jssa_decode_step with selection options (NULL = jssa_decode_step). */
+JSSA_API int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                        const float *P, void *Kt, const int32_t *seq_lens, const int32_t *pos_begin, int k,
+                        int agg, float softmax_scale, const jssa_select_opts *opts, int32_t *idx,
+                        int32_t *count, void *out, float *lse, void *ws, size_t ws_bytes,
+                        jssa_stream_t stream);
 
 /* Allocation-free variant of jssa_indexed_decode.  The method pages have no
  * counterpart: this is an integration entry point of this library.

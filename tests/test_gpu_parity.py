@@ -601,3 +601,40 @@ def test_decode_loop_graph_matches_eager_and_oracle():
     check_selection(host(loop_a.idx[0]).numpy(), host(loop_a.count[0]).numpy(), ref_s, slh.numpy(), w.k)
     ref_o, ref_l = oracle.attend(q, K, V, host(loop_a.idx[0]), host(loop_a.count[0]), slh, w.scale)
     check_attention(loop_a.out[0], loop_a.lse[0], ref_o, ref_l, torch.bfloat16)
+
+
+# ------------------------------------------- forced sink / recent tokens
+@pytest.mark.parametrize("n_sink,n_recent", [(4, 0), (0, 32), (4, 32), (300, 0)])
+def test_forced_tokens_every_form(n_sink, n_recent, form):
+    """Always-selected first / last tokens: every selection form, the fused
+    pass and score + top-k agree bit for bit, and equal the oracle's forced
+    top-k on the GPU's own fp32 scores."""
+    w, sl = W(B=3, Hkv=2, Hq=8, T=20000, k=256, seed=95), [20000, 3000, 100]
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k, n_sink=n_sink, n_recent=n_recent)
+    s = ops.score(qd, Pd, Kt, sld)
+    idx2, cnt2 = ops.topk(s, sld, w.k, n_sink=n_sink, n_recent=n_recent)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(idx).numpy(), host(idx2).numpy())
+    np.testing.assert_array_equal(host(cnt).numpy(), host(cnt2).numpy())
+    ref_idx, ref_cnt = oracle.topk(host(s).double().numpy(), slh, w.k, n_sink=n_sink, n_recent=n_recent)
+    np.testing.assert_array_equal(host(idx).numpy(), ref_idx)
+    np.testing.assert_array_equal(host(cnt).numpy(), ref_cnt)
+
+
+@pytest.mark.parametrize("fused", ["1", "0"])
+def test_forced_tokens_decode_step(fused, monkeypatch):
+    monkeypatch.setenv("JSSA_SELECT_FORM", "stream")
+    monkeypatch.setenv("JSSA_FUSED_STEP", fused)
+    w, sl = W(B=2, T=30000, k=256, seed=96), [30000, 20001]
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    pos = (slh - 1).clamp_min(0)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    out, lse, idx, cnt = ops.decode_step(qd, Kd, Vd, Pd, Kt, sld, pos.to(DEV), w.k, w.scale, n_sink=4, n_recent=64)
+    s = ops.score(qd, Pd, Kt, sld)
+    torch.cuda.synchronize()
+    ref_idx, ref_cnt = oracle.topk(host(s).double().numpy(), slh, w.k, n_sink=4, n_recent=64)
+    np.testing.assert_array_equal(host(idx).numpy(), ref_idx)
+    ref_o, ref_l = oracle.attend(q, K, V, host(idx), host(cnt), slh, w.scale)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)

@@ -347,7 +347,8 @@ void fill_attn(AttnArgs &a, const jssa_dims *d, const Shape &sh, const void *q, 
 
 int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *P, const void *Kt,
                const int32_t *seq_lens, int agg, int k, int32_t *idx, int32_t *count, void *ws, const Layout &L,
-               cudaStream_t s, bool with_project) {
+               cudaStream_t s, bool with_project, const jssa_select_opts *opts) {
+    const int n_sink = opts ? opts->n_sink : 0, n_recent = opts ? opts->n_recent : 0;
     const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
     if (with_project) {
         ProjArgs pj{q, P, at<float>(ws, L.qproj), d->B, d->Hq, d->Hkv, d->d, d->r, agg};
@@ -369,6 +370,8 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
         ca.r = d->r;
         ca.nq = nq;
         ca.k = k;
+        ca.n_sink = n_sink;
+        ca.n_recent = n_recent;
         // a null query means the source is a score array (jssa_topk)
         const int src = q == nullptr ? SRC_SCORES : (d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32);
         cudaError_t e = launch_csel(L.cp, ca, src, q == nullptr ? JSSA_AGG_SUM : agg, s, true);
@@ -393,6 +396,8 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
     sa.r = d->r;
     sa.nq = nq;
     sa.k = k;
+    sa.n_sink = n_sink;
+    sa.n_recent = n_recent;
     cudaError_t e = L.wspec ? launch_stream(L.sp, sa, s, true) : launch_scan(L.sp, sa, agg, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the selection pass");
     return JSSA_OK;
@@ -571,8 +576,21 @@ int jssa_score(const jssa_dims *dims, const void *q, const float *P, const void 
     return JSSA_OK;
 }
 
+int check_opts(const jssa_select_opts *opts) {
+    if (opts && (opts->n_sink < 0 || opts->n_recent < 0))
+        return fail(JSSA_ERR_INVALID_ARG, "negative forced-token count (n_sink=%d, n_recent=%d)", opts->n_sink,
+                    opts->n_recent);
+    return JSSA_OK;
+}
+
 int jssa_topk(const jssa_dims *dims, const float *scores, const int32_t *seq_lens, int k, int32_t *idx,
               int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    return jssa_topk_ex(dims, scores, seq_lens, k, nullptr, idx, count, ws, ws_bytes, stream);
+}
+
+int jssa_topk_ex(const jssa_dims *dims, const float *scores, const int32_t *seq_lens, int k,
+                 const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
+                 jssa_stream_t stream) {
     Shape sh;
     int st = check_dims(dims, &sh);
     if (st) return st;
@@ -585,12 +603,19 @@ int jssa_topk(const jssa_dims *dims, const float *scores, const int32_t *seq_len
     if ((st = build_layout(dims, sh, k, JSSA_OP_TOPK, 0, 0, L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
+    if ((st = check_opts(opts))) return st;
     return run_select(dims, sh, nullptr, nullptr, scores, seq_lens, JSSA_AGG_SUM, k, idx, count, ws, L, S(stream),
-                      false);
+                      false, opts);
 }
 
 int jssa_select(const jssa_dims *dims, const void *q, const float *P, const void *Kt, const int32_t *seq_lens,
                 int agg, int k, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    return jssa_select_ex(dims, q, P, Kt, seq_lens, agg, k, nullptr, idx, count, ws, ws_bytes, stream);
+}
+
+int jssa_select_ex(const jssa_dims *dims, const void *q, const float *P, const void *Kt, const int32_t *seq_lens,
+                   int agg, int k, const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *ws,
+                   size_t ws_bytes, jssa_stream_t stream) {
     Shape sh;
     int st = check_dims(dims, &sh);
     if (st) return st;
@@ -606,8 +631,9 @@ int jssa_select(const jssa_dims *dims, const void *q, const float *P, const void
     Layout L;
     if ((st = build_layout(dims, sh, k, JSSA_OP_SELECT, agg, 0, L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if ((st = check_opts(opts))) return st;
     if (dims->B == 0) return JSSA_OK;
-    return run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), true);
+    return run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), true, opts);
 }
 
 int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, const void *V, const int32_t *idx,
@@ -715,6 +741,14 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
                      const int32_t *seq_lens, const int32_t *pos_begin, int k, int agg, float softmax_scale,
                      int32_t *idx, int32_t *count, void *out, float *lse, void *ws, size_t ws_bytes,
                      jssa_stream_t stream) {
+    return jssa_decode_step_ex(dims, q, K, V, P, Kt, seq_lens, pos_begin, k, agg, softmax_scale, nullptr, idx, count,
+                               out, lse, ws, ws_bytes, stream);
+}
+
+int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, const void *V, const float *P,
+                        void *Kt, const int32_t *seq_lens, const int32_t *pos_begin, int k, int agg,
+                        float softmax_scale, const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *out,
+                        float *lse, void *ws, size_t ws_bytes, jssa_stream_t stream) {
     Shape sh;
     int st = check_dims(dims, &sh);
     if (st) return st;
@@ -735,6 +769,7 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
     Layout L;
     if ((st = build_layout(dims, sh, k, JSSA_OP_DECODE_STEP, agg, 0, L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if ((st = check_opts(opts))) return st;
     if (dims->B == 0) return JSSA_OK;
     if (L.fused) {
         ScanArgs sa;
@@ -754,6 +789,8 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
         sa.r = dims->r;
         sa.nq = 1;
         sa.k = k;
+        sa.n_sink = opts ? opts->n_sink : 0;
+        sa.n_recent = opts ? opts->n_recent : 0;
         StepExtra x;
         x.q = q;
         x.P = P;
@@ -774,7 +811,8 @@ int jssa_decode_step(const jssa_dims *dims, const void *q, const void *K, const 
     ProjArgs pj{q, P, at<float>(ws, L.qproj), dims->B, dims->Hq, dims->Hkv, dims->d, dims->r, agg};
     cudaError_t e = launch_prep(ap, pj, S(stream), true, dims->kv_dtype, dims->kt_dtype);
     if (e != cudaSuccess) return cuda_fail(e, "launching the append + projection prologue");
-    if ((st = run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), false))) return st;
+    if ((st = run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), false, opts)))
+        return st;
     if (sh.latent) return run_mla(dims, q, K, idx, count, k, seq_lens, softmax_scale, out, lse, ws, L, S(stream));
     AttnArgs a;
     fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);

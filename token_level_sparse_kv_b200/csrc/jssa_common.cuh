@@ -47,6 +47,14 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Key of a token that is always selected (forced sink / recent tokens): above
+// the key of every finite score, so a top-k by (key desc, index asc) takes
+// forced tokens first, smallest indices first.
+constexpr uint32_t kForcedKey = 0xffffffffu;
+__device__ __forceinline__ uint32_t forced_key(uint32_t key, int t, int Tb, int n_sink, int n_recent) {
+    return (t < n_sink || t >= Tb - n_recent) ? kForcedKey : key;
+}
+
 __device__ __forceinline__ int clamp_seq(int v, int cap, uint32_t *status) {
     if (v < 0 || v > cap) {
         if (status) atomicOr(status, (uint32_t)JSSA_DEV_SEQLEN);

@@ -42,6 +42,7 @@ struct ScanArgs {
     int tile_tokens, tiles_per_bh;
     long long total_tiles;
     int grid, max_seg, cap, nstages;
+    int n_sink, n_recent;  // always-selected tokens (0, 0: plain top-k)
 };
 
 struct ScanPlan {
@@ -118,6 +119,7 @@ struct CSelArgs {
     int32_t *count_out;       // [BH] or null
     uint32_t *status;
     int B, Hkv, T_cap, r, nq, k, csize, slice, nstages;
+    int n_sink, n_recent;  // always-selected tokens (0, 0: plain top-k)
 };
 struct CSelPlan {
     int csize, slice, grid_y, nstages;

@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(NT, 2) scan_kernel(ScanArgs a) {
                     if constexpr (MODE == MODE_WRITE) {
                         if (live && sub == 0) a.scores_out[(size_t)bh * a.T_cap + t0 + tt] = sc;
                     } else {
-                        const uint32_t u = score_key(sc);
+                        const uint32_t u = forced_key(score_key(sc), t0 + tt, Tb, a.n_sink, a.n_recent);
                         offer(bkey, bidx, bcount, live && sub == 0 && (!valid || u > thresh), u, t0 + tt, a.cap);
                     }
                 }
@@ -746,7 +746,7 @@ __global__ void __launch_bounds__(NT, 2) scan_kernel(ScanArgs a) {
 #pragma unroll
                 for (int u = 0; u < PASSES; ++u) {
                     const int j = tid + u * NT;
-                    const uint32_t key = score_key(v[u]);
+                    const uint32_t key = forced_key(score_key(v[u]), t0 + j, Tb, a.n_sink, a.n_recent);
                     offer(bkey, bidx, bcount, j < n && (!valid || key > thresh), key, t0 + j, a.cap);
                 }
             }

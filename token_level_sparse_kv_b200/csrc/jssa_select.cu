@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
                     }
                     sc = best;
                 }
-                if (live && sub == 0) keys[t0 + tt] = score_key(sc);
+                if (live && sub == 0) keys[t0 + tt] = forced_key(score_key(sc), lo + t0 + tt, Tb, a.n_sink, a.n_recent);
             }
             __syncthreads();  // stage s consumed
             if (tid == 0 && i + NS < ntiles) {
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = j0 + u * NT + tid;
-                if (j < n_loc) keys[j] = score_key(v[u]);
+                if (j < n_loc) keys[j] = forced_key(score_key(v[u]), lo + j, Tb, a.n_sink, a.n_recent);
             }
         }
     }

@@ -1293,7 +1293,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                 else sc = pc[0];
 #pragma unroll
                 for (int off = 1; off < LPT; off <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, off);
-                const uint32_t key = score_key(sc);
+                const uint32_t key = forced_key(score_key(sc), t0 + tt, Tb, a.n_sink, a.n_recent);
                 const bool take = live && sub == 0 && (!use || key > tk);
                 const unsigned msk = __ballot_sync(0xffffffffu, take);
                 if (msk) {
@@ -1388,7 +1388,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                 int b0 = 0;
                 if (msk) {
                     const int ld = __ffs(msk) - 1;
-                    uint32_t mn = take ? u : 0xffffffffu, mx = take ? u : 0u;
+                    // forced keys stay out of the tracked range (they sit above every bin)
+                    uint32_t mn = take ? u : 0xffffffffu, mx = (take && u != kForcedKey) ? u : 0u;
 #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) {
                         mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
