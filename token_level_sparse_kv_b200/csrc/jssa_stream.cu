@@ -1266,6 +1266,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             }
             const int t0 = t * TILE;
             const int n = max(0, min(TILE, Tb - t0));
+            // does this tile hold always-selected tokens (warp-uniform)?
+            const bool tforce = t0 < a.n_sink || t0 + TILE > Tb - a.n_recent;
             const unsigned long long tw = *thr_word;
             const bool use = (uint32_t)(tw >> 32) == tag;
             const uint32_t tk = (uint32_t)tw;
@@ -1293,7 +1295,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                 else sc = pc[0];
 #pragma unroll
                 for (int off = 1; off < LPT; off <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, off);
-                const uint32_t key = forced_key(score_key(sc), t0 + tt, Tb, a.n_sink, a.n_recent);
+                uint32_t key = score_key(sc);
+                if (tforce) key = forced_key(key, t0 + tt, Tb, a.n_sink, a.n_recent);
                 const bool take = live && sub == 0 && (!use || key > tk);
                 const unsigned msk = __ballot_sync(0xffffffffu, take);
                 if (msk) {
