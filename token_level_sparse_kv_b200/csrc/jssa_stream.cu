@@ -82,14 +82,16 @@ struct StreamSmem {
 __host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k, int fused_r = 0) {
     StreamSmem L;
     size_t o = 0;
+    // the ring and the epoch buffers first: one contiguous region that the
+    // fused step's attention epilogue reuses once the stream is done
     L.ring = o;
     o += (size_t)nstages * kTile;
-    L.bars = o;
-    o = al(o + (size_t)(2 * nstages + 2 * kEB + kMaxRows + 1) * 8, 16);
     L.ek = o;
     o = al(o + (size_t)kEB * ept * 4, 16);
     L.ei = o;
     o = al(o + (size_t)kEB * ept * 4, 16);
+    L.bars = o;
+    o = al(o + (size_t)(2 * nstages + 2 * kEB + kMaxRows + 1) * 8, 16);
     L.rk = o;
     o = al(o + (size_t)cap * 4, 16);
     L.ri = o;
@@ -685,13 +687,18 @@ struct RingPos {
 
 // End of a segment (selector).  The segment takes its arrival ticket first:
 // the last segment of the (b,h) to arrive merges the other segments'
-// published candidates straight into its own uncut candidate set (one exact
-// cut, nothing published); every other segment cuts to k, publishes, and
-// counts itself published.  The last one waits (bounded) for the publish
-// counts of segments that took their tickets before it, which are running
-// and publish without waiting on anything.  Returns the selection's size when
-// this CTA merged it, else -1.  counters[bh] = tickets, counters[BH + bh] =
-// published segments; the merger resets both.
+// published candidates into its own candidate set (nothing published);
+// every other segment cuts to k, publishes k slots (index -1 marks an empty
+// slot), and counts itself published.  The last one waits (bounded) for the
+// publish counts of segments that took their tickets before it, which are
+// running and publish without waiting on anything; while some are still
+// cutting, it cuts its own set to k, which also gives a threshold that
+// filters the merged entries.  The merge loads the slots of up to kMergeSegs
+// segments at once (one memory latency per group), as many groups as the
+// candidate capacity holds between exact cuts.  Returns the selection's size
+// when this CTA merged it, else -1.  counters[bh] = tickets, counters[BH +
+// bh] = published segments; the merger resets both.
+constexpr int kMergeSegs = 8;
 __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long long cta, int ept, int cap) {
     const int BH = a.B * a.Hkv;
     const int tpb = a.tiles_per_bh;
@@ -709,89 +716,147 @@ __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long l
             n = a.k;
         }
         const size_t cb = ((size_t)bh * a.max_seg + slot) * a.k;
-        for (int j = S.st; j < n; j += kSelT) {
-            a.cand_key[cb + j] = S.rk[j];
-            a.cand_idx[cb + j] = S.ri[j];
+        for (int j = S.st; j < a.k; j += kSelT) {
+            a.cand_key[cb + j] = j < n ? S.rk[j] : 0u;
+            a.cand_idx[cb + j] = j < n ? S.ri[j] : -1;
         }
-        if (S.st == 0) a.cand_cnt[(size_t)bh * a.max_seg + slot] = n;
         __threadfence();
         sel_sync();
         if (S.st == 0) atomicAdd(&a.counters[BH + bh], 1u);
         return -1;
     }
-    if (S.st == 0 && nseg > 1) {
-        volatile unsigned *pub = a.counters + BH + bh;
-        const uint64_t t0 = global_timer_ns();
-        while (*pub < (unsigned)(nseg - 1)) {
-            if (global_timer_ns() - t0 > 2000000000ull) {
-                if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
-                break;
+    int m = n;
+    bool valid = false;
+    uint32_t thr = 0u;
+    if (nseg > 1) {
+        if (S.st == 0) S.misc[47] = (int)__ldcg(a.counters + BH + bh);
+        sel_sync();
+        if (S.misc[47] < nseg - 1 && m > a.k) {  // others still cutting: cut this set meanwhile
+            thr = sel_reduce(S, m, a.k);
+            valid = true;
+            m = a.k;
+        }
+        if (S.st == 0) {
+            volatile unsigned *pub = a.counters + BH + bh;
+            const uint64_t t0 = global_timer_ns();
+            while (*pub < (unsigned)(nseg - 1)) {
+                if (global_timer_ns() - t0 > 2000000000ull) {
+                    if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+                    break;
+                }
+                __nanosleep(64);
             }
-            __nanosleep(64);
         }
     }
     __threadfence();
     sel_sync();
-    // merge the other segments into this one's candidates, in chunks of at
-    // most ept entries; equal keys stay candidates (order is arbitrary)
-    if (S.st == 0) S.misc[3] = n;
+    // merge the other segments' slots; equal keys stay candidates (order is arbitrary)
+    if (S.st == 0) S.misc[3] = m;
     sel_sync();
-    int m = n;
-    bool valid = false;
-    uint32_t thr = 0u;
     const int lane = S.st & 31;
-    for (int s = 0; s < nseg; ++s) {
-        if (s == slot) continue;
-        const int cnt = __ldcg(a.cand_cnt + (size_t)bh * a.max_seg + s);
-        const size_t base = ((size_t)bh * a.max_seg + s) * a.k;
-        for (int off = 0; off < cnt; off += ept) {
-            if (m > cap - ept) {
-                thr = sel_reduce(S, m, a.k);
-                valid = true;
-                m = a.k;
-                if (S.st == 0) S.misc[3] = m;
-                sel_sync();
-            }
-            const int c = min(ept, cnt - off);
-            for (int j0 = 0; j0 < c; j0 += kSelT) {
-                const int j = j0 + S.st;
-                uint32_t u = 0u;
-                int32_t ix = 0;
-                if (j < c) {
-                    u = __ldcg(a.cand_key + base + off + j);
-                    ix = __ldcg(a.cand_idx + base + off + j);
-                }
-                const bool take = j < c && (!valid || u >= thr);
-                const unsigned msk = __ballot_sync(0xffffffffu, take);
-                int b0 = 0;
-                if (msk) {
-                    const int ld = __ffs(msk) - 1;
-                    if (lane == ld) b0 = atomicAdd(&S.misc[3], __popc(msk));
-                    b0 = __shfl_sync(0xffffffffu, b0, ld);
-                }
-                if (take) {
-                    const int p = b0 + __popc(msk & lane_lt());
-                    S.rk[p] = u;
-                    S.ri[p] = ix;
-                }
-            }
+    const size_t rowbase = (size_t)bh * a.max_seg * a.k;
+    // a wave holds at most what the register-resident cut takes (the cut of
+    // a larger set reads shared memory on every level: several times slower)
+    const int wcap = max(min(cap, kRegKeys * kSelT), 2 * a.k);
+    for (int s0 = 0; s0 < nseg;) {
+        int nb = (wcap - m) / a.k;  // segments that fit before the next exact cut
+        if (nb < 1) {
+            thr = sel_reduce(S, m, a.k);
+            valid = true;
+            m = a.k;
+            if (S.st == 0) S.misc[3] = m;
             sel_sync();
-            m = S.misc[3];
-            sel_sync();
+            nb = (wcap - m) / a.k;
         }
+        const int s_end = min(nseg, s0 + nb);
+        for (int g0 = s0; g0 < s_end; g0 += kMergeSegs) {
+            const int s1 = min(s_end, g0 + kMergeSegs);
+            for (int j0 = 0; j0 < a.k; j0 += kSelT) {
+                const int j = j0 + S.st;
+                uint32_t u[kMergeSegs];
+                int32_t ix[kMergeSegs];
+#pragma unroll
+                for (int q = 0; q < kMergeSegs; ++q) {  // every load of the group in flight at once
+                    const int sg = g0 + q;
+                    u[q] = 0u;
+                    ix[q] = -1;
+                    if (sg < s1 && sg != slot && j < a.k) {
+                        const size_t o = rowbase + (size_t)sg * a.k + j;
+                        u[q] = __ldcg(a.cand_key + o);
+                        ix[q] = __ldcg(a.cand_idx + o);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kMergeSegs; ++q) {
+                    const bool take = ix[q] >= 0 && (!valid || u[q] >= thr);
+                    const unsigned msk = __ballot_sync(0xffffffffu, take);
+                    int b0 = 0;
+                    if (msk) {
+                        const int ld = __ffs(msk) - 1;
+                        if (lane == ld) b0 = atomicAdd(&S.misc[3], __popc(msk));
+                        b0 = __shfl_sync(0xffffffffu, b0, ld);
+                    }
+                    if (take) {
+                        const int p = b0 + __popc(msk & lane_lt());
+                        S.rk[p] = u[q];
+                        S.ri[p] = ix[q];
+                    }
+                }
+            }
+        }
+        s0 = s_end;
+        sel_sync();
+        m = S.misc[3];
+        sel_sync();
     }
     if (m > a.k) {
         sel_reduce(S, m, a.k);
         m = a.k;
     }
-    if (m <= 2 * kSelT) {
+    if (m <= kSelT) {
+        // bitonic sort, one value per selector thread (pads sort above every
+        // index): partners within a warp by shuffle, across warps through
+        // shared memory (the histogram is free after the cut)
+        int32_t v = S.st < m ? S.ri[S.st] : 0x7fffffff;
+        int32_t *xch = reinterpret_cast<int32_t *>(S.hist);
+#pragma unroll
+        for (int kk = 2; kk <= kSelT; kk <<= 1) {
+#pragma unroll
+            for (int j = kk >> 1; j > 0; j >>= 1) {
+                int32_t o;
+                if (j >= 32) {
+                    xch[S.st] = v;
+                    sel_sync();
+                    o = xch[S.st ^ j];
+                    sel_sync();
+                } else {
+                    o = __shfl_xor_sync(0xffffffffu, v, j);
+                }
+                const bool asc = (S.st & kk) == 0, lower = (S.st & j) == 0;
+                v = lower == asc ? min(v, o) : max(v, o);
+            }
+        }
+        if (S.st < m) S.si[S.st] = v;
+        sel_sync();
+    } else if (m <= 2 * kSelT) {
         // ascending order by rank: the indices are distinct, so each entry's
         // place is the number of smaller ones (broadcast reads, one barrier)
+        const int m4 = (m + 3) & ~3;
+        if (S.st < m4 - m) S.ri[m + S.st] = 0x7fffffff;  // pads count as larger than every index
+        sel_sync();
+        const int4 *r4 = reinterpret_cast<const int4 *>(S.ri);
         for (int j = S.st; j < m; j += kSelT) {
             const int32_t v = S.ri[j];
-            int rank = 0;
-            for (int i = 0; i < m; ++i) rank += S.ri[i] < v;
-            S.si[rank] = v;
+            int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll 4
+            for (int i = 0; i < m4 / 4; ++i) {
+                const int4 w = r4[i];
+                c0 += w.x < v;
+                c1 += w.y < v;
+                c2 += w.z < v;
+                c3 += w.w < v;
+            }
+            S.si[(c0 + c1) + (c2 + c3)] = v;
         }
         sel_sync();
     } else {
@@ -846,18 +911,42 @@ __device__ __forceinline__ float sum_parts(const float *part, int j, int nch) {
 }
 
 // Folded query of row bh: qb = P_h^T (sum of the group's queries, in head order).
+// Each work item (chunk c of kChunkD inputs, output j) loads its P column
+// slice and the group's query chunks at once and folds the queries itself:
+// one memory latency, no staging barrier.  The arithmetic order matches the
+// projection kernel's (head sum from 0 in head order, fma chain per chunk,
+// chunk partials left to right), so both give the same bits.
 template <int R>
-__device__ void sel_project(const StepExtra &x, int Hkv, int bh, float *qb, float *xs, float *part, int st) {
+__device__ void sel_project(const StepExtra &x, int Hkv, int bh, float *qb, float *part, int st) {
     const int b = bh / Hkv, h = bh - b * Hkv, G = x.G, d = x.d;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(x.q) + ((size_t)b * x.Hq + (size_t)h * G) * d;
-    for (int i = st; i < d; i += kSelT) {
-        float sum = 0.f;
-        for (int g = 0; g < G; ++g) sum += __bfloat162float(q[(size_t)g * d + i]);
-        xs[i] = sum;
+    const float *P = x.P + (size_t)h * d * R;
+    const int nch = d / kChunkD;
+    static_assert(kChunkD == 16, "two 16-byte query loads per chunk");
+    for (int p = st; p < R * nch; p += kSelT) {
+        const int c = p / R, j = p - c * R;
+        float pv[kChunkD], xr[kChunkD];
+#pragma unroll
+        for (int i = 0; i < kChunkD; ++i) {
+            pv[i] = __ldg(P + (size_t)(c * kChunkD + i) * R + j);
+            xr[i] = 0.f;
+        }
+#pragma unroll 4
+        for (int g = 0; g < G; ++g) {
+            const uint4 *qv = reinterpret_cast<const uint4 *>(q + (size_t)g * d + c * kChunkD);
+            float f[16];
+            Vec16<__nv_bfloat16>::unpack(__ldg(qv), f);
+            Vec16<__nv_bfloat16>::unpack(__ldg(qv + 1), f + 8);
+#pragma unroll
+            for (int i = 0; i < kChunkD; ++i) xr[i] += f[i];
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kChunkD; ++i) acc = fmaf(xr[i], pv[i], acc);
+        part[(size_t)j * nch + c] = acc;
     }
     sel_sync();
-    sel_dots<R>(xs, x.P + (size_t)h * d * R, d, part, st);
-    for (int j = st; j < R; j += kSelT) qb[j] = sum_parts(part, j, d / kChunkD);
+    for (int j = st; j < R; j += kSelT) qb[j] = sum_parts(part, j, nch);
     sel_sync();
 }
 
@@ -910,9 +999,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 //   O[16 x D] = P[16 x n] . V_sel        (P = softmax weights rounded to bf16)
 // The selected K and V rows of a chunk of tokens are staged by 16-byte
 // asynchronous copies straight from the cache into `buf` (16-byte chunks
-// XOR-swizzled by token so that ldmatrix reads are conflict-free); the
-// softmax runs in fp32 in the log2 domain across the warps, online across
-// chunks; the normaliser sums the bf16 weights the second product uses.
+// XOR-swizzled by token so that ldmatrix reads are conflict-free).  Each
+// warp keeps the logits of its 8-token tiles in registers; the softmax runs
+// in fp32 in the log2 domain, online across chunks, with the running max
+// and each thread's share of the normaliser (sums of the bf16 weights the
+// second product uses) in registers: three barriers per chunk.
 template <int D>
 __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int kb, unsigned char *buf,
                              size_t buf_bytes, int ct) {
@@ -922,21 +1013,24 @@ __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int 
     constexpr int QSTR = ROWB + 16;     // padded row stride of Q (bytes)
     constexpr int NTD = D / 8;          // 8-wide output tiles
     constexpr int TPW = NTD / kConsWarps;  // output tiles per warp (1 or 2)
+    constexpr int TT = 2;                  // 8-token logit tiles per warp and chunk
+    constexpr int CHMAX = kConsWarps * 8 * TT;
     static_assert(NTD % kConsWarps == 0, "head width");
     const int w = ct >> 5, lane = ct & 31, gid = lane >> 2, tig = lane & 3;
     const int G = x.G;
     const int b = bh / a.Hkv, h = bh - b * a.Hkv;
     // shared memory carve-up
     unsigned char *q_s = buf;                                  // [16][QSTR]
-    float *red = reinterpret_cast<float *>(buf + 16 * QSTR);   // [kConsWarps][16] partial max / sum
-    float *mlc = red + kConsWarps * 16;                        // m[16], l[16], corr[16]
-    unsigned char *p_s = reinterpret_cast<unsigned char *>(mlc + 48);
-    const size_t fixed = 16 * QSTR + (size_t)kConsWarps * 16 * 4 + 48 * 4;
+    float *red = reinterpret_cast<float *>(buf + 16 * QSTR);   // [kConsWarps][16] partial max, then sums
+    int32_t *idx_s = reinterpret_cast<int32_t *>(red + kConsWarps * 16);  // the token list [kb], staged once
+    unsigned char *p_s = reinterpret_cast<unsigned char *>(idx_s + ((kb + 3) & ~3));
+    const size_t fixed = 16 * QSTR + (size_t)kConsWarps * 16 * 4 + (size_t)((kb + 3) & ~3) * 4;
     // chunk of CH tokens (a multiple of 16): P [16][CH] bf16 (+16 B per row),
-    // CH staged rows, and the chunk's logits [16][CH] fp32 after them
-    int CH = (int)((buf_bytes - fixed - 16 * 16 - 256) / (ROW2 + 32 + 64)) & ~15;
+    // then CH staged K/V row pairs
+    int CH = (int)((buf_bytes - fixed - 16 * 16 - 128) / (ROW2 + 32)) & ~15;
     const int need = (kb + 15) & ~15;
     if (CH > need) CH = need;
+    if (CH > CHMAX) CH = CHMAX;
     if (CH < 16) CH = 16;
     const int PSTR = CH * 2 + 16;  // padded row stride of P (bytes)
     unsigned char *stage = p_s + (((size_t)16 * PSTR + 127) & ~(size_t)127);
@@ -948,14 +1042,17 @@ __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int 
         const int g = i / CPR, c = i - g * CPR;
         cp_async16(q_s + g * QSTR + c * 16, g < G ? qg + (size_t)g * D + c * 8 : qg, g < G ? 16u : 0u);
     }
-    if (ct < 16) {
-        mlc[ct] = -INFINITY;  // running max (log2 domain)
-        mlc[16 + ct] = 0.f;   // running sum of weights
-    }
     float o[TPW][4];
 #pragma unroll
     for (int u = 0; u < TPW; ++u) o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.f;
-    const int32_t *idx = a.idx_out + (size_t)bh * a.k;
+    float mrun[2] = {-INFINITY, -INFINITY};  // running max of rows gid, gid + 8 (log2 domain)
+    float lpart[2] = {0.f, 0.f};             // this thread's share of their normalisers
+    // the token list in shared memory: one coalesced read instead of a
+    // dependent global load before every staging copy
+    const int32_t *idx_g = a.idx_out + (size_t)bh * a.k;
+    for (int j = ct; j < kb; j += kCons) idx_s[j] = idx_g[j];
+    cons_sync();
+    const int32_t *idx = idx_s;
     const __nv_bfloat16 *Kc = static_cast<const __nv_bfloat16 *>(x.K);
     const __nv_bfloat16 *Vc = static_cast<const __nv_bfloat16 *>(x.V);
 
@@ -979,36 +1076,36 @@ __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int 
         cp_async_wait<0>();
         cons_sync();
 
-        // S = Q K^T: warp w takes 8-token tiles w, w + 16, ...
+        // S = Q K^T: warp w takes 8-token tiles w and w + 16 (logits stay in registers)
         const int ntt = n16 / 8;
+        float sv[TT][4];
         float wmax[2] = {-INFINITY, -INFINITY};
-        for (int nt = w; nt < ntt; nt += kConsWarps) {
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                uint32_t a0, a1, a2, a3, b0, b1;
-                // A: rows (lane % 16), k chunk 2*ks + lane / 16
-                ldsm_x4(q_a + (lane & 15) * QSTR + (2 * ks + (lane >> 4)) * 16, a0, a1, a2, a3);
-                // B: token rows nt*8 + lane % 8, k chunk 2*ks + (lane / 8) % 2
-                const int t = nt * 8 + (lane & 7), c = 2 * ks + ((lane >> 3) & 1);
-                ldsm_x2(st_a + t * ROW2 + ((c ^ (t & 7)) * 16), b0, b1);
-                mma_bf16_16816(sc, a0, a1, a2, a3, b0, b1);
-            }
-            // scaled logits to P (as fp32 bits for now: rows gid, gid + 8; cols 2 tig, +1)
-            const int tc = nt * 8 + 2 * tig;
-            float v[4];
+        for (int u = 0; u < TT; ++u) {
+            const int nt = w + u * kConsWarps;
+            sv[u][0] = sv[u][1] = sv[u][2] = sv[u][3] = -INFINITY;
+            if (nt < ntt) {
+                float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int row = e < 2 ? gid : gid + 8, col = tc + (e & 1);
-                v[e] = (row < G && col < n) ? sc[e] * x.scale_log2 : -INFINITY;
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    uint32_t a0, a1, a2, a3, b0, b1;
+                    // A: rows (lane % 16), k chunk 2*ks + lane / 16
+                    ldsm_x4(q_a + (lane & 15) * QSTR + (2 * ks + (lane >> 4)) * 16, a0, a1, a2, a3);
+                    // B: token rows nt*8 + lane % 8, k chunk 2*ks + (lane / 8) % 2
+                    const int t = nt * 8 + (lane & 7), c = 2 * ks + ((lane >> 3) & 1);
+                    ldsm_x2(st_a + t * ROW2 + ((c ^ (t & 7)) * 16), b0, b1);
+                    mma_bf16_16816(sc, a0, a1, a2, a3, b0, b1);
+                }
+                // scaled logits: rows gid, gid + 8; columns 2 tig, 2 tig + 1 of the tile
+                const int tc = nt * 8 + 2 * tig;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int row = e < 2 ? gid : gid + 8, col = tc + (e & 1);
+                    sv[u][e] = (row < G && col < n) ? sc[e] * x.scale_log2 : -INFINITY;
+                }
+                wmax[0] = fmaxf(wmax[0], fmaxf(sv[u][0], sv[u][1]));
+                wmax[1] = fmaxf(wmax[1], fmaxf(sv[u][2], sv[u][3]));
             }
-            wmax[0] = fmaxf(wmax[0], fmaxf(v[0], v[1]));
-            wmax[1] = fmaxf(wmax[1], fmaxf(v[2], v[3]));
-            float *srow0 = reinterpret_cast<float *>(stage + (size_t)CH * ROW2);  // [16][CH] fp32 logits
-            srow0[gid * CH + tc] = v[0];
-            srow0[gid * CH + tc + 1] = v[1];
-            srow0[(gid + 8) * CH + tc] = v[2];
-            srow0[(gid + 8) * CH + tc + 1] = v[3];
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
@@ -1020,44 +1117,47 @@ __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int 
             red[w * 16 + gid + 8] = wmax[1];
         }
         cons_sync();
-        // running max and correction per row
-        if (ct < 16) {
-            float mx = mlc[ct];
-            for (int i = 0; i < kConsWarps; ++i) mx = fmaxf(mx, red[i * 16 + ct]);
-            const float old = mlc[ct];
-            mlc[32 + ct] = old == -INFINITY ? 0.f : exp2f(old - mx);
-            mlc[ct] = mx;
+        // the chunk's row maxima (every thread of a row computes the same
+        // values) and the correction of what came before
+        float corr[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            float mx = mrun[r];
+#pragma unroll
+            for (int i = 0; i < kConsWarps; ++i) mx = fmaxf(mx, red[i * 16 + gid + 8 * r]);
+            corr[r] = mrun[r] == -INFINITY ? 0.f : exp2f(mrun[r] - mx);
+            mrun[r] = mx;
         }
-        cons_sync();
-        // weights: P = bf16(exp2(s - m)), row sums of the rounded weights
-        {
-            const float *srow0 = reinterpret_cast<const float *>(stage + (size_t)CH * ROW2);
-            for (int i = ct; i < 16 * n16; i += kCons) {
-                const int row = i / n16, col = i - row * n16;
-                const float sv = srow0[row * CH + col];
-                const float mrow = mlc[row];
-                const float pw = (sv == -INFINITY || mrow == -INFINITY) ? 0.f : exp2f(sv - mrow);
-                reinterpret_cast<__nv_bfloat16 *>(p_s + row * PSTR)[col] = __float2bfloat16_rn(pw);
+        // weights: P = bf16(exp2(s - m)) into shared memory; this thread's row
+        // sums of the rounded weights
+        float rs[2] = {0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < TT; ++u) {
+            const int nt = w + u * kConsWarps;
+            if (nt < ntt) {
+                const int tc = nt * 8 + 2 * tig;
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const float m = mrun[r];
+                    const float w0 = (sv[u][2 * r] == -INFINITY || m == -INFINITY) ? 0.f : exp2f(sv[u][2 * r] - m);
+                    const float w1 =
+                        (sv[u][2 * r + 1] == -INFINITY || m == -INFINITY) ? 0.f : exp2f(sv[u][2 * r + 1] - m);
+                    const __nv_bfloat162 pw = __floats2bfloat162_rn(w0, w1);
+                    rs[r] += __low2float(pw) + __high2float(pw);
+                    *reinterpret_cast<__nv_bfloat162 *>(p_s + (gid + 8 * r) * PSTR + tc * 2) = pw;
+                }
             }
         }
-        cons_sync();
-        if (ct < 16 * 16) {  // 16 threads per row sum the row's rounded weights
-            const int row = ct >> 4, sub = ct & 15;
-            float sum = 0.f;
-            const __nv_bfloat16 *pr = reinterpret_cast<const __nv_bfloat16 *>(p_s + row * PSTR);
-            for (int col = sub; col < n16; col += 16) sum += __bfloat162float(pr[col]);
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            if (sub == 0) mlc[16 + row] = mlc[16 + row] * mlc[32 + row] + sum;
-        }
+        for (int r = 0; r < 2; ++r) lpart[r] = lpart[r] * corr[r] + rs[r];
+        cons_sync();  // P complete (and every read of the maxima done)
         // O = O * corr + P V: warp w takes output tiles w, w + 16
-        const float cr0 = mlc[32 + gid], cr1 = mlc[32 + gid + 8];
 #pragma unroll
         for (int u = 0; u < TPW; ++u) {
-            o[u][0] *= cr0;
-            o[u][1] *= cr0;
-            o[u][2] *= cr1;
-            o[u][3] *= cr1;
+            o[u][0] *= corr[0];
+            o[u][1] *= corr[0];
+            o[u][2] *= corr[1];
+            o[u][3] *= corr[1];
             const int dt = w + u * kConsWarps;  // 8-dim tile = one 16-byte chunk of the V row
             for (int ks = 0; ks < n16 / 16; ++ks) {
                 uint32_t a0, a1, a2, a3, b0, b1;
@@ -1067,15 +1167,28 @@ __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int 
                 mma_bf16_16816(o[u], a0, a1, a2, a3, b0, b1);
             }
         }
-        cons_sync();  // before the next chunk overwrites the stage
+        if (c0 + CH < kb) cons_sync();  // before the next chunk overwrites the stage and P
     }
+    // normalisers: the four threads of a row in a warp, then the warps in order
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        lpart[r] += __shfl_xor_sync(0xffffffffu, lpart[r], 1);
+        lpart[r] += __shfl_xor_sync(0xffffffffu, lpart[r], 2);
+    }
+    if (tig == 0) {
+        red[w * 16 + gid] = lpart[0];
+        red[w * 16 + gid + 8] = lpart[1];
+    }
+    cons_sync();
     // out = O / l, lse = (m + log2 l) ln 2, rows g < G
     const size_t row0 = (size_t)b * x.Hq + (size_t)h * G;
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
         const int g = gid + 8 * hr;
         if (g >= G) continue;
-        const float l = mlc[16 + g];
+        float l = 0.f;
+#pragma unroll
+        for (int i = 0; i < kConsWarps; ++i) l += red[i * 16 + g];
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(x.out) + (row0 + g) * D;
 #pragma unroll
@@ -1085,7 +1198,7 @@ __device__ void fused_attend(const ScanArgs &a, const StepExtra &x, int bh, int 
                 __floats2bfloat162_rn(o[u][2 * hr] * inv, o[u][2 * hr + 1] * inv);
         }
         if (w == 0 && tig == 0 && x.lse)
-            x.lse[row0 + g] = l > 0.f ? (mlc[g] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            x.lse[row0 + g] = l > 0.f ? (mrun[hr] + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
     cons_sync();
 }
@@ -1346,7 +1459,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             float *xs = reinterpret_cast<float *>(smem + L.xs);
             float *part = reinterpret_cast<float *>(S.hist);
             for (int rl = 0; rl < nrows; ++rl) {
-                sel_project<R>(A.x, a.Hkv, row0 + rl, qb + (size_t)rl * R, xs, part, S.st);
+                sel_project<R>(A.x, a.Hkv, row0 + rl, qb + (size_t)rl * R, part, S.st);
                 if (S.st == 0) mbar_arrive(&qready[rl]);  // consumers of row rl may start
             }
             for (int rl = 0; rl < nrows; ++rl) {
@@ -1480,11 +1593,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
     }
     if constexpr (FUSED) {
         // epilogue: attention of the rows whose selection this CTA completed,
-        // in the (now idle) ring buffer
+        // in the (now idle) ring and epoch buffers
         if (tid >= kConsBase) {
             const int na = misc[46];
             for (int i = 0; i < na; ++i)
-                fused_attend<D>(a, A.x, misc[64 + i], misc[72 + i], smem + L.ring, (size_t)S_ * kTile, tid - kConsBase);
+                fused_attend<D>(a, A.x, misc[64 + i], misc[72 + i], smem + L.ring, L.bars - L.ring, tid - kConsBase);
         }
     }
 }
@@ -1530,6 +1643,7 @@ cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T
     // candidate capacity: the kept set after a cut (k plus up to 1024 more
     // before the next cut) and one epoch of new survivors
     P.cap = k + ept + 1024;
+    if (P.cap < 2 * k) P.cap = 2 * k;  // the merge holds k kept entries and one segment's k slots
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1612,9 +1726,11 @@ cudaError_t plan_step_fused(int B, int Hkv, int Hq, int d, int T_cap, int r, int
         if (xe > xb && (xe - 1) / p->tiles_per_bh - xb / p->tiles_per_bh + 1 > kMaxRows) return cudaErrorNotSupported;
     }
     // attention epilogue: Q, partials, and at least one 16-token chunk
-    const size_t need = 16 * (size_t)(2 * d + 16) + kConsWarps * 16 * 4 + 48 * 4 + 16 * 16 + 256 +
-                        16 * (size_t)(4 * d + 96);
-    if ((size_t)p->nstages * kTile < need) return cudaErrorNotSupported;
+    const size_t need = 16 * (size_t)(2 * d + 16) + kConsWarps * 16 * 4 + (size_t)((k + 3) & ~3) * 4 + 16 * 16 +
+                        128 + 16 * (size_t)(4 * d + 32);
+    const int tile = kTile / (r * 2), ept = tile >= kEpochTokens ? tile : kEpochTokens;
+    const StreamSmem L = stream_smem(p->nstages, ept, p->cap, k, r);
+    if (L.bars - L.ring < need) return cudaErrorNotSupported;
     return cudaSuccess;
 }
 
