@@ -156,22 +156,41 @@ size_t take(size_t &off, size_t bytes) {
     return o;
 }
 
-int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, Layout &L) {
+// Selection form: the cluster form where one wave of clusters covers the
+// rows, else the streaming form, else the block-synchronous scan.  With
+// stream_first (a decode step that runs as one fused launch of the streaming
+// kernel) the streaming form is tried first.  JSSA_SELECT_FORM overrides.
+int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, Layout &L, bool stream_first = false) {
     const int nq = (src != SRC_SCORES && agg == JSSA_AGG_MAX) ? sh.G : 1;
-    cudaError_t e = plan_csel(src, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.cp);
-    if (e == cudaSuccess) {
-        L.csel = true;
+    const int form = select_form_override();
+    stream_first = stream_first && form == 0;
+    auto try_csel = [&](bool &ok) -> int {
+        ok = false;
+        cudaError_t ec = plan_csel(src, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.cp);
+        if (ec == cudaSuccess) {
+            L.csel = true;
+            ok = true;
+            return JSSA_OK;
+        }
+        cudaGetLastError();
+        if (ec != cudaErrorNotSupported) return cuda_fail(ec, "planning the cluster selection");
         return JSSA_OK;
+    };
+    bool done = false;
+    if (!stream_first) {
+        const int st = try_csel(done);
+        if (st != JSSA_OK || done) return st;
     }
-    cudaGetLastError();
-    if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the cluster selection");
-    e = select_form_override() == 3 ? cudaErrorNotSupported
-                                    : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
+    cudaError_t e = form == 3 ? cudaErrorNotSupported : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
     if (e == cudaSuccess) {
         L.wspec = true;
     } else {
         cudaGetLastError();
         if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the streaming selection");
+        if (stream_first) {
+            const int st = try_csel(done);
+            if (st != JSSA_OK || done) return st;
+        }
         e = plan_scan(src, MODE_SELECT, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.sp);
         if (e != cudaSuccess) return cuda_fail(e, "planning the selection pass");
     }
@@ -283,21 +302,30 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
             st = layout_attend(d, sh, ATT_RANGE_BH, k, L);
             if (st == JSSA_OK) L.gcount = take(L.total, (size_t)sh.BH * 4);
             break;
-        case JSSA_OP_DECODE_STEP:
-            L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
-            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L);
-            if (st == JSSA_OK) st = layout_attend(d, sh, ATT_INDEXED, k, L);
-            if (st == JSSA_OK && L.wspec && !sh.latent && agg == JSSA_AGG_SUM && d->kv_dtype == JSSA_BF16 &&
-                d->kt_dtype == JSSA_BF16 && fused_step_allowed()) {
-                cudaError_t e = plan_step_fused(d->B, d->Hkv, d->Hq, d->d, d->T_cap, d->r, k, &L.fp);
-                if (e == cudaSuccess && L.fp.max_seg <= L.sp.max_seg) {
-                    L.fused = true;
+        case JSSA_OP_DECODE_STEP: {
+            // one fused launch where the shape allows it (it also beats the
+            // three-launch cluster form on short caches and small batches)
+            ScanPlan fp{};
+            bool fused_ok = false;
+            if (!sh.latent && agg == JSSA_AGG_SUM && d->kv_dtype == JSSA_BF16 && d->kt_dtype == JSSA_BF16 &&
+                fused_step_allowed()) {
+                cudaError_t e = plan_step_fused(d->B, d->Hkv, d->Hq, d->d, d->T_cap, d->r, k, &fp);
+                if (e == cudaSuccess) {
+                    fused_ok = true;
                 } else {
                     cudaGetLastError();
-                    if (e != cudaSuccess && e != cudaErrorNotSupported) return cuda_fail(e, "planning the fused step");
+                    if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the fused step");
                 }
             }
+            L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
+            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L, fused_ok);
+            if (st == JSSA_OK) st = layout_attend(d, sh, ATT_INDEXED, k, L);
+            if (st == JSSA_OK && fused_ok && L.wspec && fp.max_seg <= L.sp.max_seg) {
+                L.fp = fp;
+                L.fused = true;
+            }
             break;
+        }
         default: return fail(JSSA_ERR_INVALID_ARG, "unknown op %d", op);
     }
     return st;

@@ -14,8 +14,12 @@
 // (fma chains from 0), then the chunk partials added left to right.  So the
 // per-step append, the prefix append and the fused decode-step prologue give
 // bit-identical rows, and the score and select paths see the same qbar.
+#include <cooperative_groups.h>
+
 #include "jssa_common.cuh"
 #include "jssa_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace jssa {
 
@@ -162,6 +166,101 @@ __global__ void __launch_bounds__(kPrepThreadsWide) prep_kernel(AppendArgs ap, P
     project_bh<KV>(pj, blockIdx.x, xs, part);
 }
 
+// The same prologue (SUM aggregation) split over a cluster of kPrepCluster
+// CTAs per (b, h): rank s takes the d-chunks s, s + C, ...; it stages its
+// chunks of the group's queries and of P, folds the queries, and stores the
+// chunk partials of the projection and of the new key row into rank 0's
+// shared memory; rank 0 adds them in chunk order.  Every value is formed in
+// the order prep_kernel uses, so the two give the same bits; the split puts
+// many more loads in flight for wide rows (576-d latent rows, 128 heads).
+constexpr int kPrepCluster = 8;
+constexpr int kPrepClThreads = 256;
+
+template <typename KV, typename KT>
+__global__ void __launch_bounds__(kPrepClThreads) prep_cluster_kernel(AppendArgs ap, ProjArgs pj) {
+    extern __shared__ __align__(16) float sm_pc[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+    const int bh = blockIdx.x / C;
+    const int b = bh / pj.Hkv, h = bh - b * pj.Hkv;
+    const int G = pj.Hq / pj.Hkv, d = pj.d, r = pj.r, nch = d / kChunk;
+    const int cpr = (nch + C - 1) / C;                          // chunk slots per rank
+    const int mine = rank < nch ? (nch - 1 - rank) / C + 1 : 0;  // chunks rank, rank + C, ...
+    constexpr int EV = 16 / (int)sizeof(KV);                   // elements per 16-byte vector
+    float *part_all = sm_pc;                                    // [2][nch][r]: projection, key row
+    KV *qs = reinterpret_cast<KV *>(part_all + (size_t)2 * nch * r);  // [G][cpr * kChunk]
+    float *ps = reinterpret_cast<float *>(qs + (size_t)G * cpr * kChunk);  // [cpr * kChunk][r]
+    float *xq = ps + (size_t)cpr * kChunk * r;                  // folded query chunks
+    float *xk = xq + cpr * kChunk;                              // new key row chunks
+    pdl_trigger();
+    pdl_wait();
+    const int pos = ap.pos_begin[b];
+    const bool app = pos >= 0 && pos <= ap.T_cap - 1;
+    if (!app && rank == 0 && threadIdx.x == 0 && ap.status) atomicOr(ap.status, (uint32_t)JSSA_DEV_POS);
+    // stage this rank's chunks of every head's query and of P_h
+    const KV *q = static_cast<const KV *>(pj.q) + ((size_t)b * pj.Hq + (size_t)h * G) * d;
+    constexpr int VPC = kChunk / EV;  // vectors per query chunk
+    for (int v = threadIdx.x; v < G * mine * VPC; v += blockDim.x) {
+        const int g = v / (mine * VPC), rem = v - g * mine * VPC, cl = rem / VPC, e = rem - cl * VPC;
+        const int c = rank + cl * C;
+        cp_async16(qs + ((size_t)g * cpr + cl) * kChunk + e * EV, q + (size_t)g * d + c * kChunk + e * EV, 16);
+    }
+    const float *Ph = pj.P + (size_t)h * d * r;
+    const int pvr = r / 4;  // vectors per P row
+    for (int v = threadIdx.x; v < mine * kChunk * pvr; v += blockDim.x) {
+        const int row = v / pvr, e = v - row * pvr;
+        const int cl = row / kChunk, i = row - cl * kChunk;
+        cp_async16(ps + (size_t)row * r + e * 4, Ph + (size_t)((rank + cl * C) * kChunk + i) * r + e * 4, 16);
+    }
+    cp_async_commit();
+    const KV *K = static_cast<const KV *>(ap.K);
+    for (int i = threadIdx.x; i < mine * kChunk; i += blockDim.x) {
+        const int cl = i / kChunk, c = rank + cl * C;
+        xk[i] = app ? to_f32(K[(((size_t)b * ap.T_cap + pos) * ap.Hkv + h) * d + c * kChunk + (i - cl * kChunk)]) : 0.f;
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    // fold over the group in head order (eight loads in flight at a time)
+    for (int i = threadIdx.x; i < mine * kChunk; i += blockDim.x) {
+        float sum = 0.f;
+        int g = 0;
+        for (; g + 8 <= G; g += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = to_f32(qs[(size_t)(g + u) * cpr * kChunk + i]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sum += v[u];
+        }
+        for (; g < G; ++g) sum += to_f32(qs[(size_t)g * cpr * kChunk + i]);
+        xq[i] = sum;
+    }
+    __syncthreads();
+    // chunk partials (fma chain from 0 over the chunk) into rank 0's copy
+    float *dst = cluster.map_shared_rank(part_all, 0);
+    for (int p = threadIdx.x; p < 2 * mine * r; p += blockDim.x) {
+        const int o = p / (mine * r), rem = p - o * mine * r, cl = rem / r, j = rem - cl * r;
+        const float *x = (o ? xk : xq) + cl * kChunk;
+        const float *pc = ps + (size_t)cl * kChunk * r + j;
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < kChunk; ++i) acc = fmaf(x[i], pc[(size_t)i * r], acc);
+        dst[((size_t)o * nch + rank + cl * C) * r + j] = acc;
+    }
+    cluster.sync();
+    if (rank != 0) return;
+    KT *Kt = static_cast<KT *>(ap.Kt);
+    for (int t = threadIdx.x; t < 2 * r; t += blockDim.x) {
+        const int o = t / r, j = t - o * r;
+        const float *pp = part_all + (size_t)o * nch * r + j;
+        float sum = pp[0];
+        for (int c = 1; c < nch; ++c) sum += pp[(size_t)c * r];
+        if (o == 0)
+            pj.qproj[(size_t)bh * r + j] = sum;
+        else if (app)
+            store_elem(Kt + ((size_t)bh * ap.T_cap + pos) * r + j, sum);
+    }
+}
+
 size_t prep_smem(int rows, int d, int r) {
     return ((size_t)rows * d + (size_t)rows * r * (d / kChunk)) * sizeof(float);
 }
@@ -209,6 +308,40 @@ cudaError_t launch_prep(const AppendArgs &ap0, const ProjArgs &pj, cudaStream_t 
     AppendArgs ap = ap0;
     ap.n_new = 1;
     ap.rows_per_cta = 1;
+    if (pj.agg == JSSA_AGG_SUM && pj.r % 4 == 0) {
+        const int G = pj.Hq / pj.Hkv, nch = pj.d / kChunk, cpr = (nch + kPrepCluster - 1) / kPrepCluster;
+        const size_t es = kv_dtype == JSSA_BF16 ? 2 : 4;
+        const size_t smem = (size_t)2 * nch * pj.r * 4 + (size_t)G * cpr * kChunk * es +
+                            (size_t)cpr * kChunk * pj.r * 4 + (size_t)2 * cpr * kChunk * 4;
+        void (*k)(AppendArgs, ProjArgs);
+        if (kv_dtype == JSSA_BF16)
+            k = kt_dtype == JSSA_BF16 ? prep_cluster_kernel<__nv_bfloat16, __nv_bfloat16>
+                                      : prep_cluster_kernel<__nv_bfloat16, float>;
+        else
+            k = kt_dtype == JSSA_BF16 ? prep_cluster_kernel<float, __nv_bfloat16> : prep_cluster_kernel<float, float>;
+        cudaError_t e = allow_smem(k, smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pj.B * pj.Hkv * kPrepCluster);
+        cfg.blockDim = dim3(kPrepClThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        int na = 0;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = kPrepCluster;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+        if (pdl) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        return cudaLaunchKernelEx(&cfg, k, ap, pj);
+    }
     const int G = pj.Hq / pj.Hkv;
     const int nrow = pj.agg == JSSA_AGG_SUM ? 1 : G;
     size_t xs = (size_t)nrow * pj.d;
