@@ -221,38 +221,40 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     float m = -INFINITY, l = 0.f;
     if (ok) {
+        // the tile's live columns as bit masks (the same in every warp), and
+        // this head's 128 logits read from TMEM once
+        unsigned live[kTok / 32];
+#pragma unroll
+        for (int q = 0; q < kTok / 32; ++q) {
+            const int col = q * 32 + lane;
+            live[q] = __ballot_sync(0xffffffffu, col < rows && tok[col] >= 0);
+        }
+        float v[kTok / 32][32];
+#pragma unroll
+        for (int q = 0; q < kTok / 32; ++q) tmem_ld32(lane_base + q * 32, v[q]);
         float mx = -INFINITY;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kTok; c0 += 32) {
-            float v[32];
-            tmem_ld32(lane_base + c0, v);
+#pragma unroll
+        for (int q = 0; q < kTok / 32; ++q)
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (c0 + j < rows && tok[c0 + j] >= 0) mx = fmaxf(mx, v[j]);
-        }
+                if ((live[q] >> j) & 1u) mx = fmaxf(mx, v[q][j]);
         m = mx == -INFINITY ? -INFINITY : mx * a.scale_log2;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kTok; c0 += 32) {
-            float v[32];
-            tmem_ld32(lane_base + c0, v);
+#pragma unroll
+        for (int q = 0; q < kTok / 32; ++q) {
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float pr[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = c0 + g8 * 8 + e * 2 + u;
-                        const bool live = col < rows && tok[col] >= 0;
-                        const float p = live ? exp2f(v[g8 * 8 + e * 2 + u] * a.scale_log2 - m) : 0.f;
-                        l += p;
-                        pr[u] = p;
-                    }
-                    const __nv_bfloat162 pk = __floats2bfloat162_rn(pr[0], pr[1]);
+                    const int j = g8 * 8 + e * 2;
+                    const float p0 = ((live[q] >> j) & 1u) ? exp2f(v[q][j] * a.scale_log2 - m) : 0.f;
+                    const float p1 = ((live[q] >> (j + 1)) & 1u) ? exp2f(v[q][j + 1] * a.scale_log2 - m) : 0.f;
+                    l += p0;
+                    l += p1;
+                    const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<const uint32_t *>(&pk);
                 }
-                const int col8 = (c0 + g8 * 8) & 63, blk = (c0 + g8 * 8) >> 6;
+                const int c8 = q * 32 + g8 * 8, col8 = c8 & 63, blk = c8 >> 6;
                 *reinterpret_cast<uint4 *>(sP + (size_t)blk * kBlk + h * 128 + (((col8 >> 3) ^ (h & 7)) << 4)) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
@@ -304,14 +306,26 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
             }
             if (a.lse) a.lse[(size_t)b * kH + h] = l > 0.f ? (m + log2f(l)) * 0.693147180559945309417f : -INFINITY;
         } else {
-            float *po = a.part_o + (((size_t)b * a.splits + split) * kH + h) * kDv;
+            // unnormalised partial O, turned around per warp in shared memory (the
+            // K blocks are free once the second product is done) so that every
+            // store writes whole 128-byte rows: block [32 heads][32 columns]
+            float *tb = reinterpret_cast<float *>(sK) + warp * (32 * 33);
+            float *po = a.part_o + (((size_t)b * a.splits + split) * kH + warp * 32) * kDv;
 #pragma unroll 1
             for (int c0 = 0; c0 < kDv; c0 += 32) {
                 float v[32];
                 tmem_ld32(lane_base + c0, v);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(po + c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                for (int j = 0; j < 32; ++j) tb[lane * 33 + j] = v[j];
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int row = i * 4 + (lane >> 3), col = (lane & 7) * 4;
+                    const float *src = tb + row * 33 + col;
+                    *reinterpret_cast<float4 *>(po + (size_t)row * kDv + c0 + col) =
+                        make_float4(src[0], src[1], src[2], src[3]);
+                }
+                __syncwarp();
             }
             float *pml = a.part_ml + (((size_t)b * a.splits + split) * kH + h) * 2;
             pml[0] = m;
@@ -324,30 +338,44 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
 }
 
 // Log-sum-exp merge of the splits: CTA (b, 4 heads), 16 output dims per thread.
+// The splits' maxima are read first; the partial rows and (max, sum) pairs
+// are then read four splits at a time with all their loads in flight.
 __global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
     pdl_trigger();
     pdl_wait();
     const int b = blockIdx.x, h = blockIdx.y * 4 + (threadIdx.x >> 5), c0 = (threadIdx.x & 31) * 16;
     const int ns = a.splits;
+    const float2 *pml = reinterpret_cast<const float2 *>(a.part_ml) + (size_t)b * ns * kH + h;
     float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, a.part_ml[(((size_t)b * ns + s) * kH + h) * 2]);
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, pml[(size_t)s * kH].x);
     float L = 0.f, o[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) o[j] = 0.f;
-    for (int s = 0; s < ns; ++s) {
-        const float *pml = a.part_ml + (((size_t)b * ns + s) * kH + h) * 2;
-        const float ms = pml[0];
-        if (ms == -INFINITY) continue;
-        const float w = exp2f(ms - M);
-        L = fmaf(pml[1], w, L);
-        const float4 *po = reinterpret_cast<const float4 *>(a.part_o + (((size_t)b * ns + s) * kH + h) * kDv + c0);
+    const float *pbase = a.part_o + ((size_t)b * ns * kH + h) * kDv + c0;
+    for (int s0 = 0; s0 < ns; s0 += 4) {
+        float2 ml[4];
+        float4 v[4][4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 v = po[q];
-            o[4 * q] = fmaf(v.x, w, o[4 * q]);
-            o[4 * q + 1] = fmaf(v.y, w, o[4 * q + 1]);
-            o[4 * q + 2] = fmaf(v.z, w, o[4 * q + 2]);
-            o[4 * q + 3] = fmaf(v.w, w, o[4 * q + 3]);
+        for (int u = 0; u < 4; ++u) {
+            const bool in = s0 + u < ns;
+            ml[u] = in ? pml[(size_t)(s0 + u) * kH] : make_float2(-INFINITY, 0.f);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd)
+                v[u][qd] = in ? reinterpret_cast<const float4 *>(pbase + (size_t)(s0 + u) * kH * kDv)[qd]
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (ml[u].x == -INFINITY) continue;  // an empty split (or past the last)
+            const float w = exp2f(ml[u].x - M);
+            L = fmaf(ml[u].y, w, L);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                o[4 * qd] = fmaf(v[u][qd].x, w, o[4 * qd]);
+                o[4 * qd + 1] = fmaf(v[u][qd].y, w, o[4 * qd + 1]);
+                o[4 * qd + 2] = fmaf(v[u][qd].z, w, o[4 * qd + 2]);
+                o[4 * qd + 3] = fmaf(v[u][qd].w, w, o[4 * qd + 3]);
+            }
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
