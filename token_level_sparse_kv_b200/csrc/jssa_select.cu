@@ -48,7 +48,7 @@ struct CSmem {
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) / 16 * 16; }
 
-__host__ __device__ inline CSmem csel_smem(bool from_kt, int r, int nq, int slice, int nstages) {
+__host__ __device__ inline CSmem csel_smem(bool from_kt, int r, int nq, int slice, int nstages, int C) {
     CSmem L;
     size_t o = 0;
     L.stages = o;
@@ -62,7 +62,7 @@ __host__ __device__ inline CSmem csel_smem(bool from_kt, int r, int nq, int slic
     L.hist = o;
     o = align16(o + (size_t)kBins * 4);
     L.gsum = o;
-    o = align16(o + (size_t)kBins * 4 / 2);  // one slice of summed bins (C >= 2)
+    o = align16(o + (size_t)3 * (kBins / C) * 4);  // three rotating copies of this CTA's slice of summed bins
     L.gall = o;
     o = align16(o + (size_t)kBins * 4);
     L.misc = o;
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
 
     extern __shared__ __align__(128) unsigned char smem[];
     const int NS = a.nstages;
-    const CSmem L = csel_smem(FROM_KT, FROM_KT ? R : 0, a.nq, a.slice, NS);
+    const CSmem L = csel_smem(FROM_KT, FROM_KT ? R : 0, a.nq, a.slice, NS, a.csize);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
     float *qs = reinterpret_cast<float *>(smem + L.qs);
     uint32_t *keys = reinterpret_cast<uint32_t *>(smem + L.keys);
@@ -117,7 +117,15 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
         fence_barrier_init();
     }
     if (tid == 0) misc[6] = 0;
+    {
+        // copies 0 and 1 of the summed-bin slice start at zero; the cluster
+        // barrier phase opened here closes before the first remote add
+        const int bpc = kBins / a.csize;
+        uint32_t *gs = reinterpret_cast<uint32_t *>(smem + L.gsum);
+        for (int d = threadIdx.x; d < 2 * bpc; d += NT) gs[d] = 0u;
+    }
     __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     pdl_trigger();
     pdl_wait();
 
@@ -235,6 +243,7 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
         }
     }
     __syncthreads();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     const bool local_timeout = misc[6] != 0;
 
     // ---- cluster radix select of the k-th key ------------------------------
@@ -253,24 +262,26 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
                 const uint32_t u = keys[j];
                 if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
             }
-            cluster.sync();
-            // this CTA sums bins [c * bins_per_cta, (c+1) * bins_per_cta) over the cluster
-            for (int q = tid; q < bins_per_cta; q += NT) {
-                uint32_t v[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) v[r] = r < C ? *cluster.map_shared_rank(hist + c * bins_per_cta + q, r) : 0u;
-                uint32_t sum = 0u;
-#pragma unroll
-                for (int r = 0; r < 16; ++r) sum += v[r];
-                gsum[q] = sum;
+            __syncthreads();
+            // add the non-empty bins into their owners' copy lev % 3 (owner of
+            // bin d: rank d / bins_per_cta), then one cluster barrier
+            uint32_t *cur = gsum + (lev % 3) * bins_per_cta;
+            for (int d = tid; d < kBins; d += NT) {
+                const uint32_t v = hist[d];
+                if (v) atomicAdd(cluster.map_shared_rank(cur + d % bins_per_cta, d / bins_per_cta), v);
             }
             cluster.sync();
+            // every CTA has read copy (lev + 2) % 3 one level back: clear it for two levels on
+            {
+                uint32_t *nxt = gsum + ((lev + 2) % 3) * bins_per_cta;
+                for (int q = tid; q < bins_per_cta; q += NT) nxt[q] = 0u;
+            }
             {
                 uint32_t v[kBins / NT];
 #pragma unroll
                 for (int u = 0; u < kBins / NT; ++u) {
                     const int d = tid + u * NT;
-                    v[u] = *cluster.map_shared_rank(gsum + (d % bins_per_cta), d / bins_per_cta);
+                    v[u] = *cluster.map_shared_rank(cur + (d % bins_per_cta), d / bins_per_cta);
                 }
 #pragma unroll
                 for (int u = 0; u < kBins / NT; ++u) gall[tid + u * NT] = v[u];
@@ -317,56 +328,68 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
         (void)block_excl_scan<NT>(e, tmp, tot);
         if (tid == 0) misc[3] = tot;
         cluster.sync();
-        int before = 0;
-        for (int r = 0; r < c; ++r) before += *cluster.map_shared_rank(misc + 3, r);
+        // ties held by the CTAs before this one: one remote load per lane, all in flight
+        const int before = __reduce_add_sync(0xffffffffu, lane < c ? *cluster.map_shared_rank(misc + 3, lane) : 0);
         take_ties = max(0, min(tot, kk - before));
     }
 
     // ---- emit the selection in ascending token order -----------------------
+    // Warp wp takes the contiguous tokens [jb, je) of the slice, 32 at a time
+    // (lane l reads token j0 + l, conflict-free); ballots order a step's
+    // selections and ties, the warp totals are scanned across the block.
     const bool take_all = kb >= Tb;
-    const int per = (n_loc + NT - 1) / NT;
-    const int j0 = min(tid * per, n_loc), j1 = min(j0 + per, n_loc);
-    auto above = [&](uint32_t u) { return (u & mask) > prefix; };
-    auto in_group = [&](uint32_t u) { return (u & mask) == prefix; };
-    int cs = 0, ce = 0;
-    for (int j = j0; j < j1; ++j) {
-        const uint32_t u = keys[j];
-        cs += take_all || (kb > 0 && (above(u) || (in_group(u) && whole)));
-        ce += !take_all && kb > 0 && !whole && in_group(u);
+    const bool ties_on = !take_all && kb > 0 && !whole;
+    constexpr int NW = NT / 32;
+    const int wp = tid >> 5;
+    const int span = ((n_loc + NW - 1) / NW + 31) & ~31;
+    const int jb = min(wp * span, n_loc), je = min(jb + span, n_loc);
+    const unsigned lt = (1u << lane) - 1u;
+    auto sure_of = [&](uint32_t u) {
+        return take_all || (kb > 0 && ((u & mask) > prefix || ((u & mask) == prefix && whole)));
+    };
+    int cs = 0, ce = 0;  // the warp's sure selections and ties
+    for (int j0 = jb; j0 < je; j0 += 32) {
+        const int j = j0 + lane;
+        const bool ok = j < je;
+        const uint32_t u = ok ? keys[j] : 0u;
+        cs += __popc(__ballot_sync(0xffffffffu, ok && sure_of(u)));
+        ce += __popc(__ballot_sync(0xffffffffu, ok && ties_on && (u & mask) == prefix));
     }
-    int tot_e;
-    const int e0 = block_excl_scan<NT>(ce, tmp, tot_e);  // tie rank of this thread's first tie
-    {
-        int e = e0;
-        for (int j = j0; j < j1; ++j) {
-            const uint32_t u = keys[j];
-            if (!take_all && kb > 0 && !whole && in_group(u)) {
-                cs += e < take_ties;
-                ++e;
-            }
-        }
+    if (lane == 0) misc[32 + wp] = ce;
+    __syncthreads();
+    int e0 = 0;  // tie rank of the warp's first tie
+#pragma unroll
+    for (int q = 0; q < NW; ++q) e0 += q < wp ? misc[32 + q] : 0;
+    const int mine = cs + max(0, min(ce, take_ties - e0));
+    if (lane == 0) misc[40 + wp] = mine;
+    __syncthreads();
+    int w_off = 0, tot_s = 0;
+#pragma unroll
+    for (int q = 0; q < NW; ++q) {
+        const int v = misc[40 + q];
+        w_off += q < wp ? v : 0;
+        tot_s += v;
     }
-    int tot_s;
-    int w = block_excl_scan<NT>(cs, tmp, tot_s);
     if (tid == 0) misc[4] = tot_s;
     cluster.sync();
-    int base = 0;
-    for (int r = 0; r < c; ++r) base += *cluster.map_shared_rank(misc + 4, r);
+    const int base = __reduce_add_sync(0xffffffffu, lane < c ? *cluster.map_shared_rank(misc + 4, lane) : 0);
     int32_t *out = a.idx_out + (size_t)bh * a.k;
     {
-        int e = e0;
-        w += base;
-        for (int j = j0; j < j1; ++j) {
-            const uint32_t u = keys[j];
-            bool sel = take_all || (kb > 0 && (above(u) || (in_group(u) && whole)));
-            if (!take_all && kb > 0 && !whole && in_group(u)) {
-                sel = e < take_ties;
-                ++e;
-            }
+        int w = base + w_off, e = e0;
+        for (int j0 = jb; j0 < je; j0 += 32) {
+            const int j = j0 + lane;
+            const bool ok = j < je;
+            const uint32_t u = ok ? keys[j] : 0u;
+            const bool tie = ok && ties_on && (u & mask) == prefix;
+            const unsigned tb = __ballot_sync(0xffffffffu, tie);
+            const bool sel = (ok && sure_of(u)) || (tie && e + __popc(tb & lt) < take_ties);
+            const unsigned sb = __ballot_sync(0xffffffffu, sel);
             if (sel) {
-                if (w < a.k) out[w] = lo + j;
-                ++w;
+                const int p = w + __popc(sb & lt);
+                if (p < a.k) out[p] = lo + j;
             }
+            w += __popc(sb);
+            e += __popc(tb);
         }
     }
     if (c == C - 1) {
@@ -486,7 +509,7 @@ cudaError_t plan_csel_uncached(int form, int src, int agg, int B, int Hkv, int T
         // deepest ring (most bytes in flight per CTA) that keeps the wave resident
         for (int ns = kMaxStagesC; ns >= 2; --ns) {
             if (src == SRC_SCORES && ns != 2) continue;  // no ring for a score source
-            const size_t smem = csel_smem(src != SRC_SCORES, src == SRC_SCORES ? 0 : r, nq, slice, ns).total;
+            const size_t smem = csel_smem(src != SRC_SCORES, src == SRC_SCORES ? 0 : r, nq, slice, ns, C).total;
             int optin = 0, dev = 0;
             cudaError_t e = cudaGetDevice(&dev);
             if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
