@@ -303,8 +303,10 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
             if (st == JSSA_OK) L.gcount = take(L.total, (size_t)sh.BH * 4);
             break;
         case JSSA_OP_DECODE_STEP: {
-            // one fused launch where the shape allows it (it also beats the
-            // three-launch cluster form on short caches and small batches)
+            // one fused launch where the shape allows it; with k <= 256 it
+            // also beats the three-launch cluster form on short caches and
+            // small batches, so the streaming form is then tried first (with a
+            // larger k the cluster form keeps its place where it plans)
             ScanPlan fp{};
             bool fused_ok = false;
             if (!sh.latent && agg == JSSA_AGG_SUM && d->kv_dtype == JSSA_BF16 && d->kt_dtype == JSSA_BF16 &&
@@ -318,7 +320,8 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
                 }
             }
             L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
-            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L, fused_ok);
+            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L,
+                               fused_ok && k <= 256);
             if (st == JSSA_OK) st = layout_attend(d, sh, ATT_INDEXED, k, L);
             if (st == JSSA_OK && fused_ok && L.wspec && fp.max_seg <= L.sp.max_seg) {
                 L.fp = fp;
