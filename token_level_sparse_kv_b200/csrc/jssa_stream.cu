@@ -58,6 +58,7 @@ constexpr int kBins = 2048;                       // 11-bit digits
 constexpr int kBoundary = 64;                     // boundary group ranked exactly
 constexpr int kEpochTokens = 2048;                // minimum tokens per epoch
 constexpr int kMaxRows = 8;                       // (b,h) rows per CTA range on the fused step
+constexpr int kMinSegTiles = 16;                  // shortest row segment a CTA streams
 constexpr int kChunkD = 16;                       // inputs per partial sum of a projection
 
 __host__ __device__ inline int npow2(int x) {
@@ -911,39 +912,49 @@ __device__ __forceinline__ float sum_parts(const float *part, int j, int nch) {
 }
 
 // Folded query of row bh: qb = P_h^T (sum of the group's queries, in head order).
-// Each work item (chunk c of kChunkD inputs, output j) loads its P column
-// slice and the group's query chunks at once and folds the queries itself:
-// one memory latency, no staging barrier.  The arithmetic order matches the
-// projection kernel's (head sum from 0 in head order, fma chain per chunk,
-// chunk partials left to right), so both give the same bits.
+// A work pair (chunk c of kChunkD inputs; outputs j and j + R/2) issues the
+// loads of its two P column slices before the fold's query loads, so both
+// are in flight together; the fold goes through shared memory (one dim per
+// thread).  The arithmetic order matches the projection kernel's (head sum
+// from 0 in head order, fma chain per chunk, chunk partials left to right),
+// so both give the same bits.
 template <int R>
-__device__ void sel_project(const StepExtra &x, int Hkv, int bh, float *qb, float *part, int st) {
+__device__ void sel_project(const StepExtra &x, int Hkv, int bh, float *qb, float *xs, float *part, int st) {
     const int b = bh / Hkv, h = bh - b * Hkv, G = x.G, d = x.d;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(x.q) + ((size_t)b * x.Hq + (size_t)h * G) * d;
     const float *P = x.P + (size_t)h * d * R;
     const int nch = d / kChunkD;
-    static_assert(kChunkD == 16, "two 16-byte query loads per chunk");
-    for (int p = st; p < R * nch; p += kSelT) {
-        const int c = p / R, j = p - c * R;
-        float pv[kChunkD], xr[kChunkD];
+    constexpr int RH = R / 2;
+    const int npair = RH * nch;
+    float pv0[kChunkD], pv1[kChunkD];
+    auto load_pair = [&](int pp) {
+        const int c = pp / RH, j = pp - c * RH;
 #pragma unroll
         for (int i = 0; i < kChunkD; ++i) {
-            pv[i] = __ldg(P + (size_t)(c * kChunkD + i) * R + j);
-            xr[i] = 0.f;
+            pv0[i] = __ldg(P + (size_t)(c * kChunkD + i) * R + j);
+            pv1[i] = __ldg(P + (size_t)(c * kChunkD + i) * R + j + RH);
         }
+    };
+    if (st < npair) load_pair(st);
+    for (int i = st; i < d; i += kSelT) {
+        float sum = 0.f;
 #pragma unroll 4
-        for (int g = 0; g < G; ++g) {
-            const uint4 *qv = reinterpret_cast<const uint4 *>(q + (size_t)g * d + c * kChunkD);
-            float f[16];
-            Vec16<__nv_bfloat16>::unpack(__ldg(qv), f);
-            Vec16<__nv_bfloat16>::unpack(__ldg(qv + 1), f + 8);
+        for (int g = 0; g < G; ++g) sum += __bfloat162float(q[(size_t)g * d + i]);
+        xs[i] = sum;
+    }
+    sel_sync();
+    for (int pp = st; pp < npair; pp += kSelT) {
+        if (pp != st) load_pair(pp);
+        const int c = pp / RH, j = pp - c * RH;
+        const float *xr = xs + c * kChunkD;
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int i = 0; i < kChunkD; ++i) xr[i] += f[i];
+        for (int i = 0; i < kChunkD; ++i) {
+            a0 = fmaf(xr[i], pv0[i], a0);
+            a1 = fmaf(xr[i], pv1[i], a1);
         }
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < kChunkD; ++i) acc = fmaf(xr[i], pv[i], acc);
-        part[(size_t)j * nch + c] = acc;
+        part[(size_t)j * nch + c] = a0;
+        part[(size_t)(j + RH) * nch + c] = a1;
     }
     sel_sync();
     for (int j = st; j < R; j += kSelT) qb[j] = sum_parts(part, j, nch);
@@ -1455,7 +1466,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             float *xs = reinterpret_cast<float *>(smem + L.xs);
             float *part = reinterpret_cast<float *>(S.hist);
             for (int rl = 0; rl < nrows; ++rl) {
-                sel_project<R>(A.x, a.Hkv, row0 + rl, qb + (size_t)rl * R, part, S.st);
+                sel_project<R>(A.x, a.Hkv, row0 + rl, qb + (size_t)rl * R, xs, part, S.st);
                 if (S.st == 0) mbar_arrive(&qready[rl]);  // consumers of row rl may start
             }
             for (int rl = 0; rl < nrows; ++rl) {
@@ -1657,7 +1668,12 @@ cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, P.smem);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorNotSupported;
+    // one CTA per SM, but no row split into segments of fewer than
+    // kMinSegTiles tiles: a short row streams faster than the cross-CTA merge
+    // of its segments would take (a 4K-token row is one 256 KiB segment)
     long long g = device_sm_count();
+    const long long segs = (long long)B * Hkv * ((P.tiles_per_bh + kMinSegTiles - 1) / kMinSegTiles);
+    if (g > segs) g = segs;
     if (g > P.total_tiles) g = P.total_tiles;
     if (g < 1) g = 1;
     P.grid = (int)g;
