@@ -77,3 +77,21 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_flushes_l2_only_for_steps_that_fit():
+    """Steps whose bytes fit in the L2 are timed with a flush before each one
+    (and config.l2 says so); the 1 GiB headline step streams past it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from token_level_sparse_kv_b200.inputs import WORKLOADS
+
+    l2 = 126 * 2**20
+    assert bench.flushes_l2(WORKLOADS["gqa_4k_b1"], l2)
+    assert bench.flushes_l2(WORKLOADS["gqa_32k_b4"], l2)
+    assert not bench.flushes_l2(WORKLOADS["gqa_128k_b16"], l2)
+    assert not bench.flushes_l2(WORKLOADS["hybrid_global_128k_b8"], l2)
+    c = bench.config_of(WORKLOADS["gqa_4k_b1"], 1, flush=True)
+    assert c["l2"].startswith("L2 flushed before every timed step")
+    c = bench.config_of(WORKLOADS["gqa_128k_b16"], 1)
+    assert c["l2"].startswith("inputs larger than L2")

@@ -638,3 +638,26 @@ def test_forced_tokens_decode_step(fused, monkeypatch):
     np.testing.assert_array_equal(host(idx).numpy(), ref_idx)
     ref_o, ref_l = oracle.attend(q, K, V, host(idx), host(cnt), slh, w.scale)
     check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
+def test_decode_step_form_choice():
+    """The decode step runs as one fused launch where it plans and k <= 256
+    (also on short caches and small batches); a larger k keeps the
+    three-launch cluster form where that plans; the latent cache takes four
+    launches (prologue, cluster selection, attention, combine)."""
+    from token_level_sparse_kv_b200.inputs import WORKLOADS, Workload
+
+    def form(w):
+        dims = ops.Dims()
+        dims.B, dims.Hq, dims.Hkv, dims.d, dims.dv, dims.T_cap, dims.r = w.B, w.Hq, w.Hkv, w.d, w.Dv, w.T, w.r
+        dims.kv_dtype, dims.kt_dtype = ops.BF16, ops.BF16
+        return ops.plan_info(dims, w.k, ops.OP_DECODE_STEP)
+
+    for name in ("gqa_4k_b1", "gqa_32k_b4", "gqa_128k_b16", "hybrid_global_128k_b8"):
+        n, text = form(WORKLOADS[name])
+        assert n == 1 and "fused" in text, (name, n, text)
+    w = WORKLOADS["gqa_128k_b16"]
+    n, text = form(Workload(**{**w.__dict__, "B": 1, "k": 1024}))
+    assert n == 3 and "cluster" in text, (n, text)
+    n, text = form(WORKLOADS["mla_64k_b8"])
+    assert n == 4, (n, text)
