@@ -65,6 +65,8 @@
  * memory, taken when all B*Hkv clusters fit on the GPU at once; otherwise a
  * persistent streaming pass with a segment merge, warp-specialised for SUM
  * over the low-rank cache, block-synchronous for the other cases.  The
+ * decode step with k <= 256 (SUM, bf16 caches, not the latent form) tries
+ * the streaming form first, since it then runs as one fused launch.  The
  * environment variable JSSA_SELECT_FORM = "cluster", "stream" or "scan"
  * forces one form at planning time where it has a kernel (tests and
  * measurement); size the workspace after setting it.

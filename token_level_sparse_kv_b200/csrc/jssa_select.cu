@@ -8,17 +8,21 @@
 //
 // The C CTAs of a cluster split the token range of one (b, h) into C
 // contiguous slices.  Each CTA streams its slice of the low-rank key cache
-// through a two-deep ring of 32 KiB bulk asynchronous copies (or reads its
-// slice of a score array), computes the fp32 scores exactly as the score pass
-// does, and keeps their order-preserving uint32 keys in shared memory.  The
-// cluster then finds the k-th key together: three radix levels of 11, 11 and
-// 10 bits; at each level every CTA histograms its keys that match the prefix
-// found so far, each CTA sums one slice of the bins across the cluster through
-// distributed shared memory, and every CTA scans the summed histogram.  Keys
+// through a ring of 32 KiB bulk asynchronous copies (2 to 6 stages, the
+// planner's choice; or reads its slice of a score array), computes the fp32
+// scores exactly as the score pass does, and keeps their order-preserving
+// uint32 keys in shared memory.  The cluster then finds the k-th key
+// together: three radix levels of 11, 11 and 10 bits; at each level every
+// CTA histograms its keys that match the prefix found so far and adds its
+// non-empty bins into the CTA that owns them (bin d lives in rank
+// d / (2048 / C), in one of three rotating copies), one cluster barrier
+// later every CTA gathers the summed bins through distributed shared memory
+// and scans them.  Keys
 // equal to the k-th key are taken lowest token index first (CTAs hold
 // ascending token ranges, so an exclusive scan of their tie counts orders
 // them).  Each CTA finally writes its selected tokens, already ascending, at
-// its offset in the index list: no merge and no sort.  The result is the same
+// its offset in the index list (a warp's 32-token steps ordered by ballots):
+// no merge and no sort.  The result is the same
 // set, in the same order, as jssa_score + jssa_topk.
 #include <cooperative_groups.h>
 
