@@ -184,9 +184,13 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     // ---- S = Q K^T over the nine 64-column blocks -------------------------------
     constexpr uint32_t idS = mma_idesc(128, kTok, 0, 0);
     bool ok = true;
+    // Commit groups: G0..G3 = K block g + Q block g, G4 = K blocks 4..8, then
+    // R_j = Q block j + 4 (j = 0..4), committed in iteration j + 1 once the
+    // products of iteration j, which read its buffer, are done: by then they
+    // have had a whole iteration to finish, so the wait rarely stalls.
     for (int kb = 0; kb < kKB; ++kb) {
-        // groups committed after the one holding block kb (see the load order)
-        const int after = kb < kQBuf ? kQBuf : min(kQBuf - 1, kKB - 1 - kb);
+        // groups committed after the one holding block kb when this iteration starts
+        const int after = kb < kQBuf ? (kQBuf - kb) + max(0, kb - 1) : min(kQBuf, kb - 2) - kb + kQBuf;
         cp_wait_dyn<kQBuf>(after);
         fence_async_smem();
         tc_fence_before();
@@ -200,11 +204,11 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
                          (kb > 0 || kk > 0) ? 1u : 0u);
             mma_commit(&qfree[kb % kQBuf]);
         }
-        if (kb + kQBuf < kKB) {
-            // refill this Q buffer with block kb+4 once the products reading it are done
-            if (ok && !mbar_wait_bounded(&qfree[kb % kQBuf], (uint32_t)(kb / kQBuf) & 1u)) atomicOr(flag, 1);
+        const int jr = kb - 1;  // refill the buffer of the previous iteration's block
+        if (jr >= 0 && jr + kQBuf < kKB) {
+            if (ok && !mbar_wait_bounded(&qfree[jr % kQBuf], (uint32_t)(jr / kQBuf) & 1u)) atomicOr(flag, 1);
             fence_async_smem();
-            if (*flag == 0) load_q_block(kb + kQBuf, kb % kQBuf);
+            if (*flag == 0) load_q_block(jr + kQBuf, jr % kQBuf);
             cp_async_commit();
         }
         __syncthreads();
