@@ -67,9 +67,9 @@
  * over the low-rank cache, block-synchronous for the other cases.  The
  * decode step with k <= 256 (SUM, bf16 caches, not the latent form) tries
  * the streaming form first, since it then runs as one fused launch.  The
- * environment variable JSSA_SELECT_FORM = "cluster", "stream" or "scan"
- * forces one form at planning time where it has a kernel (tests and
- * measurement); size the workspace after setting it.
+ * `form` field of jssa_select_opts forces one form where it has a kernel
+ * (tests and measurement); jssa_workspace_size covers every form.  The
+ * library reads no environment variables.
  */
 #ifndef JSSA_H
 #define JSSA_H
@@ -81,7 +81,7 @@
 extern "C" {
 #endif
 
-#define JSSA_VERSION 1
+#define JSSA_VERSION 2
 
 #if defined(__GNUC__)
 #define JSSA_API __attribute__((visibility("default")))
@@ -141,9 +141,9 @@ JSSA_API const char *jssa_status_string(int status);
 JSSA_API const char *jssa_last_error(void);
 
 /* Bytes of workspace `op` needs for these dims and k (k is ignored by ops
- * without a selection).  The size covers either aggregation and any sliding
- * window, and depends on the current device's SM count.  Writes *bytes;
- * returns a status. */
+ * without a selection).  The size covers either aggregation, any sliding
+ * window and every selection form and option (jssa_select_opts), and depends
+ * on the current device's SM count.  Writes *bytes; returns a status. */
 JSSA_API int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes);
 
 /* How one call of `op` (JSSA_OP_*) with these dims, k and aggregation is
@@ -194,15 +194,32 @@ JSSA_API int jssa_select(const jssa_dims *dims, const void *q, const float *P, c
                 const int32_t *seq_lens, int agg, int k, int32_t *idx, int32_t *count,
                 void *ws, size_t ws_bytes, jssa_stream_t stream);
 
-/* Selection options: tokens that are always selected.  A variant the pages
- * do not describe (their selection is a pure top-k); the reading is the usual
- * one of sparse decoders that keep "sink" tokens and a recent window.  With
- * F = {t < n_sink} U {t >= T_b - n_recent} (t < T_b): if |F| >= k_b the
- * selection is the k_b smallest indices of F, otherwise F plus the k_b - |F|
- * best other tokens under (score desc, t asc).  NULL or zeros: plain top-k. */
+/* Selection forms (jssa_select_opts.form).  All give identical results. */
+typedef enum {
+    JSSA_FORM_AUTO = 0,    /* the library's choice for the shape */
+    JSSA_FORM_CLUSTER = 1, /* one thread-block cluster per (b, h) (several waves allowed) */
+    JSSA_FORM_STREAM = 2,  /* the warp-specialised streaming pass (SUM over the low-rank cache) */
+    JSSA_FORM_SCAN = 3     /* the block-synchronous streaming pass */
+} jssa_select_form;
+
+/* Selection options.
+ *  - n_sink, n_recent: tokens that are always selected.  A variant the pages
+ *    do not describe (their selection is a pure top-k); the reading is the
+ *    usual one of sparse decoders that keep "sink" tokens and a recent
+ *    window.  With F = {t < n_sink} U {t >= T_b - n_recent} (t < T_b): if
+ *    |F| >= k_b the selection is the k_b smallest indices of F, otherwise F
+ *    plus the k_b - |F| best other tokens under (score desc, t asc).
+ *  - form: a jssa_select_form; a forced form without a kernel for the shape
+ *    falls back to the next one (cluster -> stream -> scan).
+ *  - unfused: for jssa_decode_step_ex, nonzero keeps the step in separate
+ *    launches (prologue, selection, attention) even where the one-launch
+ *    fused form applies.
+ * NULL or all zeros: plain top-k, automatic form. */
 typedef struct {
     int32_t n_sink;   /* >= 0 */
     int32_t n_recent; /* >= 0 */
+    int32_t form;     /* jssa_select_form */
+    int32_t unfused;  /* 0 or 1 */
 } jssa_select_opts;
 
 /* jssa_topk, jssa_select and jssa_decode_step with selection options (NULL
@@ -264,6 +281,25 @@ JSSA_API int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const voi
                         int32_t *count, void *out, float *lse, void *ws, size_t ws_bytes,
                         jssa_stream_t stream);
 
+/* jssa_plan_info with selection options (NULL = jssa_plan_info): the forms
+ * and launch count of a call made with these options. */
+JSSA_API int jssa_plan_info_ex(const jssa_dims *dims, int k, int op, int agg, const jssa_select_opts *opts,
+                               int *launches, char *desc, size_t desc_len);
+
+/* Failure-detection self-check of the bounded on-chip waits.  The method
+ * pages have no counterpart.  Every wait inside the library's kernels (on an
+ * mbarrier phase, or on a device word other CTAs raise) is bounded: after a
+ * wall-time limit (2 s in the path's kernels) it gives up, the kernel sets
+ * JSSA_DEV_TIMEOUT in the status word, and it returns instead of trapping or
+ * hanging.  This call runs those same wait routines, with limit_ns, in one
+ * small kernel on a barrier and a word that nothing completes, so every wait
+ * expires: afterwards the status word (word 0 of ws) holds JSSA_DEV_TIMEOUT
+ * and the 32-bit word at byte 128 of ws holds 3, the number of waits that
+ * gave up.  ws: device memory of at least 256 bytes, 16-byte aligned (bytes
+ * 64..255 are cleared on `stream` first).  limit_ns in [1000, 1000000000].
+ * The context stays usable. */
+JSSA_API int jssa_check_wait_expiry(void *ws, size_t ws_bytes, uint64_t limit_ns, jssa_stream_t stream);
+
 /* Allocation-free variant of jssa_indexed_decode.  The method pages have no
  * counterpart: this is an integration entry point of this library.
  *
@@ -282,6 +318,10 @@ JSSA_API int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const voi
  *    JSSA_ERR_WORKSPACE and a message (use jssa_indexed_decode then).
  *  - The first call on each device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
+ *    The address stays cached for the process: after cudaDeviceReset() on a
+ *    device, unload and reload the library before calling this again.
+ *  - Latent-cache shapes (d = 576, dv = 512, Hkv = 1, 128 heads) are served
+ *    too, with their split partials in the same array.
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents.  The call clears the counters and the status word on `stream`
  *    before its kernel; calls whose execution overlaps on the GPU (other

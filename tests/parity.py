@@ -14,7 +14,11 @@ Tolerances (written here once, used by every GPU test):
     s_k - tau may be, and the counts are equal;
   * attention output: max |gpu - oracle| <= 2e-2 with bf16 K/V (fp32
     accumulation; the output itself is stored in bf16), 1e-4 with fp32 K/V;
-    lse within 1e-3.
+    lse within 1e-3;
+  * end to end (the oracle's own low-rank cache, fp64 scores, selection and
+    attention against the GPU's step): the selection rule above against the
+    oracle's own scores for every (b, h), and the output rule wherever the
+    two index sets are identical.
 """
 from __future__ import annotations
 
@@ -114,3 +118,33 @@ def check_attention(out_gpu, lse_gpu, out_ref, lse_ref, dtype):
         d = np.abs(np.where(both_inf, 0.0, l - np.where(both_inf, 0.0, lse_ref)))
         assert d.max() <= LSE_TOL, "max |lse - oracle| = %.3g" % d.max()
     return float(err.max())
+
+
+def check_end_to_end(out_gpu, lse_gpu, idx_gpu, cnt_gpu, s_or, idx_or, out_or, lse_or, seq_lens, k, G):
+    """GPU step vs the oracle's own step.  Every (b, h) selection obeys the
+    tie-window rule against the oracle's own fp64 scores; every difference
+    between the two index sets lies inside the window (rule 4); outputs (and
+    lse) agree within the attention tolerance wherever the sets are
+    identical.  Returns the number of (b, h) sets that differ."""
+    def arr(x):
+        return host(x).numpy() if isinstance(x, torch.Tensor) else np.asarray(x)
+
+    ig = arr(idx_gpu)
+    n_diff = check_selection(ig, arr(cnt_gpu), s_or, arr(seq_lens), k)
+    B, Hkv, _ = ig.shape
+    o = host(out_gpu).double().numpy()
+    l = host(lse_gpu).double().numpy() if lse_gpu is not None else None
+    same = np.all(ig == arr(idx_or), axis=2)
+    for b in range(B):
+        for h in range(Hkv):
+            if not same[b, h]:
+                continue
+            rows = slice(h * G, (h + 1) * G)
+            err = np.abs(o[b, rows] - out_or[b, rows]).max()
+            assert err <= OUT_TOL[torch.bfloat16], "end-to-end output error %.3g at (%d,%d)" % (err, b, h)
+            if l is not None:
+                fin = np.isfinite(lse_or[b, rows])
+                assert np.array_equal(np.isfinite(l[b, rows]), fin)
+                assert np.abs(l[b, rows][fin] - lse_or[b, rows][fin]).max(initial=0.0) <= LSE_TOL
+    assert n_diff == int((~same).sum())
+    return n_diff

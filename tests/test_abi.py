@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(libpath):
 
 def test_library_loads_and_host_only_calls_work(libpath):
     L = ops.lib()
-    assert L.jssa_version() == 1
+    assert L.jssa_version() == 2
     assert L.jssa_status_string(0) == b"JSSA_OK"
     assert b"INVALID" in L.jssa_status_string(-1)
     n = ctypes.c_size_t(0)
@@ -76,3 +76,19 @@ def test_product_package_has_no_oracle_dependency():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "jssa_oracle" not in txt, f
+
+
+def test_library_reads_no_environment_variables():
+    """Dispatch choices are explicit arguments (jssa_select_opts), never the
+    environment: the library source holds no getenv call."""
+    csrc = os.path.join(ROOT, "token_level_sparse_kv_b200", "csrc")
+    for f in os.listdir(csrc):
+        if f.endswith((".cu", ".cuh", ".h")):
+            assert "getenv" not in open(os.path.join(csrc, f)).read(), f
+
+
+def test_select_opts_layout_matches_the_header():
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct \{([^}]*)\} jssa_select_opts;", src).group(1)
+    fields = re.findall(r"int32_t\s+(\w+);", body)
+    assert fields == [n for n, _ in ops.SelectOpts._fields_]

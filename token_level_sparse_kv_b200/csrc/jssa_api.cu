@@ -159,14 +159,15 @@ size_t take(size_t &off, size_t bytes) {
 // Selection form: the cluster form where one wave of clusters covers the
 // rows, else the streaming form, else the block-synchronous scan.  With
 // stream_first (a decode step that runs as one fused launch of the streaming
-// kernel) the streaming form is tried first.  JSSA_SELECT_FORM overrides.
-int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, Layout &L, bool stream_first = false) {
+// kernel) the streaming form is tried first.  A forced form (form != 0,
+// jssa_select_form) overrides the choice.
+int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, int form, Layout &L,
+                  bool stream_first = false) {
     const int nq = (src != SRC_SCORES && agg == JSSA_AGG_MAX) ? sh.G : 1;
-    const int form = select_form_override();
-    stream_first = stream_first && form == 0;
+    stream_first = stream_first && form == JSSA_FORM_AUTO;
     auto try_csel = [&](bool &ok) -> int {
         ok = false;
-        cudaError_t ec = plan_csel(src, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.cp);
+        cudaError_t ec = plan_csel(form, src, agg, d->B, d->Hkv, d->T_cap, d->r, nq, k, &L.cp);
         if (ec == cudaSuccess) {
             L.csel = true;
             ok = true;
@@ -181,7 +182,7 @@ int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, 
         const int st = try_csel(done);
         if (st != JSSA_OK || done) return st;
     }
-    cudaError_t e = form == 3 ? cudaErrorNotSupported : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
+    cudaError_t e = form == JSSA_FORM_SCAN ? cudaErrorNotSupported : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
     if (e == cudaSuccess) {
         L.wspec = true;
     } else {
@@ -219,14 +220,23 @@ int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout
     return JSSA_OK;
 }
 
-// The fused decode step can be switched off with JSSA_FUSED_STEP=0 (tests of
-// the three-launch form and measurement).
-bool fused_step_allowed() {
-    const char *v = getenv("JSSA_FUSED_STEP");
-    return !(v && v[0] == '0');
+// Planning choices a caller can force (jssa_select_opts): the selection
+// form, and whether the decode step may run as one fused launch.
+struct Choice {
+    int form = JSSA_FORM_AUTO;
+    int unfused = 0;
+};
+Choice choice_of(const jssa_select_opts *opts) {
+    Choice c;
+    if (opts) {
+        c.form = opts->form;
+        c.unfused = opts->unfused ? 1 : 0;
+    }
+    return c;
 }
 
-int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L);
+int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Choice ch,
+                          Layout &L);
 
 // Layouts (workspace offsets and kernel plans) are cached per device, dims,
 // op and settings: planning costs occupancy queries and attribute calls that
@@ -247,7 +257,7 @@ LayoutEntry g_layouts[kLayoutCache];
 int g_layouts_n = 0, g_layouts_next = 0;
 std::mutex g_layouts_mu;
 
-int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L) {
+int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Choice ch, Layout &L) {
     LayoutKey key;
     memset(&key, 0, sizeof key);
     cudaError_t e = cudaGetDevice(&key.dev);
@@ -256,8 +266,8 @@ int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, in
     key.k = k;
     key.agg = agg;
     key.window = window;
-    key.form = select_form_override();
-    key.fused = fused_step_allowed() ? 1 : 0;
+    key.form = ch.form;
+    key.fused = ch.unfused ? 0 : 1;
     key.dims = *d;
     {
         std::lock_guard<std::mutex> lk(g_layouts_mu);
@@ -267,7 +277,7 @@ int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, in
                 return JSSA_OK;
             }
     }
-    const int st = build_layout_uncached(d, sh, k, op, agg, window, L);
+    const int st = build_layout_uncached(d, sh, k, op, agg, window, ch, L);
     if (st != JSSA_OK) return st;
     std::lock_guard<std::mutex> lk(g_layouts_mu);
     LayoutEntry &slot = g_layouts[g_layouts_n < kLayoutCache ? g_layouts_n++ : (g_layouts_next++ % kLayoutCache)];
@@ -276,7 +286,8 @@ int build_layout(const jssa_dims *d, const Shape &sh, int k, int op, int agg, in
     return JSSA_OK;
 }
 
-int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Layout &L) {
+int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, int agg, int window, Choice ch,
+                          Layout &L) {
     L = Layout();
     int st = JSSA_OK;
     const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
@@ -289,10 +300,10 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
             if (e != cudaSuccess) return cuda_fail(e, "planning the score pass");
             break;
         }
-        case JSSA_OP_TOPK: st = layout_select(d, sh, SRC_SCORES, k, agg, L); break;
+        case JSSA_OP_TOPK: st = layout_select(d, sh, SRC_SCORES, k, agg, ch.form, L); break;
         case JSSA_OP_SELECT:
             L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
-            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L);
+            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, ch.form, L);
             break;
         case JSSA_OP_INDEXED_DECODE: st = layout_attend(d, sh, ATT_INDEXED, k, L); break;
         case JSSA_OP_DENSE_DECODE:
@@ -310,7 +321,7 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
             ScanPlan fp{};
             bool fused_ok = false;
             if (!sh.latent && agg == JSSA_AGG_SUM && d->kv_dtype == JSSA_BF16 && d->kt_dtype == JSSA_BF16 &&
-                fused_step_allowed()) {
+                !ch.unfused) {
                 cudaError_t e = plan_step_fused(d->B, d->Hkv, d->Hq, d->d, d->T_cap, d->r, k, &fp);
                 if (e == cudaSuccess) {
                     fused_ok = true;
@@ -320,7 +331,7 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
                 }
             }
             L.qproj = take(L.total, (size_t)sh.BH * nq * d->r * 4);
-            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, L,
+            st = layout_select(d, sh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, agg, ch.form, L,
                                fused_ok && k <= 256);
             if (st == JSSA_OK) st = layout_attend(d, sh, ATT_INDEXED, k, L);
             if (st == JSSA_OK && fused_ok && L.wspec && fp.max_seg <= L.sp.max_seg) {
@@ -348,6 +359,18 @@ T *at(void *ws, size_t off) {
 }
 
 cudaStream_t S(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int check_opts(const jssa_select_opts *opts) {
+    if (!opts) return JSSA_OK;
+    if (opts->n_sink < 0 || opts->n_recent < 0)
+        return fail(JSSA_ERR_INVALID_ARG, "negative forced-token count (n_sink=%d, n_recent=%d)", opts->n_sink,
+                    opts->n_recent);
+    if (opts->form < JSSA_FORM_AUTO || opts->form > JSSA_FORM_SCAN)
+        return fail(JSSA_ERR_INVALID_ARG, "unknown selection form %d", opts->form);
+    if (opts->unfused != 0 && opts->unfused != 1)
+        return fail(JSSA_ERR_INVALID_ARG, "unfused=%d is neither 0 nor 1", opts->unfused);
+    return JSSA_OK;
+}
 
 void fill_attn(AttnArgs &a, const jssa_dims *d, const Shape &sh, const void *q, const void *K, const void *V,
                const int32_t *seq_lens, float scale, void *out, float *lse, void *ws, const Layout &L) {
@@ -489,19 +512,31 @@ int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes) {
          op == JSSA_OP_DECODE_STEP) &&
         (st = check_attn_shape(dims, sh, op == JSSA_OP_INDEXED_DECODE || op == JSSA_OP_DECODE_STEP)))
         return st;
+    const bool selects = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_DECODE_STEP;
     size_t best = 0;
     for (int agg = 0; agg < 2; ++agg) {
         if (agg == JSSA_AGG_MAX && sh.G > kMaxG) continue;
-        Layout L;
-        st = build_layout(dims, sh, k, op, agg, 0, L);
-        if (st) return st;
-        if (L.total > best) best = L.total;
+        for (int form = 0; form < (selects ? 4 : 1); ++form)
+            for (int unf = 0; unf < (op == JSSA_OP_DECODE_STEP ? 2 : 1); ++unf) {
+                Choice ch;
+                ch.form = form;
+                ch.unfused = unf;
+                Layout L;
+                st = build_layout(dims, sh, k, op, agg, 0, ch, L);
+                if (st) return st;
+                if (L.total > best) best = L.total;
+            }
     }
     *bytes = best;
     return JSSA_OK;
 }
 
 int jssa_plan_info(const jssa_dims *dims, int k, int op, int agg, int *launches, char *desc, size_t desc_len) {
+    return jssa_plan_info_ex(dims, k, op, agg, nullptr, launches, desc, desc_len);
+}
+
+int jssa_plan_info_ex(const jssa_dims *dims, int k, int op, int agg, const jssa_select_opts *opts, int *launches,
+                      char *desc, size_t desc_len) {
     Shape sh;
     int st = check_dims(dims, &sh);
     if (st) return st;
@@ -510,8 +545,9 @@ int jssa_plan_info(const jssa_dims *dims, int k, int op, int agg, int *launches,
     const bool needs_k = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_INDEXED_DECODE ||
                          op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP;
     if (needs_k && (st = check_k(k))) return st;
+    if ((st = check_opts(opts))) return st;
     Layout L;
-    if ((st = build_layout(dims, sh, k, op, agg, 0, L))) return st;
+    if ((st = build_layout(dims, sh, k, op, agg, 0, choice_of(opts), L))) return st;
     const char *sel = L.csel ? "cluster" : (L.wspec ? "stream" : "scan");
     const int att = sh.latent ? 1 + (L.ap.splits > 1 ? 1 : 0) : 1;
     int n = 0;
@@ -561,7 +597,7 @@ int jssa_append_lowrank(const jssa_dims *dims, const void *K, const float *P, vo
     REQUIRE_PTR(pos_begin);
     if (n_new < 0 || n_new > dims->T_cap) return fail(JSSA_ERR_INVALID_ARG, "n_new=%d outside [0, T_cap]", n_new);
     Layout L;
-    if ((st = build_layout(dims, sh, 1, JSSA_OP_APPEND, 0, 0, L))) return st;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_APPEND, 0, 0, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (n_new == 0 || dims->B == 0) return JSSA_OK;
     AppendArgs a{K, P, Kt, pos_begin, at<uint32_t>(ws, 0), dims->B, dims->T_cap, dims->Hkv, dims->d, dims->r, n_new, 0};
@@ -583,7 +619,7 @@ int jssa_score(const jssa_dims *dims, const void *q, const float *P, const void 
     if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
     if (agg == JSSA_AGG_MAX && sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "MAX aggregation needs G <= %d", kMaxG);
     Layout L;
-    if ((st = build_layout(dims, sh, 1, JSSA_OP_SCORE, agg, 0, L))) return st;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_SCORE, agg, 0, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
@@ -607,13 +643,6 @@ int jssa_score(const jssa_dims *dims, const void *q, const float *P, const void 
     return JSSA_OK;
 }
 
-int check_opts(const jssa_select_opts *opts) {
-    if (opts && (opts->n_sink < 0 || opts->n_recent < 0))
-        return fail(JSSA_ERR_INVALID_ARG, "negative forced-token count (n_sink=%d, n_recent=%d)", opts->n_sink,
-                    opts->n_recent);
-    return JSSA_OK;
-}
-
 int jssa_topk(const jssa_dims *dims, const float *scores, const int32_t *seq_lens, int k, int32_t *idx,
               int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream) {
     return jssa_topk_ex(dims, scores, seq_lens, k, nullptr, idx, count, ws, ws_bytes, stream);
@@ -630,11 +659,11 @@ int jssa_topk_ex(const jssa_dims *dims, const float *scores, const int32_t *seq_
     REQUIRE_PTR(seq_lens);
     REQUIRE_PTR(idx);
     OPTIONAL_PTR(count);
+    if ((st = check_opts(opts))) return st;
     Layout L;
-    if ((st = build_layout(dims, sh, k, JSSA_OP_TOPK, 0, 0, L))) return st;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_TOPK, 0, 0, choice_of(opts), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
-    if ((st = check_opts(opts))) return st;
     return run_select(dims, sh, nullptr, nullptr, scores, seq_lens, JSSA_AGG_SUM, k, idx, count, ws, L, S(stream),
                       false, opts);
 }
@@ -659,10 +688,10 @@ int jssa_select_ex(const jssa_dims *dims, const void *q, const float *P, const v
     OPTIONAL_PTR(count);
     if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
     if (agg == JSSA_AGG_MAX && sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "MAX aggregation needs G <= %d", kMaxG);
-    Layout L;
-    if ((st = build_layout(dims, sh, k, JSSA_OP_SELECT, agg, 0, L))) return st;
-    if ((st = check_ws(ws, ws_bytes, L))) return st;
     if ((st = check_opts(opts))) return st;
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_SELECT, agg, 0, choice_of(opts), L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     return run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), true, opts);
 }
@@ -684,7 +713,7 @@ int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, con
     OPTIONAL_PTR(count);
     OPTIONAL_PTR(lse);
     Layout L;
-    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, L))) return st;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     if (sh.latent) return run_mla(dims, q, K, idx, count, k, seq_lens, softmax_scale, out, lse, ws, L, S(stream));
@@ -713,7 +742,7 @@ int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const
     REQUIRE_PTR(out);
     OPTIONAL_PTR(lse);
     Layout L;
-    if ((st = build_layout(dims, sh, 1, JSSA_OP_DENSE_DECODE, 0, window, L))) return st;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_DENSE_DECODE, 0, window, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     AttnArgs a;
@@ -747,7 +776,7 @@ int jssa_gather_then_dense(const jssa_dims *dims, const void *q, const void *K, 
         return fail(JSSA_ERR_INVALID_ARG, "gather_buf of %zu bytes is below the %zu bytes needed", gather_bytes,
                     2 * half);
     Layout L;
-    if ((st = build_layout(dims, sh, k, JSSA_OP_GATHER_THEN_DENSE, 0, 0, L))) return st;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_GATHER_THEN_DENSE, 0, 0, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     void *gK = gather_buf;
@@ -797,10 +826,10 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     REQUIRE_PTR(out);
     OPTIONAL_PTR(lse);
     if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
-    Layout L;
-    if ((st = build_layout(dims, sh, k, JSSA_OP_DECODE_STEP, agg, 0, L))) return st;
-    if ((st = check_ws(ws, ws_bytes, L))) return st;
     if ((st = check_opts(opts))) return st;
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_DECODE_STEP, agg, 0, choice_of(opts), L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     if (L.fused) {
         ScanArgs sa;
@@ -855,6 +884,19 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     return JSSA_OK;
 }
 
+int jssa_check_wait_expiry(void *ws, size_t ws_bytes, uint64_t limit_ns, jssa_stream_t stream) {
+    if (!ws) return fail(JSSA_ERR_INVALID_ARG, "ws is NULL");
+    if (!aligned16(ws)) return fail(JSSA_ERR_INVALID_ARG, "ws is not 16-byte aligned");
+    if (ws_bytes < 256) return fail(JSSA_ERR_WORKSPACE, "workspace of %zu bytes is below 256", ws_bytes);
+    if (limit_ns < 1000 || limit_ns > 1000000000ull)
+        return fail(JSSA_ERR_INVALID_ARG, "limit_ns=%llu outside [1000, 1e9]", (unsigned long long)limit_ns);
+    cudaError_t e = cudaMemsetAsync(static_cast<char *>(ws) + 64, 0, 192, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the self-check words");
+    e = launch_wait_expiry(ws, limit_ns, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching the wait self-check");
+    return JSSA_OK;
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------ allocation-free ---
@@ -872,7 +914,9 @@ void *g_noalloc_ptr[kMaxDevices] = {nullptr};
 std::mutex g_noalloc_mu;
 
 // Device address of the scratch array for the current device (looked up once
-// per device, with that device current).
+// per device, with that device current).  The cached address belongs to the
+// device's primary context: after cudaDeviceReset() it is stale, and the
+// library must be unloaded and loaded again before the next call.
 int noalloc_scratch(void **ptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -909,7 +953,7 @@ extern "C" int jssa_indexed_decode_noalloc(const jssa_dims *dims, const void *q,
     OPTIONAL_PTR(count);
     OPTIONAL_PTR(lse);
     Layout L;
-    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, L))) return st;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE, 0, 0, Choice(), L))) return st;
     if (L.total > kNoAllocBytes)
         return fail(JSSA_ERR_WORKSPACE,
                     "this shape needs %zu bytes of scratch, above the %zu bytes of the allocation-free entry point; "
@@ -922,6 +966,9 @@ extern "C" int jssa_indexed_decode_noalloc(const jssa_dims *dims, const void *q,
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, S(stream));
     if (e == cudaSuccess) e = cudaMemsetAsync(at<char>(ws, L.att_ctr), 0, (size_t)sh.BH * 4, S(stream));
     if (e != cudaSuccess) return cuda_fail(e, "clearing the allocation-free scratch");
+    // the latent-cache form keeps its split partials in the same array (the
+    // layout's offsets all lie below L.total, checked above)
+    if (sh.latent) return run_mla(dims, q, K, idx, count, k, seq_lens, softmax_scale, out, lse, ws, L, S(stream));
     AttnArgs a;
     fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
     a.idx = idx;

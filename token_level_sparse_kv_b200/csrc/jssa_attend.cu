@@ -549,7 +549,7 @@ cudaError_t plan_attend(int src, int kv_dtype, int d, int G, int B, int Hkv, int
     for (;;) {
         pk = pick_attend(src, kv_dtype, d, G, stages);
         if (!pk.kern) return cudaErrorInvalidValue;
-        cudaError_t e = cudaFuncSetAttribute(pk.kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pk.smem);
+        cudaError_t e = ensure_smem(reinterpret_cast<const void *>(pk.kern), pk.smem);
         if (e != cudaSuccess) return e;
         if (src == ATT_RANGE || splits == 1) break;
         if (splits > 8) {
@@ -613,6 +613,10 @@ cudaError_t launch_attend(const AttnPlan &p, int src, const AttnArgs &a0, int kv
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
+    {
+        cudaError_t es = ensure_smem(reinterpret_cast<const void *>(pk.kern), cfg.dynamicSmemBytes);
+        if (es != cudaSuccess) return es;
+    }
     return cudaLaunchKernelEx(&cfg, pk.kern, a);
 }
 

@@ -142,14 +142,48 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Bounded wait on an mbarrier phase: gives up after ~2 s of wall time (or
-// 2^28 polls), returning false.  Normal waits last microseconds.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+// Wall-time limit of every bounded on-chip wait in the library.  Normal
+// waits last microseconds; a wait that reaches the limit gives up, the
+// kernel records JSSA_DEV_TIMEOUT and returns.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Bounded wait on an mbarrier phase: gives up after limit_ns of wall time (or
+// 2^28 polls), returning false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0; it < (1u << 28); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u && global_timer_ns() - t0 > 2000000000ull) return false;
+        if ((it & 255u) == 255u && global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return false;
+}
+
+// Bounded wait until a device word (written by other CTAs) reaches `target`:
+// false after limit_ns of wall time.
+__device__ __forceinline__ bool flag_wait_bounded(const volatile unsigned *word, unsigned target,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+    const uint64_t t0 = global_timer_ns();
+    while (*word < target) {
+        if (global_timer_ns() - t0 > limit_ns) return false;
+        __nanosleep(64);
+    }
+    return true;
+}
+
+// Bounded mbarrier wait that also gives up when another role of the CTA
+// raised the abort flag.  The thread is parked in the hardware between polls
+// (up to 20 us per poll), so waiting warps do not take issue slots from the
+// working ones.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0; it < (1u << 20); ++it) {
+        if (mbar_try_wait_for(bar, parity, 20000u)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
 }

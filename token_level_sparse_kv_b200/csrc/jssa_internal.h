@@ -125,7 +125,9 @@ struct CSelPlan {
     int csize, slice, grid_y, nstages;
     size_t smem;
 };
-cudaError_t plan_csel(int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p);
+// form: jssa_select_form (JSSA_FORM_CLUSTER relaxes the one-wave condition;
+// JSSA_FORM_STREAM / JSSA_FORM_SCAN give cudaErrorNotSupported).
+cudaError_t plan_csel(int form, int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p);
 cudaError_t launch_csel(const CSelPlan &p, const CSelArgs &a, int src, int agg, cudaStream_t s, bool pdl);
 
 // ------------------------------------------------------------------- MLA ---
@@ -184,18 +186,24 @@ struct StepExtra {
 // r in {32, 64}, G a power of two <= 16); cudaErrorNotSupported otherwise.
 cudaError_t plan_step_fused(int B, int Hkv, int Hq, int d, int T_cap, int r, int k, ScanPlan *p);
 cudaError_t launch_step_fused(const ScanPlan &p, const ScanArgs &a, const StepExtra &x, cudaStream_t s, bool pdl);
-// Selection form forced by the environment (JSSA_SELECT_FORM): 0 automatic,
-// 1 "cluster", 2 "stream", 3 "scan".
-int select_form_override();
 cudaError_t plan_attend(int src, int kv_dtype, int d, int G, int B, int Hkv, int npos, AttnPlan *p);
 cudaError_t launch_attend(const AttnPlan &p, int src, const AttnArgs &a, int kv_dtype, int d, cudaStream_t s,
                           bool pdl);
 cudaError_t launch_gather(const GatherArgs &a, int kv_dtype, cudaStream_t s, bool pdl);
 
+// Failure-detection self-check (jssa_check_wait_expiry): the bounded waits on
+// a barrier and a flag that nothing completes; ws holds the status word at
+// byte 0, the flag at byte 64 and the count of expired waits at byte 128.
+cudaError_t launch_wait_expiry(void *ws, uint64_t limit_ns, cudaStream_t s);
+
 // Launch with the programmatic-stream-serialisation attribute (PDL) if asked.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
                           Args &&...args) {
+    // planning of other shapes may have set the attribute for this kernel;
+    // it only ever grows, so one check per launch keeps it sufficient
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

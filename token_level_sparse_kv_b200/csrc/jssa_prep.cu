@@ -340,6 +340,10 @@ cudaError_t launch_prep(const AppendArgs &ap0, const ProjArgs &pj, cudaStream_t 
         }
         cfg.attrs = attr;
         cfg.numAttrs = na;
+        {
+            cudaError_t es = ensure_smem(reinterpret_cast<const void *>(k), cfg.dynamicSmemBytes);
+            if (es != cudaSuccess) return es;
+        }
         return cudaLaunchKernelEx(&cfg, k, ap, pj);
     }
     const int G = pj.Hq / pj.Hkv;

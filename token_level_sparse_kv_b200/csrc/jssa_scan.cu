@@ -837,7 +837,7 @@ cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int
         P.cap = mode == MODE_SELECT ? k + (tiles2 > chunk ? tiles2 : chunk) + slack : 0;
         P.smem = scan_smem(src, mode, src == SRC_SCORES ? 0 : r, nq, P.nstages, P.cap, mode == MODE_SELECT ? k : 0)
                      .total;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+        cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), P.smem);
         if (e != cudaSuccess) return e;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, P.smem);
         if (e != cudaSuccess) return e;

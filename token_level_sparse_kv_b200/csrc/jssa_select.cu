@@ -440,20 +440,11 @@ int csel_tile(int src, int r) {
 // (many (b,h) rows or rows too long for shared memory) a persistent streaming
 // pass is taken: the warp-specialised one for SUM over the low-rank cache,
 // the block-synchronous one for the other sources and aggregations.  All
-// return the same indices.  The environment variable JSSA_SELECT_FORM
-// overrides the choice at planning time: "cluster" takes the cluster form
-// wherever its slices fit in shared memory (several waves allowed), "stream"
-// the warp-specialised pass where it has a kernel, "scan" the
+// return the same indices.  A forced form (jssa_select_opts.form) overrides
+// the choice: JSSA_FORM_CLUSTER takes the cluster form wherever its slices fit
+// in shared memory (several waves allowed), JSSA_FORM_STREAM the
+// warp-specialised pass where it has a kernel, JSSA_FORM_SCAN the
 // block-synchronous pass.
-int select_form_override() {
-    const char *v = getenv("JSSA_SELECT_FORM");
-    if (!v) return 0;
-    if (!strcmp(v, "cluster")) return 1;
-    if (!strcmp(v, "stream")) return 2;
-    if (!strcmp(v, "scan")) return 3;
-    return 0;
-}
-
 namespace {
 
 // Resident clusters of size C for this kernel and shared-memory size (0 on error).
@@ -519,7 +510,7 @@ cudaError_t plan_csel_uncached(int form, int src, int agg, int B, int Hkv, int T
             if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
             if (e != cudaSuccess) return e;
             if (smem > (size_t)optin) continue;
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
             if (e != cudaSuccess) return e;
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (e != cudaSuccess) return e;
@@ -539,14 +530,14 @@ cudaError_t plan_csel_uncached(int form, int src, int agg, int B, int Hkv, int T
 
 }  // namespace
 
-cudaError_t plan_csel(int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p) {
+cudaError_t plan_csel(int form, int src, int agg, int B, int Hkv, int T_cap, int r, int nq, int k, CSelPlan *p) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     CSelKey key;
     memset(&key, 0, sizeof key);
     key.dev = dev;
-    key.form = select_form_override();
+    key.form = form;
     key.src = src;
     key.agg = agg;
     key.B = B;
@@ -563,8 +554,7 @@ cudaError_t plan_csel(int src, int agg, int B, int Hkv, int T_cap, int r, int nq
                     // the attributes are per device and function: set them again
                     // in case this thread planned nothing on the device yet
                     auto kern = pick_csel(src, r, agg);
-                    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)g_cache[i].plan.smem);
+                    ensure_smem(reinterpret_cast<const void *>(kern), g_cache[i].plan.smem);
                     cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
                     *p = g_cache[i].plan;
                 }
@@ -609,6 +599,10 @@ cudaError_t launch_csel(const CSelPlan &p, const CSelArgs &a0, int src, int agg,
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
+    {
+        cudaError_t es = ensure_smem(reinterpret_cast<const void *>(kern), cfg.dynamicSmemBytes);
+        if (es != cudaSuccess) return es;
+    }
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 

@@ -644,20 +644,6 @@ __device__ void sel_sort(int32_t *a, int n, int st) {
     }
 }
 
-// Bounded wait that also gives up when another role raised the abort flag.
-// The thread is parked in the hardware between polls (up to 20 us per poll),
-// so waiting warps do not take issue slots from the working ones.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 0; it < (1u << 20); ++it) {
-        if (mbar_try_wait_for(bar, parity, 20000u)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > 2000000000ull) return false;
-    }
-    return false;
-}
-
 // Tile cursor over a CTA's range: (b,h) row and tile index within the row of
 // the current tile, advanced without divisions.  An epoch ends after E tiles
 // of one segment, at a segment end, or at the end of the range; consumers and
@@ -737,17 +723,8 @@ __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long l
             valid = true;
             m = a.k;
         }
-        if (S.st == 0) {
-            volatile unsigned *pub = a.counters + BH + bh;
-            const uint64_t t0 = global_timer_ns();
-            while (*pub < (unsigned)(nseg - 1)) {
-                if (global_timer_ns() - t0 > 2000000000ull) {
-                    if (a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
+        if (S.st == 0 && !flag_wait_bounded(a.counters + BH + bh, (unsigned)(nseg - 1)) && a.status)
+            atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
     }
     __threadfence();
     sel_sync();
@@ -1662,7 +1639,7 @@ cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T
     if (ns < 3) return cudaErrorNotSupported;
     P.nstages = ns;
     P.smem = stream_smem(ns, ept, P.cap, k, fused_r).total;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P.smem);
+    e = ensure_smem(reinterpret_cast<const void *>(kern), P.smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, P.smem);

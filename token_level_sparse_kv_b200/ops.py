@@ -72,6 +72,8 @@ def lib():
     L.jssa_decode_step_ex.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.jssa_plan_info.restype = i32
     L.jssa_plan_info.argtypes = [D, i32, i32, i32, ctypes.POINTER(i32), ctypes.c_char_p, sz]
+    L.jssa_plan_info_ex.restype = i32
+    L.jssa_plan_info_ex.argtypes = [D, i32, i32, i32, vp, ctypes.POINTER(i32), ctypes.c_char_p, sz]
     L.jssa_workspace_init.restype = i32
     L.jssa_workspace_init.argtypes = [vp, sz, vp]
     L.jssa_append_lowrank.restype = i32
@@ -139,22 +141,30 @@ def make_dims(q, K, V, P=None, Kt=None, r=None):
     return Dims(B, Hq, Hkv, d, dv, r, T_cap, _dt(K), kt)
 
 
+FORMS = {"auto": 0, "cluster": 1, "stream": 2, "scan": 3}
+
+
 class SelectOpts(ctypes.Structure):
-    """jssa_select_opts: tokens [0, n_sink) and [T_b - n_recent, T_b) are always selected."""
-    _fields_ = [("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32)]
+    """jssa_select_opts: tokens [0, n_sink) and [T_b - n_recent, T_b) are always
+    selected; form forces a selection form; unfused keeps the decode step in
+    separate launches."""
+    _fields_ = [("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32), ("form", ctypes.c_int32),
+                ("unfused", ctypes.c_int32)]
 
 
-def _opts(n_sink, n_recent):
-    if not n_sink and not n_recent:
+def _opts(n_sink=0, n_recent=0, form="auto", unfused=False):
+    f = FORMS[form] if isinstance(form, str) else int(form)
+    if not n_sink and not n_recent and not f and not unfused:
         return None
-    return ctypes.byref(SelectOpts(int(n_sink), int(n_recent)))
+    return ctypes.byref(SelectOpts(int(n_sink), int(n_recent), f, 1 if unfused else 0))
 
 
-def plan_info(dims: Dims, k: int, op: int, agg: int = 0):
+def plan_info(dims: Dims, k: int, op: int, agg: int = 0, form="auto", unfused=False):
     """(kernel launches per call, description of the forms chosen) for op."""
     n = ctypes.c_int32(0)
     buf = ctypes.create_string_buffer(160)
-    _check(lib().jssa_plan_info(ctypes.byref(dims), int(k), int(op), int(agg), ctypes.byref(n), buf, 160))
+    _check(lib().jssa_plan_info_ex(ctypes.byref(dims), int(k), int(op), int(agg), _opts(0, 0, form, unfused),
+                                   ctypes.byref(n), buf, 160))
     return int(n.value), buf.value.decode()
 
 
@@ -219,23 +229,25 @@ def score(q, P, Kt, seq_lens, agg=AGG_SUM, scores=None, ws=None):
     return scores
 
 
-def topk(scores, seq_lens, k, Hq=None, d=128, ws=None, n_sink=0, n_recent=0):
+def topk(scores, seq_lens, k, Hq=None, d=128, ws=None, n_sink=0, n_recent=0, form="auto"):
     """Per-(b,h) top-k of a score array: (idx [B,Hkv,k], count [B,Hkv]).
-    n_sink / n_recent: always-selected first / last tokens (jssa_select_opts)."""
+    n_sink / n_recent: always-selected first / last tokens; form: the selection
+    form ("auto", "cluster", "stream", "scan"; jssa_select_opts)."""
     _cuda(scores, seq_lens)
     B, Hkv, T_cap = scores.shape
     dims = Dims(B, Hq or Hkv, Hkv, d, 512 if d == 576 else d, 8, T_cap, BF16, BF16)
     idx = torch.empty((B, Hkv, k), dtype=torch.int32, device=scores.device)
     cnt = torch.empty((B, Hkv), dtype=torch.int32, device=scores.device)
     ws = _ws(ws, dims, k, OP_TOPK, scores.device)
-    _check(lib().jssa_topk_ex(ctypes.byref(dims), _p(scores), _p(seq_lens), int(k), _opts(n_sink, n_recent), _p(idx),
-                              _p(cnt), _p(ws), ws.numel(), _stream(scores.device)))
+    _check(lib().jssa_topk_ex(ctypes.byref(dims), _p(scores), _p(seq_lens), int(k), _opts(n_sink, n_recent, form),
+                              _p(idx), _p(cnt), _p(ws), ws.numel(), _stream(scores.device)))
     return idx, cnt
 
 
-def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_sink=0, n_recent=0):
+def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_sink=0, n_recent=0, form="auto"):
     """Fused score + top-k: (idx [B,Hkv,k], count [B,Hkv]).
-    n_sink / n_recent: always-selected first / last tokens (jssa_select_opts)."""
+    n_sink / n_recent: always-selected first / last tokens; form: the selection
+    form (jssa_select_opts)."""
     _cuda(q, P, Kt, seq_lens)
     B, Hq, d = q.shape
     _, Hkv, T_cap, r = Kt.shape
@@ -246,7 +258,8 @@ def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_
         count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     ws = _ws(ws, dims, k, OP_SELECT, q.device)
     _check(lib().jssa_select_ex(ctypes.byref(dims), _p(q), _p(P), _p(Kt), _p(seq_lens), int(agg), int(k),
-                                _opts(n_sink, n_recent), _p(idx), _p(count), _p(ws), ws.numel(), _stream(q.device)))
+                                _opts(n_sink, n_recent, form), _p(idx), _p(count), _p(ws), ws.numel(),
+                                _stream(q.device)))
     return idx, count
 
 
@@ -305,9 +318,10 @@ def gather_then_dense(q, K, V, idx, count, seq_lens, scale, gather_buf=None, ws=
 
 
 def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=None, idx=None, count=None,
-                out=None, lse=None, n_sink=0, n_recent=0):
+                out=None, lse=None, n_sink=0, n_recent=0, form="auto", unfused=False):
     """Append the row at pos_begin, select, indexed decode: (out, lse, idx, count).
-    n_sink / n_recent: always-selected first / last tokens (jssa_select_opts)."""
+    n_sink / n_recent: always-selected first / last tokens; form: the selection
+    form; unfused: keep the step in separate launches (jssa_select_opts)."""
     _cuda(q, K, V, P, Kt, seq_lens, pos_begin, idx, count, out, lse)
     dims = make_dims(q, K, V, P=P, Kt=Kt)
     B, Hkv = dims.B, dims.Hkv
@@ -322,8 +336,8 @@ def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=N
     ws = _ws(ws, dims, k, OP_DECODE_STEP, q.device)
     _check(lib().jssa_decode_step_ex(ctypes.byref(dims), _p(q), _p(K), _p(K if V is None else V), _p(P), _p(Kt),
                                      _p(seq_lens), _p(pos_begin), int(k), int(agg), float(scale),
-                                     _opts(n_sink, n_recent), _p(idx), _p(count), _p(out), _p(lse), _p(ws), ws.numel(),
-                                     _stream(q.device)))
+                                     _opts(n_sink, n_recent, form, unfused), _p(idx), _p(count), _p(out), _p(lse),
+                                     _p(ws), ws.numel(), _stream(q.device)))
     return out, lse, idx, count
 
 
