@@ -225,6 +225,19 @@ def test_dense_decode_parity(window, dtype):
     check_attention(out, lse, ref_o, ref_l, dtype)
 
 
+@pytest.mark.parametrize("d,G,window", [(64, 1, 0), (128, 16, 0), (256, 2, 300), (64, 8, 64), (128, 3, 0)])
+def test_dense_decode_shapes_and_ragged_rows(d, G, window):
+    """The tensor-core dense pass over every head width, group sizes 1..16,
+    windows shorter and longer than a tile, and rows of 0, 1, 63, 65 and a
+    few thousand tokens (tile edges and empty rows)."""
+    w = W(B=5, d=d, Hq=2 * G, Hkv=2, T=2100, r=8, seed=34 + d + G)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[2100, 0, 1, 63, 65])
+    out, lse = ops.dense_decode(qd, Kd, Vd, sld, w.scale, window=window)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.dense(q, K, V, sl, w.scale, window=window)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
 def test_dense_decode_long_many_splits():
     w = W(B=1, T=70000, Hq=16, Hkv=2, d=256, r=8, seed=31)
     (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)

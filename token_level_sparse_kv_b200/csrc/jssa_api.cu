@@ -148,6 +148,8 @@ struct Layout {
     bool fused = false;  // decode step in one launch of the streaming kernel
     ScanPlan fp{};
     CSelPlan cp{};
+    bool tc = false;     // dense pass on the tensor cores (bf16)
+    DensePlan dp{};
 };
 
 size_t take(size_t &off, size_t bytes) {
@@ -211,6 +213,18 @@ int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout
         L.part_ml = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * 2 * 4);
         L.att_ctr = take(L.total, (size_t)sh.BH * 4);
         return JSSA_OK;
+    }
+    if (src != ATT_INDEXED && d->kv_dtype == JSSA_BF16) {
+        cudaError_t e = plan_dense(d->d, d->B, d->Hkv, npos, &L.dp);
+        if (e == cudaSuccess) {
+            L.tc = true;
+            L.part_o = take(L.total, (size_t)sh.BH * L.dp.part_stride * sh.G * d->dv * 4);
+            L.part_ml = take(L.total, (size_t)sh.BH * L.dp.part_stride * sh.G * 2 * 4);
+            L.att_ctr = take(L.total, (size_t)sh.BH * 4);
+            return JSSA_OK;
+        }
+        cudaGetLastError();
+        if (e != cudaErrorNotSupported) return cuda_fail(e, "planning the dense pass");
     }
     cudaError_t e = plan_attend(src, d->kv_dtype, d->d, sh.G, d->B, d->Hkv, npos, &L.ap);
     if (e != cudaSuccess) return cuda_fail(e, "planning the attention pass");
@@ -384,6 +398,25 @@ void fill_attn(AttnArgs &a, const jssa_dims *d, const Shape &sh, const void *q, 
     a.v_sb = (long long)d->T_cap * d->Hkv * d->dv;
     a.v_st = (long long)d->Hkv * d->dv;
     a.v_sh = d->dv;
+    a.seq_lens = seq_lens;
+    a.B = d->B;
+    a.Hq = d->Hq;
+    a.Hkv = d->Hkv;
+    a.G = sh.G;
+    a.T_cap = d->T_cap;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.part_o = at<float>(ws, L.part_o);
+    a.part_ml = at<float>(ws, L.part_ml);
+    a.counters = at<uint32_t>(ws, L.att_ctr);
+    a.out = out;
+    a.lse = lse;
+    a.status = at<uint32_t>(ws, 0);
+}
+
+void fill_dense(DenseArgs &a, const jssa_dims *d, const Shape &sh, const void *q, const int32_t *seq_lens,
+                float scale, void *out, float *lse, void *ws, const Layout &L) {
+    memset(&a, 0, sizeof a);
+    a.q = q;
     a.seq_lens = seq_lens;
     a.B = d->B;
     a.Hq = d->Hq;
@@ -745,6 +778,14 @@ int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const
     if ((st = build_layout(dims, sh, 1, JSSA_OP_DENSE_DECODE, 0, window, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
+    if (L.tc) {
+        DenseArgs da;
+        fill_dense(da, dims, sh, q, seq_lens, softmax_scale, out, lse, ws, L);
+        da.window = window;
+        cudaError_t e = launch_dense(L.dp, da, K, V, dims->d, S(stream), true);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the dense decode");
+        return JSSA_OK;
+    }
     AttnArgs a;
     fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);
     a.window = window;
@@ -785,6 +826,15 @@ int jssa_gather_then_dense(const jssa_dims *dims, const void *q, const void *K, 
                  dims->B, dims->Hkv, dims->T_cap, dims->d, k};
     cudaError_t e = launch_gather(g, dims->kv_dtype, S(stream), true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the gather");
+    if (L.tc) {
+        DenseArgs da;
+        fill_dense(da, dims, sh, q, seq_lens, softmax_scale, out, lse, ws, L);
+        da.count = at<int32_t>(ws, L.gcount);
+        da.k = k;
+        e = launch_dense(L.dp, da, gK, gV, dims->d, S(stream), true);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the dense decode over gathered rows");
+        return JSSA_OK;
+    }
     AttnArgs a;
     fill_attn(a, dims, sh, q, gK, gV, seq_lens, softmax_scale, out, lse, ws, L);
     a.k_sb = a.v_sb = (long long)dims->Hkv * k * dims->d;

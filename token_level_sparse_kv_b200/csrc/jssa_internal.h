@@ -109,6 +109,37 @@ struct GatherArgs {
     int B, Hkv, T_cap, d, k;
 };
 
+// ----------------------------------------------------- dense (tensor core) ---
+// Dense attention of bf16 rows over a contiguous token range per (b, h): the
+// cache ([B, T_cap, Hkv, d], rows [max(0, T_b - window), T_b) or [0, T_b))
+// or a gathered buffer ([B*Hkv, k, d], rows [0, count[bh])).
+struct DenseArgs {
+    const void *q;            // [B, Hq, d] bf16
+    const int32_t *seq_lens;  // [B]
+    const int32_t *count;     // gathered source: rows per (b,h); null for the cache
+    int B, Hq, Hkv, G, T_cap, window, k;
+    int row_tiles;            // plan: 64-token tiles per row
+    long long total_tiles;    // plan: rows * row_tiles
+    int grid, part_stride;    // plan: persistent CTAs; partial slots per row
+    float scale_log2;         // softmax_scale * log2(e)
+    float *part_o;            // [BH, part_stride, G, d]
+    float *part_ml;           // [BH, part_stride, G, 2]
+    uint32_t *counters;       // [BH] arrival tickets (self-resetting)
+    void *out;                // [B, Hq, d] bf16
+    float *lse;               // [B, Hq] or null
+    uint32_t *status;
+};
+struct DensePlan {
+    int row_tiles, grid, part_stride;
+    long long total_tiles;
+    size_t smem;
+};
+int dense_part_stride(int B, int Hkv);
+// cudaErrorNotSupported where it has no kernel (d outside {64, 128, 256}).
+cudaError_t plan_dense(int d, int B, int Hkv, int row_len, DensePlan *p);
+cudaError_t launch_dense(const DensePlan &p, const DenseArgs &a, const void *K, const void *V, int d,
+                         cudaStream_t s, bool pdl);
+
 // --------------------------------------------------------- cluster select ---
 // Top-k of one (b,h) by a cluster of CTAs holding the keys in shared memory.
 struct CSelArgs {
