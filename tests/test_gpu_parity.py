@@ -389,6 +389,43 @@ def test_device_status_flags_bad_data_without_fault():
     assert torch.equal(Kt[1], before[1])
 
 
+def test_rows_past_the_range_do_not_leak():
+    """Cache rows past T_b and gather-buffer rows past the count are not part
+    of the attention and may hold anything (an unwritten KV slot): NaN planted
+    there must not reach any output (dense, gathered, latent dense, latent
+    gathered)."""
+    w = W(B=2, T=700, k=128, seed=58)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[650, 100])
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    for b, tb in enumerate((650, 100)):
+        Kd[b, tb:] = float("nan")
+        Vd[b, tb:] = float("nan")
+    dims = ops.make_dims(qd, Kd, Vd, r=8)
+    gbuf = torch.full((ops.gather_buffer_bytes(dims, w.k) // 2,), float("nan"), dtype=torch.bfloat16, device=DEV)
+    do, dl = ops.dense_decode(qd, Kd, Vd, sld, w.scale)
+    go, gl = ops.gather_then_dense(qd, Kd, Vd, idx, cnt, sld, w.scale, gather_buf=gbuf.view(torch.uint8))
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.dense(q, K, V, sl, w.scale)
+    check_attention(do, dl, ref_o, ref_l, torch.bfloat16)
+    ref_o, ref_l = oracle.attend(q, K, V, host(idx), host(cnt), sl, w.scale)
+    check_attention(go, gl, ref_o, ref_l, torch.bfloat16)
+    m = MW(T=900, k=512, seed=59)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(m, seq_lens=[900, 300])
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, m.k)
+    Kd[1, 300:] = float("nan")
+    dims = ops.make_dims(qd, Kd, None, r=8)
+    gbuf = torch.full((ops.gather_buffer_bytes(dims, m.k) // 2,), float("nan"), dtype=torch.bfloat16, device=DEV)
+    do, dl = ops.dense_decode(qd, Kd, None, sld, m.scale)
+    go, gl = ops.gather_then_dense(qd, Kd, None, idx, cnt, sld, m.scale, gather_buf=gbuf.view(torch.uint8))
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.dense(q, K, None, sl, m.scale, dv=512, v_aliases_k=True)
+    check_attention(do, dl, ref_o, ref_l, torch.bfloat16)
+    ref_o, ref_l = oracle.attend(q, K, None, host(idx), host(cnt), sl, m.scale, dv=512, v_aliases_k=True)
+    check_attention(go, gl, ref_o, ref_l, torch.bfloat16)
+
+
 def test_invalid_arguments_raise():
     w = W(B=1, Hq=64, Hkv=2, T=100, k=8, seed=52)
     (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
@@ -553,6 +590,49 @@ def test_mla_indexed_decode_parity(k, sl):
     check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
 
 
+@pytest.mark.parametrize("T,sl", [(3000, [3000, 77]), (700, [129, 0]), (5000, [4097, 128])])
+def test_mla_dense_decode_parity(T, sl):
+    """Full-KV attention over the latent cache (the dense comparison path of
+    the latent-cache workload): ragged rows, an empty row, tile edges."""
+    w = MW(T=T, seed=63 + T)
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    out, lse = ops.dense_decode(qd, Kd, None, sld, w.scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.dense(q, K, None, slh, w.scale, dv=512, v_aliases_k=True)
+    check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
+
+
+def test_mla_k_equal_T_equals_dense():
+    """The pages' special case for the latent cache: with k = T every token is
+    selected and the indexed decode equals dense latent attention."""
+    w = MW(T=1900, k=1900, seed=66)
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[1900, 1900])
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    o1, l1 = ops.indexed_decode(qd, Kd, None, idx, cnt, sld, w.scale)
+    o2, l2 = ops.dense_decode(qd, Kd, None, sld, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(idx.cpu(), torch.arange(1900, dtype=torch.int32).expand(2, 1, 1900))
+    torch.testing.assert_close(o1.float(), o2.float(), rtol=0, atol=2e-2)
+    torch.testing.assert_close(l1, l2, rtol=0, atol=1e-3)
+    ref_o, ref_l = oracle.dense(q, K, None, slh, w.scale, dv=512, v_aliases_k=True)
+    check_attention(o2, l2, ref_o, ref_l, torch.bfloat16)
+
+
+@pytest.mark.parametrize("k", [300, 2048])
+def test_mla_gather_then_dense_matches_indexed_and_oracle(k):
+    w = MW(T=4000, k=k, seed=67 + k)
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[4000, 250])
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    o1, l1 = ops.indexed_decode(qd, Kd, None, idx, cnt, sld, w.scale)
+    o2, l2 = ops.gather_then_dense(qd, Kd, None, idx, cnt, sld, w.scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attend(q, K, None, host(idx), host(cnt), slh, w.scale, dv=512, v_aliases_k=True)
+    check_attention(o1, l1, ref_o, ref_l, torch.bfloat16)
+    check_attention(o2, l2, ref_o, ref_l, torch.bfloat16)
+
+
 def test_mla_decode_step_end_to_end():
     w = MW(T=5000, k=512, kind="spiked", seed=70)
     (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[5000, 4321])
@@ -588,6 +668,13 @@ def test_full_size_mla_64k_b8_sampled():
         ref_o, ref_l = oracle.attend(qs, Ks, None, host(idx[b:b + 1]), host(cnt[b:b + 1]), slh, w.scale, dv=512,
                                      v_aliases_k=True)
         check_attention(out[b:b + 1], lse[b:b + 1], ref_o, ref_l, torch.bfloat16)
+    # the dense comparison path at full size, one batch row against the oracle
+    do, dl = ops.dense_decode(q, K, None, sl, w.scale)
+    torch.cuda.synchronize()
+    b = 3
+    ref_o, ref_l = oracle.dense(host(q[b:b + 1]), host(K[b:b + 1]), None, sl[b:b + 1].cpu(), w.scale, dv=512,
+                                v_aliases_k=True)
+    check_attention(do[b:b + 1], dl[b:b + 1], ref_o, ref_l, torch.bfloat16)
     del q, K, Kt, s
     torch.cuda.empty_cache()
 

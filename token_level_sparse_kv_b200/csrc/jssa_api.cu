@@ -113,11 +113,11 @@ int check_k(int k) {
     return JSSA_OK;
 }
 
-// Attention kernels exist for GQA (G <= 16, bf16 or fp32) and, for the indexed
-// path, for the latent cache with 128 heads in bf16.
+// Attention kernels exist for GQA (G <= 16, bf16 or fp32) and for the latent
+// cache with 128 heads in bf16.
 int check_attn_shape(const jssa_dims *d, const Shape &sh, bool indexed) {
+    (void)indexed;
     if (sh.latent) {
-        if (!indexed) return fail(JSSA_ERR_UNSUPPORTED, "dense / gathered latent-cache attention has no kernel in this build");
         if (d->Hq != 128 || d->kv_dtype != JSSA_BF16)
             return fail(JSSA_ERR_UNSUPPORTED, "latent-cache attention needs Hq = 128 and bf16 (got Hq=%d)", d->Hq);
         return JSSA_OK;
@@ -150,6 +150,7 @@ struct Layout {
     CSelPlan cp{};
     bool tc = false;     // dense pass on the tensor cores (bf16)
     DensePlan dp{};
+    MlaRangePlan mp{};   // latent cache, dense or gathered rows
 };
 
 size_t take(size_t &off, size_t bytes) {
@@ -206,6 +207,14 @@ int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, 
 }
 
 int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout &L) {
+    if (sh.latent && src != ATT_INDEXED) {
+        cudaError_t e = plan_mla_range(d->B, npos, &L.mp);
+        if (e != cudaSuccess) return cuda_fail(e, "planning the latent-cache range pass");
+        L.part_o = take(L.total, (size_t)d->B * L.mp.splits * d->Hq * d->dv * 4);
+        L.part_ml = take(L.total, (size_t)d->B * L.mp.splits * d->Hq * 2 * 4);
+        L.att_ctr = take(L.total, (size_t)sh.BH * 4);
+        return JSSA_OK;
+    }
     if (sh.latent) {
         L.ap = AttnPlan();
         L.ap.splits = mla_splits(npos);
@@ -490,6 +499,27 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
     return JSSA_OK;
 }
 
+int run_mla_range(const jssa_dims *d, const void *q, const void *K, const int32_t *seq_lens, const int32_t *count,
+                  int k, float scale, void *out, float *lse, void *ws, const Layout &L, cudaStream_t s) {
+    MlaRangeArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q;
+    a.seq_lens = seq_lens;
+    a.count = count;
+    a.B = d->B;
+    a.T_cap = d->T_cap;
+    a.k = k;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.part_o = at<float>(ws, L.part_o);
+    a.part_ml = at<float>(ws, L.part_ml);
+    a.out = out;
+    a.lse = lse;
+    a.status = at<uint32_t>(ws, 0);
+    cudaError_t e = launch_mla_range(L.mp, a, K, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the latent-cache range pass");
+    return JSSA_OK;
+}
+
 int run_mla(const jssa_dims *d, const void *q, const void *K, const int32_t *idx, const int32_t *count, int k,
             const int32_t *seq_lens, float scale, void *out, float *lse, void *ws, const Layout &L, cudaStream_t s) {
     MlaArgs a;
@@ -768,6 +798,8 @@ int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const
     if (st) return st;
     if ((st = check_attn_shape(dims, sh, false))) return st;
     if (window < 0) return fail(JSSA_ERR_INVALID_ARG, "window=%d is negative", window);
+    if (sh.latent && window > 0 && window < dims->T_cap)
+        return fail(JSSA_ERR_UNSUPPORTED, "sliding-window attention over a latent cache has no kernel in this build");
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
     REQUIRE_PTR(V);
@@ -778,6 +810,8 @@ int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const
     if ((st = build_layout(dims, sh, 1, JSSA_OP_DENSE_DECODE, 0, window, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
+    if (sh.latent)
+        return run_mla_range(dims, q, K, seq_lens, nullptr, 0, softmax_scale, out, lse, ws, L, S(stream));
     if (L.tc) {
         DenseArgs da;
         fill_dense(da, dims, sh, q, seq_lens, softmax_scale, out, lse, ws, L);
@@ -813,19 +847,23 @@ int jssa_gather_then_dense(const jssa_dims *dims, const void *q, const void *K, 
     OPTIONAL_PTR(count);
     OPTIONAL_PTR(lse);
     const size_t half = (size_t)sh.BH * k * dims->d * sh.es_kv;
-    if (gather_bytes < 2 * half)
+    const size_t need = sh.latent ? half : 2 * half;  // a latent row is its own value
+    if (gather_bytes < need)
         return fail(JSSA_ERR_INVALID_ARG, "gather_buf of %zu bytes is below the %zu bytes needed", gather_bytes,
-                    2 * half);
+                    need);
     Layout L;
     if ((st = build_layout(dims, sh, k, JSSA_OP_GATHER_THEN_DENSE, 0, 0, Choice(), L))) return st;
     if ((st = check_ws(ws, ws_bytes, L))) return st;
     if (dims->B == 0) return JSSA_OK;
     void *gK = gather_buf;
-    void *gV = static_cast<char *>(gather_buf) + half;
-    GatherArgs g{K, V, idx, count, seq_lens, gK, gV, at<int32_t>(ws, L.gcount), at<uint32_t>(ws, 0),
-                 dims->B, dims->Hkv, dims->T_cap, dims->d, k};
+    void *gV = sh.latent ? nullptr : static_cast<char *>(gather_buf) + half;
+    GatherArgs g{K, sh.latent ? nullptr : V, idx, count, seq_lens, gK, gV, at<int32_t>(ws, L.gcount),
+                 at<uint32_t>(ws, 0), dims->B, dims->Hkv, dims->T_cap, dims->d, k};
     cudaError_t e = launch_gather(g, dims->kv_dtype, S(stream), true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the gather");
+    if (sh.latent)
+        return run_mla_range(dims, q, gK, seq_lens, at<int32_t>(ws, L.gcount), k, softmax_scale, out, lse, ws, L,
+                             S(stream));
     if (L.tc) {
         DenseArgs da;
         fill_dense(da, dims, sh, q, seq_lens, softmax_scale, out, lse, ws, L);

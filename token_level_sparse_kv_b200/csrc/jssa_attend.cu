@@ -443,7 +443,8 @@ __global__ void __launch_bounds__(NTH) gather_kernel(GatherArgs a) {
     const uint4 *V = static_cast<const uint4 *>(a.V);
     uint4 *gK = static_cast<uint4 *>(a.gK);
     uint4 *gV = static_cast<uint4 *>(a.gV);
-    for (int p = tid; p < (r1 - r0) * cpr * 2; p += NTH) {
+    const int copies = a.V ? 2 : 1;  // a latent cache gathers its rows once (V is K)
+    for (int p = tid; p < (r1 - r0) * cpr * copies; p += NTH) {
         const int kv = p >= (r1 - r0) * cpr;
         const int rem = p - kv * (r1 - r0) * cpr;
         const int rr = r0 + rem / cpr, ch = rem % cpr;

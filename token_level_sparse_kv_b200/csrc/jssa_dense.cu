@@ -65,6 +65,7 @@ constexpr size_t dense_smem_bytes() {
     return o + 1024;                          // alignment slack of the dynamic base
 }
 
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kNW * 32) : "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
@@ -298,6 +299,19 @@ __global__ void __launch_bounds__(kThr, 1)
             const uint32_t pa3 = pack_bf16(p[1][2], p[1][3], rs1);
             lrun[0] = lrun[0] * corr[0] + rs0;
             lrun[1] = lrun[1] * corr[1] + rs1;
+            // V rows past the row's end (the tail of its last tile) may hold
+            // anything, NaN included, and 0 * NaN is NaN: zero them first
+            if (tw + 16 > hi) {
+                unsigned char *vg = ring + (size_t)s * S::STAGE + (size_t)NB * kBoxBytes;
+                const int r0 = max(hi - t0, warp * 16), nrow = warp * 16 + 16 - r0;
+                for (int c = lane; c < nrow * NB * 8; c += 32) {
+                    const int row = r0 + c / (NB * 8), rem = c % (NB * 8);
+                    *reinterpret_cast<uint4 *>(vg + (rem >> 3) * kBoxBytes + row * 128 + (rem & 7) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_async_smem();  // before the stage is refilled by TMA
+                __syncwarp();
+            }
             // O = O * corr + P V (two 8-dim output tiles per ldmatrix)
             const int r = warp * 16 + (lane & 15);
             const int second = lane >> 4;
@@ -323,7 +337,6 @@ __global__ void __launch_bounds__(kThr, 1)
         const bool seg_end = (j == rt - 1) || (i == i1 - 1);
         if (seg_end) {
             // this warp's partial of the row: unnormalised O, max, sum
-            const int BH = a.B * a.Hkv;
             const long long first = (long long)bh * rt;
             const int c_first = (int)(((first + 1) * a.grid - 1) / total);
             const int c_last = (int)(((first + rt) * a.grid - 1) / total);
@@ -412,13 +425,21 @@ DenseKernel pick_dense(int d, size_t *smem) {
     }
 }
 
-// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time
-// dependency on the driver library).
+// Map over bf16 rows of d elements: boxes of 64 columns x 64 rows; rank 4
+// {d, Hkv, T, B} over the cache, rank 3 {d, k, B*Hkv} over a gathered buffer.
+cudaError_t encode_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides) {
+    cuuint32_t box[4] = {64, 1, 1, 1};
+    box[rank == 4 ? 2 : 1] = kNT;
+    return encode_tiled_bf16(m, base, rank, dims, strides, box);
+}
+
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
     if (!tried) {
@@ -434,22 +455,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Map over bf16 rows of d elements: boxes of 64 columns x 64 rows (128-byte
-// swizzle); rank 4 {d, Hkv, T, B} over the cache, rank 3 {d, k, B*Hkv} over
-// a gathered buffer.
-cudaError_t encode_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides) {
+bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+cudaError_t encode_tiled_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                              const cuuint64_t *strides, const cuuint32_t *box) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    cuuint32_t box[4] = {64, 1, 1, 1};
-    cuuint32_t es[4] = {1, 1, 1, 1};
-    box[rank == 4 ? 2 : 1] = kNT;
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
-
-}  // namespace
 
 int dense_part_stride(int B, int Hkv) {
     // partial slots per row: a row spans at most ceil(grid / rows) + 1 CTAs
@@ -463,7 +480,7 @@ cudaError_t plan_dense(int d, int B, int Hkv, int row_len, DensePlan *p) {
     size_t smem = 0;
     DenseKernel k = pick_dense(d, &smem);
     if (!k) return cudaErrorNotSupported;
-    if (!encode_fn()) return cudaErrorNotSupported;
+    if (!tensor_maps_available()) return cudaErrorNotSupported;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(k), smem);
     if (e != cudaSuccess) return e;
     int occ = 0;

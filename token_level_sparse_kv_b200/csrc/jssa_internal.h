@@ -2,6 +2,7 @@
 // by the translation units of libjssa.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -103,7 +104,7 @@ struct GatherArgs {
     const int32_t *count;
     const int32_t *seq_lens;
     void *gK;  // [B, Hkv, k, d]
-    void *gV;
+    void *gV;  // null with V null (latent cache: the rows are gathered once)
     int32_t *gcount;  // [BH] rows actually gathered
     uint32_t *status;
     int B, Hkv, T_cap, d, k;
@@ -139,6 +140,29 @@ int dense_part_stride(int B, int Hkv);
 cudaError_t plan_dense(int d, int B, int Hkv, int row_len, DensePlan *p);
 cudaError_t launch_dense(const DensePlan &p, const DenseArgs &a, const void *K, const void *V, int d,
                          cudaStream_t s, bool pdl);
+
+// ------------------------------------------- latent cache, token range ---
+// Attention of the 128 heads of a latent cache over [0, T_b) of the cache
+// ([B, T_cap, 1, 576]) or [0, count[b]) of a gathered buffer ([B, k, 576]).
+struct MlaRangeArgs {
+    const void *q;            // [B, 128, 576] bf16
+    const int32_t *seq_lens;  // [B]
+    const int32_t *count;     // gathered source: rows per batch row; null for the cache
+    int B, T_cap, k;
+    int row_tiles, splits;    // plan: 128-token tiles per row; CTAs (x 2 head halves) per row
+    float scale_log2;
+    float *part_o;            // [B, splits, 128, 512]
+    float *part_ml;           // [B, splits, 128, 2]
+    void *out;                // [B, 128, 512] bf16
+    float *lse;               // [B, 128] or null
+    uint32_t *status;
+};
+struct MlaRangePlan {
+    int row_tiles, splits;
+    size_t smem;
+};
+cudaError_t plan_mla_range(int B, int row_len, MlaRangePlan *p);
+cudaError_t launch_mla_range(const MlaRangePlan &p, const MlaRangeArgs &a, const void *K, cudaStream_t s, bool pdl);
 
 // --------------------------------------------------------- cluster select ---
 // Top-k of one (b,h) by a cluster of CTAs holding the keys in shared memory.
@@ -181,8 +205,18 @@ struct MlaArgs {
 };
 int mla_splits(int npos);
 cudaError_t launch_mla(const MlaArgs &a, bool indexed, cudaStream_t s, bool pdl);
+// Log-sum-exp merge of a.splits latent-cache partials into out / lse.
+cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t s, bool pdl);
 
 // --------------------------------------------------------------- helpers ---
+// A TMA tensor map over bf16 data (cuTensorMapEncodeTiled, looked up once
+// through the runtime: no link-time dependency on the driver library): rank
+// dims (innermost first), rank-1 byte strides, box extents; 128-byte
+// swizzle, 256-byte L2 promotion, zero fill outside the tensor.
+// cudaErrorNotSupported when the driver offers no encoder.
+cudaError_t encode_tiled_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                              const cuuint64_t *strides, const cuuint32_t *box);
+bool tensor_maps_available();
 int device_sm_count();
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device
 // (launch paths call it on every launch; the runtime call is made only when

@@ -22,6 +22,7 @@
 // log-sum-exp.
 #include "jssa_common.cuh"
 #include "jssa_internal.h"
+#include "jssa_tc.cuh"
 
 namespace jssa {
 
@@ -35,48 +36,6 @@ constexpr size_t kSmemK = (size_t)kKB * kBlk;
 constexpr size_t kSmemQ = (size_t)kQBuf * kBlk;
 constexpr size_t kSmemMisc = 2048;
 constexpr size_t kSmemBytes = kSmemK + kSmemQ + kSmemMisc;
-
-// Shared-memory matrix descriptor of a 128-byte-swizzled canonical layout
-// (start address, leading / stride byte offsets, descriptor version 1 for
-// this architecture, swizzle mode 128B).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor: bf16 x bf16 -> fp32, M x N, operand majorness.
-__host__ __device__ constexpr uint32_t mma_idesc(int M, int N, int a_mn, int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// 32 consecutive fp32 columns of this warp's 32 TMEM lanes.
-__device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(addr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-}
 
 template <int N>
 __device__ __forceinline__ void cp_wait_dyn(int n) {
@@ -407,6 +366,10 @@ cudaError_t launch_mla(const MlaArgs &a0, bool indexed, cudaStream_t s, bool pdl
     if (e != cudaSuccess) return e;
     e = launch_kernel(k, dim3(a.splits, a.B), dim3(kThr), kSmemBytes, s, pdl, a);
     if (e != cudaSuccess || a.splits == 1) return e;
+    return launch_mla_combine(a, s, pdl);
+}
+
+cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t s, bool pdl) {
     return launch_kernel(mla_combine_kernel, dim3(a.B, kH / 4), dim3(128), 0, s, pdl, a);
 }
 

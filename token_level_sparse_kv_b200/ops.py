@@ -295,7 +295,10 @@ def dense_decode(q, K, V, seq_lens, scale, window=0, ws=None, out=None, lse=None
 
 
 def gather_buffer_bytes(dims: Dims, k: int) -> int:
-    return 2 * dims.B * dims.Hkv * k * dims.d * (2 if dims.kv_dtype == BF16 else 4)
+    """Bytes of the gather-then-dense buffer: K and V rows, or the latent rows
+    once for a latent cache (V is K)."""
+    copies = 1 if (dims.d == 576 and dims.dv == 512 and dims.Hkv == 1) else 2
+    return copies * dims.B * dims.Hkv * k * dims.d * (2 if dims.kv_dtype == BF16 else 4)
 
 
 def gather_then_dense(q, K, V, idx, count, seq_lens, scale, gather_buf=None, ws=None, out=None, lse=None):
