@@ -621,8 +621,22 @@ int jssa_plan_info_ex(const jssa_dims *dims, int k, int op, int agg, const jssa_
         case JSSA_OP_TOPK: n = 1; snprintf(text, sizeof text, "top-k (%s form)", sel); break;
         case JSSA_OP_SELECT: n = 2; snprintf(text, sizeof text, "projection + selection (%s form)", sel); break;
         case JSSA_OP_INDEXED_DECODE: n = att; snprintf(text, sizeof text, "indexed attention"); break;
-        case JSSA_OP_DENSE_DECODE: n = 1; snprintf(text, sizeof text, "dense attention"); break;
-        case JSSA_OP_GATHER_THEN_DENSE: n = 2; snprintf(text, sizeof text, "gather + dense attention"); break;
+        case JSSA_OP_DENSE_DECODE:
+        case JSSA_OP_GATHER_THEN_DENSE: {
+            const int g = op == JSSA_OP_GATHER_THEN_DENSE ? 1 : 0;
+            if (sh.latent) {
+                n = g + 1 + (L.mp.splits > 1 ? 1 : 0);
+                snprintf(text, sizeof text, "%slatent-cache range attention (tensor cores)%s", g ? "gather + " : "",
+                         L.mp.splits > 1 ? " + combine" : "");
+            } else if (L.tc) {
+                n = g + 2;
+                snprintf(text, sizeof text, "%sdense attention (tensor cores) + combine", g ? "gather + " : "");
+            } else {
+                n = g + 1;
+                snprintf(text, sizeof text, "%sdense attention", g ? "gather + " : "");
+            }
+            break;
+        }
         case JSSA_OP_DECODE_STEP:
             if (L.fused) {
                 n = 1;

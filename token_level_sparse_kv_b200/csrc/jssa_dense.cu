@@ -26,8 +26,11 @@
 //                   S accumulators as the A operand; ldmatrix.trans of V),
 //    with an online softmax in fp32 (log2 domain) per warp;
 //  * at the end of a row's segment each warp writes its unnormalised partial
-//    (O, running max, running sum) to the workspace; the last CTA of the row
-//    to arrive (ticket, no waiting) merges the partials by log-sum-exp.
+//    (O, running max, running sum) to the workspace; a second kernel, chained
+//    with programmatic dependent launch, merges each (row, head)'s partials
+//    by log-sum-exp with one thread per output dim (a short row, such as a
+//    1024-token window, is covered by up to ten CTAs: merging its 40
+//    partials inside one CTA was latency-bound).
 // Tiles past a row's end are skipped (no load); positions past it inside a
 // tile are masked.  The CTA's rows are independent, so nothing waits on
 // another CTA.
@@ -52,7 +55,6 @@ struct DenseShape {
     static constexpr int STAGE = 2 * NB * kBoxBytes;   // K and V of one tile
     static constexpr int STAGES = (int)(kStageBudget / STAGE) > 8 ? 8 : (int)(kStageBudget / STAGE);
     static constexpr int QSTR = D * 2 + 16;            // padded row of the query tile (bytes)
-    static constexpr int DPT = D >= 128 ? D / 128 : 1; // combine: output dims per consumer thread
 };
 
 template <int D>
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(kThr, 1)
     unsigned char *q_s = ring + (size_t)STAGES * S::STAGE;
     uint64_t *full = reinterpret_cast<uint64_t *>(q_s + 16 * QSTR);
     uint64_t *empty = full + STAGES;
-    volatile int *flags = reinterpret_cast<volatile int *>(empty + STAGES);  // [0] abort, [1] last-arrival
+    volatile int *flags = reinterpret_cast<volatile int *>(empty + STAGES);  // [0] abort
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long total = a.total_tiles;
@@ -152,7 +154,6 @@ __global__ void __launch_bounds__(kThr, 1)
         }
         fence_barrier_init();
         flags[0] = 0;
-        flags[1] = 0;
     }
     __syncthreads();
     pdl_trigger();
@@ -339,8 +340,7 @@ __global__ void __launch_bounds__(kThr, 1)
             // this warp's partial of the row: unnormalised O, max, sum
             const long long first = (long long)bh * rt;
             const int c_first = (int)(((first + 1) * a.grid - 1) / total);
-            const int c_last = (int)(((first + rt) * a.grid - 1) / total);
-            const int slot = (int)blockIdx.x - c_first, nseg = c_last - c_first + 1;
+            const int slot = (int)blockIdx.x - c_first;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 lrun[r] += __shfl_xor_sync(0xffffffffu, lrun[r], 1);
@@ -359,46 +359,6 @@ __global__ void __launch_bounds__(kThr, 1)
                         *reinterpret_cast<float2 *>(a.part_ml + (pidx * G + g) * 2) = make_float2(mrun[r], lrun[r]);
                 }
             }
-            __threadfence();
-            consumer_sync();
-            if (ctid == 0) flags[1] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
-            consumer_sync();
-            if (flags[1]) {
-                // the last segment of the row merges every partial by log-sum-exp
-                __threadfence();
-                const int np = nseg * kNW;
-                const size_t pb = (size_t)bh * parts_stride;
-                const int b = bh / a.Hkv, h = bh - b * a.Hkv;
-                __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * a.Hq + (size_t)h * G) * D;
-                for (int g = 0; g < G; ++g) {
-                    float M = -INFINITY;
-                    for (int q = 0; q < np; ++q) M = fmaxf(M, __ldcg(a.part_ml + ((pb + q) * G + g) * 2));
-                    float L = 0.f, acc[S::DPT];
-#pragma unroll
-                    for (int u = 0; u < S::DPT; ++u) acc[u] = 0.f;
-                    const int d0 = ctid * S::DPT;
-                    for (int q = 0; q < np; ++q) {
-                        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.part_ml + ((pb + q) * G + g) * 2));
-                        if (ml.x == -INFINITY) continue;
-                        const float wgt = exp2f(ml.x - M);
-                        L = fmaf(ml.y, wgt, L);
-                        if (d0 < D) {
-#pragma unroll
-                            for (int u = 0; u < S::DPT; ++u)
-                                acc[u] = fmaf(__ldcg(a.part_o + ((pb + q) * G + g) * D + d0 + u), wgt, acc[u]);
-                        }
-                    }
-                    const float inv = L > 0.f ? 1.f / L : 0.f;
-                    if (d0 < D) {
-#pragma unroll
-                        for (int u = 0; u < S::DPT; ++u) out[(size_t)g * D + d0 + u] = __float2bfloat16_rn(acc[u] * inv);
-                    }
-                    if (ctid == 0 && a.lse)
-                        a.lse[(size_t)b * a.Hq + (size_t)h * G + g] =
-                            L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-                }
-                if (ctid == 0) a.counters[bh] = 0u;
-            }
             if (i + 1 < i1) {
                 ++bh;
                 j = 0;
@@ -412,6 +372,56 @@ __global__ void __launch_bounds__(kThr, 1)
             ++j;
         }
     }
+}
+
+// Log-sum-exp merge of a row's partials (every segment of every CTA that
+// covered it, one partial per consumer warp; empty partials carry O = 0 and
+// max -inf): one CTA per (row, head), one thread per output dim.  Chained
+// after the dense kernel with programmatic dependent launch.
+template <int D>
+__global__ void __launch_bounds__(D) dense_combine_kernel(DenseArgs a) {
+    __shared__ float stat[2];
+    pdl_wait();
+    const int bh = blockIdx.x, g = blockIdx.y, d = threadIdx.x;
+    const int G = a.G, rt = a.row_tiles;
+    const long long total = a.total_tiles, first = (long long)bh * rt;
+    const int c_first = (int)(((first + 1) * a.grid - 1) / total);
+    const int c_last = (int)(((first + rt) * a.grid - 1) / total);
+    const int np = (c_last - c_first + 1) * kNW;
+    const size_t pb = (size_t)bh * a.part_stride;
+    if (d < 32) {
+        float M = -INFINITY;
+        for (int q = d; q < np; q += 32) M = fmaxf(M, __ldcg(a.part_ml + ((pb + q) * G + g) * 2));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float L = 0.f;
+        if (M != -INFINITY)
+            for (int q = d; q < np; q += 32) {
+                const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.part_ml + ((pb + q) * G + g) * 2));
+                L += ml.x == -INFINITY ? 0.f : ml.y * exp2f(ml.x - M);
+            }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        if (d == 0) {
+            stat[0] = M;
+            stat[1] = L;
+        }
+    }
+    __syncthreads();
+    const float M = stat[0], L = stat[1];
+    float acc = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 8
+        for (int q = 0; q < np; ++q) {
+            const float m = __ldcg(a.part_ml + ((pb + q) * G + g) * 2);
+            const float o = __ldcg(a.part_o + ((pb + q) * G + g) * D + d);
+            acc = fmaf(o, m == -INFINITY ? 0.f : exp2f(m - M), acc);
+        }
+    }
+    const int b = bh / a.Hkv, h = bh - b * a.Hkv;
+    const size_t row = (size_t)b * a.Hq + (size_t)h * G + g;
+    static_cast<__nv_bfloat16 *>(a.out)[row * D + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+    if (d == 0 && a.lse) a.lse[row] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
 using DenseKernel = void (*)(const CUtensorMap, const CUtensorMap, DenseArgs);
@@ -523,7 +533,11 @@ cudaError_t launch_dense(const DensePlan &p, const DenseArgs &a0, const void *K,
         if (e == cudaSuccess) e = encode_map(&mv, V, 4, dims, str);
     }
     if (e != cudaSuccess) return e;
-    return launch_kernel(k, dim3(p.grid), dim3(kThr), smem, s, pdl, mk, mv, a);
+    e = launch_kernel(k, dim3(p.grid), dim3(kThr), smem, s, pdl, mk, mv, a);
+    if (e != cudaSuccess) return e;
+    void (*c)(DenseArgs) = d == 64 ? dense_combine_kernel<64> : (d == 128 ? dense_combine_kernel<128>
+                                                                          : dense_combine_kernel<256>);
+    return launch_kernel(c, dim3(a.B * a.Hkv, a.G), dim3(d), 0, s, true, a);
 }
 
 }  // namespace jssa
