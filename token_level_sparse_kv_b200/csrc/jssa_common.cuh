@@ -172,18 +172,21 @@ __device__ __forceinline__ bool flag_wait_bounded(const volatile unsigned *word,
     return true;
 }
 
+// Suspend-time hint of the waits below (ns; 0 = the hardware's own limit).
+constexpr uint32_t kParkNs = 0;
+
 // Bounded mbarrier wait that also gives up when another role of the CTA
-// raised the abort flag.  The thread is parked in the hardware between polls
-// (up to 20 us per poll), so waiting warps do not take issue slots from the
-// working ones.
+// raised the abort flag.  Each poll is a try_wait, which may suspend the
+// thread in hardware until the phase completes (or a time limit passes), so
+// waiting warps take few issue slots from the working ones.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                               uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 0; it < (1u << 20); ++it) {
-        if (mbar_try_wait_for(bar, parity, 20000u)) return true;
+    for (uint32_t it = 0; it < (1u << 28); ++it) {
+        if (kParkNs ? mbar_try_wait_for(bar, parity, kParkNs) : mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > limit_ns) return false;
+        if ((it & 15u) == 15u && global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
 }

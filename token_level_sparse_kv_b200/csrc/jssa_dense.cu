@@ -62,6 +62,8 @@ constexpr size_t dense_smem_bytes() {
     using S = DenseShape<D>;
     size_t o = (size_t)S::STAGES * S::STAGE;  // ring (1024-byte aligned stages)
     o += 16 * (size_t)S::QSTR;                // query tile
+    o += 16 * (size_t)D * 4;                  // merge buffer of the warps' O (fp32)
+    o += kNW * 16 * 8;                        // the warps' (max, sum) per row
     o += 2 * (size_t)S::STAGES * 8;           // full / empty barriers
     o += 64;                                  // flags
     return o + 1024;                          // alignment slack of the dynamic base
@@ -137,7 +139,9 @@ __global__ void __launch_bounds__(kThr, 1)
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     unsigned char *ring = smem;
     unsigned char *q_s = ring + (size_t)STAGES * S::STAGE;
-    uint64_t *full = reinterpret_cast<uint64_t *>(q_s + 16 * QSTR);
+    float *obuf = reinterpret_cast<float *>(q_s + 16 * QSTR);        // [16][D]
+    float2 *mlw = reinterpret_cast<float2 *>(obuf + 16 * D);         // [kNW][16]
+    uint64_t *full = reinterpret_cast<uint64_t *>(mlw + kNW * 16);
     uint64_t *empty = full + STAGES;
     volatile int *flags = reinterpret_cast<volatile int *>(empty + STAGES);  // [0] abort
 
@@ -337,7 +341,8 @@ __global__ void __launch_bounds__(kThr, 1)
 
         const bool seg_end = (j == rt - 1) || (i == i1 - 1);
         if (seg_end) {
-            // this warp's partial of the row: unnormalised O, max, sum
+            // the CTA's partial of the row: the four warps' (O, max, sum) merged
+            // in shared memory, then one unnormalised partial per segment
             const long long first = (long long)bh * rt;
             const int c_first = (int)(((first + 1) * a.grid - 1) / total);
             const int slot = (int)blockIdx.x - c_first;
@@ -345,19 +350,51 @@ __global__ void __launch_bounds__(kThr, 1)
             for (int r = 0; r < 2; ++r) {
                 lrun[r] += __shfl_xor_sync(0xffffffffu, lrun[r], 1);
                 lrun[r] += __shfl_xor_sync(0xffffffffu, lrun[r], 2);
+                if (tig == 0) mlw[warp * 16 + gid + 8 * r] = make_float2(mrun[r], lrun[r]);
             }
-            const size_t pidx = (size_t)bh * parts_stride + (size_t)slot * kNW + warp;
+            consumer_sync();
+            // the warps add their rescaled O into the buffer in turn (no atomics)
+            float wgt[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int g = gid + 8 * r;
-                if (g < G) {
-                    float *po = a.part_o + (pidx * G + g) * D + 2 * tig;
+                float M = -INFINITY;
 #pragma unroll
-                    for (int dt = 0; dt < D / 8; ++dt)
-                        *reinterpret_cast<float2 *>(po + dt * 8) = make_float2(o[dt][2 * r], o[dt][2 * r + 1]);
-                    if (tig == 0)
-                        *reinterpret_cast<float2 *>(a.part_ml + (pidx * G + g) * 2) = make_float2(mrun[r], lrun[r]);
+                for (int q = 0; q < kNW; ++q) M = fmaxf(M, mlw[q * 16 + g].x);
+                wgt[r] = mrun[r] == -INFINITY ? 0.f : exp2f(mrun[r] - M);
+            }
+#pragma unroll 1
+            for (int turn = 0; turn < kNW; ++turn) {
+                if (warp == turn) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int g = gid + 8 * r;
+                        if (g < G) {
+                            float2 *ob = reinterpret_cast<float2 *>(obuf + g * D + 2 * tig);
+#pragma unroll
+                            for (int dt = 0; dt < D / 8; ++dt) {
+                                float2 v = turn ? ob[dt * 4] : make_float2(0.f, 0.f);
+                                v.x = fmaf(o[dt][2 * r], wgt[r], v.x);
+                                v.y = fmaf(o[dt][2 * r + 1], wgt[r], v.y);
+                                ob[dt * 4] = v;
+                            }
+                        }
+                    }
                 }
+                consumer_sync();
+            }
+            const size_t pidx = (size_t)bh * parts_stride + slot;
+            for (int e = ctid; e < G * D; e += kNW * 32) a.part_o[pidx * G * D + e] = obuf[e];
+            if (ctid < G) {
+                float M = -INFINITY, L = 0.f;
+#pragma unroll
+                for (int q = 0; q < kNW; ++q) M = fmaxf(M, mlw[q * 16 + ctid].x);
+#pragma unroll
+                for (int q = 0; q < kNW; ++q) {
+                    const float2 v = mlw[q * 16 + ctid];
+                    if (v.x != -INFINITY) L = fmaf(v.y, exp2f(v.x - M), L);
+                }
+                *reinterpret_cast<float2 *>(a.part_ml + (pidx * G + ctid) * 2) = make_float2(M, L);
             }
             if (i + 1 < i1) {
                 ++bh;
@@ -374,9 +411,8 @@ __global__ void __launch_bounds__(kThr, 1)
     }
 }
 
-// Log-sum-exp merge of a row's partials (every segment of every CTA that
-// covered it, one partial per consumer warp; empty partials carry O = 0 and
-// max -inf): one CTA per (row, head), one thread per output dim.  Chained
+// Log-sum-exp merge of a row's partials (one per CTA segment that covered
+// it; empty partials carry O = 0 and max -inf): one CTA per (row, head), one thread per output dim.  Chained
 // after the dense kernel with programmatic dependent launch.
 template <int D>
 __global__ void __launch_bounds__(D) dense_combine_kernel(DenseArgs a) {
@@ -387,7 +423,7 @@ __global__ void __launch_bounds__(D) dense_combine_kernel(DenseArgs a) {
     const long long total = a.total_tiles, first = (long long)bh * rt;
     const int c_first = (int)(((first + 1) * a.grid - 1) / total);
     const int c_last = (int)(((first + rt) * a.grid - 1) / total);
-    const int np = (c_last - c_first + 1) * kNW;
+    const int np = c_last - c_first + 1;
     const size_t pb = (size_t)bh * a.part_stride;
     if (d < 32) {
         float M = -INFINITY;
@@ -483,7 +519,7 @@ int dense_part_stride(int B, int Hkv) {
     // of the persistent grid (grid <= SMs), whatever the row length
     const long long BH = (long long)B * Hkv;
     const long long sms = device_sm_count();
-    return (int)(((sms + BH - 1) / BH + 1) * kNW);
+    return (int)((sms + BH - 1) / BH + 1);
 }
 
 cudaError_t plan_dense(int d, int B, int Hkv, int row_len, DensePlan *p) {
