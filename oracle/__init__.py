@@ -68,6 +68,10 @@ def lib():
         L.oracle_topk_forced.argtypes = [i32, i32, i32, vp, vp, i32, i32, i32, vp, i32, vp, vp]
         L.oracle_attend.restype = i32
         L.oracle_attend.argtypes = [i32] * 6 + [vp, i32, vp, vp, i32, i32, vp, vp, i32, vp, dbl, vp, i32, vp, vp]
+        L.oracle_score_heads.restype = i32
+        L.oracle_score_heads.argtypes = [i32] * 6 + [vp, i32, vp, vp, i32, vp, vp, i32, vp]
+        L.oracle_attend_heads.restype = i32
+        L.oracle_attend_heads.argtypes = [i32] * 6 + [vp, i32, vp, vp, i32, i32, vp, vp, i32, vp, dbl, vp, i32, vp, vp]
         L.oracle_dense.restype = i32
         L.oracle_dense.argtypes = [i32] * 6 + [vp, i32, vp, vp, i32, i32, vp, i32, dbl, vp, i32, vp, vp]
         _lib = L
@@ -249,6 +253,51 @@ def attend(q, K, V, idx, count, seq_lens, scale, dv=None, bh_list=None, v_aliase
         raise ValueError("oracle_attend: an index lies outside [0, T_b) or a count outside [0, k]")
     if rc != 0:
         raise ValueError("oracle_attend: bad arguments (rc=%d)" % rc)
+    return out, lse
+
+
+def score_heads(q, P, Kt, seq_lens, bh_list=None):
+    """Per-query-head subspace scores s[b,g,t] (fp64) [B, Hq, T_cap]; t >= T_b
+    holds -inf.  bh_list lists flattened (b*Hq + g) rows."""
+    qr, qcode = raw(q)
+    B, Hq, d = qr.shape
+    Pf = _f32(P)
+    Hkv, _, r = Pf.shape
+    Ktr, ktcode = raw(Kt)
+    T_cap = Ktr.shape[2]
+    sl = _i32(seq_lens)
+    bh, nbh = _bh(bh_list)
+    out = np.full((B, Hq, T_cap), -np.inf, dtype=np.float64)
+    rc = lib().oracle_score_heads(B, Hq, Hkv, d, r, T_cap, _p(qr), qcode, _p(Pf), _p(Ktr), ktcode, _p(sl), _p(bh),
+                                  nbh, _p(out))
+    if rc != 0:
+        raise ValueError("oracle_score_heads: bad arguments (rc=%d)" % rc)
+    return out
+
+
+def attend_heads(q, K, V, idx, count, seq_lens, scale, bh_list=None):
+    """Attention of each query head over its own list: idx [B, Hq, k], count
+    [B, Hq].  Returns (out [B,Hq,dv], lse [B,Hq]) fp64."""
+    qr, qcode = raw(q)
+    B, Hq, d = qr.shape
+    Kr, kvcode = raw(K)
+    _, T_cap, Hkv, _ = Kr.shape
+    Vr, vcode = raw(V)
+    assert vcode == kvcode
+    dv = v_ld = Vr.shape[3]
+    ix = _i32(idx)
+    k = ix.shape[2]
+    cn = _i32(count)
+    sl = _i32(seq_lens)
+    bh, nbh = _bh(bh_list)
+    out = np.zeros((B, Hq, dv), dtype=np.float64)
+    lse = np.full((B, Hq), np.nan, dtype=np.float64)
+    rc = lib().oracle_attend_heads(B, Hq, Hkv, d, dv, T_cap, _p(qr), qcode, _p(Kr), _p(Vr), kvcode, v_ld, _p(ix),
+                                   _p(cn), k, _p(sl), float(scale), _p(bh), nbh, _p(out), _p(lse))
+    if rc == -2:
+        raise ValueError("oracle_attend_heads: an index lies outside [0, T_b) or a count outside [0, k]")
+    if rc != 0:
+        raise ValueError("oracle_attend_heads: bad arguments (rc=%d)" % rc)
     return out, lse
 
 

@@ -22,6 +22,10 @@
  *   4. attend      softmax attention of every query head of the KV head
  *                  over the selected tokens, full-width q.k and V   [NEWS Interp. para 3; ABS]
  *   5. dense       step 4 over all t < T_b (or the last W tokens)   [ABS: the full-KV baseline]
+ * Variant (for measurement; the method shares one set per KV head [ABS]):
+ *   2'. score_heads  s[b,g,t] = (P_h^T q_g) . Kt[b,h,t,:] per query head
+ *   3'. select       top-k_b of s per (batch, query head), as in step 3
+ *   4'. attend_heads attention of each query head over its own set
  *
  * Readings taken where the pages are silent:
  *   - the G = Hq/Hkv query heads of a KV head are h*G .. h*G+G-1;
@@ -190,6 +194,51 @@ int oracle_score(int B, int Hq, int Hkv, int d, int r, int T_cap,
     return 0;
 }
 
+/* Per-query-head subspace scores [variant: ABS and NEWS Synopsis describe one
+ * distinct set per KV head; giving every query head its own set measures what
+ * that sharing costs]:
+ *   qt_g[j] = sum_i q[b,g,i] * P[h,i,j],  s[b,g,t] = sum_j qt_g[j] * Kt[b,h,t,j]
+ * with h = g / G, for t < T_b; -inf beyond.  scores is [B, Hq, T_cap];
+ * bh_list (optional) lists flattened (b*Hq + g) rows.  With G = 1 this is
+ * oracle_score; SUM and MAX over a group are the sum and max of these rows. */
+int oracle_score_heads(int B, int Hq, int Hkv, int d, int r, int T_cap,
+                       const void *q, int q_dtype, const float *P,
+                       const void *Kt, int kt_dtype, const int32_t *seq_lens,
+                       const int32_t *bh_list, int n_bh, double *scores)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0)
+        return -1;
+    int G = Hq / Hkv;
+    int n = bh_list ? n_bh : B * Hq;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int w = 0; w < n; ++w) {
+        int bg = bh_list ? bh_list[w] : w;
+        int b = bg / Hq, g = bg % Hq, h = g / G;
+        int Tb = clamp_len(seq_lens[b], T_cap);
+        double *qt = (double *)malloc(sizeof(double) * (size_t)r);
+        for (int j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i)
+                acc += ld_elem(q, q_dtype, ((size_t)b * Hq + g) * d + i) * (double)P[((size_t)h * d + i) * r + j];
+            qt[j] = acc;
+        }
+        double *srow = scores + (size_t)bg * T_cap;
+        for (int t = 0; t < T_cap; ++t) {
+            if (t >= Tb) {
+                srow[t] = -INFINITY;
+                continue;
+            }
+            size_t krow = (((size_t)b * Hkv + h) * T_cap + t) * (size_t)r;
+            double lg = 0.0;
+            for (int j = 0; j < r; ++j)
+                lg += qt[j] * ld_elem(Kt, kt_dtype, krow + j);
+            srow[t] = lg;
+        }
+        free(qt);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- select ---
  * Per-(batch, KV head) token top-k [NEWS Synopsis: a distinct selected token
  * set for each KV head; ABS: distinct per-KV-head selections]:
@@ -311,49 +360,56 @@ int oracle_topk_forced(int B, int Hkv, int T_cap, const double *scores,
  *   lse = m + ln Z
  * An empty list gives o_g = 0 and lse = -inf.  V rows are v_ld elements apart
  * per (t, h) step: dv for a separate V cache, d when V aliases K (latent cache). */
+static void attend_head(int b, int hq, int h, int Hq, int Hkv, int d, int dv, int T_cap,
+                        const void *q, int q_dtype, const void *K, const void *V,
+                        int kv_dtype, int v_ld, const int32_t *list, int n,
+                        double scale, double *out, double *lse)
+{
+    double *o = out + ((size_t)b * Hq + hq) * dv;
+    for (int c = 0; c < dv; ++c)
+        o[c] = 0.0;
+    if (n == 0) {
+        if (lse)
+            lse[(size_t)b * Hq + hq] = -INFINITY;
+        return;
+    }
+    double *lg = (double *)malloc(sizeof(double) * (size_t)n);
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j) {
+        int t = list[j];
+        size_t krow = (((size_t)b * T_cap + t) * Hkv + h) * (size_t)d;
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i)
+            acc += ld_elem(q, q_dtype, ((size_t)b * Hq + hq) * d + i) * ld_elem(K, kv_dtype, krow + i);
+        lg[j] = scale * acc;
+        if (lg[j] > m)
+            m = lg[j];
+    }
+    double Z = 0.0;
+    for (int j = 0; j < n; ++j)
+        Z += exp(lg[j] - m);
+    for (int j = 0; j < n; ++j) {
+        int t = list[j];
+        double w = exp(lg[j] - m) / Z;
+        size_t vrow = (((size_t)b * T_cap + t) * Hkv + h) * (size_t)v_ld;
+        for (int c = 0; c < dv; ++c)
+            o[c] += w * ld_elem(V, kv_dtype, vrow + c);
+    }
+    if (lse)
+        lse[(size_t)b * Hq + hq] = m + log(Z);
+    free(lg);
+}
+
+/* every query head g of KV head h over the one list of (b, h) */
 static void attend_one(int b, int h, int Hq, int Hkv, int d, int dv, int T_cap,
                        const void *q, int q_dtype, const void *K, const void *V,
                        int kv_dtype, int v_ld, const int32_t *list, int n,
                        double scale, double *out, double *lse)
 {
     int G = Hq / Hkv;
-    double *lg = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
-    for (int g = 0; g < G; ++g) {
-        int hq = h * G + g;
-        double *o = out + ((size_t)b * Hq + hq) * dv;
-        for (int c = 0; c < dv; ++c)
-            o[c] = 0.0;
-        if (n == 0) {
-            if (lse)
-                lse[(size_t)b * Hq + hq] = -INFINITY;
-            continue;
-        }
-        double m = -INFINITY;
-        for (int j = 0; j < n; ++j) {
-            int t = list[j];
-            size_t krow = (((size_t)b * T_cap + t) * Hkv + h) * (size_t)d;
-            double acc = 0.0;
-            for (int i = 0; i < d; ++i)
-                acc += ld_elem(q, q_dtype, ((size_t)b * Hq + hq) * d + i) *
-                       ld_elem(K, kv_dtype, krow + i);
-            lg[j] = scale * acc;
-            if (lg[j] > m)
-                m = lg[j];
-        }
-        double Z = 0.0;
-        for (int j = 0; j < n; ++j)
-            Z += exp(lg[j] - m);
-        for (int j = 0; j < n; ++j) {
-            int t = list[j];
-            double w = exp(lg[j] - m) / Z;
-            size_t vrow = (((size_t)b * T_cap + t) * Hkv + h) * (size_t)v_ld;
-            for (int c = 0; c < dv; ++c)
-                o[c] += w * ld_elem(V, kv_dtype, vrow + c);
-        }
-        if (lse)
-            lse[(size_t)b * Hq + hq] = m + log(Z);
-    }
-    free(lg);
+    for (int g = 0; g < G; ++g)
+        attend_head(b, h * G + g, h, Hq, Hkv, d, dv, T_cap, q, q_dtype, K, V, kv_dtype, v_ld, list, n, scale, out,
+                    lse);
 }
 
 /* Indexed attention over per-(b,h) lists idx[b,h,0:count[b,h]] (the rest of
@@ -419,4 +475,43 @@ int oracle_dense(int B, int Hq, int Hkv, int d, int dv, int T_cap,
         free(list);
     }
     return 0;
+}
+
+/* Attention of each query head over its own list idx[b,g,0:count[b,g]]
+ * (idx [B, Hq, k], count [B, Hq]) [variant of step 4: per-query-head sets],
+ * the same arithmetic as oracle_attend.  bh_list (optional) lists flattened
+ * (b*Hq + g) rows.  Returns -2 if a listed index is outside [0, T_b). */
+int oracle_attend_heads(int B, int Hq, int Hkv, int d, int dv, int T_cap,
+                        const void *q, int q_dtype, const void *K, const void *V,
+                        int kv_dtype, int v_ld, const int32_t *idx, const int32_t *count,
+                        int k, const int32_t *seq_lens, double scale,
+                        const int32_t *bh_list, int n_bh, double *out, double *lse)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0 || dv > v_ld)
+        return -1;
+    int G = Hq / Hkv;
+    int n = bh_list ? n_bh : B * Hq;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int w = 0; w < n; ++w) {
+        int bg = bh_list ? bh_list[w] : w;
+        int b = bg / Hq, g = bg % Hq;
+        int Tb = clamp_len(seq_lens[b], T_cap);
+        int c = count[bg];
+        if (c < 0 || c > k) {
+            bad = 1;
+            continue;
+        }
+        const int32_t *list = idx + (size_t)bg * k;
+        int ok = 1;
+        for (int j = 0; j < c; ++j)
+            if (list[j] < 0 || list[j] >= Tb)
+                ok = 0;
+        if (!ok) {
+            bad = 1;
+            continue;
+        }
+        attend_head(b, g, g / G, Hq, Hkv, d, dv, T_cap, q, q_dtype, K, V, kv_dtype, v_ld, list, c, scale, out, lse);
+    }
+    return bad ? -2 : 0;
 }

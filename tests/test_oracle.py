@@ -434,3 +434,90 @@ def test_topk_forced_plain_case_and_invariants():
     # forced tokens alone exceed k: the smallest forced indices
     idx, cnt = oracle.topk(s, sl, 6, n_sink=4, n_recent=8)
     assert idx[0, 0].tolist() == [0, 1, 2, 3, 492, 493]
+
+
+# ------------------------------------- per-query-head selection (variant)
+def test_score_heads_matches_projected_matmul_and_group_relations():
+    # s[b,g,t] = (q_g P_h) . Kt_t with h = g // G, against an independent
+    # numpy statement; the SUM / MAX group scores are the sum / max of the
+    # group's rows (a dropped head, a wrong group index or a transposed P fails)
+    w = Workload("t", B=2, Hq=8, Hkv=2, d=32, T=40, r=8, k=4, seed=108)
+    q, K, V, P, _ = make_inputs(w)
+    sl = torch.tensor([40, 23], dtype=torch.int32)
+    Kt = oracle.append_lowrank(K, P, [0, 0], w.T)
+    ktd = oracle.bf16_bits_to_f64(Kt)
+    G = w.G
+    qt = np.einsum("bgi,gij->bgj", f64(q), np.repeat(P.to(torch.float64).numpy(), G, axis=0))
+    ref = np.einsum("bgj,bgtj->bgt", qt, np.repeat(ktd, G, axis=1))
+    ref[1, :, 23:] = -np.inf
+    sh = oracle.score_heads(q, P, Kt, sl)
+    np.testing.assert_allclose(sh, ref, rtol=1e-12, atol=1e-10)
+    s_sum = oracle.score(q, P, Kt, sl, oracle.AGG_SUM)
+    s_max = oracle.score(q, P, Kt, sl, oracle.AGG_MAX)
+    fin = np.isfinite(s_sum)
+    grp = sh.reshape(w.B, w.Hkv, G, w.T)
+    np.testing.assert_allclose(grp.sum(2)[fin], s_sum[fin], rtol=1e-12, atol=1e-10)
+    np.testing.assert_array_equal(grp.max(2), s_max)
+
+
+def test_score_heads_with_one_head_per_kv_head_is_the_group_score():
+    w = Workload("t", B=2, Hq=3, Hkv=3, d=16, T=30, r=8, k=4, seed=109)
+    q, K, V, P, sl = make_inputs(w)
+    Kt = oracle.append_lowrank(K, P, [0, 0], w.T)
+    np.testing.assert_array_equal(oracle.score_heads(q, P, Kt, sl), oracle.score(q, P, Kt, sl))
+
+
+def test_per_head_topk_matches_subset_brute_force():
+    # tiny T: each query head's own top-k equals the k-subset optimum of its
+    # own scores, and differs from the group's shared set where the heads disagree
+    w = Workload("t", B=1, Hq=4, Hkv=1, d=16, T=9, r=16, k=3, kind="plain", seed=110)
+    q, K, V, _, sl = make_inputs(w)
+    P = torch.eye(w.d).unsqueeze(0).contiguous()
+    Kt = oracle.append_lowrank(K, P, [0], w.T)
+    sh = oracle.score_heads(q, P, Kt, sl)
+    idx, cnt = oracle.topk(sh, sl, w.k)
+    for g in range(w.Hq):
+        assert idx[0, g].tolist() == brute.topk_by_subsets(sh[0, g].tolist(), w.k)
+        assert cnt[0, g] == w.k
+    logits = np.einsum("gi,ti->gt", f64(q[0]), f64(K[0, :, 0]))  # P = I: exact q_g . K_t
+    np.testing.assert_allclose(sh[0], logits, rtol=1e-12, atol=1e-12)
+
+
+def test_attend_heads_reduces_to_attend_and_to_loops():
+    w = Workload("t", B=2, Hq=6, Hkv=2, d=16, T=25, r=8, k=7, seed=111)
+    q, K, V, P, _ = make_inputs(w)
+    sl = torch.tensor([25, 9], dtype=torch.int32)
+    g = np.random.default_rng(5)
+    G = w.G
+    # shared lists (every head of a KV head on its group's list) equal oracle_attend
+    idx = np.full((w.B, w.Hkv, w.k), -1, np.int32)
+    cnt = np.zeros((w.B, w.Hkv), np.int32)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            c = min(w.k, int(sl[b])) - h
+            cnt[b, h] = c
+            idx[b, h, :c] = np.sort(g.choice(int(sl[b]), c, replace=False))
+    o1, l1 = oracle.attend(q, K, V, idx, cnt, sl, w.scale)
+    o2, l2 = oracle.attend_heads(q, K, V, np.repeat(idx, G, axis=1), np.repeat(cnt, G, axis=1), sl, w.scale)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    # distinct per-head lists against pure-Python loops (head g reads KV head g // G)
+    hidx = np.full((w.B, w.Hq, w.k), -1, np.int32)
+    hcnt = np.zeros((w.B, w.Hq), np.int32)
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            c = int(g.integers(0, min(w.k, int(sl[b])) + 1))
+            hcnt[b, hq] = c
+            hidx[b, hq, :c] = np.sort(g.choice(int(sl[b]), c, replace=False))
+    o, l = oracle.attend_heads(q, K, V, hidx, hcnt, sl, w.scale)
+    Kf, Vf, qf = f64(K), f64(V), f64(q)
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            rows = hidx[b, hq, :hcnt[b, hq]]
+            ro, rl = brute.attention_loops([qf[b, hq].tolist()], [Kf[b, t, hq // G].tolist() for t in rows],
+                                           [Vf[b, t, hq // G].tolist() for t in rows], w.scale)
+            if len(rows):
+                np.testing.assert_allclose(o[b, hq], ro[0], rtol=1e-12, atol=1e-13)
+                assert abs(l[b, hq] - rl[0]) < 1e-12
+            else:
+                assert np.all(o[b, hq] == 0) and np.isneginf(l[b, hq])
