@@ -405,6 +405,68 @@ def measure_decode_loop(dev, n_layers, steps, stream):
     return res
 
 
+def per_head_comparison(w, q, K, V, P, Kt, sl, pos, dims, dev, stream, flush_buf, steps, world, use_graph):
+    """The per-query-head selection variant (every query head its own top-k)
+    against the method's per-KV-head selection on the same inputs: step time
+    of both as separate calls (append, selection, indexed attention), bytes of
+    selected rows each reads, the recall of the shared per-KV-head set against
+    each query head's own top-k, and each output's distance to dense full-KV
+    attention (a proxy for what sharing one set per KV head costs)."""
+    import torch
+
+    from token_level_sparse_kv_b200 import ops
+
+    G = w.G
+    ws_a = ops.new_workspace(dims, 1, ops.OP_APPEND, dev)
+    ws_s = ops.new_workspace(dims, w.k, ops.OP_SELECT, dev)
+    ws_i = ops.new_workspace(dims, w.k, ops.OP_INDEXED_DECODE, dev)
+    ws_sh = ops.new_workspace(dims, w.k, ops.OP_SELECT_HEADS, dev)
+    ws_ih = ops.new_workspace(dims, w.k, ops.OP_INDEXED_DECODE_HEADS, dev)
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
+    idh = torch.empty((w.B, w.Hq, w.k), dtype=torch.int32, device=dev)
+    cnh = torch.empty((w.B, w.Hq), dtype=torch.int32, device=dev)
+    out_kv = torch.empty((w.B, w.Hq, w.Dv), dtype=q.dtype, device=dev)
+    out_q = torch.empty_like(out_kv)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+
+    def kv_step(i):
+        ops.append_lowrank(K, P, Kt, pos, 1, ws=ws_a)
+        ops.select(q, P, Kt, sl, w.k, ws=ws_s, idx=idx, count=cnt)
+        ops.indexed_decode(q, K, V, idx, cnt, sl, w.scale, ws=ws_i, out=out_kv, lse=lse)
+
+    def head_step(i):
+        ops.append_lowrank(K, P, Kt, pos, 1, ws=ws_a)
+        ops.select_heads(q, P, Kt, sl, w.k, ws=ws_sh, idx=idh, count=cnh)
+        ops.indexed_decode_heads(q, K, V, idh, cnh, sl, w.scale, ws=ws_ih, out=out_q, lse=lse)
+
+    res = {}
+    for name, fn in (("per_kv_head_calls", kv_step), ("per_query_head_calls", head_step)):
+        for i in range(3):
+            fn(i)
+        rep_fn = graphed(fn, dev, 1) if use_graph else fn
+        for i in range(3):
+            rep_fn(i)
+        d = time_steps(rep_fn, steps, stream, flush_buf)
+        med = max_over_ranks(percentile(d, 0.5), world)
+        res[name] = {"steps_per_s": world / med, "ms_per_step": med * 1e3}
+    torch.cuda.synchronize()
+    # recall of the shared set against each query head's own top-k
+    kv_sets = idx.repeat_interleave(G, 1)  # [B, Hq, k]
+    hit = (idh.unsqueeze(-1) == kv_sets.unsqueeze(-2)).any(-1) & (idh >= 0)
+    res["recall_of_per_kv_head_sets"] = float(hit.sum().item() / max(1, int((idh >= 0).sum().item())))
+    od, _ = ops.dense_decode(q, K, V, sl, w.scale)
+    torch.cuda.synchronize()
+    res["mean_abs_err_vs_dense"] = {"per_kv_head": float((out_kv.float() - od.float()).abs().mean().item()),
+                                    "per_query_head": float((out_q.float() - od.float()).abs().mean().item())}
+    row = (w.d + w.Dv) * 2
+    res["selected_bytes_per_step"] = {"per_kv_head": w.B * w.Hkv * min(w.k, w.T) * row,
+                                      "per_query_head": w.B * w.Hq * min(w.k, w.T) * row}
+    res["note"] = ("per-query-head selection reads G = %d times the selected rows; recall = share of each query "
+                   "head's own top-k that its KV head's shared set contains" % G)
+    return res
+
+
 def run_jssa(args, world, rank, local):
     import torch
 
@@ -570,6 +632,9 @@ def run_jssa(args, world, rank, local):
             med = max_over_ranks(percentile(d, 0.5), world)
             res[name] = {"steps_per_s": world / med, "ms_per_step": med * 1e3, "latency": latency_summary(d),
                          "launch": "cuda graph replay" if graphs else "eager"}
+        if not w.latent:
+            res["per_query_head_selection"] = per_head_comparison(w, q, K, Vv, P, Kt, sl, pos, dims, dev, stream,
+                                                                  flush_buf, cmp_steps, world, graphs is not None)
         res["speedup_vs_dense"] = value / res["dense_full_kv"]["steps_per_s"]
         res["speedup_vs_gather_then_dense"] = value / res["gather_then_dense"]["steps_per_s"]
         if w.window:

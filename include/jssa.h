@@ -122,7 +122,9 @@ typedef enum {
     JSSA_OP_INDEXED_DECODE = 4,
     JSSA_OP_DENSE_DECODE = 5,
     JSSA_OP_GATHER_THEN_DENSE = 6,
-    JSSA_OP_DECODE_STEP = 7
+    JSSA_OP_DECODE_STEP = 7,
+    JSSA_OP_SELECT_HEADS = 8,        /* jssa_select_heads */
+    JSSA_OP_INDEXED_DECODE_HEADS = 9 /* jssa_indexed_decode_heads */
 } jssa_op;
 
 typedef struct {
@@ -280,6 +282,33 @@ JSSA_API int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const voi
                         int agg, float softmax_scale, const jssa_select_opts *opts, int32_t *idx,
                         int32_t *count, void *out, float *lse, void *ws, size_t ws_bytes,
                         jssa_stream_t stream);
+
+/* Per-query-head selection: a variant for measurement.  The method selects
+ * one distinct token set per (batch, KV head), shared by the G query heads of
+ * the KV head [ABS: distinct per-KV-head selections; NEWS Synopsis]; this
+ * call gives every query head g its own set, so the two can be compared
+ * (bytes of selected rows read, recall, output error):
+ *   s[b,g,t] = (P_h^T q_g) . Kt[b,h,t,:]   (h = g / G, fp32, t < T_b)
+ *   idx[b,g,:] = the k_b tokens that come first under (s desc, t asc),
+ *                ascending, -1 padded;  count[b,g] = k_b   (count may be NULL)
+ * idx is [B, Hq, k], count [B, Hq].  The selection runs in the cluster or the
+ * block-synchronous form (opts->form JSSA_FORM_STREAM is taken as automatic).
+ * GQA shapes only (not the latent form); G <= 16. */
+JSSA_API int jssa_select_heads(const jssa_dims *dims, const void *q, const float *P, const void *Kt,
+                               const int32_t *seq_lens, int k, const jssa_select_opts *opts, int32_t *idx,
+                               int32_t *count, void *ws, size_t ws_bytes, jssa_stream_t stream);
+
+/* Attention of each query head over its own token list (the companion of
+ * jssa_select_heads): for query head g of KV head h = g / G, over t in
+ * idx[b,g,0:count[b,g]] (idx [B, Hq, k], count [B, Hq] or NULL), the same
+ * arithmetic as jssa_indexed_decode: rows read in place from the standard GQA
+ * cache, fp32 online softmax, log-sum-exp combine of the splits.  Every
+ * query head reads its own rows, so a KV head's rows are read up to G times.
+ * GQA shapes only. */
+JSSA_API int jssa_indexed_decode_heads(const jssa_dims *dims, const void *q, const void *K, const void *V,
+                                       const int32_t *idx, const int32_t *count, int k,
+                                       const int32_t *seq_lens, float softmax_scale, void *out, float *lse,
+                                       void *ws, size_t ws_bytes, jssa_stream_t stream);
 
 /* jssa_plan_info with selection options (NULL = jssa_plan_info): the forms
  * and launch count of a call made with these options. */

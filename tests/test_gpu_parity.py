@@ -479,6 +479,56 @@ def test_bounded_waits_expire_with_a_status_and_the_context_stays_usable():
     check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
 
 
+# --------------------------------------------- per-query-head selection
+@pytest.mark.parametrize("case", ["g4", "g8_r64", "g1", "fp32"])
+def test_select_heads_and_decode_heads_match_oracle(case, form):
+    """Per-query-head selection (every query head its own top-k) and attention
+    over per-head lists: bit-exact top-k on the GPU's own fp32 scores is not
+    available here, so the selection follows the tie-window rule against the
+    oracle's fp64 per-head scores on the GPU's low-rank cache, and attention
+    is compared on the GPU's indices."""
+    kt, dtype = torch.bfloat16, torch.bfloat16
+    if case == "g4":
+        w, sl = W(B=3, Hq=8, Hkv=2, T=7000, k=200, seed=120), [7000, 6999, 150]
+    elif case == "g8_r64":
+        w, sl = W(B=2, Hq=16, Hkv=2, d=256, r=64, T=5000, k=256, seed=121), [5000, 4096]
+    elif case == "g1":
+        w, sl = W(B=2, Hq=4, Hkv=4, T=3000, k=64, seed=122), [3000, 1]
+    else:
+        w, sl, kt, dtype = W(B=2, T=3000, k=100, seed=123), [3000, 2999], torch.float32, torch.float32
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, dtype=dtype, seq_lens=sl)
+    Kt = ops.build_lowrank_cache(Kd, Pd, kt_dtype=kt)
+    idx, cnt = ops.select_heads(qd, Pd, Kt, sld, w.k, form=form)
+    out, lse = ops.indexed_decode_heads(qd, Kd, Vd, idx, cnt, sld, w.scale)
+    torch.cuda.synchronize()
+    ref_s = oracle.score_heads(q, P, host(Kt), slh)
+    check_selection(host(idx).numpy(), host(cnt).numpy(), ref_s, slh.numpy(), w.k)
+    ref_o, ref_l = oracle.attend_heads(q, K, V, host(idx), host(cnt), slh, w.scale)
+    check_attention(out, lse, ref_o, ref_l, dtype)
+    if case == "g1":  # one query head per KV head: the per-KV-head selection itself
+        i2, c2 = ops.select(qd, Pd, Kt, sld, w.k, form=form)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, i2) and torch.equal(cnt, c2)
+
+
+def test_select_heads_forms_agree_and_group_lists_reduce_to_indexed():
+    w, sl = W(B=2, Hq=8, Hkv=2, T=20000, k=256, seed=124), [20000, 9000]
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    a = ops.select_heads(qd, Pd, Kt, sld, w.k, form="cluster")
+    b = ops.select_heads(qd, Pd, Kt, sld, w.k, form="scan")
+    # every head of a KV head on its group's shared list: equal to the per-KV-head attention
+    idx, cnt = ops.select(qd, Pd, Kt, sld, w.k)
+    G = w.G
+    o1, l1 = ops.indexed_decode(qd, Kd, Vd, idx, cnt, sld, w.scale)
+    o2, l2 = ops.indexed_decode_heads(qd, Kd, Vd, idx.repeat_interleave(G, 1).contiguous(),
+                                      cnt.repeat_interleave(G, 1).contiguous(), sld, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    assert (l1 - l2).abs().max().item() <= 1e-3
+
+
 # ------------------------------------------------------- full-size samples
 def _full_size_sampled(w, pairs, ks=None, dense_check=True):
     """The decode step at a full-size workload, in the launch form bench.py

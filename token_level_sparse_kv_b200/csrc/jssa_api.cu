@@ -108,6 +108,16 @@ int check_dims(const jssa_dims *d, Shape *sh) {
     return JSSA_OK;
 }
 
+// One selection (and attention) row per query head: the dims seen by the
+// row-wise planners (Hkv = Hq rows, G = 1).
+void heads_view(const jssa_dims *d, const Shape &sh, jssa_dims *dh, Shape *shh) {
+    *dh = *d;
+    dh->Hkv = d->Hq;
+    *shh = sh;
+    shh->G = 1;
+    shh->BH = d->B * d->Hq;
+}
+
 int check_k(int k) {
     if (k < 1 || k > kMaxK) return fail(JSSA_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, kMaxK);
     return JSSA_OK;
@@ -123,6 +133,14 @@ int check_attn_shape(const jssa_dims *d, const Shape &sh, bool indexed) {
         return JSSA_OK;
     }
     if (sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "G=%d query heads per KV head above %d", sh.G, kMaxG);
+    return JSSA_OK;
+}
+
+// The per-query-head variant: GQA shapes, G <= 16 (the per-head projection).
+int check_heads_shape(const jssa_dims *d, const Shape &sh) {
+    if (sh.latent) return fail(JSSA_ERR_UNSUPPORTED, "per-query-head selection is for GQA shapes, not the latent form");
+    if (sh.G > kMaxG) return fail(JSSA_ERR_UNSUPPORTED, "per-query-head selection needs G <= %d (got %d)", kMaxG, sh.G);
+    (void)d;
     return JSSA_OK;
 }
 
@@ -165,7 +183,7 @@ size_t take(size_t &off, size_t bytes) {
 // kernel) the streaming form is tried first.  A forced form (form != 0,
 // jssa_select_form) overrides the choice.
 int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, int form, Layout &L,
-                  bool stream_first = false) {
+                  bool stream_first = false, bool no_stream = false) {
     const int nq = (src != SRC_SCORES && agg == JSSA_AGG_MAX) ? sh.G : 1;
     stream_first = stream_first && form == JSSA_FORM_AUTO;
     auto try_csel = [&](bool &ok) -> int {
@@ -185,7 +203,7 @@ int layout_select(const jssa_dims *d, const Shape &sh, int src, int k, int agg, 
         const int st = try_csel(done);
         if (st != JSSA_OK || done) return st;
     }
-    cudaError_t e = form == JSSA_FORM_SCAN ? cudaErrorNotSupported : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
+    cudaError_t e = (form == JSSA_FORM_SCAN || no_stream) ? cudaErrorNotSupported : plan_stream(src, agg, d->B, d->Hkv, d->T_cap, d->r, k, &L.sp);
     if (e == cudaSuccess) {
         L.wspec = true;
     } else {
@@ -336,6 +354,22 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
             st = layout_attend(d, sh, ATT_RANGE_BH, k, L);
             if (st == JSSA_OK) L.gcount = take(L.total, (size_t)sh.BH * 4);
             break;
+        case JSSA_OP_SELECT_HEADS: {
+            L.qproj = take(L.total, (size_t)sh.BH * sh.G * d->r * 4);  // per-head projections
+            jssa_dims dh;
+            Shape shh;
+            heads_view(d, sh, &dh, &shh);
+            st = layout_select(&dh, shh, d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32, k, JSSA_AGG_SUM,
+                               ch.form == JSSA_FORM_STREAM ? JSSA_FORM_AUTO : ch.form, L, false, true);
+            break;
+        }
+        case JSSA_OP_INDEXED_DECODE_HEADS: {
+            jssa_dims dh;
+            Shape shh;
+            heads_view(d, sh, &dh, &shh);
+            st = layout_attend(&dh, shh, ATT_INDEXED, k, L);
+            break;
+        }
         case JSSA_OP_DECODE_STEP: {
             // one fused launch where the shape allows it; with k <= 256 it
             // also beats the three-launch cluster form on short caches and
@@ -443,7 +477,7 @@ void fill_dense(DenseArgs &a, const jssa_dims *d, const Shape &sh, const void *q
 
 int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *P, const void *Kt,
                const int32_t *seq_lens, int agg, int k, int32_t *idx, int32_t *count, void *ws, const Layout &L,
-               cudaStream_t s, bool with_project, const jssa_select_opts *opts) {
+               cudaStream_t s, bool with_project, const jssa_select_opts *opts, int src_div = 1) {
     const int n_sink = opts ? opts->n_sink : 0, n_recent = opts ? opts->n_recent : 0;
     const int nq = agg == JSSA_AGG_MAX ? sh.G : 1;
     if (with_project) {
@@ -468,6 +502,7 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
         ca.k = k;
         ca.n_sink = n_sink;
         ca.n_recent = n_recent;
+        ca.src_div = src_div;
         // a null query means the source is a score array (jssa_topk)
         const int src = q == nullptr ? SRC_SCORES : (d->kt_dtype == JSSA_BF16 ? SRC_KT_BF16 : SRC_KT_FP32);
         cudaError_t e = launch_csel(L.cp, ca, src, q == nullptr ? JSSA_AGG_SUM : agg, s, true);
@@ -494,6 +529,7 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
     sa.k = k;
     sa.n_sink = n_sink;
     sa.n_recent = n_recent;
+    sa.src_div = src_div;
     cudaError_t e = L.wspec ? launch_stream(L.sp, sa, s, true) : launch_scan(L.sp, sa, agg, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the selection pass");
     return JSSA_OK;
@@ -569,13 +605,17 @@ int jssa_workspace_size(const jssa_dims *dims, int k, int op, size_t *bytes) {
     if (st) return st;
     if (!bytes) return fail(JSSA_ERR_INVALID_ARG, "bytes is NULL");
     const bool needs_k = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_INDEXED_DECODE ||
-                         op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP;
+                         op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP || op == JSSA_OP_SELECT_HEADS ||
+                         op == JSSA_OP_INDEXED_DECODE_HEADS;
     if (needs_k && (st = check_k(k))) return st;
+    if ((op == JSSA_OP_SELECT_HEADS || op == JSSA_OP_INDEXED_DECODE_HEADS) && (st = check_heads_shape(dims, sh)))
+        return st;
     if ((op == JSSA_OP_INDEXED_DECODE || op == JSSA_OP_DENSE_DECODE || op == JSSA_OP_GATHER_THEN_DENSE ||
          op == JSSA_OP_DECODE_STEP) &&
         (st = check_attn_shape(dims, sh, op == JSSA_OP_INDEXED_DECODE || op == JSSA_OP_DECODE_STEP)))
         return st;
-    const bool selects = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_DECODE_STEP;
+    const bool selects = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_DECODE_STEP ||
+                         op == JSSA_OP_SELECT_HEADS;
     size_t best = 0;
     for (int agg = 0; agg < 2; ++agg) {
         if (agg == JSSA_AGG_MAX && sh.G > kMaxG) continue;
@@ -606,8 +646,11 @@ int jssa_plan_info_ex(const jssa_dims *dims, int k, int op, int agg, const jssa_
     if (!launches) return fail(JSSA_ERR_INVALID_ARG, "launches is NULL");
     if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
     const bool needs_k = op == JSSA_OP_TOPK || op == JSSA_OP_SELECT || op == JSSA_OP_INDEXED_DECODE ||
-                         op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP;
+                         op == JSSA_OP_GATHER_THEN_DENSE || op == JSSA_OP_DECODE_STEP || op == JSSA_OP_SELECT_HEADS ||
+                         op == JSSA_OP_INDEXED_DECODE_HEADS;
     if (needs_k && (st = check_k(k))) return st;
+    if ((op == JSSA_OP_SELECT_HEADS || op == JSSA_OP_INDEXED_DECODE_HEADS) && (st = check_heads_shape(dims, sh)))
+        return st;
     if ((st = check_opts(opts))) return st;
     Layout L;
     if ((st = build_layout(dims, sh, k, op, agg, 0, choice_of(opts), L))) return st;
@@ -621,6 +664,11 @@ int jssa_plan_info_ex(const jssa_dims *dims, int k, int op, int agg, const jssa_
         case JSSA_OP_TOPK: n = 1; snprintf(text, sizeof text, "top-k (%s form)", sel); break;
         case JSSA_OP_SELECT: n = 2; snprintf(text, sizeof text, "projection + selection (%s form)", sel); break;
         case JSSA_OP_INDEXED_DECODE: n = att; snprintf(text, sizeof text, "indexed attention"); break;
+        case JSSA_OP_SELECT_HEADS:
+            n = 2;
+            snprintf(text, sizeof text, "per-head projection + per-query-head selection (%s form)", sel);
+            break;
+        case JSSA_OP_INDEXED_DECODE_HEADS: n = 1; snprintf(text, sizeof text, "per-query-head indexed attention"); break;
         case JSSA_OP_DENSE_DECODE:
         case JSSA_OP_GATHER_THEN_DENSE: {
             const int g = op == JSSA_OP_GATHER_THEN_DENSE ? 1 : 0;
@@ -983,6 +1031,68 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     a.k = k;
     e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the indexed decode");
+    return JSSA_OK;
+}
+
+int jssa_select_heads(const jssa_dims *dims, const void *q, const float *P, const void *Kt, const int32_t *seq_lens,
+                      int k, const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
+                      jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    if ((st = check_heads_shape(dims, sh))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(P);
+    REQUIRE_PTR(Kt);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(idx);
+    OPTIONAL_PTR(count);
+    if ((st = check_opts(opts))) return st;
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_SELECT_HEADS, 0, 0, choice_of(opts), L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    // per-head projections (the MAX layout: [B*Hkv, G, r] = one row per query head)
+    ProjArgs pj{q, P, at<float>(ws, L.qproj), dims->B, dims->Hq, dims->Hkv, dims->d, dims->r, JSSA_AGG_MAX};
+    cudaError_t e = launch_project(pj, S(stream), true, dims->kv_dtype);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the per-head projection");
+    jssa_dims dh;
+    Shape shh;
+    heads_view(dims, sh, &dh, &shh);
+    return run_select(&dh, shh, q, P, Kt, seq_lens, JSSA_AGG_SUM, k, idx, count, ws, L, S(stream), false, opts, sh.G);
+}
+
+int jssa_indexed_decode_heads(const jssa_dims *dims, const void *q, const void *K, const void *V, const int32_t *idx,
+                              const int32_t *count, int k, const int32_t *seq_lens, float softmax_scale, void *out,
+                              float *lse, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if ((st = check_k(k))) return st;
+    if ((st = check_heads_shape(dims, sh))) return st;
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(out);
+    OPTIONAL_PTR(count);
+    OPTIONAL_PTR(lse);
+    Layout L;
+    if ((st = build_layout(dims, sh, k, JSSA_OP_INDEXED_DECODE_HEADS, 0, 0, Choice(), L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    if (dims->B == 0) return JSSA_OK;
+    AttnArgs a;
+    fill_attn(a, dims, sh, q, K, V, seq_lens, softmax_scale, out, lse, ws, L);  // strides of the real cache
+    a.Hkv = dims->Hq;  // one attention row per query head ...
+    a.G = 1;
+    a.head_div = sh.G;  // ... reading KV head g / G
+    a.idx = idx;
+    a.count = count;
+    a.k = k;
+    cudaError_t e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the per-query-head indexed decode");
     return JSSA_OK;
 }
 

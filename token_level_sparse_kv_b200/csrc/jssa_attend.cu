@@ -156,8 +156,9 @@ __global__ void __launch_bounds__(NTH) attend_kernel(AttnArgs a) {
             const int t = tk[row];
             unsigned char *dst = ks + (size_t)kv * NT * STRIDE + (size_t)row * STRIDE + ch * 16;
             if (t >= 0) {
-                const long long off = kv ? ((long long)b * a.v_sb + (long long)t * a.v_st + (long long)h * a.v_sh)
-                                         : ((long long)b * a.k_sb + (long long)t * a.k_st + (long long)h * a.k_sh);
+                const long long hp = a.head_div > 1 ? h / a.head_div : h;  // the K/V head this row reads
+                const long long off = kv ? ((long long)b * a.v_sb + (long long)t * a.v_st + hp * a.v_sh)
+                                         : ((long long)b * a.k_sb + (long long)t * a.k_st + hp * a.k_sh);
                 cp_async16(dst, (kv ? Vb : Kb) + off * S::ES + ch * 16, 16);
             } else {
                 cp_async16(dst, Kb, 0);

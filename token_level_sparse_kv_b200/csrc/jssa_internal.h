@@ -44,6 +44,7 @@ struct ScanArgs {
     long long total_tiles;
     int grid, max_seg, cap, nstages;
     int n_sink, n_recent;  // always-selected tokens (0, 0: plain top-k)
+    int src_div;           // selection row bh reads source row bh / src_div (0 or 1: the same row)
 };
 
 struct ScanPlan {
@@ -90,6 +91,7 @@ struct AttnArgs {
     void *out;               // [B, Hq, D]
     float *lse;              // [B, Hq] or null
     uint32_t *status;
+    int head_div;            // row head h reads K/V head h / head_div (0 or 1: head h)
 };
 
 struct AttnPlan {
@@ -175,6 +177,7 @@ struct CSelArgs {
     uint32_t *status;
     int B, Hkv, T_cap, r, nq, k, csize, slice, nstages;
     int n_sink, n_recent;  // always-selected tokens (0, 0: plain top-k)
+    int src_div;           // selection row bh reads source row bh / src_div (0 or 1: the same row)
 };
 struct CSelPlan {
     int csize, slice, grid_y, nstages;

@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(NT, 2) scan_kernel(ScanArgs a) {
             const int t0 = p_t * TILE, n = min(TILE, Tb_p - t0);
             if (n > 0) {
                 mbar_arrive_expect_tx(&bars[p_s], (uint32_t)n * ROWB);
-                bulk_g2s(smem + L.stages + (size_t)p_s * kTileBytes, src_base + ((size_t)p_bh * a.T_cap + t0) * ROWB,
+                bulk_g2s(smem + L.stages + (size_t)p_s * kTileBytes, src_base + ((size_t)(a.src_div > 1 ? p_bh / a.src_div : p_bh) * a.T_cap + t0) * ROWB,
                          (uint32_t)n * ROWB, &bars[p_s], pol);
             } else {
                 mbar_arrive(&bars[p_s]);
@@ -723,7 +723,8 @@ __global__ void __launch_bounds__(NT, 2) scan_kernel(ScanArgs a) {
                 if (np > 0) {
                     mbar_arrive_expect_tx(&bars[p_s], (uint32_t)np * ROWB);
                     bulk_g2s(smem + L.stages + (size_t)p_s * kTileBytes,
-                             src_base + ((size_t)p_bh * a.T_cap + tp0) * ROWB, (uint32_t)np * ROWB, &bars[p_s], pol);
+                             src_base + ((size_t)(a.src_div > 1 ? p_bh / a.src_div : p_bh) * a.T_cap + tp0) * ROWB,
+                             (uint32_t)np * ROWB, &bars[p_s], pol);
                 } else {
                     mbar_arrive(&bars[p_s]);
                 }

@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
 
     // ---- scores of this slice into shared memory ---------------------------
     if constexpr (FROM_KT) {
-        const char *src = static_cast<const char *>(a.src) + ((size_t)bh * a.T_cap + lo) * ROWB;
+        const int srow = a.src_div > 1 ? bh / a.src_div : bh;
+        const char *src = static_cast<const char *>(a.src) + ((size_t)srow * a.T_cap + lo) * ROWB;
         uint64_t pol = 0;
         if (tid == 0) {
             pol = policy_evict_first();

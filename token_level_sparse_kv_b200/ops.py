@@ -24,6 +24,7 @@ BF16, FP32 = 0, 1
 AGG_SUM, AGG_MAX = 0, 1
 OP_APPEND, OP_SCORE, OP_TOPK, OP_SELECT, OP_INDEXED_DECODE, OP_DENSE_DECODE, OP_GATHER_THEN_DENSE, OP_DECODE_STEP = \
     range(8)
+OP_SELECT_HEADS, OP_INDEXED_DECODE_HEADS = 8, 9
 DEV_SEQLEN, DEV_INDEX, DEV_POS, DEV_TIMEOUT = 1, 2, 4, 8
 
 
@@ -72,6 +73,10 @@ def lib():
     L.jssa_decode_step_ex.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.jssa_plan_info.restype = i32
     L.jssa_plan_info.argtypes = [D, i32, i32, i32, ctypes.POINTER(i32), ctypes.c_char_p, sz]
+    L.jssa_select_heads.restype = i32
+    L.jssa_select_heads.argtypes = [D, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    L.jssa_indexed_decode_heads.restype = i32
+    L.jssa_indexed_decode_heads.argtypes = [D, vp, vp, vp, vp, vp, i32, vp, f32, vp, vp, vp, sz, vp]
     L.jssa_plan_info_ex.restype = i32
     L.jssa_plan_info_ex.argtypes = [D, i32, i32, i32, vp, ctypes.POINTER(i32), ctypes.c_char_p, sz]
     L.jssa_workspace_init.restype = i32
@@ -261,6 +266,39 @@ def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_
                                 _opts(n_sink, n_recent, form), _p(idx), _p(count), _p(ws), ws.numel(),
                                 _stream(q.device)))
     return idx, count
+
+
+def select_heads(q, P, Kt, seq_lens, k, ws=None, idx=None, count=None, form="auto"):
+    """Per-query-head selection (a variant for measurement): every query head g
+    gets its own top-k over (P_h^T q_g) . Kt.  Returns (idx [B,Hq,k], count [B,Hq])."""
+    _cuda(q, P, Kt, seq_lens)
+    B, Hq, d = q.shape
+    _, Hkv, T_cap, r = Kt.shape
+    dims = Dims(B, Hq, Hkv, d, d, r, T_cap, _dt(q), _dt(Kt))
+    if idx is None:
+        idx = torch.empty((B, Hq, k), dtype=torch.int32, device=q.device)
+    if count is None:
+        count = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+    ws = _ws(ws, dims, k, OP_SELECT_HEADS, q.device)
+    _check(lib().jssa_select_heads(ctypes.byref(dims), _p(q), _p(P), _p(Kt), _p(seq_lens), int(k),
+                                   _opts(0, 0, form), _p(idx), _p(count), _p(ws), ws.numel(), _stream(q.device)))
+    return idx, count
+
+
+def indexed_decode_heads(q, K, V, idx, count, seq_lens, scale, ws=None, out=None, lse=None):
+    """Attention of each query head over its own list idx [B,Hq,k]: (out, lse)."""
+    _cuda(q, K, V, idx, count, seq_lens, out, lse)
+    k = idx.shape[2]
+    dims = make_dims(q, K, V, r=8)
+    if out is None:
+        out = torch.empty((dims.B, dims.Hq, dims.dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((dims.B, dims.Hq), dtype=torch.float32, device=q.device)
+    ws = _ws(ws, dims, k, OP_INDEXED_DECODE_HEADS, q.device)
+    _check(lib().jssa_indexed_decode_heads(ctypes.byref(dims), _p(q), _p(K), _p(V), _p(idx), _p(count), int(k),
+                                           _p(seq_lens), float(scale), _p(out), _p(lse), _p(ws), ws.numel(),
+                                           _stream(q.device)))
+    return out, lse
 
 
 def indexed_decode(q, K, V, idx, count, seq_lens, scale, ws=None, out=None, lse=None):
