@@ -645,28 +645,39 @@ def run_jssa(args, world, rank, local):
         line["comparison"] = res
 
     if not args.quick:
-        # end to end through the session API with host buffers
-        sess = ops.DecodeSession(K, Vv, P, sl, w.k, w.scale, Kt=Kt)
-        qh = [x.cpu().pin_memory() for x in qs]
-        kh = torch.randn((w.B, w.Hkv, w.d), dtype=torch.float32).to(q.dtype).pin_memory()
-        vh = None if w.latent else torch.randn((w.B, w.Hkv, w.Dv), dtype=torch.float32).to(q.dtype).pin_memory()
+        # end to end through the C-ABI call with host buffers: every step copies
+        # the packed [q | new K rows | new V rows] block from pinned host memory,
+        # writes the new rows into the cache, runs the step and copies the
+        # output back to pinned host memory; the host waits for it every step
+        nbytes = ops.host_step_bytes(dims)
+        g = torch.Generator().manual_seed(1234 + rank)
+        hosts = []
+        for j in range(4):
+            kn = torch.randn((w.B, w.Hkv, w.d), generator=g).to(q.dtype)
+            parts = [qs[j].cpu().reshape(-1), kn.reshape(-1)]
+            if not w.latent:
+                parts.append(torch.randn((w.B, w.Hkv, w.Dv), generator=g).to(q.dtype).reshape(-1))
+            blob = torch.cat(parts).view(torch.uint8)
+            hosts.append(torch.empty(nbytes, dtype=torch.uint8).pin_memory().copy_(blob))
+        stage = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         e2e_steps = max(5, min(args.steps, args.e2e_steps))
-        use_graph = graphs is not None
+
+        def host_step(i):
+            ops.decode_step_host(hosts[i & 3], stage, K, Vv, P, Kt, sl, pos, w.k, w.scale, out_host, ws, idx, cnt,
+                                 out, lse, dims=dims)
+            stream.synchronize()  # the host reads the output every step
+
         for i in range(3):
-            sess.step_from_host(qh[i & 3], kh, vh, graph=use_graph)
-            stream.synchronize()
+            host_step(i)
         barrier(world)
         t0 = time.perf_counter()
         for i in range(e2e_steps):
-            o = sess.step_from_host(qh[i & 3], kh, vh, graph=use_graph)
-            stream.synchronize()  # the host reads the output every step
+            host_step(i)
         te = max_over_ranks(time.perf_counter() - t0, world)
-        h2d = qh[0].numel() * qh[0].element_size() + kh.numel() * kh.element_size() + (
-            0 if vh is None else vh.numel() * vh.element_size())
-        d2h = o.numel() * o.element_size()
-        line["e2e"] = {"value": world * e2e_steps / te, "unit": "steps/s", "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h,
-                       "api": "DecodeSession.step_from_host (pinned host in/out%s)" % (", graph=True" if use_graph else "")}
+        line["e2e"] = {"value": world * e2e_steps / te, "unit": "steps/s", "h2d_bytes_per_step": nbytes,
+                       "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+                       "api": "jssa_decode_step_host (C ABI; pinned host in/out, one stream sync per step)"}
 
     if not args.quick and world == 1:
         line["decode_loop"] = measure_decode_loop(dev, 32, 20, stream)

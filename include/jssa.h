@@ -283,6 +283,32 @@ JSSA_API int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const voi
                         int32_t *count, void *out, float *lse, void *ws, size_t ws_bytes,
                         jssa_stream_t stream);
 
+/* Bytes of host input (and of the device staging buffer) that
+ * jssa_decode_step_host takes: the queries [B, Hq, d], then the new token's
+ * K rows [B, Hkv, d], then its V rows [B, Hkv, dv] (none for a latent
+ * cache), packed back to back in kv_dtype. */
+JSSA_API int jssa_host_step_bytes(const jssa_dims *dims, size_t *bytes);
+
+/* One decode step driven from host memory: the call a serving loop makes per
+ * token.  Enqueued on `stream`, in order:
+ *   1. one host-to-device copy of in_host (jssa_host_step_bytes bytes, layout
+ *      above) into the device buffer `stage` (same size, 16-byte aligned);
+ *   2. the new K / V rows written into the cache at position pos_begin[b]
+ *      (K[b, pos, :, :], V[b, pos, :, :]); a position outside [0, T_cap) is
+ *      skipped and sets JSSA_DEV_POS;
+ *   3. jssa_decode_step_ex with q = the staged queries (append of the
+ *      low-rank row at pos_begin, selection, indexed attention) into the
+ *      device buffers idx, count, out, lse;
+ *   4. one device-to-host copy of out into out_host ([B, Hq, dv] kv_dtype).
+ * in_host and out_host should be pinned (page-locked) host memory for the
+ * copies to run asynchronously; the host must synchronise the stream before
+ * reading out_host.  Other arguments and errors as jssa_decode_step_ex. */
+JSSA_API int jssa_decode_step_host(const jssa_dims *dims, const void *in_host, void *stage, void *K, void *V,
+                                   const float *P, void *Kt, const int32_t *seq_lens, const int32_t *pos_begin,
+                                   int k, int agg, float softmax_scale, const jssa_select_opts *opts,
+                                   int32_t *idx, int32_t *count, void *out, float *lse, void *out_host, void *ws,
+                                   size_t ws_bytes, jssa_stream_t stream);
+
 /* Per-query-head selection: a variant for measurement.  The method selects
  * one distinct token set per (batch, KV head), shared by the G query heads of
  * the KV head [ABS: distinct per-KV-head selections; NEWS Synopsis]; this

@@ -479,6 +479,48 @@ def test_bounded_waits_expire_with_a_status_and_the_context_stays_usable():
     check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
 
 
+def test_host_buffer_step_equals_device_step():
+    """jssa_decode_step_host (pinned host input block -> staged copy -> new
+    K/V rows written at pos -> decode step -> output copied to the host) gives
+    bit for bit what writing the rows on the device and calling
+    jssa_decode_step gives; the GQA and the latent form."""
+    for w, sl in ((W(B=3, T=5000, k=256, seed=130), [5000, 4000, 77]), (MW(T=3000, k=512, seed=131), [3000, 2500])):
+        (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+        pos = (sld - 1).clamp_min(0).contiguous()
+        g = torch.Generator().manual_seed(9)
+        kn = torch.randn((w.B, w.Hkv, w.d), generator=g).to(torch.bfloat16)
+        vn = None if Vd is None else torch.randn((w.B, w.Hkv, w.Dv), generator=g).to(torch.bfloat16)
+        # device path: write the rows, then the step
+        K1, V1 = Kd.clone(), None if Vd is None else Vd.clone()
+        Kt1 = ops.build_lowrank_cache(K1, Pd)
+        for b in range(w.B):
+            K1[b, int(pos[b])] = kn[b].to(DEV)
+            if V1 is not None:
+                V1[b, int(pos[b])] = vn[b].to(DEV)
+        o1, l1, i1, c1 = ops.decode_step(qd, K1, V1, Pd, Kt1, sld, pos, w.k, w.scale)
+        # host path
+        K2, V2 = Kd.clone(), None if Vd is None else Vd.clone()
+        Kt2 = ops.build_lowrank_cache(K2, Pd)
+        dims = ops.make_dims(qd, K2, V2, P=Pd, Kt=Kt2)
+        parts = [q.reshape(-1), kn.reshape(-1)] + ([] if vn is None else [vn.reshape(-1)])
+        blob = torch.cat(parts).view(torch.uint8)
+        in_host = torch.empty(ops.host_step_bytes(dims), dtype=torch.uint8).pin_memory()
+        assert in_host.numel() == blob.numel()
+        in_host.copy_(blob)
+        stage = torch.empty_like(in_host, device=DEV)
+        out_host = torch.empty(o1.shape, dtype=o1.dtype).pin_memory()
+        ws = ops.new_workspace(dims, w.k, ops.OP_DECODE_STEP, qd.device)
+        o2, l2 = torch.empty_like(o1), torch.empty_like(l1)
+        i2, c2 = torch.empty_like(i1), torch.empty_like(c1)
+        ops.decode_step_host(in_host, stage, K2, V2, Pd, Kt2, sld, pos, w.k, w.scale, out_host, ws, i2, c2, o2, l2,
+                             dims=dims)
+        torch.cuda.synchronize()
+        assert torch.equal(K1, K2) and (V1 is None or torch.equal(V1, V2)) and torch.equal(Kt1, Kt2)
+        assert torch.equal(i1, i2) and torch.equal(c1, c2)
+        assert torch.equal(o1.cpu(), out_host) and torch.equal(o1, o2)
+        assert ops.device_status(ws) == 0
+
+
 # --------------------------------------------- per-query-head selection
 @pytest.mark.parametrize("case", ["g4", "g8_r64", "g1", "fp32"])
 def test_select_heads_and_decode_heads_match_oracle(case, form):

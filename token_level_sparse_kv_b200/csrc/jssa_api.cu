@@ -1034,6 +1034,63 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     return JSSA_OK;
 }
 
+int jssa_host_step_bytes(const jssa_dims *dims, size_t *bytes) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if (!bytes) return fail(JSSA_ERR_INVALID_ARG, "bytes is NULL");
+    const size_t q = (size_t)dims->B * dims->Hq * dims->d, kr = (size_t)sh.BH * dims->d;
+    const size_t vr = sh.latent ? 0 : (size_t)sh.BH * dims->dv;
+    *bytes = (q + kr + vr) * sh.es_kv;
+    return JSSA_OK;
+}
+
+int jssa_decode_step_host(const jssa_dims *dims, const void *in_host, void *stage, void *K, void *V, const float *P,
+                          void *Kt, const int32_t *seq_lens, const int32_t *pos_begin, int k, int agg,
+                          float softmax_scale, const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *out,
+                          float *lse, void *out_host, void *ws, size_t ws_bytes, jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if (!in_host) return fail(JSSA_ERR_INVALID_ARG, "in_host is NULL");
+    if (!out_host) return fail(JSSA_ERR_INVALID_ARG, "out_host is NULL");
+    REQUIRE_PTR(stage);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(V);
+    size_t in_bytes = 0;
+    if ((st = jssa_host_step_bytes(dims, &in_bytes))) return st;
+    const size_t q_bytes = (size_t)dims->B * dims->Hq * dims->d * sh.es_kv;
+    const size_t krow = (size_t)dims->Hkv * dims->d * sh.es_kv, vrow = (size_t)dims->Hkv * dims->dv * sh.es_kv;
+    if (q_bytes % 16 || krow % 16 || vrow % 16)
+        return fail(JSSA_ERR_UNSUPPORTED, "host-buffer step needs rows of whole 16-byte chunks");
+    // argument checks of the step itself, before anything is enqueued
+    {
+        Layout L;
+        if ((st = check_k(k))) return st;
+        if ((st = check_attn_shape(dims, sh, true))) return st;
+        if ((st = check_opts(opts))) return st;
+        if (agg != JSSA_AGG_SUM && agg != JSSA_AGG_MAX) return fail(JSSA_ERR_INVALID_ARG, "bad agg %d", agg);
+        if ((st = build_layout(dims, sh, k, JSSA_OP_DECODE_STEP, agg, 0, choice_of(opts), L))) return st;
+        if ((st = check_ws(ws, ws_bytes, L))) return st;
+    }
+    if (dims->B == 0) return JSSA_OK;
+    cudaError_t e = cudaMemcpyAsync(stage, in_host, in_bytes, cudaMemcpyHostToDevice, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "copying the step's inputs to the device");
+    char *sg = static_cast<char *>(stage);
+    const char *k_new = sg + q_bytes;
+    const char *v_new = sh.latent ? nullptr : k_new + (size_t)dims->B * krow;
+    e = launch_place_rows(k_new, v_new, K, sh.latent ? nullptr : V, pos_begin, dims->B, dims->T_cap, krow, vrow,
+                          at<uint32_t>(ws, 0), S(stream), false);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the new-row write");
+    st = jssa_decode_step_ex(dims, stage, K, V, P, Kt, seq_lens, pos_begin, k, agg, softmax_scale, opts, idx, count,
+                             out, lse, ws, ws_bytes, stream);
+    if (st) return st;
+    e = cudaMemcpyAsync(out_host, out, (size_t)dims->B * dims->Hq * dims->dv * sh.es_kv, cudaMemcpyDeviceToHost,
+                        S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "copying the output to the host");
+    return JSSA_OK;
+}
+
 int jssa_select_heads(const jssa_dims *dims, const void *q, const float *P, const void *Kt, const int32_t *seq_lens,
                       int k, const jssa_select_opts *opts, int32_t *idx, int32_t *count, void *ws, size_t ws_bytes,
                       jssa_stream_t stream) {

@@ -173,7 +173,7 @@ __device__ __forceinline__ bool flag_wait_bounded(const volatile unsigned *word,
 }
 
 // Suspend-time hint of the waits below (ns; 0 = the hardware's own limit).
-constexpr uint32_t kParkNs = 0;
+constexpr uint32_t kParkNs = 20000;
 
 // Bounded mbarrier wait that also gives up when another role of the CTA
 // raised the abort flag.  Each poll is a try_wait, which may suspend the

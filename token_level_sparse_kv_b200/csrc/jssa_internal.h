@@ -226,6 +226,11 @@ int device_sm_count();
 // the requested size grows).
 cudaError_t ensure_smem(const void *kern, size_t smem);
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype);
+// Write each batch row's new K row (row_k_bytes, all KV heads) and V row into
+// the cache at position pos[b]; v_new / V null for a latent cache.
+cudaError_t launch_place_rows(const void *k_new, const void *v_new, void *K, void *V, const int32_t *pos, int B,
+                              int T_cap, size_t row_k_bytes, size_t row_v_bytes, uint32_t *status, cudaStream_t s,
+                              bool pdl);
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s, bool pdl, int kv_dtype, int kt_dtype);
 cudaError_t launch_prep(const AppendArgs &ap, const ProjArgs &pj, cudaStream_t s, bool pdl, int kv_dtype,
                         int kt_dtype);

@@ -261,6 +261,28 @@ __global__ void __launch_bounds__(kPrepClThreads) prep_cluster_kernel(AppendArgs
     }
 }
 
+// The new token's K and V rows of each batch row, staged contiguously
+// ([B, Hkv, d] then [B, Hkv, dv]), written into the cache at pos[b] (the
+// host-buffer decode step).  A position outside [0, T_cap) is skipped and
+// flagged.  16-byte copies; one CTA per batch row.
+__global__ void __launch_bounds__(128) place_rows_kernel(const uint4 *k_new, const uint4 *v_new, uint4 *K, uint4 *V,
+                                                         const int32_t *pos, int T_cap, int row_k16, int row_v16,
+                                                         uint32_t *status) {
+    pdl_trigger();
+    pdl_wait();
+    const int b = blockIdx.x;
+    const int p = pos[b];
+    if (p < 0 || p >= T_cap) {
+        if (threadIdx.x == 0 && status) atomicOr(status, (uint32_t)JSSA_DEV_POS);
+        return;
+    }
+    for (int c = threadIdx.x; c < row_k16; c += blockDim.x)
+        K[((size_t)b * T_cap + p) * row_k16 + c] = k_new[(size_t)b * row_k16 + c];
+    if (V)
+        for (int c = threadIdx.x; c < row_v16; c += blockDim.x)
+            V[((size_t)b * T_cap + p) * row_v16 + c] = v_new[(size_t)b * row_v16 + c];
+}
+
 size_t prep_smem(int rows, int d, int r) {
     return ((size_t)rows * d + (size_t)rows * r * (d / kChunk)) * sizeof(float);
 }
@@ -289,6 +311,14 @@ cudaError_t launch_append(const AppendArgs &a0, cudaStream_t s, bool pdl, int kv
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
     return launch_kernel(k, grid, dim3(prep_threads(a.d)), smem, s, pdl, a);
+}
+
+cudaError_t launch_place_rows(const void *k_new, const void *v_new, void *K, void *V, const int32_t *pos, int B,
+                              int T_cap, size_t row_k_bytes, size_t row_v_bytes, uint32_t *status, cudaStream_t s,
+                              bool pdl) {
+    return launch_kernel(place_rows_kernel, dim3(B), dim3(128), 0, s, pdl, static_cast<const uint4 *>(k_new),
+                         static_cast<const uint4 *>(v_new), static_cast<uint4 *>(K), static_cast<uint4 *>(V), pos,
+                         T_cap, (int)(row_k_bytes / 16), (int)(row_v_bytes / 16), status);
 }
 
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype) {

@@ -73,6 +73,11 @@ def lib():
     L.jssa_decode_step_ex.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.jssa_plan_info.restype = i32
     L.jssa_plan_info.argtypes = [D, i32, i32, i32, ctypes.POINTER(i32), ctypes.c_char_p, sz]
+    L.jssa_host_step_bytes.restype = i32
+    L.jssa_host_step_bytes.argtypes = [D, ctypes.POINTER(sz)]
+    L.jssa_decode_step_host.restype = i32
+    L.jssa_decode_step_host.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, vp,
+                                        sz, vp]
     L.jssa_select_heads.restype = i32
     L.jssa_select_heads.argtypes = [D, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
     L.jssa_indexed_decode_heads.restype = i32
@@ -380,6 +385,33 @@ def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=N
                                      _opts(n_sink, n_recent, form, unfused), _p(idx), _p(count), _p(out), _p(lse),
                                      _p(ws), ws.numel(), _stream(q.device)))
     return out, lse, idx, count
+
+
+def host_step_bytes(dims: Dims) -> int:
+    """Bytes of the packed host input of decode_step_host: q [B,Hq,d], then the
+    new K rows [B,Hkv,d], then the new V rows [B,Hkv,dv] (none for a latent cache)."""
+    n = ctypes.c_size_t(0)
+    _check(lib().jssa_host_step_bytes(ctypes.byref(dims), ctypes.byref(n)))
+    return int(n.value)
+
+
+def decode_step_host(in_host, stage, K, V, P, Kt, seq_lens, pos_begin, k, scale, out_host, ws, idx, count, out, lse,
+                     agg=AGG_SUM, dims=None):
+    """One step driven from (pinned) host memory through jssa_decode_step_host:
+    in_host (uint8, host_step_bytes) is copied to the device buffer stage, the
+    new K/V rows are written at pos_begin, the step runs, and out is copied to
+    out_host.  Asynchronous: synchronise the stream before reading out_host."""
+    _cuda(stage, K, V, P, Kt, seq_lens, pos_begin, ws, idx, count, out, lse)
+    if dims is None:
+        B, T_cap, Hkv, d = K.shape
+        Hq = out.shape[1]
+        dv = out.shape[2]
+        dims = Dims(B, Hq, Hkv, d, dv, P.shape[2], T_cap, _dt(K), _dt(Kt))
+    _check(lib().jssa_decode_step_host(ctypes.byref(dims), ctypes.c_void_p(in_host.data_ptr()), _p(stage), _p(K),
+                                       _p(K if V is None else V), _p(P), _p(Kt), _p(seq_lens), _p(pos_begin), int(k),
+                                       int(agg), float(scale), None, _p(idx), _p(count), _p(out), _p(lse),
+                                       ctypes.c_void_p(out_host.data_ptr()), _p(ws), ws.numel(), _stream(K.device)))
+    return out_host
 
 
 class StepGraph:
