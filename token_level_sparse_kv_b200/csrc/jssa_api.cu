@@ -228,7 +228,7 @@ int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout
     if (sh.latent && src != ATT_INDEXED) {
         cudaError_t e = plan_mla_range(d->B, npos, &L.mp);
         if (e != cudaSuccess) return cuda_fail(e, "planning the latent-cache range pass");
-        L.part_o = take(L.total, (size_t)d->B * L.mp.splits * d->Hq * d->dv * 4);
+        L.part_o = take(L.total, (size_t)d->B * L.mp.splits * d->Hq * d->dv * 2);  // bf16
         L.part_ml = take(L.total, (size_t)d->B * L.mp.splits * d->Hq * 2 * 4);
         L.att_ctr = take(L.total, (size_t)sh.BH * 4);
         return JSSA_OK;
@@ -236,7 +236,7 @@ int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout
     if (sh.latent) {
         L.ap = AttnPlan();
         L.ap.splits = mla_splits(npos);
-        L.part_o = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * d->dv * 4);
+        L.part_o = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * d->dv * 2);  // bf16
         L.part_ml = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * 2 * 4);
         L.att_ctr = take(L.total, (size_t)sh.BH * 4);
         return JSSA_OK;
@@ -546,7 +546,7 @@ int run_mla_range(const jssa_dims *d, const void *q, const void *K, const int32_
     a.T_cap = d->T_cap;
     a.k = k;
     a.scale_log2 = scale * 1.4426950408889634f;
-    a.part_o = at<float>(ws, L.part_o);
+    a.part_o = at<__nv_bfloat16>(ws, L.part_o);
     a.part_ml = at<float>(ws, L.part_ml);
     a.out = out;
     a.lse = lse;
@@ -570,7 +570,7 @@ int run_mla(const jssa_dims *d, const void *q, const void *K, const int32_t *idx
     a.B = d->B;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.splits = L.ap.splits;
-    a.part_o = at<float>(ws, L.part_o);
+    a.part_o = at<__nv_bfloat16>(ws, L.part_o);
     a.part_ml = at<float>(ws, L.part_ml);
     a.out = out;
     a.lse = lse;

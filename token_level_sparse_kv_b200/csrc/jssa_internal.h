@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -153,7 +154,7 @@ struct MlaRangeArgs {
     int B, T_cap, k;
     int row_tiles, splits;    // plan: 128-token tiles per row; CTAs (x 2 head halves) per row
     float scale_log2;
-    float *part_o;            // [B, splits, 128, 512]
+    __nv_bfloat16 *part_o;    // [B, splits, 128, 512] bf16 (unnormalised O of each split)
     float *part_ml;           // [B, splits, 128, 2]
     void *out;                // [B, 128, 512] bf16
     float *lse;               // [B, 128] or null
@@ -200,7 +201,7 @@ struct MlaArgs {
     int k, T_cap, B;
     float scale_log2;
     int splits;               // CTAs per batch row (128 tokens each)
-    float *part_o;            // [B, splits, 128, 512]
+    __nv_bfloat16 *part_o;    // [B, splits, 128, 512] bf16 (unnormalised O of each split)
     float *part_ml;           // [B, splits, 128, 2]
     void *out;                // [B, 128, 512] bf16
     float *lse;               // [B, 128] or null

@@ -269,24 +269,32 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
             }
             if (a.lse) a.lse[(size_t)b * kH + h] = l > 0.f ? (m + log2f(l)) * 0.693147180559945309417f : -INFINITY;
         } else {
-            // unnormalised partial O, turned around per warp in shared memory (the
-            // K blocks are free once the second product is done) so that every
-            // store writes whole 128-byte rows: block [32 heads][32 columns]
-            float *tb = reinterpret_cast<float *>(sK) + warp * (32 * 33);
-            float *po = a.part_o + (((size_t)b * a.splits + split) * kH + warp * 32) * kDv;
+            // unnormalised partial O in bf16, turned around per warp in shared
+            // memory (the K blocks are free once the second product is done) so
+            // that every store writes whole 128-byte rows: block [32 heads][64 columns]
+            float *tb = reinterpret_cast<float *>(sK) + warp * (32 * 65);
+            __nv_bfloat16 *po = a.part_o + (((size_t)b * a.splits + split) * kH + warp * 32) * kDv;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kDv; c0 += 32) {
+            for (int c0 = 0; c0 < kDv; c0 += 64) {
                 float v[32];
                 tmem_ld32(lane_base + c0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) tb[lane * 33 + j] = v[j];
+                for (int j = 0; j < 32; ++j) tb[lane * 65 + j] = v[j];
+                tmem_ld32(lane_base + c0 + 32, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) tb[lane * 65 + 32 + j] = v[j];
                 __syncwarp();
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int row = i * 4 + (lane >> 3), col = (lane & 7) * 4;
-                    const float *src = tb + row * 33 + col;
-                    *reinterpret_cast<float4 *>(po + (size_t)row * kDv + c0 + col) =
-                        make_float4(src[0], src[1], src[2], src[3]);
+                    const int row = i * 4 + (lane >> 3), col = (lane & 7) * 8;
+                    const float *src = tb + row * 65 + col;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 pk = __floats2bfloat162_rn(src[2 * e], src[2 * e + 1]);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&pk);
+                    }
+                    *reinterpret_cast<uint4 *>(po + (size_t)row * kDv + c0 + col) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
                 __syncwarp();
             }
@@ -314,30 +322,30 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
     float L = 0.f, o[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) o[j] = 0.f;
-    const float *pbase = a.part_o + ((size_t)b * ns * kH + h) * kDv + c0;
-    for (int s0 = 0; s0 < ns; s0 += 4) {
-        float2 ml[4];
-        float4 v[4][4];
+    const __nv_bfloat16 *pbase = a.part_o + ((size_t)b * ns * kH + h) * kDv + c0;
+    for (int s0 = 0; s0 < ns; s0 += 8) {
+        float2 ml[8];
+        uint4 v[8][2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const bool in = s0 + u < ns;
             ml[u] = in ? pml[(size_t)(s0 + u) * kH] : make_float2(-INFINITY, 0.f);
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd)
-                v[u][qd] = in ? reinterpret_cast<const float4 *>(pbase + (size_t)(s0 + u) * kH * kDv)[qd]
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int qd = 0; qd < 2; ++qd)
+                v[u][qd] = in ? reinterpret_cast<const uint4 *>(pbase + (size_t)(s0 + u) * kH * kDv)[qd]
+                              : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             if (ml[u].x == -INFINITY) continue;  // an empty split (or past the last)
             const float w = exp2f(ml[u].x - M);
             L = fmaf(ml[u].y, w, L);
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-                o[4 * qd] = fmaf(v[u][qd].x, w, o[4 * qd]);
-                o[4 * qd + 1] = fmaf(v[u][qd].y, w, o[4 * qd + 1]);
-                o[4 * qd + 2] = fmaf(v[u][qd].z, w, o[4 * qd + 2]);
-                o[4 * qd + 3] = fmaf(v[u][qd].w, w, o[4 * qd + 3]);
+            for (int qd = 0; qd < 2; ++qd) {
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(v[u][qd], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[8 * qd + e] = fmaf(f[e], w, o[8 * qd + e]);
             }
         }
     }

@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kThr, 1)
                 for (int j = 0; j < 32; ++j) {
                     const int h = hbase + half * 32 + j;
                     if (part) {
-                        a.part_o[(((size_t)b * a.splits + split) * kH + h) * kDv + dv] = v[j];
+                        a.part_o[(((size_t)b * a.splits + split) * kH + h) * kDv + dv] = __float2bfloat16_rn(v[j]);
                     } else {
                         const float l = lsum[half * 32 + j];
                         static_cast<__nv_bfloat16 *>(a.out)[((size_t)b * kH + h) * kDv + dv] =
