@@ -521,3 +521,54 @@ def test_attend_heads_reduces_to_attend_and_to_loops():
                 assert abs(l[b, hq] - rl[0]) < 1e-12
             else:
                 assert np.all(o[b, hq] == 0) and np.isneginf(l[b, hq])
+
+
+# ------------------------------------------ calibration of P (NEXT-4 reading)
+from oracle import calib  # noqa: E402
+
+
+def test_calib_key_positions_rule():
+    assert calib.key_positions(5, 8).tolist() == [0, 1, 2, 3, 4]
+    p = calib.key_positions(1000, 7)
+    assert p[0] == 0 and np.all(np.diff(p) > 0) and p[-1] < 1000
+    assert p.tolist() == [j * 1000 // 7 for j in range(7)]
+
+
+def test_calib_moments_match_explicit_loops():
+    w = Workload("t", B=2, Hq=4, Hkv=2, d=4, T=9, r=2, k=2, seed=140)
+    q, K, V, P, _ = make_inputs(w)
+    sl = torch.tensor([9, 5], dtype=torch.int32)
+    Sq, Sk = calib.moments(q[:1], K, sl, n_keys=3)
+    qf, Kf = f64(q), f64(K)
+    for h in range(2):
+        ref_q = [[0.0] * 4 for _ in range(4)]
+        for g in (2 * h, 2 * h + 1):
+            for i in range(4):
+                for j in range(4):
+                    ref_q[i][j] += qf[0, g, i] * qf[0, g, j]
+        np.testing.assert_allclose(Sq[h], ref_q, rtol=1e-15, atol=1e-15)
+        ref_k = [[0.0] * 4 for _ in range(4)]
+        for b, tb in ((0, 9), (1, 5)):
+            for t in ([0, 3, 6] if tb == 9 else [0, 1, 3]):
+                for i in range(4):
+                    for j in range(4):
+                        ref_k[i][j] += Kf[b, t, h, i] * Kf[b, t, h, j]
+        np.testing.assert_allclose(Sk[h], ref_k, rtol=1e-15, atol=1e-15)
+    M = calib.joint_matrix(Sq, Sk)
+    np.testing.assert_allclose([np.trace(M[h]) for h in range(2)], [2.0, 2.0], rtol=1e-14)
+    np.testing.assert_allclose(M, np.transpose(M, (0, 2, 1)), rtol=0, atol=0)
+
+
+def test_calib_recovers_a_planted_subspace():
+    # queries and keys drawn inside a 3-dim subspace U of R^16: M has rank 3
+    # and the top-r (r = 5) basis contains U exactly (principal angles 0)
+    g = torch.Generator().manual_seed(141)
+    d, r0, r = 16, 3, 5
+    U = torch.linalg.qr(torch.randn(d, r0, generator=g, dtype=torch.float64))[0]
+    q = (torch.randn(6, 2, r0, generator=g, dtype=torch.float64) @ U.T).to(torch.float32)
+    K = (torch.randn(1, 50, 1, r0, generator=g, dtype=torch.float64) @ U.T).to(torch.float32)
+    Pc, lam, M = calib.calibrate(q, K, torch.tensor([50], dtype=torch.int32), r, n_keys=20)
+    Ud = U.numpy()
+    assert abs(np.linalg.norm(Ud.T @ Pc[0]) ** 2 - r0) < 1e-9
+    assert np.all(lam[0, r0:] < 1e-9)
+    np.testing.assert_allclose(calib.captured_energy(M, Pc), lam[:, :r].sum(1), rtol=1e-12)
