@@ -405,6 +405,45 @@ def measure_decode_loop(dev, n_layers, steps, stream):
     return res
 
 
+def calibration_recall(w, q, K, P, sl, dev, stream, n_keys=4096, iters=30):
+    """Selection quality against the exact top-k of the full-width group
+    scores (sum_g q_g . K_t, by the library's own selection with an identity
+    basis, r = d): recall of the k selected tokens per (b, h) with the random
+    orthonormal basis and with the basis calibrated from the step's queries
+    and sampled keys (jssa_calibrate_basis), and the calibration's time."""
+    import torch
+
+    from token_level_sparse_kv_b200 import ops
+
+    eye = torch.eye(w.d, dtype=torch.float32, device=dev).expand(w.Hkv, w.d, w.d).contiguous()
+    Kt_full = ops.build_lowrank_cache(K, eye)
+    idx_exact, _ = ops.select(q, eye, Kt_full, sl, w.k)
+    del Kt_full
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ops.calibrate_basis(q, K, sl, P, n_keys=n_keys, iters=iters)  # warm (planning)
+    a.record(stream)
+    P_cal = ops.calibrate_basis(q, K, sl, P, n_keys=n_keys, iters=iters)
+    b.record(stream)
+    torch.cuda.synchronize()
+    cal_ms = a.elapsed_time(b)
+
+    def recall(basis):
+        Kt = ops.build_lowrank_cache(K, basis)
+        idx, _ = ops.select(q, basis, Kt, sl, w.k)
+        hit = (idx.unsqueeze(-1) == idx_exact.unsqueeze(-2)).any(-1) & (idx >= 0)
+        r = float(hit.sum().item() / max(1, int((idx_exact >= 0).sum().item())))
+        del Kt
+        torch.cuda.empty_cache()
+        return r
+
+    res = {"recall_random_P": recall(P), "recall_calibrated_P": recall(P_cal), "calibration_ms": cal_ms,
+           "samples": "the step's queries (%d rows) and %d evenly spaced keys per batch row; %d iterations"
+                      % (w.B, n_keys, iters),
+           "reference": "exact top-k of the full-width group scores (identity basis, r = d)"}
+    torch.cuda.synchronize()
+    return res
+
+
 def per_head_comparison(w, q, K, V, P, Kt, sl, pos, dims, dev, stream, flush_buf, steps, world, use_graph):
     """The per-query-head selection variant (every query head its own top-k)
     against the method's per-KV-head selection on the same inputs: step time
@@ -632,6 +671,8 @@ def run_jssa(args, world, rank, local):
             med = max_over_ranks(percentile(d, 0.5), world)
             res[name] = {"steps_per_s": world / med, "ms_per_step": med * 1e3, "latency": latency_summary(d),
                          "launch": "cuda graph replay" if graphs else "eager"}
+        if not w.latent and w.d <= 128:
+            res["calibration_of_P"] = calibration_recall(w, q, K, P, sl, dev, stream)
         if not w.latent:
             res["per_query_head_selection"] = per_head_comparison(w, q, K, Vv, P, Kt, sl, pos, dims, dev, stream,
                                                                   flush_buf, cmp_steps, world, graphs is not None)

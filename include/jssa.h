@@ -124,7 +124,8 @@ typedef enum {
     JSSA_OP_GATHER_THEN_DENSE = 6,
     JSSA_OP_DECODE_STEP = 7,
     JSSA_OP_SELECT_HEADS = 8,        /* jssa_select_heads */
-    JSSA_OP_INDEXED_DECODE_HEADS = 9 /* jssa_indexed_decode_heads */
+    JSSA_OP_INDEXED_DECODE_HEADS = 9, /* jssa_indexed_decode_heads */
+    JSSA_OP_CALIBRATE = 10            /* jssa_calibrate_basis (k ignored) */
 } jssa_op;
 
 typedef struct {
@@ -308,6 +309,25 @@ JSSA_API int jssa_decode_step_host(const jssa_dims *dims, const void *in_host, v
                                    int k, int agg, float softmax_scale, const jssa_select_opts *opts,
                                    int32_t *idx, int32_t *count, void *out, float *lse, void *out_host, void *ws,
                                    size_t ws_bytes, jssa_stream_t stream);
+
+/* Calibration of the shared basis P from sampled queries and keys: the step
+ * before the decode path [ABS: a spectral solution for the shared query-key
+ * subspace; NEWS Interpretation para 2: queries and keys preserved jointly].
+ * The pages give no objective or formula; the reading computed is, per KV
+ * head h,
+ *   S_q = sum of q q^T over the rows of q_cal [n_q, Hq, d] of the head's G
+ *         query heads,   S_k = sum of k k^T over n_keys sampled tokens per
+ *         batch row (t_j = floor(j * T_b / n_keys), j < n_keys; all t < T_b
+ *         when T_b <= n_keys),
+ *   M = S_q / tr(S_q) + S_k / tr(S_k)  (fp32),
+ *   P_out[h] = an orthonormal basis of the dominant r-dimensional
+ *              eigen-subspace of M, by `iters` rounds of subspace iteration
+ *              X <- orth(M X) from P_init[h] (Gram-Schmidt applied twice).
+ * P_init, P_out: [Hkv, d, r] fp32 (may not alias).  r <= 64; d in {64, 128,
+ * 256}; GQA shapes.  Workspace: jssa_workspace_size(.., JSSA_OP_CALIBRATE). */
+JSSA_API int jssa_calibrate_basis(const jssa_dims *dims, const void *q_cal, int n_q, const void *K,
+                                  const int32_t *seq_lens, int n_keys, int iters, const float *P_init,
+                                  float *P_out, void *ws, size_t ws_bytes, jssa_stream_t stream);
 
 /* Per-query-head selection: a variant for measurement.  The method selects
  * one distinct token set per (batch, KV head), shared by the G query heads of

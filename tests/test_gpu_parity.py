@@ -521,6 +521,48 @@ def test_host_buffer_step_equals_device_step():
         assert ops.device_status(ws) == 0
 
 
+# ------------------------------------------------------- calibration of P
+@pytest.mark.parametrize("d,r,Hkv,G", [(128, 32, 2, 4), (256, 64, 2, 8), (64, 8, 3, 1)])
+def test_calibrated_basis_keeps_the_dominant_joint_energy(d, r, Hkv, G):
+    """jssa_calibrate_basis against the oracle's fp64 statement of the same
+    reading: the GPU basis is orthonormal and keeps at least 99.9% of the
+    joint energy the exact top-r eigen-subspace keeps (tr(P^T M P) with the
+    oracle's M; any basis of a dominant subspace does, even where eigenvalues
+    of the noise bulk are too close for the iteration to single one out)."""
+    from oracle import calib
+
+    w = W(B=3, Hq=G * Hkv, Hkv=Hkv, d=d, r=r, T=3000, k=8, seed=150 + d)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=[3000, 2000, 700])
+    Pc = ops.calibrate_basis(qd, Kd, sld, Pd, n_keys=512, iters=40)
+    torch.cuda.synchronize()
+    Pg = host(Pc).double().numpy()
+    Pref, lam, M = calib.calibrate(q, K, sl, r, 512)
+    for h in range(Hkv):
+        np.testing.assert_allclose(Pg[h].T @ Pg[h], np.eye(r), atol=2e-5)
+    best = lam[:, :r].sum(1)
+    got = calib.captured_energy(M, Pg)
+    assert np.all(got >= 0.999 * best), (got, best)
+
+
+def test_calibrated_basis_recovers_a_planted_subspace():
+    """Queries and keys drawn inside a 5-dim subspace U: the calibrated basis
+    (r = 16) contains U (||U^T P||_F^2 = 5), from a random start."""
+    g = torch.Generator().manual_seed(151)
+    d, r0, r, Hkv, G = 128, 5, 16, 2, 4
+    U = torch.linalg.qr(torch.randn(Hkv, d, r0, generator=g, dtype=torch.float64))[0]
+    q = torch.einsum("nhgz,hdz->nhgd", torch.randn(2, Hkv, G, r0, generator=g, dtype=torch.float64), U)
+    K = torch.einsum("bthz,hdz->bthd", torch.randn(2, 600, Hkv, r0, generator=g, dtype=torch.float64), U)
+    qd = q.reshape(2, Hkv * G, d).to(torch.bfloat16).contiguous().to(DEV)
+    Kd = K.to(torch.bfloat16).contiguous().to(DEV)
+    P0 = torch.linalg.qr(torch.randn(Hkv, d, r, generator=g, dtype=torch.float64))[0].float().contiguous().to(DEV)
+    sl = torch.tensor([600, 450], dtype=torch.int32, device=DEV)
+    Pc = ops.calibrate_basis(qd, Kd, sl, P0, n_keys=256, iters=30)
+    torch.cuda.synchronize()
+    for h in range(Hkv):
+        cap = float((U[h].T @ host(Pc[h]).double()).norm() ** 2)
+        assert abs(cap - r0) < 1e-3, cap
+
+
 # --------------------------------------------- per-query-head selection
 @pytest.mark.parametrize("case", ["g4", "g8_r64", "g1", "fp32"])
 def test_select_heads_and_decode_heads_match_oracle(case, form):

@@ -158,6 +158,8 @@ int check_heads_shape(const jssa_dims *d, const Shape &sh) {
 struct Layout {
     size_t qproj = 0, cand_key = 0, cand_idx = 0, cand_cnt = 0, sel_ctr = 0;
     size_t part_o = 0, part_ml = 0, att_ctr = 0, gcount = 0;
+    size_t cal_sk = 0, cal_sq = 0, cal_m = 0;
+    int cal_chunks = 0;
     size_t total = 256;  // [0, 256): status word
     ScanPlan sp{};
     AttnPlan ap{};
@@ -354,6 +356,14 @@ int build_layout_uncached(const jssa_dims *d, const Shape &sh, int k, int op, in
             st = layout_attend(d, sh, ATT_RANGE_BH, k, L);
             if (st == JSSA_OK) L.gcount = take(L.total, (size_t)sh.BH * 4);
             break;
+        case JSSA_OP_CALIBRATE: {
+            const size_t dd = (size_t)d->d * d->d;
+            L.cal_chunks = calib_chunks(d->Hkv);
+            L.cal_sk = take(L.total, (size_t)d->Hkv * L.cal_chunks * dd * 4);
+            L.cal_sq = take(L.total, (size_t)d->Hkv * dd * 4);
+            L.cal_m = take(L.total, (size_t)d->Hkv * dd * 4);
+            break;
+        }
         case JSSA_OP_SELECT_HEADS: {
             L.qproj = take(L.total, (size_t)sh.BH * sh.G * d->r * 4);  // per-head projections
             jssa_dims dh;
@@ -1031,6 +1041,50 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     a.k = k;
     e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the indexed decode");
+    return JSSA_OK;
+}
+
+int jssa_calibrate_basis(const jssa_dims *dims, const void *q_cal, int n_q, const void *K, const int32_t *seq_lens,
+                         int n_keys, int iters, const float *P_init, float *P_out, void *ws, size_t ws_bytes,
+                         jssa_stream_t stream) {
+    Shape sh;
+    int st = check_dims(dims, &sh);
+    if (st) return st;
+    if (sh.latent) return fail(JSSA_ERR_UNSUPPORTED, "calibration is for GQA shapes");
+    if (dims->r > 64) return fail(JSSA_ERR_UNSUPPORTED, "calibration needs r <= 64 (got %d)", dims->r);
+    if (n_q < 0 || n_keys < 0 || iters < 0 || iters > 1000)
+        return fail(JSSA_ERR_INVALID_ARG, "bad counts (n_q=%d n_keys=%d iters=%d)", n_q, n_keys, iters);
+    if (n_q > 0) REQUIRE_PTR(q_cal);
+    REQUIRE_PTR(K);
+    REQUIRE_PTR(seq_lens);
+    REQUIRE_PTR(P_init);
+    REQUIRE_PTR(P_out);
+    if (P_init == P_out) return fail(JSSA_ERR_INVALID_ARG, "P_init and P_out alias");
+    Layout L;
+    if ((st = build_layout(dims, sh, 1, JSSA_OP_CALIBRATE, 0, 0, Choice(), L))) return st;
+    if ((st = check_ws(ws, ws_bytes, L))) return st;
+    CalibArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q_cal;
+    a.K = K;
+    a.seq_lens = seq_lens;
+    a.B = dims->B;
+    a.Hq = dims->Hq;
+    a.Hkv = dims->Hkv;
+    a.T_cap = dims->T_cap;
+    a.Nq = n_q;
+    a.n_keys = n_keys;
+    a.chunks = L.cal_chunks;
+    a.r = dims->r;
+    a.iters = iters;
+    a.P_init = P_init;
+    a.P_out = P_out;
+    a.Sk = at<float>(ws, L.cal_sk);
+    a.Sq = at<float>(ws, L.cal_sq);
+    a.M = at<float>(ws, L.cal_m);
+    a.status = at<uint32_t>(ws, 0);
+    cudaError_t e = launch_calib(a, dims->kv_dtype, dims->d, S(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching the calibration");
     return JSSA_OK;
 }
 

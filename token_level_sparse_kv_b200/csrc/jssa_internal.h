@@ -144,6 +144,22 @@ cudaError_t plan_dense(int d, int B, int Hkv, int row_len, DensePlan *p);
 cudaError_t launch_dense(const DensePlan &p, const DenseArgs &a, const void *K, const void *V, int d,
                          cudaStream_t s, bool pdl);
 
+// ----------------------------------------------------------- calibration ---
+struct CalibArgs {
+    const void *q;            // [Nq, Hq, d] calibration queries (kv dtype)
+    const void *K;            // [B, T_cap, Hkv, d]
+    const int32_t *seq_lens;  // [B]
+    int B, Hq, Hkv, T_cap, Nq, n_keys, chunks, r, iters;
+    const float *P_init;      // [Hkv, d, r] start of the subspace iteration
+    float *P_out;             // [Hkv, d, r]
+    float *Sk;                // [Hkv, chunks, d, d] partial key sums
+    float *Sq;                // [Hkv, d, d] query sums
+    float *M;                 // [Hkv, d, d] the joint matrix
+    uint32_t *status;
+};
+int calib_chunks(int Hkv);
+cudaError_t launch_calib(const CalibArgs &a, int kv_dtype, int d, cudaStream_t s);
+
 // ------------------------------------------- latent cache, token range ---
 // Attention of the 128 heads of a latent cache over [0, T_b) of the cache
 // ([B, T_cap, 1, 576]) or [0, count[b]) of a gathered buffer ([B, k, 576]).

@@ -24,7 +24,7 @@ BF16, FP32 = 0, 1
 AGG_SUM, AGG_MAX = 0, 1
 OP_APPEND, OP_SCORE, OP_TOPK, OP_SELECT, OP_INDEXED_DECODE, OP_DENSE_DECODE, OP_GATHER_THEN_DENSE, OP_DECODE_STEP = \
     range(8)
-OP_SELECT_HEADS, OP_INDEXED_DECODE_HEADS = 8, 9
+OP_SELECT_HEADS, OP_INDEXED_DECODE_HEADS, OP_CALIBRATE = 8, 9, 10
 DEV_SEQLEN, DEV_INDEX, DEV_POS, DEV_TIMEOUT = 1, 2, 4, 8
 
 
@@ -73,6 +73,8 @@ def lib():
     L.jssa_decode_step_ex.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.jssa_plan_info.restype = i32
     L.jssa_plan_info.argtypes = [D, i32, i32, i32, ctypes.POINTER(i32), ctypes.c_char_p, sz]
+    L.jssa_calibrate_basis.restype = i32
+    L.jssa_calibrate_basis.argtypes = [D, vp, i32, vp, vp, i32, i32, vp, vp, vp, sz, vp]
     L.jssa_host_step_bytes.restype = i32
     L.jssa_host_step_bytes.argtypes = [D, ctypes.POINTER(sz)]
     L.jssa_decode_step_host.restype = i32
@@ -385,6 +387,23 @@ def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=N
                                      _opts(n_sink, n_recent, form, unfused), _p(idx), _p(count), _p(out), _p(lse),
                                      _p(ws), ws.numel(), _stream(q.device)))
     return out, lse, idx, count
+
+
+def calibrate_basis(q_cal, K, seq_lens, P_init, n_keys, iters=30, ws=None):
+    """Calibrated basis [Hkv, d, r] fp32 (jssa_calibrate_basis): the dominant
+    r-dim eigen-subspace of S_q/tr(S_q) + S_k/tr(S_k) per KV head, from the
+    query rows q_cal [N, Hq, d] and n_keys sampled keys per batch row, by
+    `iters` rounds of subspace iteration from P_init."""
+    _cuda(q_cal, K, seq_lens, P_init)
+    N, Hq, d = q_cal.shape
+    B, T_cap, Hkv, _ = K.shape
+    r = P_init.shape[2]
+    dims = Dims(B, Hq, Hkv, d, d, r, T_cap, _dt(K), BF16)
+    P_out = torch.empty_like(P_init)
+    ws = _ws(ws, dims, 1, OP_CALIBRATE, K.device)
+    _check(lib().jssa_calibrate_basis(ctypes.byref(dims), _p(q_cal), int(N), _p(K), _p(seq_lens), int(n_keys),
+                                      int(iters), _p(P_init), _p(P_out), _p(ws), ws.numel(), _stream(K.device)))
+    return P_out
 
 
 def host_step_bytes(dims: Dims) -> int:
