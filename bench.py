@@ -405,6 +405,42 @@ def measure_decode_loop(dev, n_layers, steps, stream):
     return res
 
 
+def screening_comparison(w, qs, K, V, P, Kt, sl, pos, dims, dev, stream, flush_buf, steps, world, use_graph):
+    """The decode step with exact block screening (per-128-token norm bounds
+    of the low-rank cache): its time and the tiles it skipped per step, on
+    the same inputs as the timed step (results are bit-identical)."""
+    import torch
+
+    from token_level_sparse_kv_b200 import ops
+
+    nrm = ops.block_norms(Kt)
+    ws = ops.new_workspace(dims, w.k, ops.OP_DECODE_STEP, dev)
+    idx = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.Hkv), dtype=torch.int32, device=dev)
+    out = torch.empty((w.B, w.Hq, w.Dv), dtype=qs[0].dtype, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+
+    def step(i):
+        ops.decode_step(qs[i & 3], K, V, P, Kt, sl, pos, w.k, w.scale, ws=ws, idx=idx, count=cnt, out=out, lse=lse,
+                        block_norms=nrm)
+
+    for i in range(3):
+        step(i)
+    rep_fn = graphed(step, dev) if use_graph else step
+    for i in range(3):
+        rep_fn(i)
+    torch.cuda.synchronize()
+    before = ops.skip_count(ws)
+    d = time_steps(rep_fn, steps, stream, flush_buf)
+    skipped = ops.skip_count(ws) - before
+    med = max_over_ranks(percentile(d, 0.5), world)
+    tiles = w.B * w.Hkv * ((w.T * w.r * 2 + 32767) // 32768)
+    return {"steps_per_s": world / med, "ms_per_step": med * 1e3, "skipped_tiles_per_step": skipped / steps,
+            "tiles_per_step": tiles,
+            "note": "Cauchy-Schwarz bound ||qbar|| * max ||Kt_t|| per 128-token block against the segment's k-th "
+                    "key; on these inputs the bound rarely falls below it"}
+
+
 def calibration_recall(w, q, K, P, sl, dev, stream, n_keys=4096, iters=30):
     """Selection quality against the exact top-k of the full-width group
     scores (sum_g q_g . K_t, by the library's own selection with an identity
@@ -671,6 +707,9 @@ def run_jssa(args, world, rank, local):
             med = max_over_ranks(percentile(d, 0.5), world)
             res[name] = {"steps_per_s": world / med, "ms_per_step": med * 1e3, "latency": latency_summary(d),
                          "launch": "cuda graph replay" if graphs else "eager"}
+        if not w.latent:
+            res["block_screening"] = screening_comparison(w, qs, K, Vv, P, Kt, sl, pos, dims, dev, stream, flush_buf,
+                                                          cmp_steps, world, graphs is not None)
         if not w.latent and w.d <= 128:
             res["calibration_of_P"] = calibration_recall(w, q, K, P, sl, dev, stream)
         if not w.latent:

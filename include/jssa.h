@@ -217,13 +217,37 @@ typedef enum {
  *  - unfused: for jssa_decode_step_ex, nonzero keeps the step in separate
  *    launches (prologue, selection, attention) even where the one-launch
  *    fused form applies.
- * NULL or all zeros: plain top-k, automatic form. */
+ *  - block_norms: exact block screening (a lossless cut of the low-rank
+ *    stream; the method pages on DoSA-style screening describe the bound).
+ *    NULL: off.  Else [B, Hkv, ceil(T_cap / JSSA_NORM_BLOCK)] fp32 upper
+ *    bounds of ||Kt[b,h,t,:]|| over each block of JSSA_NORM_BLOCK tokens (see
+ *    jssa_block_norms).  The streaming form then skips reading a tile of the
+ *    low-rank cache when ||qbar|| times its blocks' bound (inflated by 1e-4
+ *    to cover fp32 rounding) cannot beat the k-th best key its segment has
+ *    already seen; the selection is bit-identical either way (other forms
+ *    ignore the bound).  Tiles holding forced tokens are never skipped.  The
+ *    decode step keeps the bound of the block of the appended row current
+ *    (raised with an atomic max); an append made with jssa_append_lowrank
+ *    needs jssa_block_norms afterwards.  Skipped tiles are counted in word 1
+ *    of the workspace (uint32, cumulative; jssa_workspace_init clears it).
+ * NULL or all zeros: plain top-k, automatic form, no screening. */
 typedef struct {
-    int32_t n_sink;   /* >= 0 */
-    int32_t n_recent; /* >= 0 */
-    int32_t form;     /* jssa_select_form */
-    int32_t unfused;  /* 0 or 1 */
+    int32_t n_sink;     /* >= 0 */
+    int32_t n_recent;   /* >= 0 */
+    int32_t form;       /* jssa_select_form */
+    int32_t unfused;    /* 0 or 1 */
+    float *block_norms; /* screening bounds, or NULL */
 } jssa_select_opts;
+
+#define JSSA_NORM_BLOCK 128
+
+/* Block norm bounds of the low-rank cache for screening: norms[b,h,j] = the
+ * largest ||Kt[b,h,t,:]|| (fp32, from the stored values) over t in
+ * [j*JSSA_NORM_BLOCK, min(T_cap, (j+1)*JSSA_NORM_BLOCK)), every row b.
+ * norms: [B, Hkv, ceil(T_cap / JSSA_NORM_BLOCK)] fp32 device memory.  Only
+ * B, Hkv, T_cap, r and kt_dtype of dims are read.  The pages have no API for
+ * it; it is the screening variant's bookkeeping. */
+JSSA_API int jssa_block_norms(const jssa_dims *dims, const void *Kt, float *norms, jssa_stream_t stream);
 
 /* jssa_topk, jssa_select and jssa_decode_step with selection options (NULL
  * = the plain calls).  jssa_select_ex stays bit-identical to jssa_score +

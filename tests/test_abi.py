@@ -91,4 +91,5 @@ def test_select_opts_layout_matches_the_header():
     src = open(HEADER).read()
     body = re.search(r"typedef struct \{([^}]*)\} jssa_select_opts;", src).group(1)
     fields = re.findall(r"int32_t\s+(\w+);", body)
+    fields += re.findall(r"float \*(\w+);", body)
     assert fields == [n for n, _ in ops.SelectOpts._fields_]

@@ -521,6 +521,63 @@ def test_host_buffer_step_equals_device_step():
         assert ops.device_status(ws) == 0
 
 
+# ------------------------------------------------ exact block screening
+def test_block_norms_match_numpy():
+    w = W(B=2, Hq=8, Hkv=2, T=1000, r=32, seed=159)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    nrm = ops.block_norms(Kt)
+    torch.cuda.synchronize()
+    kt = host(Kt).double().numpy()
+    rn = np.sqrt((kt * kt).sum(-1))  # [B, Hkv, T]
+    nb = (w.T + 127) // 128
+    ref = np.stack([rn[:, :, j * 128:(j + 1) * 128].max(-1) for j in range(nb)], -1)
+    np.testing.assert_allclose(host(nrm).double().numpy(), ref, rtol=1e-5)
+
+
+def test_block_screening_is_exact_and_skips():
+    """Exact screening over the low-rank cache: with block norm bounds the
+    streaming form skips tiles that cannot beat its segment's k-th key, and
+    every result stays bit-identical (selection alone, fused and unfused
+    decode step; the other selection forms ignore the bounds).  Inputs where
+    it must trigger: every row's keys past token 1024 are zero, so once a
+    segment holds k candidates its remaining tiles are bounded by 0."""
+    w = W(B=16, Hq=32, Hkv=8, T=16384, k=64, kind="plain", seed=160)
+    (q, K, V, P, sl), (qd, Kd, Vd, Pd, sld) = draw(w)
+    Kd[:, 1024:] = 0
+    Kt = ops.build_lowrank_cache(Kd, Pd)
+    nrm = ops.block_norms(Kt)
+    dims = ops.make_dims(qd, Kd, Vd, P=Pd, Kt=Kt)
+    i1, c1 = ops.select(qd, Pd, Kt, sld, w.k, form="stream")
+    ws = ops.new_workspace(dims, w.k, ops.OP_SELECT, qd.device)
+    i2, c2 = ops.select(qd, Pd, Kt, sld, w.k, form="stream", ws=ws, block_norms=nrm)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    skipped = ops.skip_count(ws)
+    assert skipped > 0, "no tile was screened out"
+    for f in ("cluster", "scan", "auto"):
+        i3, c3 = ops.select(qd, Pd, Kt, sld, w.k, form=f, block_norms=nrm)
+        torch.cuda.synchronize()
+        assert torch.equal(i1, i3) and torch.equal(c1, c3), f
+    # the selection against the oracle on a few rows (the GPU's own low-rank cache)
+    ref_s = oracle.score(q[:2], P, host(Kt[:2]), sl[:2])
+    check_selection(host(i2[:2]).numpy(), host(c2[:2]).numpy(), ref_s, sl[:2].numpy(), w.k)
+    # the decode step, fused and unfused, with and without screening
+    pos = (sld - 1).clamp_min(0)
+    for unfused in (False, True):
+        Kt1, Kt2, n2 = Kt.clone(), Kt.clone(), nrm.clone()
+        wsd = ops.new_workspace(dims, w.k, ops.OP_DECODE_STEP, qd.device)
+        o1, l1, j1, d1 = ops.decode_step(qd, Kd, Vd, Pd, Kt1, sld, pos, w.k, w.scale, form="stream", unfused=unfused)
+        o2, l2, j2, d2 = ops.decode_step(qd, Kd, Vd, Pd, Kt2, sld, pos, w.k, w.scale, form="stream", unfused=unfused,
+                                         ws=wsd, block_norms=n2)
+        torch.cuda.synchronize()
+        assert torch.equal(Kt1, Kt2) and torch.equal(j1, j2) and torch.equal(d1, d2)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        assert ops.skip_count(wsd) > 0
+        # the bounds still cover every row of the cache after the append
+        assert torch.all(n2 >= ops.block_norms(Kt2) * (1 - 1e-6))
+
+
 # ------------------------------------------------------- calibration of P
 @pytest.mark.parametrize("d,r,Hkv,G", [(128, 32, 2, 4), (256, 64, 2, 8), (64, 8, 3, 1)])
 def test_calibrated_basis_keeps_the_dominant_joint_energy(d, r, Hkv, G):

@@ -427,6 +427,14 @@ T *at(void *ws, size_t off) {
 
 cudaStream_t S(jssa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Screening fields of a streaming-form launch (opts->block_norms non-null).
+void fill_screen(ScanArgs &sa, const jssa_dims *d, const jssa_select_opts *opts, void *ws) {
+    if (!opts || !opts->block_norms) return;
+    sa.norms = opts->block_norms;
+    sa.norm_blocks = (d->T_cap + JSSA_NORM_BLOCK - 1) / JSSA_NORM_BLOCK;
+    sa.skip_count = at<uint32_t>(ws, 4);
+}
+
 int check_opts(const jssa_select_opts *opts) {
     if (!opts) return JSSA_OK;
     if (opts->n_sink < 0 || opts->n_recent < 0)
@@ -436,6 +444,8 @@ int check_opts(const jssa_select_opts *opts) {
         return fail(JSSA_ERR_INVALID_ARG, "unknown selection form %d", opts->form);
     if (opts->unfused != 0 && opts->unfused != 1)
         return fail(JSSA_ERR_INVALID_ARG, "unfused=%d is neither 0 nor 1", opts->unfused);
+    if (opts->block_norms && !aligned16(opts->block_norms))
+        return fail(JSSA_ERR_INVALID_ARG, "block_norms is not 16-byte aligned");
     return JSSA_OK;
 }
 
@@ -540,6 +550,7 @@ int run_select(const jssa_dims *d, const Shape &sh, const void *q, const float *
     sa.n_sink = n_sink;
     sa.n_recent = n_recent;
     sa.src_div = src_div;
+    if (L.wspec && q != nullptr && src_div <= 1) fill_screen(sa, d, opts, ws);
     cudaError_t e = L.wspec ? launch_stream(L.sp, sa, s, true) : launch_scan(L.sp, sa, agg, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the selection pass");
     return JSSA_OK;
@@ -1011,6 +1022,7 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
         sa.k = k;
         sa.n_sink = opts ? opts->n_sink : 0;
         sa.n_recent = opts ? opts->n_recent : 0;
+        fill_screen(sa, dims, opts, ws);
         StepExtra x;
         x.q = q;
         x.P = P;
@@ -1031,6 +1043,11 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     ProjArgs pj{q, P, at<float>(ws, L.qproj), dims->B, dims->Hq, dims->Hkv, dims->d, dims->r, agg};
     cudaError_t e = launch_prep(ap, pj, S(stream), true, dims->kv_dtype, dims->kt_dtype);
     if (e != cudaSuccess) return cuda_fail(e, "launching the append + projection prologue");
+    if (opts && opts->block_norms && !sh.latent) {
+        e = launch_norm_raise(Kt, dims->kt_dtype, opts->block_norms, pos_begin, dims->B, dims->Hkv, dims->T_cap,
+                              dims->r, S(stream), true);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the screening-bound update");
+    }
     if ((st = run_select(dims, sh, q, P, Kt, seq_lens, agg, k, idx, count, ws, L, S(stream), false, opts)))
         return st;
     if (sh.latent) return run_mla(dims, q, K, idx, count, k, seq_lens, softmax_scale, out, lse, ws, L, S(stream));
@@ -1041,6 +1058,24 @@ int jssa_decode_step_ex(const jssa_dims *dims, const void *q, const void *K, con
     a.k = k;
     e = launch_attend(L.ap, ATT_INDEXED, a, dims->kv_dtype, dims->d, S(stream), true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the indexed decode");
+    return JSSA_OK;
+}
+
+int jssa_block_norms(const jssa_dims *dims, const void *Kt, float *norms, jssa_stream_t stream) {
+    // only the low-rank cache's dims matter here: B, Hkv, T_cap, r, kt_dtype
+    if (!dims) return fail(JSSA_ERR_INVALID_ARG, "dims is NULL");
+    if (dims->B < 0 || dims->Hkv < 1 || dims->T_cap < 1 || dims->r < 1)
+        return fail(JSSA_ERR_INVALID_ARG, "bad dimension (B=%d Hkv=%d r=%d T_cap=%d)", dims->B, dims->Hkv, dims->r,
+                    dims->T_cap);
+    if (dims->kt_dtype != JSSA_BF16 && dims->kt_dtype != JSSA_FP32)
+        return fail(JSSA_ERR_INVALID_ARG, "bad dtype code (kt=%d)", dims->kt_dtype);
+    if ((long long)dims->B * dims->Hkv > 65535) return fail(JSSA_ERR_UNSUPPORTED, "B*Hkv above 65535");
+    REQUIRE_PTR(Kt);
+    REQUIRE_PTR(norms);
+    if (dims->B == 0) return JSSA_OK;
+    cudaError_t e = launch_block_norms(Kt, dims->kt_dtype, norms, dims->B * dims->Hkv, dims->T_cap, dims->r,
+                                       S(stream), true);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the block norms");
     return JSSA_OK;
 }
 

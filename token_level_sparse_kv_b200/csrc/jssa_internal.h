@@ -46,6 +46,9 @@ struct ScanArgs {
     int grid, max_seg, cap, nstages;
     int n_sink, n_recent;  // always-selected tokens (0, 0: plain top-k)
     int src_div;           // selection row bh reads source row bh / src_div (0 or 1: the same row)
+    float *norms;          // screening: [BH, norm_blocks] block norm bounds, or null (streaming form)
+    int norm_blocks;       // blocks of JSSA_NORM_BLOCK tokens per row
+    uint32_t *skip_count;  // screening: tiles skipped (cumulative)
 };
 
 struct ScanPlan {
@@ -243,6 +246,12 @@ int device_sm_count();
 // the requested size grows).
 cudaError_t ensure_smem(const void *kern, size_t smem);
 cudaError_t launch_project(const ProjArgs &a, cudaStream_t s, bool pdl, int kv_dtype);
+// Block norm bounds of the low-rank cache (jssa_block_norms), and the raise of
+// the bound of the block holding each row's appended row at pos[b].
+cudaError_t launch_block_norms(const void *Kt, int kt_dtype, float *norms, int BH, int T_cap, int r,
+                               cudaStream_t s, bool pdl);
+cudaError_t launch_norm_raise(const void *Kt, int kt_dtype, float *norms, const int32_t *pos, int B, int Hkv,
+                              int T_cap, int r, cudaStream_t s, bool pdl);
 // Write each batch row's new K row (row_k_bytes, all KV heads) and V row into
 // the cache at position pos[b]; v_new / V null for a latent cache.
 cudaError_t launch_place_rows(const void *k_new, const void *v_new, void *K, void *V, const int32_t *pos, int B,

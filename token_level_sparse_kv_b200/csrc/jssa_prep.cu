@@ -283,6 +283,50 @@ __global__ void __launch_bounds__(128) place_rows_kernel(const uint4 *k_new, con
             V[((size_t)b * T_cap + p) * row_v16 + c] = v_new[(size_t)b * row_v16 + c];
 }
 
+// ||row|| of r stored values (fp32 sum of squares of the exact stored values)
+template <typename KT>
+__device__ __forceinline__ float row_norm(const KT *row, int r, int lane) {
+    float s = 0.f;
+    for (int j = lane; j < r; j += 32) {
+        const float v = to_f32(row[j]);
+        s = fmaf(v, v, s);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return sqrtf(s);
+}
+
+// One warp per block of JSSA_NORM_BLOCK tokens of a row.
+template <typename KT>
+__global__ void __launch_bounds__(256) block_norms_kernel(const KT *Kt, float *norms, int BH, int T_cap, int r,
+                                                          int nblk) {
+    pdl_trigger();
+    pdl_wait();
+    const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= (long long)BH * nblk) return;
+    const int bh = (int)(w / nblk), j = (int)(w - (long long)bh * nblk);
+    const int t1 = min(T_cap, (j + 1) * JSSA_NORM_BLOCK);
+    float m = 0.f;
+    for (int t = j * JSSA_NORM_BLOCK; t < t1; ++t) m = fmaxf(m, row_norm(Kt + ((size_t)bh * T_cap + t) * r, r, lane));
+    if (lane == 0) norms[w] = m;
+}
+
+// One warp per (b,h): the bound of the block holding the row at pos[b] is
+// raised to cover the row (an atomic max on the non-negative float's bits).
+template <typename KT>
+__global__ void __launch_bounds__(256) norm_raise_kernel(const KT *Kt, float *norms, const int32_t *pos, int B,
+                                                         int Hkv, int T_cap, int r, int nblk) {
+    pdl_trigger();
+    pdl_wait();
+    const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (w >= B * Hkv) return;
+    const int p = pos[w / Hkv];
+    if (p < 0 || p >= T_cap) return;
+    const float n = row_norm(Kt + ((size_t)w * T_cap + p) * r, r, lane);
+    if (lane == 0) atomicMax(reinterpret_cast<int *>(norms + (size_t)w * nblk + p / JSSA_NORM_BLOCK), __float_as_int(n));
+}
+
 size_t prep_smem(int rows, int d, int r) {
     return ((size_t)rows * d + (size_t)rows * r * (d / kChunk)) * sizeof(float);
 }
@@ -311,6 +355,29 @@ cudaError_t launch_append(const AppendArgs &a0, cudaStream_t s, bool pdl, int kv
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return e;
     return launch_kernel(k, grid, dim3(prep_threads(a.d)), smem, s, pdl, a);
+}
+
+cudaError_t launch_block_norms(const void *Kt, int kt_dtype, float *norms, int BH, int T_cap, int r,
+                               cudaStream_t s, bool pdl) {
+    const int nblk = (T_cap + JSSA_NORM_BLOCK - 1) / JSSA_NORM_BLOCK;
+    const long long warps = (long long)BH * nblk;
+    const dim3 grid((unsigned)((warps + 7) / 8));
+    if (kt_dtype == JSSA_BF16)
+        return launch_kernel(block_norms_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, pdl,
+                             static_cast<const __nv_bfloat16 *>(Kt), norms, BH, T_cap, r, nblk);
+    return launch_kernel(block_norms_kernel<float>, grid, dim3(256), 0, s, pdl, static_cast<const float *>(Kt), norms,
+                         BH, T_cap, r, nblk);
+}
+
+cudaError_t launch_norm_raise(const void *Kt, int kt_dtype, float *norms, const int32_t *pos, int B, int Hkv,
+                              int T_cap, int r, cudaStream_t s, bool pdl) {
+    const int nblk = (T_cap + JSSA_NORM_BLOCK - 1) / JSSA_NORM_BLOCK;
+    const dim3 grid((unsigned)((B * Hkv + 7) / 8));
+    if (kt_dtype == JSSA_BF16)
+        return launch_kernel(norm_raise_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, pdl,
+                             static_cast<const __nv_bfloat16 *>(Kt), norms, pos, B, Hkv, T_cap, r, nblk);
+    return launch_kernel(norm_raise_kernel<float>, grid, dim3(256), 0, s, pdl, static_cast<const float *>(Kt), norms,
+                         pos, B, Hkv, T_cap, r, nblk);
 }
 
 cudaError_t launch_place_rows(const void *k_new, const void *v_new, void *K, void *V, const int32_t *pos, int B,

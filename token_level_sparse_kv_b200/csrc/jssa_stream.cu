@@ -78,7 +78,7 @@ struct StreamSmem {
 // (u64), [40..42] epoch buffer counts, [44..45] smallest / largest key
 // appended to the segment's candidates, [48..63] reduction scratch.
 // misc words, fused step: [46] rows to attend, [64..71] their (b,h), [72..79]
-// their token counts.  qb: folded queries of the range's rows [kMaxRows][r];
+// their token counts.  [80..87]: stage s holds a tile skipped by screening.  qb: folded queries of the range's rows [kMaxRows][r];
 // xs: one input row of a projection [256].
 __host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k, int fused_r = 0) {
     StreamSmem L;
@@ -950,6 +950,16 @@ __device__ void sel_append(const ScanArgs &a, const StepExtra &x, int bh, int po
     __nv_bfloat16 *Kt = static_cast<__nv_bfloat16 *>(const_cast<void *>(a.src));
     for (int j = st; j < R; j += kSelT)
         Kt[((size_t)bh * a.T_cap + pos) * R + j] = __float2bfloat16_rn(sum_parts(part, j, d / kChunkD));
+    if (a.norms && st == 0) {
+        // screening bound of the row's block raised to cover the new row
+        float ss = 0.f;
+        for (int j = 0; j < R; ++j) {
+            const float v = __bfloat162float(__float2bfloat16_rn(sum_parts(part, j, d / kChunkD)));
+            ss = fmaf(v, v, ss);
+        }
+        atomicMax(reinterpret_cast<int *>(a.norms + (size_t)bh * a.norm_blocks + pos / JSSA_NORM_BLOCK),
+                  __float_as_int(sqrtf(ss)));
+    }
     fence_proxy_async_global();
     sel_sync();
 }
@@ -1271,6 +1281,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             RingPos rp(S_);
             int Tb = 0, atile = -1;
             bool appended = false;
+            float qn = -1.f;  // ||qbar|| of the current row (screening), -1 while unknown
             for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
                 const int s = rp.s;
                 if (i >= S_ && !wait_or_abort(&empty[s], rp.ph ^ 1u, abort_flag)) {
@@ -1279,6 +1290,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                 }
                 const int bh = cur.bh, t0 = cur.t * TILE;
                 if (i == 0 || cur.t == 0) {
+                    qn = -1.f;
                     Tb = clamp_seq(__ldg(a.seq_lens + bh / a.Hkv), a.T_cap, nullptr);
                     if constexpr (FUSED) {
                         const int pos = __ldg(A.x.pos_begin + bh / a.Hkv);
@@ -1294,12 +1306,47 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                     appended = true;
                 }
                 const int n = min(TILE, Tb - t0);
-                if (n > 0) {
+                // exact screening: skip the tile when ||qbar|| times its blocks'
+                // norm bound (inflated for fp32 rounding) cannot beat the key
+                // the row's segment already holds k candidates above
+                bool skip = false;
+                if (a.norms && n > 0) {
+                    const bool tforce = t0 < a.n_sink || t0 + TILE > Tb - a.n_recent;
+                    const unsigned long long tw = *thr_word;
+                    if (!tforce && (uint32_t)(tw >> 32) == (uint32_t)bh + 1u) {
+                        if (qn < 0.f) {
+                            const float *qp = nullptr;
+                            if constexpr (FUSED) {
+                                if (mbar_try_wait(&qready[bh - row0], 0u)) qp = qb + (size_t)(bh - row0) * R;
+                            } else {
+                                qp = a.qproj + (size_t)bh * R;
+                            }
+                            if (qp) {
+                                float ss = 0.f;
+                                for (int j = 0; j < R; ++j) {
+                                    const float v = FUSED ? qp[j] : __ldcg(qp + j);
+                                    ss = fmaf(v, v, ss);
+                                }
+                                qn = sqrtf(ss);
+                            }
+                        }
+                        if (qn >= 0.f) {
+                            const float *nr = a.norms + (size_t)bh * a.norm_blocks;
+                            float nb = 0.f;
+                            for (int j = t0 / JSSA_NORM_BLOCK; j <= (t0 + n - 1) / JSSA_NORM_BLOCK; ++j)
+                                nb = fmaxf(nb, __ldcg(nr + j));
+                            skip = score_key(qn * nb * 1.0001f) <= (uint32_t)tw;
+                        }
+                    }
+                }
+                misc[80 + s] = skip ? 1 : 0;
+                if (n > 0 && !skip) {
                     mbar_arrive_expect_tx(&full[s], (uint32_t)n * ROWB);
                     bulk_g2s(smem + L.ring + (size_t)s * kTile, src + ((size_t)bh * a.T_cap + t0) * ROWB,
                              (uint32_t)n * ROWB, &full[s], pol);
                 } else {
                     mbar_arrive(&full[s]);
+                    if (skip && a.skip_count) atomicAdd(a.skip_count, 1u);
                 }
                 issued = i + 1;
             }
@@ -1362,7 +1409,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                 }
             }
             const int t0 = t * TILE;
-            const int n = max(0, min(TILE, Tb - t0));
+            const int n = misc[80 + s] ? 0 : max(0, min(TILE, Tb - t0));  // a screened-out tile holds nothing
             // does this tile hold always-selected tokens (warp-uniform)?
             const bool tforce = t0 < a.n_sink || t0 + TILE > Tb - a.n_recent;
             const unsigned long long tw = *thr_word;

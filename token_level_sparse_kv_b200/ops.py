@@ -73,6 +73,8 @@ def lib():
     L.jssa_decode_step_ex.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.jssa_plan_info.restype = i32
     L.jssa_plan_info.argtypes = [D, i32, i32, i32, ctypes.POINTER(i32), ctypes.c_char_p, sz]
+    L.jssa_block_norms.restype = i32
+    L.jssa_block_norms.argtypes = [D, vp, vp, vp]
     L.jssa_calibrate_basis.restype = i32
     L.jssa_calibrate_basis.argtypes = [D, vp, i32, vp, vp, i32, i32, vp, vp, vp, sz, vp]
     L.jssa_host_step_bytes.restype = i32
@@ -161,14 +163,36 @@ class SelectOpts(ctypes.Structure):
     selected; form forces a selection form; unfused keeps the decode step in
     separate launches."""
     _fields_ = [("n_sink", ctypes.c_int32), ("n_recent", ctypes.c_int32), ("form", ctypes.c_int32),
-                ("unfused", ctypes.c_int32)]
+                ("unfused", ctypes.c_int32), ("block_norms", ctypes.c_void_p)]
 
 
-def _opts(n_sink=0, n_recent=0, form="auto", unfused=False):
+NORM_BLOCK = 128
+
+
+def _opts(n_sink=0, n_recent=0, form="auto", unfused=False, block_norms=None):
     f = FORMS[form] if isinstance(form, str) else int(form)
-    if not n_sink and not n_recent and not f and not unfused:
+    if not n_sink and not n_recent and not f and not unfused and block_norms is None:
         return None
-    return ctypes.byref(SelectOpts(int(n_sink), int(n_recent), f, 1 if unfused else 0))
+    if block_norms is not None:
+        _cuda(block_norms)
+    nb = None if block_norms is None else block_norms.data_ptr()
+    return ctypes.byref(SelectOpts(int(n_sink), int(n_recent), f, 1 if unfused else 0, nb))
+
+
+def block_norms(Kt, norms=None):
+    """Screening bounds [B, Hkv, ceil(T_cap / 128)] fp32: the largest ||Kt[b,h,t,:]|| per block of 128 tokens."""
+    _cuda(Kt, norms)
+    B, Hkv, T_cap, r = Kt.shape
+    if norms is None:
+        norms = torch.empty((B, Hkv, (T_cap + NORM_BLOCK - 1) // NORM_BLOCK), dtype=torch.float32, device=Kt.device)
+    dims = Dims(B, Hkv, Hkv, r, r, r, T_cap, BF16, _dt(Kt))
+    _check(lib().jssa_block_norms(ctypes.byref(dims), _p(Kt), _p(norms), _stream(Kt.device)))
+    return norms
+
+
+def skip_count(ws: torch.Tensor) -> int:
+    """Tiles the screening skipped (workspace word 1, cumulative); synchronises."""
+    return int(ws[4:8].view(torch.int32).item()) & 0xFFFFFFFF
 
 
 def plan_info(dims: Dims, k: int, op: int, agg: int = 0, form="auto", unfused=False):
@@ -256,7 +280,8 @@ def topk(scores, seq_lens, k, Hq=None, d=128, ws=None, n_sink=0, n_recent=0, for
     return idx, cnt
 
 
-def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_sink=0, n_recent=0, form="auto"):
+def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_sink=0, n_recent=0, form="auto",
+           block_norms=None):
     """Fused score + top-k: (idx [B,Hkv,k], count [B,Hkv]).
     n_sink / n_recent: always-selected first / last tokens; form: the selection
     form (jssa_select_opts)."""
@@ -270,8 +295,8 @@ def select(q, P, Kt, seq_lens, k, agg=AGG_SUM, ws=None, idx=None, count=None, n_
         count = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
     ws = _ws(ws, dims, k, OP_SELECT, q.device)
     _check(lib().jssa_select_ex(ctypes.byref(dims), _p(q), _p(P), _p(Kt), _p(seq_lens), int(agg), int(k),
-                                _opts(n_sink, n_recent, form), _p(idx), _p(count), _p(ws), ws.numel(),
-                                _stream(q.device)))
+                                _opts(n_sink, n_recent, form, block_norms=block_norms), _p(idx), _p(count), _p(ws),
+                                ws.numel(), _stream(q.device)))
     return idx, count
 
 
@@ -366,7 +391,7 @@ def gather_then_dense(q, K, V, idx, count, seq_lens, scale, gather_buf=None, ws=
 
 
 def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=None, idx=None, count=None,
-                out=None, lse=None, n_sink=0, n_recent=0, form="auto", unfused=False):
+                out=None, lse=None, n_sink=0, n_recent=0, form="auto", unfused=False, block_norms=None):
     """Append the row at pos_begin, select, indexed decode: (out, lse, idx, count).
     n_sink / n_recent: always-selected first / last tokens; form: the selection
     form; unfused: keep the step in separate launches (jssa_select_opts)."""
@@ -384,7 +409,8 @@ def decode_step(q, K, V, P, Kt, seq_lens, pos_begin, k, scale, agg=AGG_SUM, ws=N
     ws = _ws(ws, dims, k, OP_DECODE_STEP, q.device)
     _check(lib().jssa_decode_step_ex(ctypes.byref(dims), _p(q), _p(K), _p(K if V is None else V), _p(P), _p(Kt),
                                      _p(seq_lens), _p(pos_begin), int(k), int(agg), float(scale),
-                                     _opts(n_sink, n_recent, form, unfused), _p(idx), _p(count), _p(out), _p(lse),
+                                     _opts(n_sink, n_recent, form, unfused, block_norms), _p(idx), _p(count), _p(out),
+                                     _p(lse),
                                      _p(ws), ws.numel(), _stream(q.device)))
     return out, lse, idx, count
 
