@@ -1282,12 +1282,20 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             int Tb = 0, atile = -1;
             bool appended = false;
             float qn = -1.f;  // ||qbar|| of the current row (screening), -1 while unknown
+            // screening: the block bounds of a tile are loaded one tile ahead
+            // (after the previous tile's copy is issued), so that their
+            // latency hides behind the ring
+            constexpr int NBT = (TILE + JSSA_NORM_BLOCK - 1) / JSSA_NORM_BLOCK;
+            float nbv[NBT];
+            auto load_bounds = [&](int bh_, int t0_) {
+                const float *nr = a.norms + (size_t)bh_ * a.norm_blocks + t0_ / JSSA_NORM_BLOCK;
+                const int nblk = min(NBT, a.norm_blocks - t0_ / JSSA_NORM_BLOCK);
+#pragma unroll
+                for (int j = 0; j < NBT; ++j) nbv[j] = j < nblk ? __ldcg(nr + j) : 0.f;
+            };
+            if (a.norms && ntiles > 0) load_bounds(cur.bh, cur.t * TILE);
             for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
                 const int s = rp.s;
-                if (i >= S_ && !wait_or_abort(&empty[s], rp.ph ^ 1u, abort_flag)) {
-                    *abort_flag = 1;
-                    break;
-                }
                 const int bh = cur.bh, t0 = cur.t * TILE;
                 if (i == 0 || cur.t == 0) {
                     qn = -1.f;
@@ -1297,6 +1305,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                         atile = (pos >= 0 && pos < a.T_cap) ? pos / TILE : -1;
                     }
                 }
+                if (i >= S_ && !wait_or_abort(&empty[s], rp.ph ^ 1u, abort_flag)) {
+                    *abort_flag = 1;
+                    break;
+                }
                 if (FUSED && !appended && cur.t == atile) {
                     // this tile holds the row appended in the prologue
                     if (!wait_or_abort(aready, 0u, abort_flag)) {
@@ -1304,6 +1316,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                         break;
                     }
                     appended = true;
+                    if (a.norms) load_bounds(bh, t0);  // its block's bound was raised for the new row
                 }
                 const int n = min(TILE, Tb - t0);
                 // exact screening: skip the tile when ||qbar|| times its blocks'
@@ -1331,10 +1344,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                             }
                         }
                         if (qn >= 0.f) {
-                            const float *nr = a.norms + (size_t)bh * a.norm_blocks;
                             float nb = 0.f;
-                            for (int j = t0 / JSSA_NORM_BLOCK; j <= (t0 + n - 1) / JSSA_NORM_BLOCK; ++j)
-                                nb = fmaxf(nb, __ldcg(nr + j));
+#pragma unroll
+                            for (int j = 0; j < NBT; ++j)
+                                if (j * JSSA_NORM_BLOCK < n) nb = fmaxf(nb, nbv[j]);
                             skip = score_key(qn * nb * 1.0001f) <= (uint32_t)tw;
                         }
                     }
@@ -1349,6 +1362,11 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                     if (skip && a.skip_count) atomicAdd(a.skip_count, 1u);
                 }
                 issued = i + 1;
+                if (a.norms && i + 1 < ntiles) {
+                    Cursor nx = cur;
+                    nx.next();
+                    load_bounds(nx.bh, nx.t * TILE);
+                }
             }
             misc[24] = issued;
         }
