@@ -147,9 +147,18 @@ __global__ void __launch_bounds__(kThr, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long total = a.total_tiles;
-    const long long i0 = (long long)blockIdx.x * total / a.grid;
-    const long long i1 = (long long)(blockIdx.x + 1) * total / a.grid;
     const int rt = a.row_tiles;
+    // the CTA's tiles: a contiguous share of the flattened (row, tile) list,
+    // or (short problems) one of row_split equal parts of a single row
+    long long i0, i1;
+    if (a.row_split > 0) {
+        const int bhs = blockIdx.x / a.row_split, part = blockIdx.x - bhs * a.row_split;
+        i0 = (long long)bhs * rt + (long long)part * rt / a.row_split;
+        i1 = (long long)bhs * rt + (long long)(part + 1) * rt / a.row_split;
+    } else {
+        i0 = (long long)blockIdx.x * total / a.grid;
+        i1 = (long long)(blockIdx.x + 1) * total / a.grid;
+    }
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -344,8 +353,8 @@ __global__ void __launch_bounds__(kThr, 1)
             // the CTA's partial of the row: the four warps' (O, max, sum) merged
             // in shared memory, then one unnormalised partial per segment
             const long long first = (long long)bh * rt;
-            const int c_first = (int)(((first + 1) * a.grid - 1) / total);
-            const int slot = (int)blockIdx.x - c_first;
+            const int slot = a.row_split > 0 ? (int)blockIdx.x % a.row_split
+                                             : (int)blockIdx.x - (int)(((first + 1) * a.grid - 1) / total);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 lrun[r] += __shfl_xor_sync(0xffffffffu, lrun[r], 1);
@@ -421,9 +430,8 @@ __global__ void __launch_bounds__(D) dense_combine_kernel(DenseArgs a) {
     const int bh = blockIdx.x, g = blockIdx.y, d = threadIdx.x;
     const int G = a.G, rt = a.row_tiles;
     const long long total = a.total_tiles, first = (long long)bh * rt;
-    const int c_first = (int)(((first + 1) * a.grid - 1) / total);
-    const int c_last = (int)(((first + rt) * a.grid - 1) / total);
-    const int np = c_last - c_first + 1;
+    const int np = a.row_split > 0 ? a.row_split
+                                   : (int)(((first + rt) * a.grid - 1) / total) - (int)(((first + 1) * a.grid - 1) / total) + 1;
     const size_t pb = (size_t)bh * a.part_stride;
     if (d < 32) {
         float M = -INFINITY;
@@ -536,11 +544,22 @@ cudaError_t plan_dense(int d, int B, int Hkv, int row_len, DensePlan *p) {
     if (row_len < 1) row_len = 1;
     p->row_tiles = (row_len + kNT - 1) / kNT;
     p->total_tiles = (long long)B * Hkv * p->row_tiles;
-    long long g = device_sm_count();
+    const long long sms = device_sm_count(), BH = (long long)B * Hkv;
+    long long g = sms;
     if (g > p->total_tiles) g = p->total_tiles;
     if (g < 1) g = 1;
     p->grid = (int)g;
+    p->row_split = 0;
     p->part_stride = dense_part_stride(B, Hkv);
+    // short problems (under four tiles per SM): split each row evenly, so that
+    // no CTA covers the end of one row and the start of the next
+    if (p->total_tiles < 4 * sms && BH <= sms) {
+        long long sp = sms / BH;
+        if (sp > p->row_tiles) sp = p->row_tiles;
+        if (sp < 1) sp = 1;
+        p->row_split = (int)sp;
+        p->grid = (int)(BH * sp);
+    }
     p->smem = smem;
     return cudaSuccess;
 }
@@ -555,6 +574,7 @@ cudaError_t launch_dense(const DensePlan &p, const DenseArgs &a0, const void *K,
     a.total_tiles = p.total_tiles;
     a.grid = p.grid;
     a.part_stride = p.part_stride;
+    a.row_split = p.row_split;
     CUtensorMap mk, mv;
     cudaError_t e;
     if (a.count) {  // gathered [B*Hkv, k, d]

@@ -128,6 +128,7 @@ struct DenseArgs {
     int row_tiles;            // plan: 64-token tiles per row
     long long total_tiles;    // plan: rows * row_tiles
     int grid, part_stride;    // plan: persistent CTAs; partial slots per row
+    int row_split;            // plan: > 0 = each row split into row_split parts, one CTA each (short problems)
     float scale_log2;         // softmax_scale * log2(e)
     float *part_o;            // [BH, part_stride, G, d]
     float *part_ml;           // [BH, part_stride, G, 2]
@@ -137,7 +138,7 @@ struct DenseArgs {
     uint32_t *status;
 };
 struct DensePlan {
-    int row_tiles, grid, part_stride;
+    int row_tiles, grid, part_stride, row_split;
     long long total_tiles;
     size_t smem;
 };

@@ -1330,7 +1330,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                         if (qn < 0.f) {
                             const float *qp = nullptr;
                             if constexpr (FUSED) {
-                                if (mbar_try_wait(&qready[bh - row0], 0u)) qp = qb + (size_t)(bh - row0) * R;
+                                // a test, not a wait: the producer must not stall on the prologue
+                                if (mbar_test_wait(&qready[bh - row0], 0u)) qp = qb + (size_t)(bh - row0) * R;
                             } else {
                                 qp = a.qproj + (size_t)bh * R;
                             }
