@@ -48,11 +48,13 @@ struct ScanArgs {
     int src_div;           // selection row bh reads source row bh / src_div (0 or 1: the same row)
     float *norms;          // screening: [BH, norm_blocks] block norm bounds, or null (streaming form)
     int norm_blocks;       // blocks of JSSA_NORM_BLOCK tokens per row
+    int nb_cap;            // streaming form: tile bounds staged in shared memory per CTA (plan)
     uint32_t *skip_count;  // screening: tiles skipped (cumulative)
 };
 
 struct ScanPlan {
     int src, mode, tile_tokens, tiles_per_bh, grid, max_seg, cap, nstages;
+    int nb_cap;  // streaming form: tile bounds a CTA stages in shared memory for screening
     long long total_tiles;
     size_t smem;
 };

@@ -818,6 +818,7 @@ cudaError_t plan_scan(int src, int mode, int agg, int B, int Hkv, int T_cap, int
     auto kern = pick_scan(src, mode, r, agg);
     if (!kern) return cudaErrorInvalidValue;
     ScanPlan P;
+    P.nb_cap = 0;
     P.src = src;
     P.mode = mode;
     P.tile_tokens = scan_tile_tokens(src, r);

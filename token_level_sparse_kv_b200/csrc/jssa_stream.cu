@@ -69,7 +69,7 @@ __host__ __device__ inline int npow2(int x) {
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct StreamSmem {
-    size_t ring, bars, ek, ei, rk, ri, sk, si, hist, misc, qb, xs, total;
+    size_t ring, bars, ek, ei, rk, ri, sk, si, hist, misc, qb, xs, nb, total;
 };
 
 // misc words (int): [0] abort, [3] candidate count, [4..6] select results,
@@ -79,8 +79,10 @@ struct StreamSmem {
 // appended to the segment's candidates, [48..63] reduction scratch.
 // misc words, fused step: [46] rows to attend, [64..71] their (b,h), [72..79]
 // their token counts.  [80..87]: stage s holds a tile skipped by screening.  qb: folded queries of the range's rows [kMaxRows][r];
-// xs: one input row of a projection [256].
-__host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k, int fused_r = 0) {
+// xs: one input row of a projection [256].  nb: screening bounds of the CTA's
+// first nb_cap tiles (the space left over by the ring, never a stage of it).
+__host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap, int k, int fused_r = 0,
+                                                  int nb_cap = 0) {
     StreamSmem L;
     size_t o = 0;
     // the ring and the epoch buffers first: one contiguous region that the
@@ -92,7 +94,7 @@ __host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap,
     L.ei = o;
     o = al(o + (size_t)kEB * ept * 4, 16);
     L.bars = o;
-    o = al(o + (size_t)(2 * nstages + 2 * kEB + kMaxRows + 1) * 8, 16);
+    o = al(o + (size_t)(2 * nstages + 2 * kEB + kMaxRows + 2) * 8, 16);
     L.rk = o;
     o = al(o + (size_t)cap * 4, 16);
     L.ri = o;
@@ -108,7 +110,9 @@ __host__ __device__ inline StreamSmem stream_smem(int nstages, int ept, int cap,
     L.qb = o;
     o = al(o + (size_t)kMaxRows * fused_r * 4, 16);
     L.xs = o;
-    o = al(o + (fused_r ? 256 * 4 : 0), 128);
+    o = al(o + (fused_r ? 256 * 4 : 0), 16);
+    L.nb = o;
+    o = al(o + (size_t)nb_cap * 4, 128);
     L.total = o;
     return L;
 }
@@ -948,17 +952,23 @@ __device__ void sel_append(const ScanArgs &a, const StepExtra &x, int bh, int po
     sel_sync();
     sel_dots<R>(xs, x.P + (size_t)h * d * R, d, part, st);
     __nv_bfloat16 *Kt = static_cast<__nv_bfloat16 *>(const_cast<void *>(a.src));
-    for (int j = st; j < R; j += kSelT)
-        Kt[((size_t)bh * a.T_cap + pos) * R + j] = __float2bfloat16_rn(sum_parts(part, j, d / kChunkD));
-    if (a.norms && st == 0) {
-        // screening bound of the row's block raised to cover the new row
-        float ss = 0.f;
-        for (int j = 0; j < R; ++j) {
-            const float v = __bfloat162float(__float2bfloat16_rn(sum_parts(part, j, d / kChunkD)));
-            ss = fmaf(v, v, ss);
+    for (int j = st; j < R; j += kSelT) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(sum_parts(part, j, d / kChunkD));
+        Kt[((size_t)bh * a.T_cap + pos) * R + j] = v;
+        if (a.norms) {
+            const float f = __bfloat162float(v);
+            xs[j] = f * f;  // the input row is no longer read (sel_dots ended on a barrier)
         }
-        atomicMax(reinterpret_cast<int *>(a.norms + (size_t)bh * a.norm_blocks + pos / JSSA_NORM_BLOCK),
-                  __float_as_int(sqrtf(ss)));
+    }
+    if (a.norms) {
+        // screening bound of the row's block raised to cover the new row
+        sel_sync();
+        if (st == 0) {
+            float ss = 0.f;
+            for (int j = 0; j < R; ++j) ss += xs[j];
+            atomicMax(reinterpret_cast<int *>(a.norms + (size_t)bh * a.norm_blocks + pos / JSSA_NORM_BLOCK),
+                      __float_as_int(sqrtf(ss)));
+        }
     }
     fence_proxy_async_global();
     sel_sync();
@@ -1221,13 +1231,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
 
     extern __shared__ __align__(128) unsigned char smem[];
     const int S_ = a.nstages;
-    const StreamSmem L = stream_smem(S_, EPT, a.cap, a.k, FUSED ? R : 0);
+    const StreamSmem L = stream_smem(S_, EPT, a.cap, a.k, FUSED ? R : 0, a.nb_cap);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + S_;
     uint64_t *efull = empty + S_;  // [kEB]
     uint64_t *efree = efull + kEB; // [kEB]
     uint64_t *qready = efree + kEB;       // fused: folded query of row i in shared memory [kMaxRows]
     uint64_t *aready = qready + kMaxRows;  // fused: new low-rank rows stored
+    uint64_t *nbready = aready + 1;        // screening: staged tile bounds written
     uint32_t *ek = reinterpret_cast<uint32_t *>(smem + L.ek);
     int32_t *ei = reinterpret_cast<int32_t *>(smem + L.ei);
     int *misc = reinterpret_cast<int *>(smem + L.misc);
@@ -1259,6 +1270,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
         }
         for (int i = 0; i < kMaxRows; ++i) mbar_init(&qready[i], 1);
         mbar_init(aready, 1);
+        mbar_init(nbready, 1);
         misc[46] = 0;
         fence_barrier_init();
         misc[0] = 0;
@@ -1273,7 +1285,35 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
 
     if (tid >= kProdBase && tid < kConsBase) {
         // ------------------------------------------------------ producer
-        if (tid == kProdBase) {
+        // Screening bound of a tile: the largest block norm over the blocks
+        // holding its n tokens (tiles and blocks align, or a tile lies in one block).
+        auto tile_bound = [&](int bh_, int t0_, int n_) {
+            const float *nr = a.norms + (size_t)bh_ * a.norm_blocks + t0_ / JSSA_NORM_BLOCK;
+            float m = 0.f;
+            for (int j = 0; j * JSSA_NORM_BLOCK < n_; ++j) m = fmaxf(m, __ldcg(nr + j));
+            return m;
+        };
+        float *nbs = reinterpret_cast<float *>(smem + L.nb);
+        const int nstaged = a.norms ? min(ntiles, a.nb_cap) : 0;
+        if (tid != kProdBase) {
+            // the warp's other lanes stage the bounds of the CTA's first
+            // nstaged tiles, so that none of their loads sits on the path of
+            // the copies (the ring is only a few stages deep)
+            for (int i = lane - 1; i < nstaged; i += 31) {
+                const int tt = c0.t + i, rr = tt / c0.tpb;  // tile i of the range: row c0.bh + rr
+                const int bh_ = c0.bh + rr, t0_ = (tt - rr * c0.tpb) * TILE;
+                const int Tb_ = clamp_seq(__ldg(a.seq_lens + bh_ / a.Hkv), a.T_cap, nullptr);
+                const float *nr = a.norms + (size_t)bh_ * a.norm_blocks + t0_ / JSSA_NORM_BLOCK;
+                const int n_ = min(TILE, Tb_ - t0_);
+                float m = 0.f;
+#pragma unroll
+                for (int j = 0; j < (TILE + JSSA_NORM_BLOCK - 1) / JSSA_NORM_BLOCK; ++j)
+                    if (j * JSSA_NORM_BLOCK < n_) m = fmaxf(m, __ldcg(nr + j));
+                nbs[i] = m;
+            }
+            __syncwarp(0xfffffffeu);
+            if (lane == 1) mbar_arrive(nbready);
+        } else {
             const char *src = static_cast<const char *>(a.src);
             const uint64_t pol = policy_evict_first();
             int issued = 0;
@@ -1281,19 +1321,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
             RingPos rp(S_);
             int Tb = 0, atile = -1;
             bool appended = false;
+            bool staged = nstaged == 0;  // staged bounds visible to this thread
             float qn = -1.f;  // ||qbar|| of the current row (screening), -1 while unknown
-            // screening: the block bounds of a tile are loaded one tile ahead
-            // (after the previous tile's copy is issued), so that their
-            // latency hides behind the ring
-            constexpr int NBT = (TILE + JSSA_NORM_BLOCK - 1) / JSSA_NORM_BLOCK;
-            float nbv[NBT];
-            auto load_bounds = [&](int bh_, int t0_) {
-                const float *nr = a.norms + (size_t)bh_ * a.norm_blocks + t0_ / JSSA_NORM_BLOCK;
-                const int nblk = min(NBT, a.norm_blocks - t0_ / JSSA_NORM_BLOCK);
-#pragma unroll
-                for (int j = 0; j < NBT; ++j) nbv[j] = j < nblk ? __ldcg(nr + j) : 0.f;
-            };
-            if (a.norms && ntiles > 0) load_bounds(cur.bh, cur.t * TILE);
             for (int i = 0; i < ntiles; ++i, cur.next(), rp.next()) {
                 const int s = rp.s;
                 const int bh = cur.bh, t0 = cur.t * TILE;
@@ -1309,21 +1338,23 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                     *abort_flag = 1;
                     break;
                 }
+                bool newrow = false;  // this tile holds the row appended in the prologue
                 if (FUSED && !appended && cur.t == atile) {
-                    // this tile holds the row appended in the prologue
                     if (!wait_or_abort(aready, 0u, abort_flag)) {
                         *abort_flag = 1;
                         break;
                     }
                     appended = true;
-                    if (a.norms) load_bounds(bh, t0);  // its block's bound was raised for the new row
+                    newrow = true;
                 }
                 const int n = min(TILE, Tb - t0);
                 // exact screening: skip the tile when ||qbar|| times its blocks'
                 // norm bound (inflated for fp32 rounding) cannot beat the key
-                // the row's segment already holds k candidates above
+                // the row's segment already holds k candidates above.  The tile
+                // of the new row is not screened: its staged bound may predate
+                // the prologue's raise.
                 bool skip = false;
-                if (a.norms && n > 0) {
+                if (a.norms && n > 0 && !newrow) {
                     const bool tforce = t0 < a.n_sink || t0 + TILE > Tb - a.n_recent;
                     const unsigned long long tw = *thr_word;
                     if (!tforce && (uint32_t)(tw >> 32) == (uint32_t)bh + 1u) {
@@ -1344,13 +1375,14 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                                 qn = sqrtf(ss);
                             }
                         }
-                        if (qn >= 0.f) {
-                            float nb = 0.f;
-#pragma unroll
-                            for (int j = 0; j < NBT; ++j)
-                                if (j * JSSA_NORM_BLOCK < n) nb = fmaxf(nb, nbv[j]);
-                            skip = score_key(qn * nb * 1.0001f) <= (uint32_t)tw;
+                        float nb = -1.f;
+                        if (i < nstaged) {
+                            if (!staged) staged = mbar_test_wait(nbready, 0u);
+                            if (staged) nb = nbs[i];
+                        } else {
+                            nb = tile_bound(bh, t0, n);
                         }
+                        if (qn >= 0.f && nb >= 0.f) skip = score_key(qn * nb * 1.0001f) <= (uint32_t)tw;
                     }
                 }
                 misc[80 + s] = skip ? 1 : 0;
@@ -1363,11 +1395,6 @@ __global__ void __launch_bounds__(kThreads, 1) stream_select_kernel(StreamArgs A
                     if (skip && a.skip_count) atomicAdd(a.skip_count, 1u);
                 }
                 issued = i + 1;
-                if (a.norms && i + 1 < ntiles) {
-                    Cursor nx = cur;
-                    nx.next();
-                    load_bounds(nx.bh, nx.t * TILE);
-                }
             }
             misc[24] = issued;
         }
@@ -1704,13 +1731,6 @@ cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T
     while (ns >= 3 && stream_smem(ns, ept, P.cap, k, fused_r).total > (size_t)optin) --ns;
     if (ns < 3) return cudaErrorNotSupported;
     P.nstages = ns;
-    P.smem = stream_smem(ns, ept, P.cap, k, fused_r).total;
-    e = ensure_smem(reinterpret_cast<const void *>(kern), P.smem);
-    if (e != cudaSuccess) return e;
-    int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, P.smem);
-    if (e != cudaSuccess) return e;
-    if (occ < 1) return cudaErrorNotSupported;
     // one CTA per SM, but no row split into segments of fewer than
     // kMinSegTiles tiles: a short row streams faster than the cross-CTA merge
     // of its segments would take (a 4K-token row is one 256 KiB segment)
@@ -1720,6 +1740,20 @@ cudaError_t plan_common(void (*kern)(StreamArgs), int src, int B, int Hkv, int T
     if (g > P.total_tiles) g = P.total_tiles;
     if (g < 1) g = 1;
     P.grid = (int)g;
+    // screening bounds staged per CTA: as many tiles of its range as the
+    // space the ring leaves over holds (the rest load as they are needed)
+    const size_t base = stream_smem(ns, ept, P.cap, k, fused_r).total;
+    const long long per_cta = (P.total_tiles + g - 1) / g;
+    long long nb = ((long long)optin - (long long)base - 128) / 4;
+    if (nb > per_cta) nb = per_cta;
+    P.nb_cap = nb > 0 ? (int)nb : 0;
+    P.smem = stream_smem(ns, ept, P.cap, k, fused_r, P.nb_cap).total;
+    e = ensure_smem(reinterpret_cast<const void *>(kern), P.smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, P.smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorNotSupported;
     int ms = 1;
     const long long BH = (long long)B * Hkv;
     for (long long bh = 0; bh < BH; ++bh) {
@@ -1753,6 +1787,7 @@ void fill_plan(StreamArgs &A, const ScanPlan &p) {
     A.s.max_seg = p.max_seg;
     A.s.cap = p.cap;
     A.s.nstages = p.nstages;
+    A.s.nb_cap = p.nb_cap;
 }
 }  // namespace
 
