@@ -19,7 +19,10 @@
 // swizzled 16 KiB buffers; P is written to shared memory in the A-operand
 // layout.  TMEM holds S in columns 0..127, then O in columns 0..511.  Splits
 // write (unnormalised O, row max, row sum) and a combine kernel merges them by
-// log-sum-exp.
+// log-sum-exp.  Sixteen warps: warp w reads TMEM lanes 32 (w mod 4) .. +31
+// (its heads) and a quarter of the columns, w / 4, so that the softmax (32
+// logits per thread) and the readout of O (128 columns per thread) are four
+// short chains instead of one long one.
 #include "jssa_common.cuh"
 #include "jssa_internal.h"
 #include "jssa_tc.cuh"
@@ -28,13 +31,14 @@ namespace jssa {
 
 namespace {
 
-constexpr int kD = 576, kDv = 512, kH = 128, kTok = 128, kThr = 128;
+constexpr int kD = 576, kDv = 512, kH = 128, kTok = 128, kThr = 512;
+constexpr int kWG = kThr / 128;  // warpgroups: column quarters of S and O
 constexpr int kKB = 9;          // 64-column blocks of a latent row
 constexpr int kQBuf = 4;        // Q block buffers
 constexpr int kBlk = 16384;     // one block: 128 rows x 128 bytes
 constexpr size_t kSmemK = (size_t)kKB * kBlk;
 constexpr size_t kSmemQ = (size_t)kQBuf * kBlk;
-constexpr size_t kSmemMisc = 2048;
+constexpr size_t kSmemMisc = 2048 + 2 * kWG * kH * 4;  // barriers, tokens; row max / sum per quarter
 constexpr size_t kSmemBytes = kSmemK + kSmemQ + kSmemMisc;
 
 template <int N>
@@ -58,6 +62,8 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     uint32_t *tptr = reinterpret_cast<uint32_t *>(qfree + kQBuf + 2);
     int *flag = reinterpret_cast<int *>(tptr + 1);
     int *tok = reinterpret_cast<int *>(qfree + 8);  // [kTok]
+    float *red_m = reinterpret_cast<float *>(smem + kSmemK + kSmemQ + 2048);  // [kWG][kH]
+    float *red_l = red_m + kWG * kH;                                          // [kWG][kH]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, b = blockIdx.y;
@@ -95,7 +101,7 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
                      "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
     }
-    {
+    if (tid < kTok) {
         int t = -1;
         if (tid < rows) {
             t = INDEXED ? __ldg(a.idx + (size_t)b * a.k + p0 + tid) : p0 + tid;
@@ -179,54 +185,58 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     __syncthreads();
     ok = *flag == 0;
 
-    // ---- softmax over the tile's tokens, one head per thread (TMEM lane) --------
-    const int h = warp * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // ---- softmax over the tile's tokens: head = TMEM lane, 32 columns per warp --
+    const int q4 = warp & 3, cg = warp >> 2;  // lane quarter (heads), column quarter
+    const int h = q4 * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
     float m = -INFINITY, l = 0.f;
     if (ok) {
-        // the tile's live columns as bit masks (the same in every warp), and
-        // this head's 128 logits read from TMEM once
-        unsigned live[kTok / 32];
-#pragma unroll
-        for (int q = 0; q < kTok / 32; ++q) {
-            const int col = q * 32 + lane;
-            live[q] = __ballot_sync(0xffffffffu, col < rows && tok[col] >= 0);
-        }
-        float v[kTok / 32][32];
-#pragma unroll
-        for (int q = 0; q < kTok / 32; ++q) tmem_ld32(lane_base + q * 32, v[q]);
+        // this quarter's live columns as a bit mask (the same in every warp),
+        // and the head's 32 logits of the quarter read from TMEM once
+        const int col = cg * 32 + lane;
+        const unsigned live = __ballot_sync(0xffffffffu, col < rows && tok[col] >= 0);
+        float v[32];
+        tmem_ld32(lane_base + cg * 32, v);
         float mx = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < kTok / 32; ++q)
+        for (int j = 0; j < 32; ++j)
+            if ((live >> j) & 1u) mx = fmaxf(mx, v[j]);
+        red_m[cg * kH + h] = mx;
+        __syncthreads();
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if ((live[q] >> j) & 1u) mx = fmaxf(mx, v[q][j]);
+        for (int g = 0; g < kWG; ++g) mx = fmaxf(mx, red_m[g * kH + h]);
         m = mx == -INFINITY ? -INFINITY : mx * a.scale_log2;
+        float lp = 0.f;
 #pragma unroll
-        for (int q = 0; q < kTok / 32; ++q) {
+        for (int g8 = 0; g8 < 4; ++g8) {
+            uint32_t w[4];
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = g8 * 8 + e * 2;
-                    const float p0 = ((live[q] >> j) & 1u) ? exp2f(v[q][j] * a.scale_log2 - m) : 0.f;
-                    const float p1 = ((live[q] >> (j + 1)) & 1u) ? exp2f(v[q][j + 1] * a.scale_log2 - m) : 0.f;
-                    l += p0;
-                    l += p1;
-                    const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&pk);
-                }
-                const int c8 = q * 32 + g8 * 8, col8 = c8 & 63, blk = c8 >> 6;
-                *reinterpret_cast<uint4 *>(sP + (size_t)blk * kBlk + h * 128 + (((col8 >> 3) ^ (h & 7)) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 4; ++e) {
+                const int j = g8 * 8 + e * 2;
+                const float p0 = ((live >> j) & 1u) ? exp2f(v[j] * a.scale_log2 - m) : 0.f;
+                const float p1 = ((live >> (j + 1)) & 1u) ? exp2f(v[j + 1] * a.scale_log2 - m) : 0.f;
+                lp += p0;
+                lp += p1;
+                const __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+                w[e] = *reinterpret_cast<const uint32_t *>(&pk);
             }
+            const int c8 = cg * 32 + g8 * 8, col8 = c8 & 63, blk = c8 >> 6;
+            *reinterpret_cast<uint4 *>(sP + (size_t)blk * kBlk + h * 128 + (((col8 >> 3) ^ (h & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
         }
+        red_l[cg * kH + h] = lp;
+    } else {
+        __syncthreads();  // the exchange barrier of the branch above
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (ok) {
+        // the row sum in quarter order (every warp of the head adds the same way)
+#pragma unroll
+        for (int g = 0; g < kWG; ++g) l += red_l[g * kH + h];
+    }
 
     // ---- O = P V: V is the first 512 columns of the same rows (MN-major) --------
     constexpr uint32_t idO = mma_idesc(128, 256, 0, 1);
@@ -247,13 +257,14 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     ok = *flag == 0;
     if (!ok && tid == 0 && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
 
-    // ---- epilogue --------------------------------------------------------------
+    // ---- epilogue: this warp's heads, columns [128 cg, 128 cg + 128) of O ----------
     if (ok) {
+        const int cb = cg * (kDv / kWG);
         if (a.splits == 1) {
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * kH + h) * kDv;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kDv; c0 += 32) {
+            for (int c0 = cb; c0 < cb + kDv / kWG; c0 += 32) {
                 float v[32];
                 tmem_ld32(lane_base + c0, v);
 #pragma unroll
@@ -267,15 +278,16 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
                     *reinterpret_cast<uint4 *>(orow + c0 + j) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            if (a.lse) a.lse[(size_t)b * kH + h] = l > 0.f ? (m + log2f(l)) * 0.693147180559945309417f : -INFINITY;
+            if (a.lse && cg == 0)
+                a.lse[(size_t)b * kH + h] = l > 0.f ? (m + log2f(l)) * 0.693147180559945309417f : -INFINITY;
         } else {
             // unnormalised partial O in bf16, turned around per warp in shared
             // memory (the K blocks are free once the second product is done) so
             // that every store writes whole 128-byte rows: block [32 heads][64 columns]
             float *tb = reinterpret_cast<float *>(sK) + warp * (32 * 65);
-            __nv_bfloat16 *po = a.part_o + (((size_t)b * a.splits + split) * kH + warp * 32) * kDv;
+            __nv_bfloat16 *po = a.part_o + (((size_t)b * a.splits + split) * kH + q4 * 32) * kDv;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kDv; c0 += 64) {
+            for (int c0 = cb; c0 < cb + kDv / kWG; c0 += 64) {
                 float v[32];
                 tmem_ld32(lane_base + c0, v);
 #pragma unroll
@@ -298,9 +310,11 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
                 }
                 __syncwarp();
             }
-            float *pml = a.part_ml + (((size_t)b * a.splits + split) * kH + h) * 2;
-            pml[0] = m;
-            pml[1] = l;
+            if (cg == 0) {
+                float *pml = a.part_ml + (((size_t)b * a.splits + split) * kH + h) * 2;
+                pml[0] = m;
+                pml[1] = l;
+            }
         }
     }
     tc_fence_before();
