@@ -697,7 +697,7 @@ __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long l
     const long long c_first = ((first + 1) * a.grid - 1) / a.total_tiles;
     const long long c_last = ((first + tpb) * a.grid - 1) / a.total_tiles;
     const int slot = (int)(cta - c_first), nseg = (int)(c_last - c_first + 1);
-    if (S.st == 0) S.misc[9] = atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
+    if (S.st == 0) S.misc[9] = nseg == 1 || atomicAdd(&a.counters[bh], 1u) == (unsigned)(nseg - 1);
     sel_sync();
     const bool last = S.misc[9] != 0;
     sel_sync();
@@ -729,18 +729,20 @@ __device__ int sel_finish(const ScanArgs &a, const Sel &S, int n, int bh, long l
         }
         if (S.st == 0 && !flag_wait_bounded(a.counters + BH + bh, (unsigned)(nseg - 1)) && a.status)
             atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+        __threadfence();
     }
-    __threadfence();
-    sel_sync();
     // merge the other segments' slots; equal keys stay candidates (order is arbitrary)
-    if (S.st == 0) S.misc[3] = m;
-    sel_sync();
+    if (nseg > 1) {
+        sel_sync();
+        if (S.st == 0) S.misc[3] = m;
+        sel_sync();
+    }
     const int lane = S.st & 31;
     const size_t rowbase = (size_t)bh * a.max_seg * a.k;
     // a wave holds at most what the register-resident cut takes (the cut of
     // a larger set reads shared memory on every level: several times slower)
     const int wcap = max(min(cap, kRegKeys * kSelT), 2 * a.k);
-    for (int s0 = 0; s0 < nseg;) {
+    for (int s0 = 0; nseg > 1 && s0 < nseg;) {
         int nb = (wcap - m) / a.k;  // segments that fit before the next exact cut
         if (nb < 1) {
             thr = sel_reduce(S, m, a.k);
