@@ -781,6 +781,40 @@ def test_mla_indexed_decode_parity(k, sl):
     check_attention(out, lse, ref_o, ref_l, torch.bfloat16)
 
 
+@pytest.mark.parametrize("B", [3, 12])
+def test_mla_split_merge_forms(B):
+    """The 16 splits of a k = 2048 latent-cache decode merge inside the
+    attention kernel when all its CTAs fit on the GPU at once (B = 3: 48
+    CTAs), else in a second kernel (B = 12: 192 CTAs, above the 148 SMs);
+    both against the oracle, and twice in a row (the merge counters reset
+    themselves)."""
+    k = 2048
+    w = MW(B=B, T=2200, k=k, seed=70 + B)
+    sl = [2200 - 37 * b for b in range(B)]
+    (q, K, V, P, slh), (qd, Kd, Vd, Pd, sld) = draw(w, seq_lens=sl)
+    g = torch.Generator().manual_seed(71)
+    idx = torch.full((B, 1, k), -1, dtype=torch.int32)
+    cnt = torch.zeros((B, 1), dtype=torch.int32)
+    for b in range(B):
+        c = min(k, int(slh[b]))
+        cnt[b, 0] = c
+        idx[b, 0, :c] = torch.sort(torch.randperm(int(slh[b]), generator=g)[:c])[0].to(torch.int32)
+    dims = ops.make_dims(qd, Kd, None)
+    n, _ = ops.plan_info(dims, k, ops.OP_INDEXED_DECODE)
+    sms = torch.cuda.get_device_properties(DEV).multi_processor_count
+    assert n == (1 if 16 * B <= sms else 2), (n, B, sms)
+    ws = ops.new_workspace(dims, k, ops.OP_INDEXED_DECODE, DEV)
+    res = []
+    for _ in range(2):
+        out, lse = ops.indexed_decode(qd, Kd, None, idx.to(DEV), cnt.to(DEV), sld, w.scale, ws=ws)
+        torch.cuda.synchronize()
+        assert ops.device_status(ws) == 0
+        res.append((out.clone(), lse.clone()))
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    ref_o, ref_l = oracle.attend(q, K, None, idx, cnt, slh, w.scale, dv=512, v_aliases_k=True)
+    check_attention(res[0][0], res[0][1], ref_o, ref_l, torch.bfloat16)
+
+
 @pytest.mark.parametrize("T,sl", [(3000, [3000, 77]), (700, [129, 0]), (5000, [4097, 128])])
 def test_mla_dense_decode_parity(T, sl):
     """Full-KV attention over the latent cache (the dense comparison path of
@@ -979,8 +1013,9 @@ def test_forced_tokens_decode_step(fused):
 def test_decode_step_form_choice():
     """The decode step runs as one fused launch where it plans and k <= 256
     (also on short caches and small batches); a larger k keeps the
-    three-launch cluster form where that plans; the latent cache takes four
-    launches (prologue, cluster selection, attention, combine)."""
+    three-launch cluster form where that plans; the latent cache takes three
+    launches (prologue, cluster selection, attention with the split merge
+    inside: its 128 CTAs fit on the GPU at once), four where they do not."""
     from token_level_sparse_kv_b200.inputs import WORKLOADS, Workload
 
     def form(w):
@@ -996,4 +1031,5 @@ def test_decode_step_form_choice():
     n, text = form(Workload(**{**w.__dict__, "B": 1, "k": 1024}))
     assert n == 3 and "cluster" in text, (n, text)
     n, text = form(WORKLOADS["mla_64k_b8"])
-    assert n == 4, (n, text)
+    sms = torch.cuda.get_device_properties(DEV).multi_processor_count
+    assert n == (3 if 16 * 8 <= sms else 4), (n, text)

@@ -240,7 +240,7 @@ int layout_attend(const jssa_dims *d, const Shape &sh, int src, int npos, Layout
         L.ap.splits = mla_splits(npos);
         L.part_o = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * d->dv * 2);  // bf16
         L.part_ml = take(L.total, (size_t)d->B * L.ap.splits * d->Hq * 2 * 4);
-        L.att_ctr = take(L.total, (size_t)sh.BH * 4);
+        L.att_ctr = take(L.total, (size_t)sh.BH * 2 * 4);  // arrival and done counters of the split merge
         return JSSA_OK;
     }
     if (src != ATT_INDEXED && d->kv_dtype == JSSA_BF16) {
@@ -596,6 +596,7 @@ int run_mla(const jssa_dims *d, const void *q, const void *K, const int32_t *idx
     a.out = out;
     a.lse = lse;
     a.status = at<uint32_t>(ws, 0);
+    a.ctr = at<uint32_t>(ws, L.att_ctr);
     cudaError_t e = launch_mla(a, true, s, true);
     if (e != cudaSuccess) return cuda_fail(e, "launching the latent-cache indexed decode");
     return JSSA_OK;
@@ -676,7 +677,7 @@ int jssa_plan_info_ex(const jssa_dims *dims, int k, int op, int agg, const jssa_
     Layout L;
     if ((st = build_layout(dims, sh, k, op, agg, 0, choice_of(opts), L))) return st;
     const char *sel = L.csel ? "cluster" : (L.wspec ? "stream" : "scan");
-    const int att = sh.latent ? 1 + (L.ap.splits > 1 ? 1 : 0) : 1;
+    const int att = sh.latent ? 1 + (L.ap.splits > 1 && !mla_inline_combine(L.ap.splits, dims->B) ? 1 : 0) : 1;
     int n = 0;
     char text[160];
     switch (op) {
@@ -1322,7 +1323,8 @@ extern "C" int jssa_indexed_decode_noalloc(const jssa_dims *dims, const void *q,
     if ((st = noalloc_scratch(&ws))) return st;
     // the status word and the arrival counters must start at zero
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, S(stream));
-    if (e == cudaSuccess) e = cudaMemsetAsync(at<char>(ws, L.att_ctr), 0, (size_t)sh.BH * 4, S(stream));
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(at<char>(ws, L.att_ctr), 0, (size_t)sh.BH * 4 * (sh.latent ? 2 : 1), S(stream));
     if (e != cudaSuccess) return cuda_fail(e, "clearing the allocation-free scratch");
     // the latent-cache form keeps its split partials in the same array (the
     // layout's offsets all lie below L.total, checked above)

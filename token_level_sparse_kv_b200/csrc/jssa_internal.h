@@ -228,8 +228,13 @@ struct MlaArgs {
     void *out;                // [B, 128, 512] bf16
     float *lse;               // [B, 128] or null
     uint32_t *status;
+    uint32_t *ctr;            // [2 B] arrival / done counters of the in-kernel merge (self-resetting, start at 0)
+    int inline_combine;       // set by launch_mla: the splits merge inside the kernel
 };
 int mla_splits(int npos);
+// true when the splits of a latent-cache indexed decode merge inside its kernel
+// (every CTA of the grid resident at once) rather than in a second kernel
+bool mla_inline_combine(int splits, int B);
 cudaError_t launch_mla(const MlaArgs &a, bool indexed, cudaStream_t s, bool pdl);
 // Log-sum-exp merge of a.splits latent-cache partials into out / lse.
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t s, bool pdl);

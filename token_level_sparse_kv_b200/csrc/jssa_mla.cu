@@ -50,6 +50,65 @@ __device__ __forceinline__ void cp_wait_dyn(int n) {
     }
 }
 
+// The log-sum-exp merge of heads [h0, h1) of batch row b over the splits'
+// partials: one 8-column chunk of one head per thread and pass; the splits
+// are read sixteen at a time, every (max, sum) pair and partial of a group in
+// flight at once, and merged online (the running sums rescaled when a group
+// raises the maximum).
+__device__ void merge_heads(const MlaArgs &a, int b, int h0, int h1, int tid, int nthr) {
+    constexpr int GS = 16;
+    const int ns = a.splits;
+    const int items = (h1 - h0) * (kDv / 8);
+    for (int it = tid; it < items; it += nthr) {
+        const int h = h0 + it / (kDv / 8), c0 = (it % (kDv / 8)) * 8;
+        const float2 *pml = reinterpret_cast<const float2 *>(a.part_ml) + (size_t)b * ns * kH + h;
+        const __nv_bfloat16 *pbase = a.part_o + ((size_t)b * ns * kH + h) * kDv + c0;
+        float M = -INFINITY, L = 0.f, o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = 0.f;
+        for (int s0 = 0; s0 < ns; s0 += GS) {
+            float2 ml[GS];
+            uint4 v[GS];
+#pragma unroll
+            for (int u = 0; u < GS; ++u) {
+                const bool in = s0 + u < ns;
+                ml[u] = in ? __ldcg(pml + (size_t)(s0 + u) * kH) : make_float2(-INFINITY, 0.f);
+                v[u] = in ? __ldcg(reinterpret_cast<const uint4 *>(pbase + (size_t)(s0 + u) * kH * kDv))
+                          : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float mg = M;
+#pragma unroll
+            for (int u = 0; u < GS; ++u) mg = fmaxf(mg, ml[u].x);
+            if (mg == -INFINITY) continue;  // nothing live so far
+            const float r = exp2f(M - mg);  // 0 while M is -inf
+            L *= r;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] *= r;
+            M = mg;
+#pragma unroll
+            for (int u = 0; u < GS; ++u) {
+                if (ml[u].x == -INFINITY) continue;  // an empty split (or past the last)
+                const float w = exp2f(ml[u].x - M);
+                L = fmaf(ml[u].y, w, L);
+                float f[8];
+                Vec16<__nv_bfloat16>::unpack(v[u], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = fmaf(f[e], w, o[e]);
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pk = __floats2bfloat162_rn(o[2 * e] * inv, o[2 * e + 1] * inv);
+            w4[e] = *reinterpret_cast<const uint32_t *>(&pk);
+        }
+        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + ((size_t)b * kH + h) * kDv + c0) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        if (a.lse && c0 == 0) a.lse[(size_t)b * kH + h] = L > 0.f ? (M + log2f(L)) * 0.693147180559945309417f : -INFINITY;
+    }
+}
+
 template <bool INDEXED>
 __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -320,6 +379,33 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
     tc_fence_before();
     __syncthreads();
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    if (a.splits > 1 && a.inline_combine) {
+        // In-kernel merge (every CTA of the grid is resident at once, which
+        // the launch checks): each split publishes its partial (stores, then a
+        // fence and an arrival), waits for the other splits of its batch row,
+        // and merges its share of the heads.  The last CTA to finish resets
+        // the two counters for the next call.  A wait that runs out sets the
+        // timeout status and skips the merge.
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(a.ctr + b, 1u);
+            const bool all = flag_wait_bounded(a.ctr + b, (unsigned)a.splits);
+            __threadfence();
+            *flag = all ? 0 : 1;
+            if (!all && a.status) atomicOr(a.status, (uint32_t)JSSA_DEV_TIMEOUT);
+        }
+        __syncthreads();
+        if (*flag == 0) {
+            const int hps = (kH + a.splits - 1) / a.splits;
+            const int h0 = min(kH, split * hps), h1 = min(kH, h0 + hps);
+            merge_heads(a, b, h0, h1, tid, kThr);
+        }
+        __syncthreads();
+        if (tid == 0 && atomicAdd(a.ctr + a.B + b, 1u) == (unsigned)(a.splits - 1)) {
+            a.ctr[b] = 0u;
+            a.ctr[a.B + b] = 0u;
+        }
+    }
 }
 
 // Log-sum-exp merge of the splits: CTA (b, 4 heads), 16 output dims per thread.
@@ -381,13 +467,18 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(MlaArgs a) {
 
 int mla_splits(int npos) { return npos <= kTok ? 1 : (npos + kTok - 1) / kTok; }
 
+bool mla_inline_combine(int splits, int B) { return splits > 1 && (long long)splits * B <= device_sm_count(); }
+
 cudaError_t launch_mla(const MlaArgs &a0, bool indexed, cudaStream_t s, bool pdl) {
     MlaArgs a = a0;
     void (*k)(MlaArgs) = indexed ? mla_kernel<true> : mla_kernel<false>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(k), kSmemBytes);
     if (e != cudaSuccess) return e;
+    // the splits merge inside the kernel when every CTA fits on the GPU at
+    // once (one CTA per SM: its shared memory); else a second kernel merges
+    a.inline_combine = a.ctr && mla_inline_combine(a.splits, a.B);
     e = launch_kernel(k, dim3(a.splits, a.B), dim3(kThr), kSmemBytes, s, pdl, a);
-    if (e != cudaSuccess || a.splits == 1) return e;
+    if (e != cudaSuccess || a.splits == 1 || a.inline_combine) return e;
     return launch_mla_combine(a, s, pdl);
 }
 
