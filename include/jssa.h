@@ -270,7 +270,13 @@ JSSA_API int jssa_select_ex(const jssa_dims *dims, const void *q, const float *P
  * fp32 accumulation, split over the index list, log-sum-exp combine.
  * count may be NULL (then the count is the number of leading non-negative
  * slots).  An empty set gives out = 0, lse = -inf.  An index outside [0, T_b)
- * is skipped and sets JSSA_DEV_INDEX.  lse may be NULL. */
+ * is skipped and sets JSSA_DEV_INDEX.  lse may be NULL.
+ * Latent form: the 128-token splits of a batch row merge inside the attention
+ * kernel when all B * ceil(k / 128) of its CTAs fit on the device at once
+ * (one per SM), else in a second kernel.  The in-kernel merge waits, bounded,
+ * for the other splits of the batch row: if concurrent work on another stream
+ * keeps SMs from the kernel for longer than the limit, the call completes with
+ * JSSA_DEV_TIMEOUT in the status word and the affected rows undefined. */
 JSSA_API int jssa_indexed_decode(const jssa_dims *dims, const void *q, const void *K, const void *V,
                         const int32_t *idx, const int32_t *count, int k,
                         const int32_t *seq_lens, float softmax_scale, void *out, float *lse,
