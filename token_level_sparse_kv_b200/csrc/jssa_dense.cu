@@ -168,6 +168,12 @@ __global__ void __launch_bounds__(kThr, 1)
         fence_barrier_init();
         flags[0] = 0;
     }
+    if (tid == kNW * 32) {
+        // the tensor maps are kernel parameters: fetch them into the TMA
+        // unit's cache while the previous kernel may still be running
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+    }
     __syncthreads();
     pdl_trigger();
     pdl_wait();
@@ -426,6 +432,7 @@ __global__ void __launch_bounds__(kThr, 1)
 template <int D>
 __global__ void __launch_bounds__(D) dense_combine_kernel(DenseArgs a) {
     __shared__ float stat[2];
+    pdl_trigger();
     pdl_wait();
     const int bh = blockIdx.x, g = blockIdx.y, d = threadIdx.x;
     const int G = a.G, rt = a.row_tiles;
