@@ -883,7 +883,7 @@ int jssa_dense_decode(const jssa_dims *dims, const void *q, const void *K, const
     if ((st = check_attn_shape(dims, sh, false))) return st;
     if (window < 0) return fail(JSSA_ERR_INVALID_ARG, "window=%d is negative", window);
     if (sh.latent && window > 0 && window < dims->T_cap)
-        return fail(JSSA_ERR_UNSUPPORTED, "sliding-window attention over a latent cache has no kernel in this build");
+        return fail(JSSA_ERR_UNSUPPORTED, "sliding-window attention over a latent cache has no kernel in this library");
     REQUIRE_PTR(q);
     REQUIRE_PTR(K);
     REQUIRE_PTR(V);
