@@ -340,35 +340,33 @@ __global__ void __launch_bounds__(kThr, 1) mla_kernel(MlaArgs a) {
             if (a.lse && cg == 0)
                 a.lse[(size_t)b * kH + h] = l > 0.f ? (m + log2f(l)) * 0.693147180559945309417f : -INFINITY;
         } else {
-            // unnormalised partial O in bf16, turned around per warp in shared
-            // memory (the K blocks are free once the second product is done) so
-            // that every store writes whole 128-byte rows: block [32 heads][64 columns]
-            float *tb = reinterpret_cast<float *>(sK) + warp * (32 * 65);
-            __nv_bfloat16 *po = a.part_o + (((size_t)b * a.splits + split) * kH + q4 * 32) * kDv;
+            // unnormalised partial O in bf16: each thread converts its head's 128
+            // columns into a shared-memory row (the K blocks are free once the
+            // second product is done; a 1040-byte row stride keeps the 16-byte
+            // stores of a warp on distinct banks) and copies its 256-byte segment
+            // to the partial with one bulk copy
+            constexpr int kRowS = kDv * 2 + 16;
+            unsigned char *srow = sK + (size_t)h * kRowS + (size_t)cb * 2;
 #pragma unroll 1
-            for (int c0 = cb; c0 < cb + kDv / kWG; c0 += 64) {
+            for (int c0 = 0; c0 < kDv / kWG; c0 += 32) {
                 float v[32];
-                tmem_ld32(lane_base + c0, v);
+                tmem_ld32(lane_base + cb + c0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) tb[lane * 65 + j] = v[j];
-                tmem_ld32(lane_base + c0 + 32, v);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) tb[lane * 65 + 32 + j] = v[j];
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int row = i * 4 + (lane >> 3), col = (lane & 7) * 8;
-                    const float *src = tb + row * 65 + col;
+                for (int j = 0; j < 32; j += 8) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 pk = __floats2bfloat162_rn(src[2 * e], src[2 * e + 1]);
+                        const __nv_bfloat162 pk = __floats2bfloat162_rn(v[j + 2 * e], v[j + 2 * e + 1]);
                         w[e] = *reinterpret_cast<const uint32_t *>(&pk);
                     }
-                    *reinterpret_cast<uint4 *>(po + (size_t)row * kDv + c0 + col) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(srow + (size_t)(c0 + j) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-                __syncwarp();
             }
+            fence_async_smem();
+            __nv_bfloat16 *po = a.part_o + (((size_t)b * a.splits + split) * kH + h) * kDv + cb;
+            bulk_s2g(po, srow, (uint32_t)(kDv / kWG) * 2);
+            bulk_wait_all();  // the segment is in global memory before the split is published,
+            asm volatile("fence.proxy.async.global;" ::: "memory");  // and ordered before the arrival
             if (cg == 0) {
                 float *pml = a.part_ml + (((size_t)b * a.splits + split) * kH + h) * 2;
                 pml[0] = m;
