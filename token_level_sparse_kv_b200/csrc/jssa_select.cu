@@ -340,8 +340,11 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
 
     // ---- emit the selection in ascending token order -----------------------
     // Warp wp takes the contiguous tokens [jb, je) of the slice, 32 at a time
-    // (lane l reads token j0 + l, conflict-free); ballots order a step's
-    // selections and ties, the warp totals are scanned across the block.
+    // (lane l reads token j0 + l, conflict-free), and compacts its selected
+    // tokens and ties, in order, into the front of its own span of the key
+    // array (the keys are not read again; a step only writes entries it has
+    // already read): token index, bit 31 for a tie.  The warp totals are
+    // scanned across the block, and each warp then writes from its short list.
     const bool take_all = kb >= Tb;
     const bool ties_on = !take_all && kb > 0 && !whole;
     constexpr int NW = NT / 32;
@@ -357,8 +360,12 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
         const int j = j0 + lane;
         const bool ok = j < je;
         const uint32_t u = ok ? keys[j] : 0u;
-        cs += __popc(__ballot_sync(0xffffffffu, ok && sure_of(u)));
-        ce += __popc(__ballot_sync(0xffffffffu, ok && ties_on && (u & mask) == prefix));
+        const bool sure = ok && sure_of(u);
+        const bool tie = ok && ties_on && (u & mask) == prefix;
+        const unsigned mb = __ballot_sync(0xffffffffu, sure || tie);
+        if (sure || tie) keys[jb + cs + ce + __popc(mb & lt)] = (uint32_t)j | (tie ? 0x80000000u : 0u);
+        cs += __popc(__ballot_sync(0xffffffffu, sure));
+        ce += __popc(__ballot_sync(0xffffffffu, tie));
     }
     if (lane == 0) misc[32 + wp] = ce;
     __syncthreads();
@@ -381,17 +388,18 @@ __global__ void __launch_bounds__(NT, 2) select_cluster_kernel(CSelArgs a) {
     int32_t *out = a.idx_out + (size_t)bh * a.k;
     {
         int w = base + w_off, e = e0;
-        for (int j0 = jb; j0 < je; j0 += 32) {
-            const int j = j0 + lane;
-            const bool ok = j < je;
-            const uint32_t u = ok ? keys[j] : 0u;
-            const bool tie = ok && ties_on && (u & mask) == prefix;
+        const int cnt = cs + ce;
+        for (int i0 = 0; i0 < cnt; i0 += 32) {
+            const int i = i0 + lane;
+            const bool ok = i < cnt;
+            const uint32_t v = ok ? keys[jb + i] : 0u;
+            const bool tie = ok && (v >> 31);
             const unsigned tb = __ballot_sync(0xffffffffu, tie);
-            const bool sel = (ok && sure_of(u)) || (tie && e + __popc(tb & lt) < take_ties);
+            const bool sel = ok && (!tie || e + __popc(tb & lt) < take_ties);
             const unsigned sb = __ballot_sync(0xffffffffu, sel);
             if (sel) {
                 const int p = w + __popc(sb & lt);
-                if (p < a.k) out[p] = lo + j;
+                if (p < a.k) out[p] = lo + (int)(v & 0x7fffffffu);
             }
             w += __popc(sb);
             e += __popc(tb);
