@@ -18,8 +18,9 @@
 // the MN-major V operand of the second product); Q streams through four
 // swizzled 16 KiB buffers; P is written to shared memory in the A-operand
 // layout.  TMEM holds S in columns 0..127, then O in columns 0..511.  Splits
-// write (unnormalised O, row max, row sum) and a combine kernel merges them by
-// log-sum-exp.  Sixteen warps: warp w reads TMEM lanes 32 (w mod 4) .. +31
+// write (unnormalised O, row max, row sum), merged by log-sum-exp inside the
+// kernel when all its CTAs fit on the GPU at once, else by a second kernel
+// (mla_combine_kernel).  Sixteen warps: warp w reads TMEM lanes 32 (w mod 4) .. +31
 // (its heads) and a quarter of the columns, w / 4, so that the softmax (32
 // logits per thread) and the readout of O (128 columns per thread) are four
 // short chains instead of one long one.
